@@ -1,0 +1,345 @@
+"""Pins for the CPU oracle: each test checks the oracle against something other than itself
+(a library routine, a closed form, an invariant the mathematics fixes, or brute force on tiny
+inputs). Sources: "Technical Summary: ParisKV" (gist.science/paper/2602.07721), Methodology,
+Core Algorithmic Innovations 1-2."""
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+from long_context_kv_srht_b200 import workload
+
+D, M = 128, 8
+B = D // M
+
+
+def _signs(d, seed=0):
+    return np.where(np.random.default_rng(seed).integers(0, 2, d) == 1, -1, 1).astype(np.int8)
+
+
+def _rotation_matrix(d, signs):
+    """R built by applying the oracle to basis vectors (column j = R e_j)."""
+    cols = [oracle.rotate_f64(np.eye(d)[j], signs) for j in range(d)]
+    return np.stack(cols, axis=1)
+
+
+# ----------------------------------------------------------------------------- rotation
+@pytest.mark.parametrize("d", [4, 16, 128])
+def test_rotation_is_orthogonal(d):
+    R = _rotation_matrix(d, _signs(d, d))
+    np.testing.assert_allclose(R @ R.T, np.eye(d), atol=1e-12)
+
+
+@pytest.mark.parametrize("d", [8, 128])
+def test_rotation_is_sylvester_hadamard_times_signs(d):
+    s = _signs(d, 7)
+    R = _rotation_matrix(d, s)
+    ref = scipy.linalg.hadamard(d).astype(np.float64) * s[None, :].astype(np.float64) / np.sqrt(d)
+    np.testing.assert_allclose(R, ref, atol=1e-12)
+
+
+def test_rotation_closed_form_d4():
+    s = np.array([1, 1, 1, 1], np.int8)
+    np.testing.assert_allclose(oracle.rotate_f64(np.array([1.0, 0, 0, 0]), s), [0.5] * 4)
+    np.testing.assert_allclose(oracle.rotate_f64(np.array([0, 1.0, 0, 0]), s),
+                               [0.5, -0.5, 0.5, -0.5])
+    s2 = np.array([1, -1, 1, 1], np.int8)
+    np.testing.assert_allclose(oracle.rotate_f64(np.array([0, 1.0, 0, 0]), s2),
+                               [-0.5, 0.5, -0.5, 0.5])
+
+
+def test_normalized_rotation_unit_norm_and_norms():
+    rng = np.random.default_rng(1)
+    x = (rng.standard_normal((10000, D)) * rng.uniform(0.1, 30, (10000, 1))).astype(np.float32)
+    y, nr = oracle.normalize_rotate(x, _signs(D))
+    ny = np.linalg.norm(y.astype(np.float64), axis=1)
+    assert np.max(np.abs(ny - 1.0)) <= 1e-5
+    np.testing.assert_allclose(nr, np.linalg.norm(x.astype(np.float64), axis=1), rtol=1e-6)
+
+
+def test_normalized_rotation_zero_row():
+    x = np.zeros((2, D), np.float32)
+    x[1, 3] = 2.0
+    y, nr = oracle.normalize_rotate(x, _signs(D))
+    assert np.all(y[0] == 0) and nr[0] == 0
+    assert nr[1] == 2.0
+
+
+def test_rotation_preserves_inner_products():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((64, D)).astype(np.float32)
+    y, nr = oracle.normalize_rotate(x, _signs(D, 3))
+    xh = x.astype(np.float64) / np.linalg.norm(x.astype(np.float64), axis=1, keepdims=True)
+    np.testing.assert_allclose(y.astype(np.float64) @ y.T.astype(np.float64), xh @ xh.T, atol=2e-6)
+
+
+# ----------------------------------------------------------------------------- bucket ids
+def _centroids(m):
+    c = np.arange(1 << m)[:, None]
+    bits = (c >> np.arange(m)[None, :]) & 1
+    return np.where(bits == 1, -1.0, 1.0) / np.sqrt(m)   # [2^m, m], centroid id c
+
+
+@pytest.mark.parametrize("m", [2, 4, 8])
+def test_bucket_id_is_nearest_analytic_centroid(m):
+    rng = np.random.default_rng(4)
+    d = 16 * m if m < 8 else D
+    y = rng.standard_normal((300, d)).astype(np.float32)
+    y[::3, ::5] = 0.0          # exact zeros: ties between centroids -> lower id
+    y[1::7, 2] = -0.0
+    nr = np.ones(300, np.float32)
+    enc = oracle.encode_rotated(y, nr, m)
+    C = _centroids(m)
+    for i in range(y.shape[0]):
+        for b in range(d // m):
+            yb = y[i, b * m:(b + 1) * m].astype(np.float64)
+            ip = C @ yb
+            dist = np.sum((C - yb[None, :]) ** 2, axis=1)
+            best_ip = int(np.flatnonzero(ip == ip.max())[0])       # lowest id among ties
+            best_dist = int(np.flatnonzero(dist == dist.min())[0])
+            assert enc.ids[i, b] == best_ip == best_dist
+
+
+# ----------------------------------------------------------------------------- RSQ codes
+def test_codes_uniform_levels_exact_values():
+    mx = 0.5
+    yb = np.array([mx, -mx, mx * 3 / 7, -mx * 2.49 / 7, mx * 2.51 / 7, 0.0, -0.0, -mx * 0.4 / 7],
+                  np.float32)
+    y = np.zeros((1, D), np.float32)
+    y[0, :8] = yb
+    enc = oracle.encode_rotated(y, np.ones(1, np.float32), M)
+    assert list(enc.mag[0, :8]) == [7, 7, 3, 2, 3, 0, 0, 0]
+    assert list(enc.neg[0, :8]) == [0, 1, 0, 1, 0, 0, 0, 1]
+    assert list(enc.codes[0, :8]) == [7, 15, 3, 10, 3, 0, 0, 8]
+    # all-zero subspaces: codes 0, factor 0
+    assert np.all(enc.mag[0, 8:] == 0) and np.all(enc.factor[0, 1:] == 0)
+
+
+def test_codes_nearest_uniform_level():
+    rng = np.random.default_rng(5)
+    y = rng.standard_normal((2000, D)).astype(np.float32)
+    enc = oracle.encode_rotated(y, np.ones(2000, np.float32), M)
+    yb = np.abs(y.reshape(2000, B, M)).astype(np.float64)
+    mx = yb.max(axis=2, keepdims=True)
+    lvl = enc.mag.reshape(2000, B, M) * mx / 7.0
+    assert np.all(np.abs(yb - lvl) <= mx / 14.0 * (1 + 1e-6))       # nearest of 8 levels
+    assert np.all(enc.mag.reshape(2000, B, M).max(axis=2) == 7)      # the max maps to level 7
+    np.testing.assert_array_equal(enc.neg, (y < 0).astype(np.uint8))
+
+
+# ----------------------------------------------------------------------------- estimator
+def _literal_terms(enc, y, knorm, qt):
+    """The page's estimator written literally in fp64: w = ||k|| ||y_b|| / <u_b, v_b>,
+    term_b = w * <v_b, q~_b> with v_b the normalised dequantised direction."""
+    n = y.shape[0]
+    yb = y.reshape(n, B, M).astype(np.float64)
+    vt = enc.vt.reshape(n, B, M)
+    nyb = np.linalg.norm(yb, axis=2)
+    nvt = np.linalg.norm(vt, axis=2)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        u = yb / nyb[..., None]
+        v = vt / nvt[..., None]
+        w = knorm.astype(np.float64)[:, None] * nyb / np.sum(u * v, axis=2)
+        terms = w * np.sum(v * qt.reshape(B, M).astype(np.float64)[None], axis=2)
+    return np.nan_to_num(terms)
+
+
+def test_folded_factor_equals_literal_page_form():
+    rng = np.random.default_rng(6)
+    sg = _signs(D, 9)
+    k = (rng.standard_normal((500, D)) * 3 + 1).astype(np.float32)
+    q = rng.standard_normal((1, D)).astype(np.float32)
+    y, kn = oracle.normalize_rotate(k, sg)
+    qt, qn = oracle.normalize_rotate(q, sg)
+    enc = oracle.encode_rotated(y, kn, M)
+    lit = _literal_terms(enc, y, kn, qt[0])
+    folded = enc.factor.astype(np.float64) * np.sum(
+        enc.vt.reshape(500, B, M) * qt[0].reshape(B, M).astype(np.float64)[None], axis=2)
+    scale = kn.astype(np.float64)[:, None]
+    assert np.max(np.abs(folded - lit) / scale) <= 1e-5
+    # full estimate from the fp32 rerank vs the literal fp64 sum
+    cand = np.arange(500, dtype=np.int32)
+    S = oracle.rerank(enc, cand, qt[0], M).astype(np.float64)
+    est = float(qn[0]) * S
+    est_lit = float(qn[0]) * lit.sum(axis=1)
+    assert np.max(np.abs(est - est_lit) / (kn * qn[0])) <= 1e-5
+
+
+def test_estimate_of_key_with_itself_is_squared_norm():
+    rng = np.random.default_rng(7)
+    sg = _signs(D, 11)
+    k = (rng.standard_normal((200, D)) * rng.uniform(0.5, 5, (200, 1))).astype(np.float32)
+    y, kn = oracle.normalize_rotate(k, sg)
+    enc = oracle.encode_rotated(y, kn, M)
+    for i in range(0, 200, 20):
+        one = oracle.Encoded(enc.ids[i:i + 1], enc.mag[i:i + 1], enc.neg[i:i + 1],
+                             enc.factor[i:i + 1])
+        lit = _literal_terms(one, y[i:i + 1], kn[i:i + 1], y[i])
+        k2 = float(kn[i]) ** 2
+        # in real arithmetic the estimate of <k,k> is ||k||^2 ||y||^2 exactly (||y|| = 1 up to
+        # the fp32 rounding of y)
+        y2 = float(np.sum(y[i].astype(np.float64) ** 2))
+        assert abs(float(kn[i]) * lit.sum() - k2 * y2) <= 1e-12 * k2
+        assert abs(y2 - 1.0) <= 1e-6
+        S = oracle.rerank(enc, np.array([i], np.int32), y[i], M)[0]
+        assert abs(float(kn[i]) * float(S) - k2) <= 2e-6 * k2
+
+
+def test_exact_subspaces_single_coordinate_and_equal_magnitudes():
+    rng = np.random.default_rng(8)
+    y = np.zeros((1, D), np.float32)
+    y[0, 3] = 0.6                                  # subspace 0: one non-zero coordinate
+    y[0, 8:16] = 0.2 * np.array([1, -1, 1, 1, -1, -1, 1, -1])   # subspace 1: equal magnitudes
+    y[0, 16:] = rng.standard_normal(D - 16).astype(np.float32) * 0.05
+    kn = np.array([3.0], np.float32)
+    enc = oracle.encode_rotated(y, kn, M)
+    qt = rng.standard_normal(D).astype(np.float32)
+    lit = _literal_terms(enc, y, kn, qt)[0]
+    exact = 3.0 * np.array([np.dot(y[0, 0:8].astype(np.float64), qt[0:8]),
+                            np.dot(y[0, 8:16].astype(np.float64), qt[8:16])])
+    np.testing.assert_allclose(lit[:2], exact, rtol=1e-6, atol=1e-7)
+
+
+def test_estimate_converges_as_levels_refine():
+    rng = np.random.default_rng(9)
+    sg = _signs(D, 13)
+    k = (rng.standard_normal((400, D)) + 0.3).astype(np.float32)
+    q = rng.standard_normal((1, D)).astype(np.float32)
+    y, kn = oracle.normalize_rotate(k, sg)
+    qt, qn = oracle.normalize_rotate(q, sg)
+    exact = k.astype(np.float64) @ q[0].astype(np.float64)
+    denom = np.linalg.norm(k.astype(np.float64), axis=1) * np.linalg.norm(q[0].astype(np.float64))
+    errs = []
+    for bits in range(3, 21):
+        L = (1 << bits) - 1
+        enc = oracle.encode_rotated(y, kn, M, levels=L)
+        lit = _literal_terms(enc, y, kn, qt[0])
+        est = float(qn[0]) * lit.sum(axis=1)
+        errs.append(float(np.mean(np.abs(est - exact) / denom)))
+    for a, b in zip(errs[:-1], errs[1:]):
+        assert b <= a * 1.05, errs             # non-increasing up to sampling noise
+    assert errs[-1] <= 1e-4 and errs[0] > 10 * errs[-1]
+
+
+# ----------------------------------------------------------------------------- query LUT
+@pytest.mark.parametrize("rho", [1, 2, 4, 16, 256])
+def test_query_top_rho_is_brute_force(rho):
+    rng = np.random.default_rng(10 + rho)
+    C = _centroids(M)
+    checked = 0
+    for trial in range(20):
+        qt = rng.standard_normal(D).astype(np.float32)
+        lut = oracle.query_lut(qt, M, rho, 2, 1)
+        for b in range(B):
+            ip = C @ qt[b * M:(b + 1) * M].astype(np.float64)
+            order = np.argsort(-ip, kind="stable")   # descending, ties -> lower id
+            if rho < 256 and ip[order[rho - 1]] - ip[order[rho]] <= 1e-6:
+                continue
+            sel = set(np.flatnonzero(lut[b]).tolist())
+            assert sel == set(order[:rho].tolist())
+            assert lut[b, order[0]] == 2
+            assert all(lut[b, c] == 1 for c in order[1:rho])
+            c1 = sum(1 << j for j in range(M) if qt[b * M + j] < 0)
+            assert order[0] == c1
+            checked += 1
+    assert checked > 200
+
+
+# ----------------------------------------------------------------------------- vote
+def test_vote_invariants():
+    rng = np.random.default_rng(11)
+    sg = _signs(D, 5)
+    q = rng.standard_normal((1, D)).astype(np.float32)
+    qt, _ = oracle.normalize_rotate(q, sg)
+    lut = oracle.query_lut(qt[0], M, 4, 2, 1)
+    # keys: the query itself at several positive scales, random keys, and a key whose every
+    # subspace sits in the rank-2 bucket
+    keys = np.concatenate([q * 0.5, q * 7.0, rng.standard_normal((200, D)).astype(np.float32)])
+    y, kn = oracle.normalize_rotate(keys, sg)
+    enc = oracle.encode_rotated(y, kn, M)
+    rank2 = np.array([[int(np.flatnonzero(lut[b] == 1)[0]) for b in range(B)]], np.uint8)
+    ids = np.concatenate([enc.ids, rank2])
+    sc = oracle.vote(ids, lut, M)
+    assert sc[0] == sc[1] == 2 * B
+    assert sc[-1] == B
+    assert np.all((sc >= 0) & (sc <= 2 * B))
+    assert np.bincount(sc, minlength=2 * B + 1).sum() == ids.shape[0]
+
+
+# ----------------------------------------------------------------------------- selections
+@pytest.mark.parametrize("n,k,bp,want", [(4096, 64, 1000, 410), (131072, 2048, 500, 6554),
+                                          (1 << 20, 4096, 500, 52429), (100, 64, 500, 64),
+                                          (50, 50, 500, 50), (33, 1, 10000, 33)])
+def test_candidate_count(n, k, bp, want):
+    assert oracle.candidate_count(n, k, bp) == want
+
+
+@pytest.mark.parametrize("n,C", [(1, 1), (31, 7), (4096, 410), (5000, 5000)])
+def test_select_candidates_is_stable_sort(n, C):
+    rng = np.random.default_rng(n)
+    sc = rng.integers(0, 6, n).astype(np.int32)        # many ties
+    got = oracle.select_candidates(sc, C)
+    order = np.argsort(-sc, kind="stable")[:C]
+    np.testing.assert_array_equal(got, np.sort(order))
+
+
+@pytest.mark.parametrize("C,k", [(1, 1), (410, 64), (3000, 3000), (6554, 2048)])
+def test_topk_is_stable_sort(C, k):
+    rng = np.random.default_rng(C + k)
+    S = rng.standard_normal(C).astype(np.float32)
+    S[::5] = S[0]                                       # ties -> lower key index wins
+    cand = np.sort(rng.choice(10 * C + 10, C, replace=False)).astype(np.int32)
+    idx, so = oracle.topk(S, cand, k)
+    order = np.lexsort((cand, -S.astype(np.float64)))[:k]
+    keep = np.sort(cand[order])
+    np.testing.assert_array_equal(idx, keep)
+    np.testing.assert_array_equal(so, S[np.searchsorted(cand, keep)])
+
+
+# ----------------------------------------------------------------------------- attention
+def test_attend_dense_equals_sdpa():
+    rng = np.random.default_rng(12)
+    n = 300
+    q = rng.standard_normal(D).astype(np.float32)
+    K = rng.standard_normal((n, D)).astype(np.float32)
+    V = rng.standard_normal((n, D)).astype(np.float32)
+    out = oracle.attend(q, K, V, np.arange(n, dtype=np.int32), 1 / np.sqrt(D))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).double()[None, None, None], torch.from_numpy(K).double()[None, None],
+        torch.from_numpy(V).double()[None, None])[0, 0, 0].numpy()
+    np.testing.assert_allclose(out, ref, atol=1e-12)
+    # a subset equals dense attention over the gathered rows
+    idx = np.sort(rng.choice(n, 40, replace=False)).astype(np.int32)
+    sub = oracle.attend(q, K, V, idx, 0.1)
+    ref2 = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).double()[None, None, None],
+        torch.from_numpy(K[idx]).double()[None, None], torch.from_numpy(V[idx]).double()[None, None],
+        scale=0.1)[0, 0, 0].numpy()
+    np.testing.assert_allclose(sub, ref2, atol=1e-12)
+
+
+def test_attend_equal_logits_is_mean():
+    rng = np.random.default_rng(13)
+    K = np.tile(rng.standard_normal(D).astype(np.float32), (50, 1))
+    V = rng.standard_normal((50, D)).astype(np.float32)
+    out = oracle.attend(rng.standard_normal(D).astype(np.float32), K, V,
+                        np.arange(50, dtype=np.int32), 0.3)
+    np.testing.assert_allclose(out, V.astype(np.float64).mean(axis=0), atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- end to end
+def test_tiny_workload_retrieves_planted_keys():
+    """Informational check of the method on the tiny workload: the planted near-duplicates of
+    the query are retrieved, and top-k recall against the exact <k,q> top-k is high."""
+    sp = workload.SPECS["tiny"]
+    w = workload.generate(sp)
+    p = oracle.SearchParams(m=sp.m, rho=sp.rho, cand_bp=sp.cand_bp)
+    enc = oracle.build_unit(w.keys[0, 0], w.signs, sp.m)
+    idx, s, est, cand, sc = oracle.search(enc, w.queries[0, 0], w.signs, sp.k, p)
+    planted = set(w.planted[0, 0].tolist())
+    assert len(planted & set(idx.tolist())) / len(planted) >= 0.9
+    exact = w.keys[0, 0].astype(np.float64) @ w.queries[0, 0].astype(np.float64)
+    true_top = set(np.argsort(-exact, kind="stable")[:sp.k].tolist())
+    recall = len(true_top & set(idx.tolist())) / sp.k
+    assert recall >= 0.5, recall
