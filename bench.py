@@ -1,0 +1,395 @@
+#!/usr/bin/env python
+"""Benchmark of the ParisKV decode-step retrieval path on B200.
+
+Metric: keys searched per second per decode step (query prep + collision vote + candidate
+select + RSQ-IP rerank + top-k), i.e. batch * query heads * cached keys / search time, and
+the achieved fraction of the HBM roofline of the dominant kernel.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload million_offload]
+    python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+Default workload: the million-token offload decode step (batch 1, 32 query / 8 KV heads,
+d = 128, N = 1,048,576 cached keys, 5% candidates, k = 4096; index in HBM, bf16 K/V in pinned
+host memory read over UVA by the sparse attention). Inputs are synthetic (seeded, see
+long_context_kv_srht_b200/workload.py). Multi-GPU runs are weak-scaled replicas: every rank
+holds its own sequences; the only collectives are the timing barrier and max-reduction.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_FLUSH_BYTES = 256 << 20
+APPEND_SLACK = 64
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="million_offload")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------------ dist
+def dist_setup(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def dist_max(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(ws: int):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampled every 100 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: int):
+        try:
+            import torch
+            self.gpu = "GPU-" + str(torch.cuda.get_device_properties(gpu).uuid)
+        except Exception:
+            self.gpu = str(gpu)
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
+        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------ helpers
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, only while the kernel source is
+    unchanged since the capture (its sha256 is stored next to the figure)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload)
+    if not e:
+        return None
+    src = os.path.join(ROOT, "long_context_kv_srht_b200", "csrc", e["source"])
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    return e["dram_bytes_per_launch"] if sha == e["sha256"] else None
+
+
+def algorithmic_bytes(stage: str, sp, C: int) -> int:
+    """Bytes a stage must move per launch: the vote reads 16 B of ids per key per KV head;
+    the rerank reads one 128 B record per candidate per query head."""
+    units = sp.batch * sp.num_kv_heads
+    packs = -(-sp.group // 4)
+    if stage == "vote":
+        return units * packs * sp.n * 16
+    if stage == "rerank":
+        return sp.batch * sp.num_q_heads * C * 128
+    return 0
+
+
+def candidate_count(n, k, bp):
+    return min(n, max(k, -(-n * bp // 10000)))
+
+
+# ------------------------------------------------------------------------------------ oracle
+def oracle_sample(sp, data, reps: int, heads: int = 4):
+    """Times the CPU oracle (as it stands) on one (sequence, KV head) unit of the workload:
+    index build untimed, then `reps` searches of `heads` query heads over all n keys."""
+    import oracle
+    keys = data["keys"][0, 0, :sp.n].float().cpu().numpy()
+    qs = data["queries"][0, :heads].float().cpu().numpy()
+    signs = data["signs"].numpy()
+    p = oracle.SearchParams(m=sp.m, rho=sp.rho, cand_bp=sp.cand_bp)
+    enc = oracle.build_unit(keys, signs, sp.m)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        for g in range(heads):
+            oracle.search(enc, qs[g], signs, sp.k, p)
+    dt = time.perf_counter() - t0
+    keys_done = reps * heads * keys.shape[0]
+    return keys_done / dt, dt, oracle.num_threads()
+
+
+def run_reference(args, ws, rank):
+    """The reference arm: the CPU oracle on the host cores, for the same metric/workload."""
+    if rank != 0:
+        return
+    import torch
+    from long_context_kv_srht_b200 import workload
+    sp = workload.spec(args.workload)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    one = workload.spec(args.workload, batch=1, num_kv_heads=1)
+    data = workload.generate_torch(one, dev)
+    import oracle
+    keys = data["keys"][0, 0].float().cpu().numpy()
+    qs = data["queries"][0].float().cpu().numpy()
+    signs = data["signs"].numpy()
+    p = oracle.SearchParams(m=sp.m, rho=sp.rho, cand_bp=sp.cand_bp)
+    enc = oracle.build_unit(keys, signs, sp.m)
+    for i in range(args.warmup):
+        oracle.search(enc, qs[i % sp.group], signs, sp.k, p)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.search(enc, qs[i % sp.group], signs, sp.k, p)
+    dt = time.perf_counter() - t0
+    value = args.steps * keys.shape[0] / dt
+    line = {
+        "impl": "reference", "metric": "keys searched/s per decode step (vote+rerank+top-k)",
+        "value": value, "unit": "keys/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": sp.name, "sample": "1 query head x 1 (sequence, KV head) unit",
+                   "n": sp.n, "k": sp.k, "cand_bp": sp.cand_bp},
+        "cpu_baseline": {"value": value, "unit": "keys/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: one query head over one unit's {sp.n} keys"},
+        "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------ main
+def main():
+    args = parse()
+    ws, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, ws, rank)
+        return
+    import numpy as np
+    import torch
+    from long_context_kv_srht_b200 import pariskv as pk
+    from long_context_kv_srht_b200 import workload
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    base = workload.spec(args.workload)
+    sp = workload.spec(args.workload, seed=base.seed + 1000 * rank)
+    kv_host = sp.name == "million_offload"
+    # K/V hold APPEND_SLACK extra tokens after the n indexed ones: the decode-step measurement
+    # appends them to the index, so every index the search can return has a K/V row
+    data = workload.generate_torch(sp, dev, n=sp.n + APPEND_SLACK, kv_on_host=kv_host)
+    keys, vals, qs = data["keys"], data["values"], data["queries"]
+    cfg = pk.config(batch=sp.batch, num_kv_heads=sp.num_kv_heads, group=sp.group,
+                    capacity=sp.n + APPEND_SLACK, dtype=sp.dtype, rho=sp.rho,
+                    cand_bp=sp.cand_bp)
+    ix = pk.build_index(cfg, data["signs"], keys, n=sp.n)
+    H = sp.batch * sp.num_q_heads
+    k = sp.k
+    C = candidate_count(sp.n, k, sp.cand_bp)
+    idx = torch.empty((H, k), dtype=torch.int32, device=dev)
+    est = torch.empty((H, k), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ix.profile(True)
+    for _ in range(args.warmup):
+        ix.search(qs, k, idx, est)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    dist_barrier(ws)
+    torch.cuda.synchronize()
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stage_tot = {}
+    launches = 0
+    for s in range(args.steps):
+        flush.fill_(s & 255)                    # L2 flushed between timed steps
+        ev0[s].record()
+        ix.search(qs, k, idx, est)
+        ev1[s].record()
+        launches += pk.last_launch_count()
+        for name, ms in ix.stage_ms().items():
+            stage_tot[name] = stage_tot.get(name, 0.0) + ms
+    torch.cuda.synchronize()
+    dist_barrier(ws)
+    clk = clocks.stop()
+    step_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev0, ev1)]))
+    step_ms_max = dist_max(step_ms, ws)
+    keys_per_step = sp.batch * sp.num_q_heads * sp.n
+    value = ws * keys_per_step / (step_ms_max / 1e3)
+    stage_avg = {kname: v / args.steps for kname, v in stage_tot.items()}
+
+    # roofline of the dominant kernel (HBM-bound; no tensor-core work on this path)
+    dom = max(stage_avg, key=stage_avg.get)
+    peak, peak_kind = measured_peaks()
+    abytes = algorithmic_bytes(dom, sp, C)
+    achieved = abytes / (stage_avg[dom] / 1e3) / 1e9 if abytes else None
+    step_bytes = algorithmic_bytes("vote", sp, C) + algorithmic_bytes("rerank", sp, C)
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": (achieved / peak) if achieved else None,
+                "peak_kind": peak_kind, "algorithmic_bytes_per_launch": abytes,
+                "traffic": kernel_traffic(dom, sp.name),
+                "step_algorithmic_bytes": step_bytes,
+                "step_frac": step_bytes / (step_ms_max / 1e3) / 1e9 / peak}
+
+    # end to end through the C ABI: pinned host query in, top-k indices and estimates out
+    e2e = None
+    if not args.no_e2e:
+        q_host = qs.cpu().pin_memory()
+        q_dev = torch.empty_like(qs)
+        i_host = torch.empty((H, k), dtype=torch.int32).pin_memory()
+        e_host = torch.empty((H, k), dtype=torch.float32).pin_memory()
+        ix.profile(False)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        tot = 0.0
+        nrep = max(3, min(args.steps, 50))
+        for s in range(nrep + 2):
+            flush.fill_(s & 255)
+            e0.record()
+            q_dev.copy_(q_host, non_blocking=True)
+            ix.search(q_dev, k, idx, est)
+            i_host.copy_(idx, non_blocking=True)
+            e_host.copy_(est, non_blocking=True)
+            e1.record()
+            e1.synchronize()
+            if s >= 2:
+                tot += e0.elapsed_time(e1)
+        e2e_ms = dist_max(tot / nrep, ws)
+        e2e = {"value": ws * keys_per_step / (e2e_ms / 1e3), "unit": "keys/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),
+               "d2h_bytes_per_step": i_host.numel() * 4 + e_host.numel() * 4}
+
+    # the full decode step around the search: append one key per (sequence, KV head), search,
+    # sparse attention over the top-k (K/V read from pinned host memory over UVA here)
+    e0 = torch.cuda.Event(enable_timing=True)
+    ea = torch.cuda.Event(enable_timing=True)
+    es = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    app_ms = srch_ms = att_ms = 0.0
+    nrep = 5
+    out = torch.empty_like(qs)
+    assert nrep <= APPEND_SLACK
+    for s in range(nrep):
+        new_k = keys[:, :, ix.size:ix.size + 1].to(dev)
+        e0.record()
+        ix.append(new_k)
+        ea.record()
+        ix.search(qs, k, idx, est)
+        es.record()
+        pk.sparse_attend(cfg, qs, keys, vals, idx, k, 1.0 / float(np.sqrt(sp.d)), n=ix.size,
+                         out=out)
+        e1.record()
+        e1.synchronize()
+        app_ms += e0.elapsed_time(ea) / nrep
+        srch_ms += ea.elapsed_time(es) / nrep
+        att_ms += es.elapsed_time(e1) / nrep
+    kv_bytes = H * k * 2 * sp.d * 2
+    decode = {"append_ms": app_ms, "search_ms": srch_ms, "sparse_attend_ms": att_ms,
+              "total_ms": app_ms + srch_ms + att_ms,
+              "kv_source": "pinned host (UVA)" if kv_host else "HBM",
+              "attend_gbs": kv_bytes / (att_ms / 1e3) / 1e9}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        v, dt, cores = oracle_sample(sp, data, reps=1)
+        cpu = {"value": v, "unit": "keys/s", "cores": cores, "kind": "oracle",
+               "sample": f"one (sequence, KV head) unit: 4 query heads x {sp.n} keys, "
+                         f"index build untimed ({dt:.1f} s timed)"}
+
+    if rank == 0:
+        line = {
+            "metric": "keys searched/s per decode step (vote+rerank+top-k)",
+            "value": value, "unit": "keys/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms_max, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": sp.name, "batch": sp.batch, "q_heads": sp.num_q_heads,
+                       "kv_heads": sp.num_kv_heads, "d": sp.d, "n": sp.n, "k": k,
+                       "candidates": C, "B": sp.B, "m": sp.m, "rho": sp.rho,
+                       "key_dtype": sp.dtype, "kv_in": "pinned host" if kv_host else "HBM",
+                       "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"},
+            "stage_ms": stage_avg,
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "decode_step": decode,
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    ix.destroy()
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,160 @@
+/*
+ * pariskv.h -- C ABI of libpariskv.so, the B200 (sm_100a) ParisKV KV-cache retrieval path.
+ *
+ * The method ("Technical Summary: ParisKV", gist.science/paper/2602.07721, Methodology and
+ * System-Level Innovations; "ParisKV: Fast and Drift-Robust KV-Cache Retrieval for
+ * Long-Context LLMs", ICML 2026 poster abstract): keys are indexed once at prefill and kept
+ * fresh as decoding appends new keys; each decode step returns, for every query head, the
+ * top-k cached keys found on the GPU from compact metadata (no CPU-side search); the
+ * selected full-precision K/V rows, which may live in pinned host memory, feed a sparse
+ * decode attention.
+ *
+ * Conventions for every call:
+ *  - Plain pointers and sizes only. A "device pointer" is memory the current CUDA device can
+ *    dereference: cudaMalloc'd memory, or pinned host memory allocated with cudaHostAlloc /
+ *    registered with cudaHostRegister (UVA makes its host address usable on the device).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Work is
+ *    enqueued asynchronously on it; argument errors are reported synchronously and leave
+ *    nothing enqueued.
+ *  - The caller owns every buffer it passes; no call keeps a caller pointer after it
+ *    returns. The library owns the index and its scratch memory.
+ *  - An index is bound to the device that was current when it was built, and is not
+ *    thread-safe: calls on one index must not overlap.
+ *  - Floating point follows IEEE fp32 (no fast-math); search results are deterministic.
+ */
+#ifndef PARISKV_H_
+#define PARISKV_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PARISKV_API __attribute__((visibility("default")))
+#else
+#define PARISKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PARISKV_OK = 0,
+    PARISKV_EINVAL = 1,     /* an argument is invalid; nothing was done */
+    PARISKV_ENOMEM = 2,     /* a device allocation failed; nothing was changed */
+    PARISKV_ECUDA = 3,      /* a CUDA call or a kernel launch failed (pariskv_last_error()) */
+    PARISKV_ECAPACITY = 4,  /* an append would exceed the index capacity; nothing appended */
+    PARISKV_ETIMEOUT = 5    /* a bounded device-side wait expired; results are invalid */
+} pariskv_status;
+
+enum { PARISKV_F32 = 0, PARISKV_BF16 = 1 };
+
+/* Hyper-parameters and shapes. "Coarse Candidate Generation" and "Candidate Reranking" in
+ * the methodology of the technical summary name B, m, rho, the tiered vote weights and the
+ * 5-10% candidate fraction. Constraints checked by every call that takes a config:
+ *   d == 128, m == 8, B * m == d (the kernels are specialised for d = 128, m = 8);
+ *   1 <= rho <= 2^m; 0 <= w_rest <= w_rank1 <= 3, w_rank1 >= 1 (so a score fits 6 bits);
+ *   1 <= cand_bp <= 10000; batch, num_kv_heads, group >= 1; capacity >= 0;
+ *   dtype is PARISKV_F32 or PARISKV_BF16. */
+typedef struct {
+    int32_t d;            /* head dimension */
+    int32_t B;            /* number of subspaces */
+    int32_t m;            /* dimensions per subspace */
+    int32_t rho;          /* centroids selected per subspace by each query */
+    int32_t w_rank1;      /* vote weight of a query's nearest centroid (default 2) */
+    int32_t w_rest;       /* vote weight of its ranks 2..rho (default 1) */
+    int32_t cand_bp;      /* candidate fraction in basis points (500 = 5%) */
+    int32_t batch;        /* sequences */
+    int32_t num_kv_heads; /* KV heads per sequence */
+    int32_t group;        /* query heads per KV head (GQA group size) */
+    int64_t capacity;     /* maximum tokens per (sequence, KV head) in the index */
+    int32_t dtype;        /* element type of keys, queries, values and outputs */
+    int32_t reserved;     /* must be 0 */
+} pariskv_config;
+
+typedef struct pariskv_index pariskv_index;  /* opaque; owns device memory */
+
+/* Fills *cfg with d=128, B=16, m=8, rho=4, w_rank1=2, w_rest=1, cand_bp=500, batch=1,
+ * num_kv_heads=1, group=1, capacity=0, dtype=PARISKV_BF16. */
+PARISKV_API pariskv_status pariskv_config_default(pariskv_config* cfg);
+
+/* Builds an index over the first n keys of every (sequence, KV head).
+ * Definition: "Normalization and Rotation" and "Coarse Candidate Generation" /
+ * "Quantization" / "Calibration" (technical summary, Core Algorithmic Innovations 1-2):
+ * each key is l2-normalised and rotated by the SRHT R = H diag(signs) / sqrt(d) shared by
+ * keys and queries, then stored as B one-byte bucket ids (the nearest sign centroid of each
+ * m-dim subspace), d 4-bit codes (sign bit + 3-bit uniform magnitude level) and B fp32
+ * calibration factors ("precomputed during the prefill phase").
+ *   srht_signs: host array of d int8 values, each +1 or -1 (copied).
+ *   keys:       device pointer, element (s, t, j) at keys[(s * ld_tok + t) * d + j] with
+ *               s = sequence * num_kv_heads + kv_head, t < n, j < d; dtype cfg->dtype.
+ *   ld_tok:     token slab stride of `keys` (>= n when n > 0).
+ *   n:          0 <= n <= cfg->capacity.
+ *   out:        receives the new index (NULL on failure).
+ * Errors: EINVAL (config, NULL pointer, misaligned keys, n/ld_tok), ENOMEM, ECUDA. */
+PARISKV_API pariskv_status pariskv_build_index(const pariskv_config* cfg, const int8_t* srht_signs,
+                                   const void* keys, int64_t ld_tok, int64_t n, void* stream,
+                                   pariskv_index** out);
+
+/* Appends t new keys to every (sequence, KV head): the decode-time update that keeps the
+ * index fresh under distribution drift ("Drift-Robust Analytic Centroids": the centroids
+ * are data-independent, so new keys are encoded exactly like prefill keys).
+ *   keys: device pointer, element (s, r, j) at keys[(s * ld_tok + r) * d + j], r < t.
+ * Errors: EINVAL, ECAPACITY (size + t > capacity; nothing appended), ECUDA. */
+PARISKV_API pariskv_status pariskv_append(pariskv_index* index, const void* keys, int64_t ld_tok, int64_t t,
+                              void* stream);
+
+/* One decode-step retrieval for every query head ("Two-Stage GPU-Native Retrieval
+ * Pipeline"): rotate the query; per subspace select its top-rho centroids (tiered weights
+ * w_rank1, w_rest); collision-vote an integer coarse score for every cached key; keep the
+ * C = min(n, max(k, ceil(n * cand_bp / 10000))) best-scoring keys (ties to the lower key
+ * index); rerank them with the RSQ-IP estimator est = ||q|| * sum_b w_{i,b} <v_{i,b}, q~_b>;
+ * return the k best (ties to the lower key index).
+ *   q:         device pointer [batch][num_kv_heads * group][d], dtype cfg->dtype; query head
+ *              h uses KV head h / group.
+ *   k:         1 <= k <= current size.
+ *   topk_idx:  device pointer [batch][num_kv_heads * group][k] int32: the selected key
+ *              indices in ascending index order.
+ *   topk_est:  device pointer with the same shape (fp32 estimates of <k, q>), or NULL.
+ * Scratch memory is owned by the index; the first search with a larger candidate count
+ * allocates (so run one search before capturing a CUDA graph).
+ * Errors: EINVAL, ENOMEM, ECUDA, ETIMEOUT. */
+PARISKV_API pariskv_status pariskv_search(pariskv_index* index, const void* q, int32_t k, int32_t* topk_idx,
+                              float* topk_est, void* stream);
+
+/* Sparse decode attention over the retrieved tokens (Problem Statement: attend to a Top-k
+ * subset; System-Level Innovations 1: the selected full-precision K/V rows are fetched by
+ * the GPU kernel directly, from HBM or from pinned host memory over UVA, with no memcpy):
+ *   out[s][h] = sum_{t in topk[s][h]} softmax_t(scale * <q[s][h], K[s][h/group][t]>) V[..][t]
+ *   q:        device pointer [batch][Hq][d]; K, V: device or pinned-host pointers with the
+ *             layout of pariskv_build_index's keys (slab stride ld_tok, n valid tokens);
+ *   topk_idx: device pointer [batch][Hq][k] with values in [0, n);
+ *   out:      device pointer [batch][Hq][d]. Element type cfg->dtype everywhere; fp32
+ *             accumulation. Uses a library-owned per-device workspace.
+ * Errors: EINVAL, ENOMEM, ECUDA. */
+PARISKV_API pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, const void* K,
+                                     const void* V, int64_t ld_tok, int64_t n,
+                                     const int32_t* topk_idx, int32_t k, float scale, void* out,
+                                     void* stream);
+
+/* Waits for the index's stream work and reports any asynchronous error or expired wait. */
+PARISKV_API pariskv_status pariskv_sync(pariskv_index* index, void* stream);
+
+/* Frees the index (NULL is a no-op). Waits for the device first. */
+PARISKV_API pariskv_status pariskv_destroy(pariskv_index* index);
+
+/* Current number of indexed tokens per (sequence, KV head); -1 for NULL. */
+PARISKV_API int64_t pariskv_size(const pariskv_index* index);
+
+/* Number of kernels the last search / attend call launched (for launch accounting). */
+PARISKV_API int32_t pariskv_last_launch_count(void);
+
+PARISKV_API const char* pariskv_status_string(pariskv_status status);
+
+/* Message of the last failure on the calling thread ("" when none). */
+PARISKV_API const char* pariskv_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PARISKV_H_ */

@@ -1,0 +1,563 @@
+// api.cu -- the C ABI of libpariskv.so: argument validation, memory ownership and the
+// launch sequence of each call. Every step of the retrieval path runs in the kernels of this
+// library; the host only validates, allocates and launches.
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.hpp"
+#include "pariskv_debug.h"
+
+using namespace pkv;
+
+namespace {
+
+thread_local char g_err[512] = "";
+thread_local int32_t g_launches = 0;
+
+void set_err(const char* fmt, va_list ap) { vsnprintf(g_err, sizeof(g_err), fmt, ap); }
+
+// Test hook: PARISKV_FAULT=alloc makes every device allocation of the library fail, so the
+// ENOMEM paths (and their cleanup) can be exercised without exhausting a real device.
+bool fault_alloc() {
+    const char* f = getenv("PARISKV_FAULT");
+    return f && strcmp(f, "alloc") == 0;
+}
+
+template <typename T>
+bool dalloc(T** p, size_t count) {
+    *p = nullptr;
+    if (count == 0) count = 1;
+    if (fault_alloc()) return false;
+    if (cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T)) != cudaSuccess) {
+        cudaGetLastError();
+        *p = nullptr;
+        return false;
+    }
+    return true;
+}
+
+template <typename T>
+void dfree(T*& p) {
+    if (p) cudaFree(p);
+    p = nullptr;
+}
+
+int64_t candidate_count(int64_t n, int64_t k, int32_t bp) {
+    int64_t c = (n * bp + 9999) / 10000;
+    if (c < k) c = k;
+    if (c > n) c = n;
+    return c;
+}
+
+pariskv_status check_config(const pariskv_config* c) {
+    if (!c) return fail(PARISKV_EINVAL, "config is NULL");
+    if (c->d != D || c->m != M || c->B != NB)
+        return fail(PARISKV_EINVAL, "shape d=%d B=%d m=%d unsupported (need d=128, B=16, m=8)",
+                    c->d, c->B, c->m);
+    if (c->rho < 1 || c->rho > NC) return fail(PARISKV_EINVAL, "rho=%d not in [1, 256]", c->rho);
+    if (c->w_rank1 < 1 || c->w_rank1 > 3 || c->w_rest < 0 || c->w_rest > c->w_rank1)
+        return fail(PARISKV_EINVAL, "vote weights (%d, %d) need 1 <= w_rank1 <= 3 and "
+                    "0 <= w_rest <= w_rank1", c->w_rank1, c->w_rest);
+    if (c->cand_bp < 1 || c->cand_bp > 10000)
+        return fail(PARISKV_EINVAL, "cand_bp=%d not in [1, 10000]", c->cand_bp);
+    if (c->batch < 1 || c->num_kv_heads < 1 || c->group < 1)
+        return fail(PARISKV_EINVAL, "batch, num_kv_heads and group must be >= 1");
+    const int64_t heads = static_cast<int64_t>(c->batch) * c->num_kv_heads * c->group;
+    if (heads > 65535) return fail(PARISKV_EINVAL, "batch * query heads = %lld > 65535",
+                                   static_cast<long long>(heads));
+    if (c->capacity < 0 || c->capacity > (int64_t(1) << 31) - CHUNK)
+        return fail(PARISKV_EINVAL, "capacity %lld out of range",
+                    static_cast<long long>(c->capacity));
+    if (c->dtype != PARISKV_F32 && c->dtype != PARISKV_BF16)
+        return fail(PARISKV_EINVAL, "dtype %d unknown", c->dtype);
+    if (c->reserved != 0) return fail(PARISKV_EINVAL, "reserved field must be 0");
+    return PARISKV_OK;
+}
+
+// A pointer the current device can dereference: device memory, managed memory, or host
+// memory that is pinned/registered (UVA maps it into the device address space).
+pariskv_status check_dev_ptr(const void* p, size_t align, const char* name) {
+    if (!p) return fail(PARISKV_EINVAL, "%s is NULL", name);
+    if (reinterpret_cast<uintptr_t>(p) % align)
+        return fail(PARISKV_EINVAL, "%s is not %zu-byte aligned", name, align);
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(PARISKV_EINVAL, "%s is not a CUDA-visible pointer", name);
+    }
+    if (a.type == cudaMemoryTypeUnregistered)
+        return fail(PARISKV_EINVAL, "%s is pageable host memory (pin or register it)", name);
+    if (a.type == cudaMemoryTypeHost && a.devicePointer != p)
+        return fail(PARISKV_EINVAL, "%s: pinned host memory without an identical device "
+                    "mapping", name);
+    return PARISKV_OK;
+}
+
+pariskv_status check_index(const pariskv_index* ix) {
+    if (!ix) return fail(PARISKV_EINVAL, "index is NULL");
+    int dev = -1;
+    cudaGetDevice(&dev);
+    if (dev != ix->device)
+        return fail(PARISKV_EINVAL, "index lives on device %d but device %d is current",
+                    ix->device, dev);
+    return PARISKV_OK;
+}
+
+void free_index(pariskv_index* ix) {
+    if (!ix) return;
+    dfree(ix->signs); dfree(ix->ids); dfree(ix->rec); dfree(ix->lut); dfree(ix->qt);
+    dfree(ix->qnorm); dfree(ix->scores); dfree(ix->hist); dfree(ix->thr); dfree(ix->cbase);
+    dfree(ix->cand); dfree(ix->S); dfree(ix->status);
+    for (auto& e : ix->ev)
+        if (e) cudaEventDestroy(e);
+    delete ix;
+}
+
+pariskv_status create_index(const pariskv_config* cfg, const int8_t* signs, cudaStream_t st,
+                            pariskv_index** out) {
+    *out = nullptr;
+    for (int j = 0; j < D; ++j)
+        if (signs[j] != 1 && signs[j] != -1)
+            return fail(PARISKV_EINVAL, "srht_signs[%d] = %d is not +-1", j, signs[j]);
+    pariskv_index* ix = new (std::nothrow) pariskv_index();
+    if (!ix) return fail(PARISKV_ENOMEM, "host allocation failed");
+    ix->cfg = *cfg;
+    cudaGetDevice(&ix->device);
+    ix->units = cfg->batch * cfg->num_kv_heads;
+    ix->hq = cfg->num_kv_heads * cfg->group;
+    ix->packs = static_cast<int>(ceil_div(cfg->group, PACK));
+    ix->cap_pad = round_up(cfg->capacity > 0 ? cfg->capacity : 1, CHUNK);
+    const int64_t up = static_cast<int64_t>(ix->units) * ix->packs;
+    const int64_t heads = static_cast<int64_t>(ix->units) * cfg->group;
+    const int64_t nch = ix->cap_pad / CHUNK;
+    bool ok = dalloc(&ix->signs, D) && dalloc(&ix->ids, ix->units * ix->cap_pad * 16) &&
+              dalloc(&ix->rec, ix->units * ix->cap_pad * REC) &&
+              dalloc(&ix->lut, up * NB * NC) && dalloc(&ix->qt, heads * D) &&
+              dalloc(&ix->qnorm, heads) && dalloc(&ix->scores, up * ix->cap_pad) &&
+              dalloc(&ix->hist, up * nch * PACK * NBINS) && dalloc(&ix->thr, heads * 4) &&
+              dalloc(&ix->cbase, heads * nch * 2) && dalloc(&ix->status, 1);
+    if (!ok) {
+        free_index(ix);
+        return fail(PARISKV_ENOMEM, "device allocation for the index failed");
+    }
+    float hs[D];
+    for (int j = 0; j < D; ++j) hs[j] = static_cast<float>(signs[j]);
+    cudaError_t e = cudaMemcpyAsync(ix->signs, hs, sizeof(hs), cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ix->lut, 0, up * NB * NC * sizeof(uint32_t), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ix->status, 0, sizeof(int), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);  // hs lives on this stack frame
+    if (e != cudaSuccess) {
+        free_index(ix);
+        return cuda_fail(e, "index initialisation");
+    }
+    *out = ix;
+    return PARISKV_OK;
+}
+
+pariskv_status ensure_candidates(pariskv_index* ix, int64_t C) {
+    if (C <= ix->cmax) return PARISKV_OK;
+    const int64_t heads = static_cast<int64_t>(ix->units) * ix->cfg.group;
+    int32_t* c2 = nullptr;
+    float* s2 = nullptr;
+    if (!dalloc(&c2, heads * C) || !dalloc(&s2, heads * C)) {
+        dfree(c2);
+        dfree(s2);
+        return fail(PARISKV_ENOMEM, "candidate buffers (%lld per head)", static_cast<long long>(C));
+    }
+    dfree(ix->cand);
+    dfree(ix->S);
+    ix->cand = c2;
+    ix->S = s2;
+    ix->cmax = C;
+    return PARISKV_OK;
+}
+
+pariskv_status run_search(pariskv_index* ix, const void* q, const float* qt, const float* qn,
+                          bool rotated, int32_t k, int32_t* topk_idx, float* topk_est,
+                          cudaStream_t st) {
+    if (k < 1 || k > ix->n)
+        return fail(PARISKV_EINVAL, "k=%d not in [1, size=%lld]", k, static_cast<long long>(ix->n));
+    const int64_t C = candidate_count(ix->n, k, ix->cfg.cand_bp);
+    pariskv_status s = ensure_candidates(ix, C);
+    if (s != PARISKV_OK) return s;
+    g_launches = 0;
+    int ne = 0;
+    auto mark = [&]() {
+        if (ix->profile) cudaEventRecord(ix->ev[ne++], st);
+    };
+    mark();
+    cudaError_t e = launch_query_prep(ix, q, qt, qn, rotated, st);
+    if (e == cudaSuccess) { ++g_launches; mark(); e = launch_vote(ix, st); }
+    if (e == cudaSuccess) { ++g_launches; mark(); e = launch_threshold(ix, C, st); }
+    if (e == cudaSuccess) { ++g_launches; mark(); e = launch_compact(ix, st); }
+    if (e == cudaSuccess) { ++g_launches; mark(); e = launch_rerank(ix, C, st); }
+    if (e == cudaSuccess) { ++g_launches; mark(); e = launch_topk(ix, C, k, topk_idx, topk_est, st); }
+    if (e == cudaSuccess) { ++g_launches; mark(); }
+    ix->nev = ne;
+    if (e != cudaSuccess) return cuda_fail(e, "search launch");
+    ix->last_C = C;
+    ix->last_k = k;
+    ix->searched = true;
+    return PARISKV_OK;
+}
+
+}  // namespace
+
+namespace pkv {
+
+pariskv_status fail(pariskv_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    set_err(fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+pariskv_status cuda_fail(cudaError_t e, const char* what) {
+    cudaGetLastError();
+    snprintf(g_err, sizeof(g_err), "%s: %s", what, cudaGetErrorString(e));
+    return e == cudaErrorMemoryAllocation ? PARISKV_ENOMEM : PARISKV_ECUDA;
+}
+
+}  // namespace pkv
+
+// =========================================================================================
+// Product surface
+// =========================================================================================
+extern "C" {
+
+pariskv_status pariskv_config_default(pariskv_config* cfg) {
+    if (!cfg) return fail(PARISKV_EINVAL, "config is NULL");
+    memset(cfg, 0, sizeof(*cfg));
+    cfg->d = D; cfg->B = NB; cfg->m = M; cfg->rho = 4; cfg->w_rank1 = 2; cfg->w_rest = 1;
+    cfg->cand_bp = 500; cfg->batch = 1; cfg->num_kv_heads = 1; cfg->group = 1;
+    cfg->capacity = 0; cfg->dtype = PARISKV_BF16;
+    return PARISKV_OK;
+}
+
+static pariskv_status build_common(const pariskv_config* cfg, const int8_t* srht_signs,
+                                   const void* keys, const float* knorm, bool rotated,
+                                   int64_t ld_tok, int64_t n, void* stream,
+                                   pariskv_index** out) {
+    if (!out) return fail(PARISKV_EINVAL, "out is NULL");
+    *out = nullptr;
+    pariskv_status s = check_config(cfg);
+    if (s != PARISKV_OK) return s;
+    if (!srht_signs) return fail(PARISKV_EINVAL, "srht_signs is NULL");
+    if (n < 0 || n > cfg->capacity)
+        return fail(PARISKV_EINVAL, "n=%lld not in [0, capacity=%lld]", static_cast<long long>(n),
+                    static_cast<long long>(cfg->capacity));
+    if (n > 0) {
+        if (ld_tok < n) return fail(PARISKV_EINVAL, "ld_tok < n");
+        s = check_dev_ptr(keys, rotated ? 16 : (cfg->dtype == PARISKV_BF16 ? 8 : 16), "keys");
+        if (s != PARISKV_OK) return s;
+        if (rotated && (s = check_dev_ptr(knorm, 4, "knorm")) != PARISKV_OK) return s;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    pariskv_index* ix = nullptr;
+    s = create_index(cfg, srht_signs, st, &ix);
+    if (s != PARISKV_OK) return s;
+    cudaError_t e = launch_encode(ix, keys, knorm, ld_tok, n, 0, rotated, st);
+    if (e != cudaSuccess) {
+        free_index(ix);
+        return cuda_fail(e, "encode launch");
+    }
+    ix->n = n;
+    *out = ix;
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_build_index(const pariskv_config* cfg, const int8_t* srht_signs,
+                                   const void* keys, int64_t ld_tok, int64_t n, void* stream,
+                                   pariskv_index** out) {
+    return build_common(cfg, srht_signs, keys, nullptr, false, ld_tok, n, stream, out);
+}
+
+static pariskv_status append_common(pariskv_index* ix, const void* keys, const float* knorm,
+                                    bool rotated, int64_t ld_tok, int64_t t, void* stream) {
+    pariskv_status s = check_index(ix);
+    if (s != PARISKV_OK) return s;
+    if (t < 0) return fail(PARISKV_EINVAL, "t < 0");
+    if (t == 0) return PARISKV_OK;
+    if (ix->n + t > ix->cfg.capacity)
+        return fail(PARISKV_ECAPACITY, "append of %lld keys exceeds capacity %lld (size %lld)",
+                    static_cast<long long>(t), static_cast<long long>(ix->cfg.capacity),
+                    static_cast<long long>(ix->n));
+    if (ld_tok < t) return fail(PARISKV_EINVAL, "ld_tok < t");
+    s = check_dev_ptr(keys, rotated ? 16 : (ix->cfg.dtype == PARISKV_BF16 ? 8 : 16), "keys");
+    if (s != PARISKV_OK) return s;
+    if (rotated && (s = check_dev_ptr(knorm, 4, "knorm")) != PARISKV_OK) return s;
+    cudaError_t e = launch_encode(ix, keys, knorm, ld_tok, t, ix->n, rotated,
+                                  static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "encode launch");
+    ix->n += t;
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_append(pariskv_index* index, const void* keys, int64_t ld_tok, int64_t t,
+                              void* stream) {
+    return append_common(index, keys, nullptr, false, ld_tok, t, stream);
+}
+
+pariskv_status pariskv_search(pariskv_index* index, const void* q, int32_t k, int32_t* topk_idx,
+                              float* topk_est, void* stream) {
+    pariskv_status s = check_index(index);
+    if (s != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(q, index->cfg.dtype == PARISKV_BF16 ? 8 : 16, "q")) != PARISKV_OK)
+        return s;
+    if ((s = check_dev_ptr(topk_idx, 4, "topk_idx")) != PARISKV_OK) return s;
+    if (topk_est && (s = check_dev_ptr(topk_est, 4, "topk_est")) != PARISKV_OK) return s;
+    return run_search(index, q, nullptr, nullptr, false, k, topk_idx, topk_est,
+                      static_cast<cudaStream_t>(stream));
+}
+
+pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, const void* K,
+                                     const void* V, int64_t ld_tok, int64_t n,
+                                     const int32_t* topk_idx, int32_t k, float scale, void* out,
+                                     void* stream) {
+    pariskv_status s = check_config(cfg);
+    if (s != PARISKV_OK) return s;
+    const size_t al = cfg->dtype == PARISKV_BF16 ? 8 : 16;
+    if (k < 1 || k > n) return fail(PARISKV_EINVAL, "k=%d not in [1, n=%lld]", k,
+                                    static_cast<long long>(n));
+    if (ld_tok < n) return fail(PARISKV_EINVAL, "ld_tok < n");
+    if ((s = check_dev_ptr(q, al, "q")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(K, al, "K")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(V, al, "V")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(topk_idx, 4, "topk_idx")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(out, al, "out")) != PARISKV_OK) return s;
+    if (!(scale == scale)) return fail(PARISKV_EINVAL, "scale is NaN");
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int heads = cfg->batch * cfg->num_kv_heads * cfg->group;
+    const int nsplit = attend_splits(heads, k, sms);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* work = nullptr;
+    if (fault_alloc()) return fail(PARISKV_ENOMEM, "attention workspace");
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&work),
+                                    attend_workspace_floats(heads, nsplit) * sizeof(float), st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention workspace");
+    g_launches = 0;
+    e = launch_attend(cfg, q, K, V, ld_tok, n, topk_idx, k, scale, out, work, nsplit, st);
+    if (e == cudaSuccess) g_launches = 2;
+    cudaFreeAsync(work, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_sync(pariskv_index* index, void* stream) {
+    pariskv_status s = check_index(index);
+    if (s != PARISKV_OK) return s;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronise");
+    int st = 0;
+    e = cudaMemcpy(&st, index->status, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "status read");
+    if (st != ST_OK) {
+        cudaMemset(index->status, 0, sizeof(int));
+        if (st == ST_TIMEOUT) return fail(PARISKV_ETIMEOUT, "a bounded device-side wait expired");
+        return fail(PARISKV_ECUDA, "internal consistency check failed on the device (%d)", st);
+    }
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_destroy(pariskv_index* index) {
+    if (!index) return PARISKV_OK;
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(index->device);
+    cudaDeviceSynchronize();
+    free_index(index);
+    cudaSetDevice(prev);
+    return PARISKV_OK;
+}
+
+int64_t pariskv_size(const pariskv_index* index) { return index ? index->n : -1; }
+
+int32_t pariskv_last_launch_count(void) { return g_launches; }
+
+const char* pariskv_status_string(pariskv_status s) {
+    switch (s) {
+        case PARISKV_OK: return "ok";
+        case PARISKV_EINVAL: return "invalid argument";
+        case PARISKV_ENOMEM: return "out of device memory";
+        case PARISKV_ECUDA: return "CUDA error";
+        case PARISKV_ECAPACITY: return "index capacity exceeded";
+        case PARISKV_ETIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+const char* pariskv_last_error(void) { return g_err; }
+
+// =========================================================================================
+// Test-only surface (pariskv_debug.h)
+// =========================================================================================
+pariskv_status pariskv_debug_rotate(const pariskv_config* cfg, const int8_t* srht_signs,
+                                    const void* x, int64_t n, float* y, float* norm,
+                                    void* stream) {
+    pariskv_status s = check_config(cfg);
+    if (s != PARISKV_OK) return s;
+    if (!srht_signs) return fail(PARISKV_EINVAL, "srht_signs is NULL");
+    if (n < 0) return fail(PARISKV_EINVAL, "n < 0");
+    if (n == 0) return PARISKV_OK;
+    if ((s = check_dev_ptr(x, cfg->dtype == PARISKV_BF16 ? 8 : 16, "x")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(y, 16, "y")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(norm, 4, "norm")) != PARISKV_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float hs[D];
+    for (int j = 0; j < D; ++j) hs[j] = static_cast<float>(srht_signs[j]);
+    float* ds = nullptr;
+    if (!dalloc(&ds, D)) return fail(PARISKV_ENOMEM, "signs");
+    cudaError_t e = cudaMemcpy(ds, hs, sizeof(hs), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = launch_rotate(cfg, ds, x, n, y, norm, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    dfree(ds);
+    if (e != cudaSuccess) return cuda_fail(e, "rotate");
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_debug_build_index_rotated(const pariskv_config* cfg,
+                                                 const int8_t* srht_signs, const float* y,
+                                                 const float* knorm, int64_t ld_tok, int64_t n,
+                                                 void* stream, pariskv_index** out) {
+    return build_common(cfg, srht_signs, y, knorm, true, ld_tok, n, stream, out);
+}
+
+pariskv_status pariskv_debug_append_rotated(pariskv_index* index, const float* y,
+                                            const float* knorm, int64_t ld_tok, int64_t t,
+                                            void* stream) {
+    return append_common(index, y, knorm, true, ld_tok, t, stream);
+}
+
+pariskv_status pariskv_debug_search_rotated(pariskv_index* index, const float* qt,
+                                            const float* qnorm, int32_t k, int32_t* topk_idx,
+                                            float* topk_est, void* stream) {
+    pariskv_status s = check_index(index);
+    if (s != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(qt, 16, "qt")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(qnorm, 4, "qnorm")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(topk_idx, 4, "topk_idx")) != PARISKV_OK) return s;
+    if (topk_est && (s = check_dev_ptr(topk_est, 4, "topk_est")) != PARISKV_OK) return s;
+    return run_search(index, nullptr, qt, qnorm, true, k, topk_idx, topk_est,
+                      static_cast<cudaStream_t>(stream));
+}
+
+pariskv_status pariskv_debug_profile(pariskv_index* ix, int32_t enable) {
+    pariskv_status s = check_index(ix);
+    if (s != PARISKV_OK) return s;
+    if (enable && !ix->ev[0]) {
+        for (auto& e : ix->ev) {
+            cudaError_t r = cudaEventCreate(&e);
+            if (r != cudaSuccess) return cuda_fail(r, "event create");
+        }
+    }
+    ix->profile = enable != 0;
+    ix->nev = 0;
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_debug_stage_ms(pariskv_index* ix, float* ms, int32_t* nstages) {
+    pariskv_status s = check_index(ix);
+    if (s != PARISKV_OK) return s;
+    if (!ms || !nstages) return fail(PARISKV_EINVAL, "NULL output");
+    *nstages = 0;
+    if (ix->nev < 2) return fail(PARISKV_EINVAL, "no profiled search has run");
+    cudaError_t e = cudaEventSynchronize(ix->ev[ix->nev - 1]);
+    if (e != cudaSuccess) return cuda_fail(e, "event synchronise");
+    for (int i = 0; i + 1 < ix->nev; ++i) {
+        e = cudaEventElapsedTime(&ms[i], ix->ev[i], ix->ev[i + 1]);
+        if (e != cudaSuccess) return cuda_fail(e, "event elapsed");
+    }
+    *nstages = ix->nev - 1;
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_debug_export_index(pariskv_index* ix, uint8_t* ids, uint8_t* codes,
+                                          float* factors) {
+    pariskv_status s = check_index(ix);
+    if (s != PARISKV_OK) return s;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "synchronise");
+    const int64_t n = ix->n;
+    std::vector<uint8_t> hid, hrec;
+    try {
+        hid.resize(static_cast<size_t>(n) * 16);
+        hrec.resize(static_cast<size_t>(n) * REC);
+    } catch (...) {
+        return fail(PARISKV_ENOMEM, "host staging");
+    }
+    for (int u = 0; u < ix->units; ++u) {
+        if (n == 0) break;
+        e = cudaMemcpy(hid.data(), ix->ids + u * ix->cap_pad * 16, n * 16, cudaMemcpyDeviceToHost);
+        if (e == cudaSuccess)
+            e = cudaMemcpy(hrec.data(), ix->rec + u * ix->cap_pad * REC, n * REC,
+                           cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail(e, "export copy");
+        for (int64_t i = 0; i < n; ++i) {
+            const int64_t o = static_cast<int64_t>(u) * n + i;
+            for (int b = 0; b < NB; ++b) {
+                if (ids) ids[o * NB + b] = hid[i * 16 + ((b - i) & 15)];
+                uint32_t w;
+                memcpy(&w, &hrec[i * REC + 4 * b], 4);
+                if (codes)
+                    for (int j = 0; j < M; ++j) codes[o * D + b * M + j] = (w >> (4 * j)) & 15u;
+                if (factors) memcpy(&factors[o * NB + b], &hrec[i * REC + 64 + 4 * b], 4);
+            }
+        }
+    }
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_debug_export_search(pariskv_index* ix, uint8_t* lut, int32_t* scores,
+                                           int64_t* ncand, int32_t* cand, float* S) {
+    pariskv_status s = check_index(ix);
+    if (s != PARISKV_OK) return s;
+    if (!ix->searched) return fail(PARISKV_EINVAL, "no search has run on this index");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "synchronise");
+    const int G = ix->cfg.group;
+    const int64_t n = ix->n, C = ix->last_C;
+    if (ncand) *ncand = C;
+    std::vector<uint32_t> buf;
+    for (int u = 0; u < ix->units; ++u) {
+        for (int g = 0; g < G; ++g) {
+            const int64_t head = static_cast<int64_t>(u) * G + g;
+            const int64_t up = static_cast<int64_t>(u) * ix->packs + g / PACK;
+            const int sh = 8 * (g % PACK);
+            if (lut) {
+                buf.resize(NB * NC);
+                e = cudaMemcpy(buf.data(), ix->lut + up * NB * NC, NB * NC * 4,
+                               cudaMemcpyDeviceToHost);
+                if (e != cudaSuccess) return cuda_fail(e, "export lut");
+                for (int i = 0; i < NB * NC; ++i) lut[head * NB * NC + i] = (buf[i] >> sh) & 0xff;
+            }
+            if (scores && n > 0) {
+                buf.resize(n);
+                e = cudaMemcpy(buf.data(), ix->scores + up * ix->cap_pad, n * 4,
+                               cudaMemcpyDeviceToHost);
+                if (e != cudaSuccess) return cuda_fail(e, "export scores");
+                for (int64_t i = 0; i < n; ++i) scores[head * n + i] = (buf[i] >> sh) & 0xff;
+            }
+            if (cand && C > 0) {
+                e = cudaMemcpy(cand + head * C, ix->cand + head * ix->cmax, C * 4,
+                               cudaMemcpyDeviceToHost);
+                if (e != cudaSuccess) return cuda_fail(e, "export candidates");
+            }
+            if (S && C > 0) {
+                e = cudaMemcpy(S + head * C, ix->S + head * ix->cmax, C * 4,
+                               cudaMemcpyDeviceToHost);
+                if (e != cudaSuccess) return cuda_fail(e, "export S");
+            }
+        }
+    }
+    return PARISKV_OK;
+}
+
+}  // extern "C"

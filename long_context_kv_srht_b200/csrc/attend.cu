@@ -1,0 +1,169 @@
+// attend.cu -- sparse decode attention over the retrieved top-k tokens.
+//
+// "Technical Summary: ParisKV", Problem Statement (attend only to a Top-k subset of past
+// tokens) and System-Level Innovations 1 (Unified Virtual Addressing offloading: the GPU
+// kernel fetches only the selected full-precision K/V rows, from HBM or directly from pinned
+// host memory, without memcpy or CPU scheduling):
+//     o_h = sum_{t in topk_h} softmax_t(scale * <q_h, K_t>) V_t,   K/V of KV head h / group.
+//
+// Split-K: CTA (split, head) processes a contiguous slice of the head's k indices; each of
+// its 4 warps walks every 4th token of the slice, a lane holding 4 of the 128 dims, and
+// keeps an online-softmax state (running max, denominator, 4 accumulators). Four tokens
+// are loaded before any is used so that each warp has 8 row reads in flight (this matters
+// for K/V in host memory, where a read crosses PCIe). The warps are merged in shared memory
+// and the CTA writes (max, denominator, 128 accumulators) to the workspace; a second kernel
+// merges the splits with the log-sum-exp rule and writes the output in the input dtype.
+#include "common.cuh"
+#include "internal.hpp"
+
+namespace pkv {
+
+namespace {
+
+constexpr int kAW = 4;            // warps per CTA
+constexpr int kUnroll = 4;        // tokens in flight per warp
+constexpr int kPart = 2 + D;      // floats per partial: max, denominator, accumulators
+
+template <typename T> __device__ __forceinline__ void store4(T* p, const float v[4]);
+template <> __device__ __forceinline__ void store4<float>(float* p, const float v[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <> __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, const float v[4]) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kAW * 32)
+attend_partial_kernel(const T* __restrict__ q, const T* __restrict__ K, const T* __restrict__ V,
+                      int64_t ld_tok, int64_t n, const int32_t* __restrict__ topk, int32_t k,
+                      float scale, int group, int nsplit, float* __restrict__ work) {
+    __shared__ float sm[kAW][kPart];
+    const int head = blockIdx.y, split = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t unit = head / group;
+    const int64_t t0 = static_cast<int64_t>(k) * split / nsplit;
+    const int64_t t1 = static_cast<int64_t>(k) * (split + 1) / nsplit;
+
+    float qv[4];
+    Elem<T>::load4(q + static_cast<int64_t>(head) * D + 4 * lane, qv);
+    const T* Kb = K + unit * ld_tok * D + 4 * lane;
+    const T* Vb = V + unit * ld_tok * D + 4 * lane;
+    const int32_t* idx = topk + static_cast<int64_t>(head) * k;
+
+    float mx = -INFINITY, den = 0.0f, acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int64_t t = t0 + warp; t < t1; t += kAW * kUnroll) {
+        float kv[kUnroll][4], vv[kUnroll][4];
+        bool ok[kUnroll], valid[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t tt = t + static_cast<int64_t>(u) * kAW;
+            ok[u] = tt < t1;
+            const int64_t row = ok[u] ? idx[tt] : 0;
+            // rows outside [0, n) are skipped (the caller's indices are not trusted)
+            valid[u] = ok[u] && row >= 0 && row < n;
+            if (valid[u]) {
+                Elem<T>::load4(Kb + row * D, kv[u]);
+                Elem<T>::load4(Vb + row * D, vv[u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            if (!ok[u]) break;
+            if (!valid[u]) continue;
+            float s = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s = __fmaf_rn(qv[i], kv[u][i], s);
+            s = warp_sum(s) * scale;
+            const float mn = fmaxf(mx, s);
+            const float corr = expf(mx - mn);
+            const float p = expf(s - mn);
+            den = den * corr + p;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[i] = acc[i] * corr + p * vv[u][i];
+            mx = mn;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sm[warp][2 + 4 * lane + i] = acc[i];
+    if (lane == 0) { sm[warp][0] = mx; sm[warp][1] = den; }
+    __syncthreads();
+    if (warp == 0) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kAW; ++w) M = fmaxf(M, sm[w][0]);
+        float dsum = 0.0f, a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int w = 0; w < kAW; ++w) {
+            const float f = sm[w][0] == -INFINITY ? 0.0f : expf(sm[w][0] - M);
+            dsum += sm[w][1] * f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] += sm[w][2 + 4 * lane + i] * f;
+        }
+        float* out = work + (static_cast<int64_t>(head) * nsplit + split) * kPart;
+        *reinterpret_cast<float4*>(out + 2 + 4 * lane) = make_float4(a[0], a[1], a[2], a[3]);
+        if (lane == 0) { out[0] = M; out[1] = dsum; }
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(32)
+attend_combine_kernel(const float* __restrict__ work, int nsplit, T* __restrict__ out) {
+    const int head = blockIdx.x, lane = threadIdx.x;
+    const float* w = work + static_cast<int64_t>(head) * nsplit * kPart;
+    float M = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, w[s * kPart]);
+    float den = 0.0f, a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int s = 0; s < nsplit; ++s) {
+        const float ms = w[s * kPart];
+        const float f = ms == -INFINITY ? 0.0f : expf(ms - M);
+        den += w[s * kPart + 1] * f;
+        const float4 v = *reinterpret_cast<const float4*>(w + s * kPart + 2 + 4 * lane);
+        a[0] += v.x * f; a[1] += v.y * f; a[2] += v.z * f; a[3] += v.w * f;
+    }
+    const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+    float o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = a[i] * inv;
+    store4<T>(out + static_cast<int64_t>(head) * D + 4 * lane, o);
+}
+
+}  // namespace
+
+int attend_splits(int heads, int32_t k, int num_sms) {
+    const int want = static_cast<int>(ceil_div(4LL * num_sms, heads));
+    const int most = static_cast<int>(ceil_div(k, 64));
+    return max(1, min(want, most));
+}
+
+size_t attend_workspace_floats(int heads, int nsplit) {
+    return static_cast<size_t>(heads) * nsplit * kPart;
+}
+
+cudaError_t launch_attend(const pariskv_config* cfg, const void* q, const void* K,
+                          const void* V, int64_t ld_tok, int64_t n, const int32_t* topk_idx,
+                          int32_t k,
+                          float scale, void* out, float* work, int nsplit, cudaStream_t st) {
+    const int heads = cfg->batch * cfg->num_kv_heads * cfg->group;
+    dim3 grid(nsplit, heads);
+    if (cfg->dtype == PARISKV_BF16) {
+        using T = __nv_bfloat16;
+        attend_partial_kernel<T><<<grid, kAW * 32, 0, st>>>(
+            static_cast<const T*>(q), static_cast<const T*>(K), static_cast<const T*>(V),
+            ld_tok, n, topk_idx, k, scale, cfg->group, nsplit, work);
+        attend_combine_kernel<T><<<heads, 32, 0, st>>>(work, nsplit, static_cast<T*>(out));
+    } else {
+        attend_partial_kernel<float><<<grid, kAW * 32, 0, st>>>(
+            static_cast<const float*>(q), static_cast<const float*>(K),
+            static_cast<const float*>(V), ld_tok, n, topk_idx, k, scale, cfg->group, nsplit,
+            work);
+        attend_combine_kernel<float><<<heads, 32, 0, st>>>(work, nsplit, static_cast<float*>(out));
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace pkv

@@ -1,0 +1,84 @@
+// internal.hpp -- the index object and the kernel launchers behind the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pariskv.h"
+
+struct pariskv_index {
+    pariskv_config cfg;
+    int device = 0;
+    int64_t n = 0;        // tokens indexed per unit
+    int64_t cap_pad = 0;  // capacity rounded up to a whole histogram chunk
+    int units = 0;        // batch * num_kv_heads
+    int hq = 0;           // query heads per sequence
+    int packs = 0;        // ceil(group / 4): vote-table packs per KV head
+
+    float* signs = nullptr;     // [128] +-1.0f
+    uint8_t* ids = nullptr;     // [units][cap_pad][16] bucket ids, byte-rotated per key
+    uint8_t* rec = nullptr;     // [units][cap_pad][128] codes (64 B) + factors (16 x f32)
+
+    // per-search scratch (library-owned)
+    uint32_t* lut = nullptr;    // [units*packs][16][256] packed vote weights
+    float* qt = nullptr;        // [units*group][128] rotated queries
+    float* qnorm = nullptr;     // [units*group]
+    uint32_t* scores = nullptr; // [units*packs][cap_pad] packed coarse scores
+    uint32_t* hist = nullptr;   // [units*packs][chunks][4][64] per-chunk score histograms
+    int32_t* thr = nullptr;     // [units*group][4] threshold T, ties E, candidate count C
+    int32_t* cbase = nullptr;   // [units*group][chunks][2] selected/ties before each chunk
+    int32_t* cand = nullptr;    // [units*group][cmax] candidate indices (ascending)
+    float* S = nullptr;         // [units*group][cmax] rerank values
+    int64_t cmax = 0;
+    int* status = nullptr;      // device status word (ST_OK / ST_TIMEOUT)
+
+    // optional per-stage timing of searches (test and benchmark use)
+    bool profile = false;
+    cudaEvent_t ev[8] = {};
+    int nev = 0;
+
+    int64_t last_C = 0;
+    int32_t last_k = 0;
+    bool searched = false;
+};
+
+namespace pkv {
+
+// status helpers (defined in api.cu)
+pariskv_status fail(pariskv_status s, const char* fmt, ...);
+pariskv_status cuda_fail(cudaError_t e, const char* what);
+
+// encode.cu
+cudaError_t launch_encode(const pariskv_index* ix, const void* keys, const float* knorm,
+                          int64_t ld_tok, int64_t t, int64_t pos0, bool rotated,
+                          cudaStream_t st);
+cudaError_t launch_rotate(const pariskv_config* cfg, const float* signs, const void* x,
+                          int64_t n, float* y, float* norm, cudaStream_t st);
+
+// query.cu
+cudaError_t launch_query_prep(const pariskv_index* ix, const void* q, const float* qt_in,
+                              const float* qn_in, bool rotated, cudaStream_t st);
+
+// vote.cu
+cudaError_t launch_vote(const pariskv_index* ix, cudaStream_t st);
+
+// select.cu
+cudaError_t launch_threshold(const pariskv_index* ix, int64_t C, cudaStream_t st);
+cudaError_t launch_compact(const pariskv_index* ix, cudaStream_t st);
+
+// rerank.cu
+cudaError_t launch_rerank(const pariskv_index* ix, int64_t C, cudaStream_t st);
+
+// topk.cu
+cudaError_t launch_topk(const pariskv_index* ix, int64_t C, int32_t k, int32_t* topk_idx,
+                        float* topk_est, cudaStream_t st);
+
+// attend.cu
+cudaError_t launch_attend(const pariskv_config* cfg, const void* q, const void* K,
+                          const void* V, int64_t ld_tok, int64_t n, const int32_t* topk_idx,
+                          int32_t k,
+                          float scale, void* out, float* work, int nsplit, cudaStream_t st);
+int attend_splits(int heads, int32_t k, int num_sms);
+size_t attend_workspace_floats(int heads, int nsplit);
+
+}  // namespace pkv

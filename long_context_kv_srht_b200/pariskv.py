@@ -1,0 +1,281 @@
+"""Thin ctypes binding over libpariskv.so (the C ABI declared in include/pariskv.h and
+include/pariskv_debug.h).
+
+Only argument marshalling happens here: tensors become data pointers and strides become the
+library's slab strides; every step of the retrieval path runs in the library's CUDA kernels.
+Importing this module loads the library and raises if it is missing (there is no fallback).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "libpariskv.so")
+HEADERS = [os.path.join(os.path.dirname(_PKG), "include", h)
+           for h in ("pariskv.h", "pariskv_debug.h")]
+
+OK, EINVAL, ENOMEM, ECUDA, ECAPACITY, ETIMEOUT = range(6)
+F32, BF16 = 0, 1
+
+
+class PariskvError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__(f"{where}: status {status} ({_status_name(status)}): {message}")
+        self.status = status
+
+
+def _status_name(s: int) -> str:
+    return ["OK", "EINVAL", "ENOMEM", "ECUDA", "ECAPACITY", "ETIMEOUT"][s] if 0 <= s < 6 else "?"
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("B", ctypes.c_int32), ("m", ctypes.c_int32),
+                ("rho", ctypes.c_int32), ("w_rank1", ctypes.c_int32), ("w_rest", ctypes.c_int32),
+                ("cand_bp", ctypes.c_int32), ("batch", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("capacity", ctypes.c_int64), ("dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+    @property
+    def num_q_heads(self) -> int:
+        return self.num_kv_heads * self.group
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python -m long_context_kv_srht_b200.build`")
+lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I32, _I64 = ctypes.c_int32, ctypes.c_int64
+_S = ctypes.c_int
+_SIGS = {
+    "pariskv_config_default": (_S, [ctypes.POINTER(Config)]),
+    "pariskv_build_index": (_S, [ctypes.POINTER(Config), _P, _P, _I64, _I64, _P, ctypes.POINTER(_P)]),
+    "pariskv_append": (_S, [_P, _P, _I64, _I64, _P]),
+    "pariskv_search": (_S, [_P, _P, _I32, _P, _P, _P]),
+    "pariskv_sparse_attend": (_S, [ctypes.POINTER(Config), _P, _P, _P, _I64, _I64, _P, _I32,
+                                   ctypes.c_float, _P, _P]),
+    "pariskv_sync": (_S, [_P, _P]),
+    "pariskv_destroy": (_S, [_P]),
+    "pariskv_size": (_I64, [_P]),
+    "pariskv_last_launch_count": (_I32, []),
+    "pariskv_status_string": (ctypes.c_char_p, [_S]),
+    "pariskv_last_error": (ctypes.c_char_p, []),
+    "pariskv_debug_rotate": (_S, [ctypes.POINTER(Config), _P, _P, _I64, _P, _P, _P]),
+    "pariskv_debug_build_index_rotated": (_S, [ctypes.POINTER(Config), _P, _P, _P, _I64, _I64, _P,
+                                               ctypes.POINTER(_P)]),
+    "pariskv_debug_append_rotated": (_S, [_P, _P, _P, _I64, _I64, _P]),
+    "pariskv_debug_search_rotated": (_S, [_P, _P, _P, _I32, _P, _P, _P]),
+    "pariskv_debug_export_index": (_S, [_P, _P, _P, _P]),
+    "pariskv_debug_export_search": (_S, [_P, _P, _P, ctypes.POINTER(_I64), _P, _P]),
+    "pariskv_debug_profile": (_S, [_P, _I32]),
+    "pariskv_debug_stage_ms": (_S, [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_I32)]),
+}
+
+STAGES = ("query_prep", "vote", "threshold", "compact", "rerank", "topk")
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+def declared_symbols() -> list:
+    """Every function declared in the public and test-only headers."""
+    names = []
+    for h in HEADERS:
+        with open(h) as f:
+            names += re.findall(r"PARISKV_API\s+[\w\s\*]+?\b(pariskv_\w+)\s*\(", f.read())
+    return names
+
+
+def last_error() -> str:
+    return lib.pariskv_last_error().decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise PariskvError(status, where, last_error())
+
+
+def config(**kw) -> Config:
+    c = Config()
+    _check(lib.pariskv_config_default(ctypes.byref(c)), "pariskv_config_default")
+    for k, v in kw.items():
+        if k == "dtype" and isinstance(v, str):
+            v = BF16 if v == "bf16" else F32
+        setattr(c, k, v)
+    return c
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _signs_ptr(signs) -> tuple:
+    a = np.ascontiguousarray(np.asarray(signs.cpu() if hasattr(signs, "cpu") else signs,
+                                        dtype=np.int8))
+    return a, a.ctypes.data
+
+
+def _slab(t, d: int = 128) -> int:
+    """Token slab stride of a [units..., tokens, d] view (rows contiguous, d elements each)."""
+    assert t.stride(-1) == 1 and t.stride(-2) == d, "rows must be contiguous d-vectors"
+    if t.dim() <= 2:
+        return t.shape[-2] if t.dim() == 2 else 1
+    return t.stride(-3) // d
+
+
+class Index:
+    """Owner of a ``pariskv_index*``; methods map one-to-one onto the C calls."""
+
+    def __init__(self, handle: int, cfg: Config):
+        self.handle = ctypes.c_void_p(handle)
+        self.cfg = cfg
+
+    # -- product calls ------------------------------------------------------------------
+    def append(self, keys, t: Optional[int] = None, stream=None) -> None:
+        t = keys.shape[-2] if t is None else t
+        _check(lib.pariskv_append(self.handle, keys.data_ptr(), _slab(keys), t, _stream(stream)),
+               "pariskv_append")
+
+    def search(self, q, k: int, topk_idx=None, topk_est=None, want_est: bool = True,
+               stream=None):
+        import torch
+        H = self.cfg.batch * self.cfg.num_q_heads
+        if topk_idx is None:
+            topk_idx = torch.empty((H, k), dtype=torch.int32, device=q.device)
+        if topk_est is None and want_est:
+            topk_est = torch.empty((H, k), dtype=torch.float32, device=q.device)
+        _check(lib.pariskv_search(self.handle, q.data_ptr(), k, topk_idx.data_ptr(),
+                                  topk_est.data_ptr() if topk_est is not None else None,
+                                  _stream(stream)), "pariskv_search")
+        return topk_idx, topk_est
+
+    def sync(self, stream=None) -> None:
+        _check(lib.pariskv_sync(self.handle, _stream(stream)), "pariskv_sync")
+
+    @property
+    def size(self) -> int:
+        return int(lib.pariskv_size(self.handle))
+
+    def destroy(self) -> None:
+        if self.handle:
+            lib.pariskv_destroy(self.handle)
+            self.handle = ctypes.c_void_p(0)
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+    # -- test-only calls ----------------------------------------------------------------
+    def append_rotated(self, y, knorm, stream=None) -> None:
+        _check(lib.pariskv_debug_append_rotated(self.handle, y.data_ptr(), knorm.data_ptr(),
+                                                _slab(y), y.shape[-2], _stream(stream)),
+               "pariskv_debug_append_rotated")
+
+    def search_rotated(self, qt, qnorm, k: int, stream=None):
+        import torch
+        H = self.cfg.batch * self.cfg.num_q_heads
+        idx = torch.empty((H, k), dtype=torch.int32, device=qt.device)
+        est = torch.empty((H, k), dtype=torch.float32, device=qt.device)
+        _check(lib.pariskv_debug_search_rotated(self.handle, qt.data_ptr(), qnorm.data_ptr(), k,
+                                                idx.data_ptr(), est.data_ptr(), _stream(stream)),
+               "pariskv_debug_search_rotated")
+        return idx, est
+
+    def profile(self, enable: bool = True) -> None:
+        _check(lib.pariskv_debug_profile(self.handle, int(enable)), "pariskv_debug_profile")
+
+    def stage_ms(self) -> dict:
+        ms = (ctypes.c_float * 8)()
+        n = _I32(0)
+        _check(lib.pariskv_debug_stage_ms(self.handle, ms, ctypes.byref(n)),
+               "pariskv_debug_stage_ms")
+        return {STAGES[i]: float(ms[i]) for i in range(n.value)}
+
+    def export_index(self):
+        units = self.cfg.batch * self.cfg.num_kv_heads
+        n = self.size
+        ids = np.empty((units, n, 16), np.uint8)
+        codes = np.empty((units, n, 128), np.uint8)
+        fac = np.empty((units, n, 16), np.float32)
+        _check(lib.pariskv_debug_export_index(self.handle, ids.ctypes.data, codes.ctypes.data,
+                                              fac.ctypes.data), "pariskv_debug_export_index")
+        return ids, codes, fac
+
+    def export_search(self):
+        H = self.cfg.batch * self.cfg.num_q_heads
+        n = self.size
+        C = _I64(0)
+        _check(lib.pariskv_debug_export_search(self.handle, None, None, ctypes.byref(C), None,
+                                               None), "pariskv_debug_export_search")
+        C = int(C.value)
+        lut = np.empty((H, 16, 256), np.uint8)
+        scores = np.empty((H, n), np.int32)
+        cand = np.empty((H, C), np.int32)
+        S = np.empty((H, C), np.float32)
+        _check(lib.pariskv_debug_export_search(self.handle, lut.ctypes.data, scores.ctypes.data,
+                                               None, cand.ctypes.data, S.ctypes.data),
+               "pariskv_debug_export_search")
+        return lut, scores, cand, S
+
+
+def build_index(cfg: Config, signs, keys, n: Optional[int] = None, stream=None) -> Index:
+    """keys: tensor [batch, num_kv_heads, L, d] (device or pinned host); n <= L tokens used."""
+    n = keys.shape[-2] if n is None else n
+    sa, sp = _signs_ptr(signs)
+    h = _P()
+    _check(lib.pariskv_build_index(ctypes.byref(cfg), sp, keys.data_ptr(), _slab(keys), n,
+                                   _stream(stream), ctypes.byref(h)), "pariskv_build_index")
+    return Index(h.value, cfg)
+
+
+def build_index_rotated(cfg: Config, signs, y, knorm, n: Optional[int] = None,
+                        stream=None) -> Index:
+    n = y.shape[-2] if n is None else n
+    sa, sp = _signs_ptr(signs)
+    h = _P()
+    _check(lib.pariskv_debug_build_index_rotated(ctypes.byref(cfg), sp, y.data_ptr(),
+                                                 knorm.data_ptr(), _slab(y), n, _stream(stream),
+                                                 ctypes.byref(h)),
+           "pariskv_debug_build_index_rotated")
+    return Index(h.value, cfg)
+
+
+def rotate(cfg: Config, signs, x, stream=None):
+    import torch
+    n = x.numel() // 128
+    y = torch.empty((n, 128), dtype=torch.float32, device=x.device)
+    nr = torch.empty((n,), dtype=torch.float32, device=x.device)
+    sa, sp = _signs_ptr(signs)
+    _check(lib.pariskv_debug_rotate(ctypes.byref(cfg), sp, x.data_ptr(), n, y.data_ptr(),
+                                    nr.data_ptr(), _stream(stream)), "pariskv_debug_rotate")
+    return y, nr
+
+
+def sparse_attend(cfg: Config, q, K, V, topk_idx, k: int, scale: float, n: Optional[int] = None,
+                  out=None, stream=None):
+    """q [batch, Hq, d]; K, V [batch, Hkv, L, d] (device or pinned host); topk [batch*Hq, k]."""
+    import torch
+    n = K.shape[-2] if n is None else n
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
+    _check(lib.pariskv_sparse_attend(ctypes.byref(cfg), q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                     _slab(K), n, topk_idx.data_ptr(), k, float(scale),
+                                     out.data_ptr(), _stream(stream)), "pariskv_sparse_attend")
+    return out
+
+
+def last_launch_count() -> int:
+    return int(lib.pariskv_last_launch_count())

@@ -83,8 +83,10 @@ def spec(name: str, **overrides) -> Spec:
 def bf16_round(x: np.ndarray) -> np.ndarray:
     """fp32 -> nearest bf16 (ties to even), returned as fp32 values (exactly representable)."""
     u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
-    r = ((u.astype(np.uint64) + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint32) << 16
-    return r.astype(np.uint32).view(np.float32)
+    # finite inputs never wrap: the largest finite pattern plus 0x8000 rounds up to infinity
+    r = u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    r &= np.uint32(0xFFFF0000)
+    return r.view(np.float32)
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:

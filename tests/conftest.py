@@ -28,3 +28,12 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+# The CUDA library and the oracle are compiled in-tree on first use (nvcc cross-compiles for
+# sm_100a without a GPU); an up-to-date build is reused.
+def pytest_sessionstart(session):
+    from long_context_kv_srht_b200 import build as kbuild
+    kbuild.build()
+    import oracle
+    oracle.build()
