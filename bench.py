@@ -41,6 +41,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
     return ap.parse_args()
 
 
@@ -225,6 +226,45 @@ def run_reference(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+def decode_step(args, ix, cfg, sp, keys, vals, qs, idx, est, k, H, dev, kv_host):
+    import numpy as np
+    import torch
+    from long_context_kv_srht_b200 import pariskv as pk
+    ix.profile(True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    ea = torch.cuda.Event(enable_timing=True)
+    es = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    app_ms = srch_ms = att_ms = 0.0
+    stage = {}
+    nrep = 5
+    out = torch.empty(qs.shape, dtype=torch.float32, device=dev)
+    assert nrep <= APPEND_SLACK
+    for s in range(nrep):
+        new_k = keys[:, :, ix.size:ix.size + 1].to(dev)
+        e0.record()
+        ix.append(new_k)
+        ea.record()
+        ix.search(qs, k, idx, est)
+        es.record()
+        pk.sparse_attend(cfg, qs, keys, vals, idx, k, 1.0 / float(np.sqrt(sp.d)), n=ix.size,
+                         out=out)
+        e1.record()
+        e1.synchronize()
+        for name, ms in ix.stage_ms().items():
+            stage[name] = stage.get(name, 0.0) + ms / nrep
+        app_ms += e0.elapsed_time(ea) / nrep
+        srch_ms += ea.elapsed_time(es) / nrep
+        att_ms += es.elapsed_time(e1) / nrep
+    kv_bytes = H * k * 2 * sp.d * 2
+    decode = {"append_ms": app_ms, "search_ms": srch_ms, "sparse_attend_ms": att_ms,
+              "total_ms": app_ms + srch_ms + att_ms,
+              "kv_source": "pinned host (UVA)" if kv_host else "HBM",
+              "attend_gbs": kv_bytes / (att_ms / 1e3) / 1e9}
+    decode["search_stage_ms"] = stage
+    return decode
+
+
 # ------------------------------------------------------------------------------------ main
 def main():
     args = parse()
@@ -330,34 +370,11 @@ def main():
 
     # the full decode step around the search: append one key per (sequence, KV head), search,
     # sparse attention over the top-k (K/V read from pinned host memory over UVA here)
-    e0 = torch.cuda.Event(enable_timing=True)
-    ea = torch.cuda.Event(enable_timing=True)
-    es = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    app_ms = srch_ms = att_ms = 0.0
-    nrep = 5
-    out = torch.empty_like(qs)
-    assert nrep <= APPEND_SLACK
-    for s in range(nrep):
-        new_k = keys[:, :, ix.size:ix.size + 1].to(dev)
-        e0.record()
-        ix.append(new_k)
-        ea.record()
-        ix.search(qs, k, idx, est)
-        es.record()
-        pk.sparse_attend(cfg, qs, keys, vals, idx, k, 1.0 / float(np.sqrt(sp.d)), n=ix.size,
-                         out=out)
-        e1.record()
-        e1.synchronize()
-        app_ms += e0.elapsed_time(ea) / nrep
-        srch_ms += ea.elapsed_time(es) / nrep
-        att_ms += es.elapsed_time(e1) / nrep
-    kv_bytes = H * k * 2 * sp.d * 2
-    decode = {"append_ms": app_ms, "search_ms": srch_ms, "sparse_attend_ms": att_ms,
-              "total_ms": app_ms + srch_ms + att_ms,
-              "kv_source": "pinned host (UVA)" if kv_host else "HBM",
-              "attend_gbs": kv_bytes / (att_ms / 1e3) / 1e9}
+    decode = None
+    if not args.no_decode:
+        decode = decode_step(args, ix, cfg, sp, keys, vals, qs, idx, est, k, H, dev, kv_host)
 
+    cpu = None
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         v, dt, cores = oracle_sample(sp, data, reps=1)

@@ -127,14 +127,17 @@ PARISKV_API pariskv_status pariskv_search(pariskv_index* index, const void* q, i
  *   out[s][h] = sum_{t in topk[s][h]} softmax_t(scale * <q[s][h], K[s][h/group][t]>) V[..][t]
  *   q:        device pointer [batch][Hq][d]; K, V: device or pinned-host pointers with the
  *             layout of pariskv_build_index's keys (slab stride ld_tok, n valid tokens);
- *   topk_idx: device pointer [batch][Hq][k] with values in [0, n);
- *   out:      device pointer [batch][Hq][d]. Element type cfg->dtype everywhere; fp32
- *             accumulation. Uses a library-owned per-device workspace.
+ *   topk_idx: device pointer [batch][Hq][k]; entries outside [0, n) are skipped;
+ *   out:      device pointer [batch][Hq][d] of element type out_dtype (PARISKV_F32 keeps the
+ *             fp32 accumulator precision; PARISKV_BF16 rounds to nearest even).
+ * q, K and V have element type cfg->dtype; accumulation is fp32. The split-K partials live in
+ * a stream-ordered workspace (cudaMallocAsync / cudaFreeAsync on `stream`).
  * Errors: EINVAL, ENOMEM, ECUDA. */
-PARISKV_API pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, const void* K,
-                                     const void* V, int64_t ld_tok, int64_t n,
-                                     const int32_t* topk_idx, int32_t k, float scale, void* out,
-                                     void* stream);
+PARISKV_API pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q,
+                                                 const void* K, const void* V, int64_t ld_tok,
+                                                 int64_t n, const int32_t* topk_idx, int32_t k,
+                                                 float scale, void* out, int32_t out_dtype,
+                                                 void* stream);
 
 /* Waits for the index's stream work and reports any asynchronous error or expired wait. */
 PARISKV_API pariskv_status pariskv_sync(pariskv_index* index, void* stream);

@@ -319,7 +319,7 @@ pariskv_status pariskv_search(pariskv_index* index, const void* q, int32_t k, in
 pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, const void* K,
                                      const void* V, int64_t ld_tok, int64_t n,
                                      const int32_t* topk_idx, int32_t k, float scale, void* out,
-                                     void* stream) {
+                                     int32_t out_dtype, void* stream) {
     pariskv_status s = check_config(cfg);
     if (s != PARISKV_OK) return s;
     const size_t al = cfg->dtype == PARISKV_BF16 ? 8 : 16;
@@ -330,7 +330,10 @@ pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, c
     if ((s = check_dev_ptr(K, al, "K")) != PARISKV_OK) return s;
     if ((s = check_dev_ptr(V, al, "V")) != PARISKV_OK) return s;
     if ((s = check_dev_ptr(topk_idx, 4, "topk_idx")) != PARISKV_OK) return s;
-    if ((s = check_dev_ptr(out, al, "out")) != PARISKV_OK) return s;
+    if (out_dtype != PARISKV_F32 && out_dtype != PARISKV_BF16)
+        return fail(PARISKV_EINVAL, "out_dtype %d unknown", out_dtype);
+    if ((s = check_dev_ptr(out, out_dtype == PARISKV_BF16 ? 8 : 16, "out")) != PARISKV_OK)
+        return s;
     if (!(scale == scale)) return fail(PARISKV_EINVAL, "scale is NaN");
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
@@ -344,7 +347,8 @@ pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, c
                                     attend_workspace_floats(heads, nsplit) * sizeof(float), st);
     if (e != cudaSuccess) return cuda_fail(e, "attention workspace");
     g_launches = 0;
-    e = launch_attend(cfg, q, K, V, ld_tok, n, topk_idx, k, scale, out, work, nsplit, st);
+    e = launch_attend(cfg, q, K, V, ld_tok, n, topk_idx, k, scale, out, out_dtype, work, nsplit,
+                      st);
     if (e == cudaSuccess) g_launches = 2;
     cudaFreeAsync(work, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");

@@ -11,7 +11,7 @@
 // keeps an online-softmax state (running max, denominator, 4 accumulators). Four tokens
 // are loaded before any is used so that each warp has 8 row reads in flight (this matters
 // for K/V in host memory, where a read crosses PCIe). The warps are merged in shared memory
-// and the CTA writes (max, denominator, 128 accumulators) to the workspace; a second kernel
+// and the CTA writes (128 accumulators, max, denominator) to the workspace; a second kernel
 // merges the splits with the log-sum-exp rule and writes the output in the input dtype.
 #include "common.cuh"
 #include "internal.hpp"
@@ -22,7 +22,11 @@ namespace {
 
 constexpr int kAW = 4;            // warps per CTA
 constexpr int kUnroll = 4;        // tokens in flight per warp
-constexpr int kPart = 2 + D;      // floats per partial: max, denominator, accumulators
+// floats per partial: 128 accumulators, then max and denominator, padded to a multiple of 4
+// so that every partial (and its accumulators) starts on a 16-byte boundary
+constexpr int kPart = D + 4;
+constexpr int kMax = D, kDen = D + 1;
+static_assert((kPart * sizeof(float)) % 16 == 0, "partials must stay 16-byte aligned");
 
 template <typename T> __device__ __forceinline__ void store4(T* p, const float v[4]);
 template <> __device__ __forceinline__ void store4<float>(float* p, const float v[4]) {
@@ -42,7 +46,7 @@ __global__ void __launch_bounds__(kAW * 32)
 attend_partial_kernel(const T* __restrict__ q, const T* __restrict__ K, const T* __restrict__ V,
                       int64_t ld_tok, int64_t n, const int32_t* __restrict__ topk, int32_t k,
                       float scale, int group, int nsplit, float* __restrict__ work) {
-    __shared__ float sm[kAW][kPart];
+    __shared__ __align__(16) float sm[kAW][kPart];
     const int head = blockIdx.y, split = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t unit = head / group;
@@ -89,24 +93,24 @@ attend_partial_kernel(const T* __restrict__ q, const T* __restrict__ K, const T*
         }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) sm[warp][2 + 4 * lane + i] = acc[i];
-    if (lane == 0) { sm[warp][0] = mx; sm[warp][1] = den; }
+    for (int i = 0; i < 4; ++i) sm[warp][4 * lane + i] = acc[i];
+    if (lane == 0) { sm[warp][kMax] = mx; sm[warp][kDen] = den; }
     __syncthreads();
     if (warp == 0) {
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kAW; ++w) M = fmaxf(M, sm[w][0]);
+        for (int w = 0; w < kAW; ++w) M = fmaxf(M, sm[w][kMax]);
         float dsum = 0.0f, a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
         for (int w = 0; w < kAW; ++w) {
-            const float f = sm[w][0] == -INFINITY ? 0.0f : expf(sm[w][0] - M);
-            dsum += sm[w][1] * f;
+            const float f = sm[w][kMax] == -INFINITY ? 0.0f : expf(sm[w][kMax] - M);
+            dsum += sm[w][kDen] * f;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] += sm[w][2 + 4 * lane + i] * f;
+            for (int i = 0; i < 4; ++i) a[i] += sm[w][4 * lane + i] * f;
         }
         float* out = work + (static_cast<int64_t>(head) * nsplit + split) * kPart;
-        *reinterpret_cast<float4*>(out + 2 + 4 * lane) = make_float4(a[0], a[1], a[2], a[3]);
-        if (lane == 0) { out[0] = M; out[1] = dsum; }
+        *reinterpret_cast<float4*>(out + 4 * lane) = make_float4(a[0], a[1], a[2], a[3]);
+        if (lane == 0) { out[kMax] = M; out[kDen] = dsum; }
     }
 }
 
@@ -116,13 +120,13 @@ attend_combine_kernel(const float* __restrict__ work, int nsplit, T* __restrict_
     const int head = blockIdx.x, lane = threadIdx.x;
     const float* w = work + static_cast<int64_t>(head) * nsplit * kPart;
     float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, w[s * kPart]);
+    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, w[s * kPart + kMax]);
     float den = 0.0f, a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     for (int s = 0; s < nsplit; ++s) {
-        const float ms = w[s * kPart];
+        const float ms = w[s * kPart + kMax];
         const float f = ms == -INFINITY ? 0.0f : expf(ms - M);
-        den += w[s * kPart + 1] * f;
-        const float4 v = *reinterpret_cast<const float4*>(w + s * kPart + 2 + 4 * lane);
+        den += w[s * kPart + kDen] * f;
+        const float4 v = *reinterpret_cast<const float4*>(w + s * kPart + 4 * lane);
         a[0] += v.x * f; a[1] += v.y * f; a[2] += v.z * f; a[3] += v.w * f;
     }
     const float inv = den > 0.0f ? 1.0f / den : 0.0f;
@@ -146,8 +150,8 @@ size_t attend_workspace_floats(int heads, int nsplit) {
 
 cudaError_t launch_attend(const pariskv_config* cfg, const void* q, const void* K,
                           const void* V, int64_t ld_tok, int64_t n, const int32_t* topk_idx,
-                          int32_t k,
-                          float scale, void* out, float* work, int nsplit, cudaStream_t st) {
+                          int32_t k, float scale, void* out, int32_t out_dtype, float* work,
+                          int nsplit, cudaStream_t st) {
     const int heads = cfg->batch * cfg->num_kv_heads * cfg->group;
     dim3 grid(nsplit, heads);
     if (cfg->dtype == PARISKV_BF16) {
@@ -155,14 +159,17 @@ cudaError_t launch_attend(const pariskv_config* cfg, const void* q, const void* 
         attend_partial_kernel<T><<<grid, kAW * 32, 0, st>>>(
             static_cast<const T*>(q), static_cast<const T*>(K), static_cast<const T*>(V),
             ld_tok, n, topk_idx, k, scale, cfg->group, nsplit, work);
-        attend_combine_kernel<T><<<heads, 32, 0, st>>>(work, nsplit, static_cast<T*>(out));
     } else {
         attend_partial_kernel<float><<<grid, kAW * 32, 0, st>>>(
             static_cast<const float*>(q), static_cast<const float*>(K),
             static_cast<const float*>(V), ld_tok, n, topk_idx, k, scale, cfg->group, nsplit,
             work);
-        attend_combine_kernel<float><<<heads, 32, 0, st>>>(work, nsplit, static_cast<float*>(out));
     }
+    if (out_dtype == PARISKV_BF16)
+        attend_combine_kernel<__nv_bfloat16><<<heads, 32, 0, st>>>(
+            work, nsplit, static_cast<__nv_bfloat16*>(out));
+    else
+        attend_combine_kernel<float><<<heads, 32, 0, st>>>(work, nsplit, static_cast<float*>(out));
     return cudaGetLastError();
 }
 

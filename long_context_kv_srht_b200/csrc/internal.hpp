@@ -76,8 +76,8 @@ cudaError_t launch_topk(const pariskv_index* ix, int64_t C, int32_t k, int32_t* 
 // attend.cu
 cudaError_t launch_attend(const pariskv_config* cfg, const void* q, const void* K,
                           const void* V, int64_t ld_tok, int64_t n, const int32_t* topk_idx,
-                          int32_t k,
-                          float scale, void* out, float* work, int nsplit, cudaStream_t st);
+                          int32_t k, float scale, void* out, int32_t out_dtype, float* work,
+                          int nsplit, cudaStream_t st);
 int attend_splits(int heads, int32_t k, int num_sms);
 size_t attend_workspace_floats(int heads, int nsplit);
 

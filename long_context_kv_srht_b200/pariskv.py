@@ -60,7 +60,7 @@ _SIGS = {
     "pariskv_append": (_S, [_P, _P, _I64, _I64, _P]),
     "pariskv_search": (_S, [_P, _P, _I32, _P, _P, _P]),
     "pariskv_sparse_attend": (_S, [ctypes.POINTER(Config), _P, _P, _P, _I64, _I64, _P, _I32,
-                                   ctypes.c_float, _P, _P]),
+                                   ctypes.c_float, _P, _I32, _P]),
     "pariskv_sync": (_S, [_P, _P]),
     "pariskv_destroy": (_S, [_P]),
     "pariskv_size": (_I64, [_P]),
@@ -265,15 +265,18 @@ def rotate(cfg: Config, signs, x, stream=None):
 
 
 def sparse_attend(cfg: Config, q, K, V, topk_idx, k: int, scale: float, n: Optional[int] = None,
-                  out=None, stream=None):
-    """q [batch, Hq, d]; K, V [batch, Hkv, L, d] (device or pinned host); topk [batch*Hq, k]."""
+                  out=None, out_dtype=None, stream=None):
+    """q [batch, Hq, d]; K, V [batch, Hkv, L, d] (device or pinned host); topk [batch*Hq, k].
+    out_dtype: torch.float32 (fp32 accumulator precision) or torch.bfloat16; defaults to the
+    dtype of ``out`` when given, else to q's dtype."""
     import torch
     n = K.shape[-2] if n is None else n
     if out is None:
-        out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    od = BF16 if out.dtype == torch.bfloat16 else F32
     _check(lib.pariskv_sparse_attend(ctypes.byref(cfg), q.data_ptr(), K.data_ptr(), V.data_ptr(),
                                      _slab(K), n, topk_idx.data_ptr(), k, float(scale),
-                                     out.data_ptr(), _stream(stream)), "pariskv_sparse_attend")
+                                     out.data_ptr(), od, _stream(stream)), "pariskv_sparse_attend")
     return out
 
 

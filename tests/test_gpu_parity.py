@@ -4,7 +4,7 @@ Bit-exact gates (identical rotated fp32 inputs on both sides): bucket ids, 4-bit
 calibration factors, vote lookup tables, coarse scores, candidate sets, rerank values, top-k
 indices and estimates. Tolerance gates: rotation <= 1e-5 absolute per coordinate of the
 unit vector; end-to-end top-k recall from raw inputs >= 0.999; sparse attention <= 2e-3
-absolute (bf16 output)."""
+absolute with fp32 output (bf16 output adds its own rounding bound)."""
 import numpy as np
 import pytest
 import torch
@@ -181,7 +181,11 @@ def test_end_to_end_recall_from_raw_inputs(name, n):
 @pytest.mark.parametrize("dtype,G,n,k", [("bf16", 4, 5000, 512), ("f32", 1, 3000, 3000),
                                          ("bf16", 2, 70, 1), ("bf16", 4, 20000, 2048)])
 @pytest.mark.parametrize("host_kv", [False, True])
-def test_sparse_attend_matches_oracle(dtype, G, n, k, host_kv):
+@pytest.mark.parametrize("out_f32", [True, False])
+def test_sparse_attend_matches_oracle(dtype, G, n, k, host_kv, out_f32):
+    """fp32 output: |gpu - oracle| <= 2e-3. bf16 output additionally carries its own
+    round-to-nearest error, at most 2^-9 |x| (8 significand bits), so the bound there is
+    2e-3 + 2^-8 |oracle| (one rounding of the result plus fp32 accumulation slack)."""
     rng = np.random.default_rng(n + k)
     batch, hkv = 2, 2
     K = rng.standard_normal((batch, hkv, n, 128)).astype(np.float32) * 0.5
@@ -199,14 +203,16 @@ def test_sparse_attend_matches_oracle(dtype, G, n, k, host_kv):
         Kt, Vt = Kt.pin_memory(), Vt.pin_memory()
     else:
         Kt, Vt = Kt.to(DEV), Vt.to(DEV)
+    od = torch.float32 if out_f32 else torch.bfloat16
     out = pk.sparse_attend(cfg, conv(q).to(DEV), Kt, Vt, _t(topk.astype(np.int32)), k,
-                           1 / np.sqrt(128))
+                           1 / np.sqrt(128), out_dtype=od)
     got = out.float().cpu().numpy()
     for b in range(batch):
         for h in range(hkv * G):
             ref = oracle.attend(q[b, h], K[b, h // G], V[b, h // G],
                                 topk[b * hkv * G + h].astype(np.int32), 1 / np.sqrt(128))
-            assert np.max(np.abs(got[b, h] - ref)) <= 2e-3
+            tol = 2e-3 if out_f32 else 2e-3 + np.abs(ref) * 2.0 ** -8
+            assert np.all(np.abs(got[b, h] - ref) <= tol)
 
 
 # ------------------------------------------------------------------------------- errors
