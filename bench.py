@@ -340,6 +340,42 @@ def main():
                 "step_algorithmic_bytes": step_bytes,
                 "step_frac": step_bytes / (step_ms_max / 1e3) / 1e9 / peak}
 
+    # host cost of enqueueing one search (the device is kept busy meanwhile), and the same
+    # search replayed as a CUDA graph (one launch per step, no host work between kernels)
+    ix.profile(False)
+    big = torch.empty(4 << 30, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    big.fill_(1)
+    t0 = time.perf_counter()
+    for _ in range(10):
+        ix.search(qs, k, idx, est)
+    host_us = (time.perf_counter() - t0) / 10 * 1e6
+    torch.cuda.synchronize()
+    del big
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        ix.search(qs, k, idx, est)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+        ix.search(qs, k, idx, est)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    gtimes = []
+    for s in range(args.steps):
+        flush.fill_(s & 255)
+        ev0[s].record()
+        graph.replay()
+        ev1[s].record()
+    torch.cuda.synchronize()
+    graph_ms = dist_max(float(np.mean([a.elapsed_time(b) for a, b in zip(ev0, ev1)])), ws)
+    graph_value = ws * keys_per_step / (graph_ms / 1e3)
+    del graph
+    ix.profile(True)
+
     # end to end through the C ABI: pinned host query in, top-k indices and estimates out
     e2e = None
     if not args.no_e2e:
@@ -394,6 +430,8 @@ def main():
                        "key_dtype": sp.dtype, "kv_in": "pinned host" if kv_host else "HBM",
                        "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"},
             "stage_ms": stage_avg,
+            "host_enqueue_us_per_search": host_us,
+            "graph": {"ms_per_step": graph_ms, "value": graph_value},
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -402,6 +440,7 @@ def main():
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
+    ix.sync()   # raises if a device-side consistency flag or bounded wait fired
     ix.destroy()
     if ws > 1:
         import torch.distributed as dist

@@ -508,11 +508,12 @@ pariskv_status pariskv_debug_export_index(pariskv_index* ix, uint8_t* ids, uint8
             const int64_t o = static_cast<int64_t>(u) * n + i;
             for (int b = 0; b < NB; ++b) {
                 if (ids) ids[o * NB + b] = hid[i * 16 + ((b - i) & 15)];
+                const int64_t at = i * REC + 32 * (b >> 2) + 4 * (b & 3);
                 uint32_t w;
-                memcpy(&w, &hrec[i * REC + 4 * b], 4);
+                memcpy(&w, &hrec[at], 4);
                 if (codes)
                     for (int j = 0; j < M; ++j) codes[o * D + b * M + j] = (w >> (4 * j)) & 15u;
-                if (factors) memcpy(&factors[o * NB + b], &hrec[i * REC + 64 + 4 * b], 4);
+                if (factors) memcpy(&factors[o * NB + b], &hrec[at + 16], 4);
             }
         }
     }

@@ -61,28 +61,15 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
-}
 
-__device__ __forceinline__ uint4 lds_u128(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-    return v;
-}
-
-__device__ __forceinline__ void red_shared_add(uint32_t addr, uint32_t v) {
-    asm volatile("red.shared.add.u32 [%0], %1;" :: "r"(addr), "r"(v) : "memory");
-}
-
-// 128-bit read-only global load that does not allocate in L1 (streamed data).
-__device__ __forceinline__ uint4 ldg_stream_u128(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+// 256-bit read-only global load that does not allocate in L1 (sm_100): 8 consecutive words.
+struct u32x8 { uint32_t w[8]; };
+__device__ __forceinline__ u32x8 ldg_stream_u256(const void* p) {
+    u32x8 v;
+    asm("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]),
+          "=r"(v.w[6]), "=r"(v.w[7])
+        : "l"(p));
     return v;
 }
 

@@ -23,8 +23,10 @@
 //  ids: 16 bytes at (unit * cap_pad + i) * 16; subspace b is stored at byte (b - i) mod 16.
 //       The rotation by the key index lets the vote scan read, at each step, 32 different
 //       subspaces across a warp and so hit 32 different shared-memory banks.
-//  rec: 128 bytes at (unit * cap_pad + i) * 128: bytes 4b..4b+3 hold the 8 codes of
-//       subspace b (dim j in nibble j, sign in bit 3 of the nibble); bytes 64 + 4b hold f_b.
+//  rec: 128 bytes at (unit * cap_pad + i) * 128, four 32-byte chunks; chunk p serves
+//       subspaces 4p..4p+3: its first 16 bytes are their code words (subspace b's 8 codes in
+//       one 32-bit word, dim j in nibble j, sign in bit 3 of the nibble), its last 16 bytes
+//       their factors f_b. The rerank reads one chunk per lane with a single 32-byte load.
 #include "common.cuh"
 #include "internal.hpp"
 #include "rotate.cuh"
@@ -108,9 +110,9 @@ encode_kernel(const T* __restrict__ src, const float* __restrict__ knorm_in, int
         const int64_t key = pos0 + r;
         const int64_t slot = unit * cap_pad + key;
         ids[slot * 16 + ((b - key) & 15)] = static_cast<uint8_t>(id);
-        uint8_t* rr = rec + slot * REC;
-        reinterpret_cast<uint32_t*>(rr)[b] = code;
-        reinterpret_cast<float*>(rr + 64)[b] = f;
+        uint8_t* rr = rec + slot * REC + 32 * (b >> 2) + 4 * (b & 3);
+        *reinterpret_cast<uint32_t*>(rr) = code;
+        *reinterpret_cast<float*>(rr + 16) = f;
     }
 }
 

@@ -11,11 +11,14 @@
 // score == T.
 //
 //  threshold_kernel (one CTA per query head): sums the per-chunk histograms written by the
-//    vote scan, finds T and E, and writes for every 8192-key chunk how many candidates and
-//    how many score-T keys precede it (exclusive scans over chunks).
-//  compact_kernel (one CTA per chunk and vote pack): each thread owns 32 consecutive keys;
-//    two block-wide scans (tie counts, then candidate counts, four heads packed in 16-bit
-//    lanes of a 64-bit word) give every candidate its output position.
+//    vote scan (warp per chunk, lane per pair of bins), finds T and E with suffix sums and
+//    ballots, and writes for every 8192-key chunk how many candidates and how many score-T
+//    keys precede it (exclusive scans over chunks).
+//  compact_kernel (one CTA per chunk and vote pack): each thread owns 16 consecutive keys.
+//    SWAR byte arithmetic tests the four packed scores of a key against the four heads'
+//    thresholds at once (two adds and masks); byte counters count keys above T and ties;
+//    two block-wide scans (four heads in 16-bit lanes of a 64-bit word) give every
+//    candidate its output position, and the ties each thread may keep follow from E.
 #include "common.cuh"
 #include "internal.hpp"
 
@@ -23,13 +26,16 @@ namespace pkv {
 
 namespace {
 
-constexpr int kThr = 256;
+constexpr int kThr = 256;                  // threshold kernel
+constexpr int kKeysPerThread = 16;         // compaction: keys per thread
+constexpr int kCThr = CHUNK / kKeysPerThread;  // compaction: one chunk per block
 
-// Block-wide exclusive scan of a 64-bit value (4 packed 16-bit counters; no lane overflows
-// because a block's total per counter is at most CHUNK = 8192). Returns the exclusive
-// prefix; *total receives the block total. All threads must call it.
+// Block-wide exclusive scan of a 64-bit value (4 packed 16-bit counters in the compaction,
+// none of which overflows because a block's total per counter is at most CHUNK = 8192).
+// Returns the exclusive prefix; *total receives the block total. All threads must call it.
+template <int NT>
 __device__ __forceinline__ uint64_t block_excl_scan_u64(uint64_t v, uint64_t* total,
-                                                        uint64_t* sh /* >= 9 entries */) {
+                                                        uint64_t* sh /* >= NT/32+1 */) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint64_t x = v;
 #pragma unroll
@@ -41,16 +47,16 @@ __device__ __forceinline__ uint64_t block_excl_scan_u64(uint64_t v, uint64_t* to
     __syncthreads();
     if (threadIdx.x == 0) {
         uint64_t run = 0;
-        for (int w = 0; w < kThr / 32; ++w) {
+        for (int w = 0; w < NT / 32; ++w) {
             const uint64_t t = sh[w];
             sh[w] = run;
             run += t;
         }
-        sh[kThr / 32] = run;
+        sh[NT / 32] = run;
     }
     __syncthreads();
     const uint64_t res = sh[warp] + x - v;
-    *total = sh[kThr / 32];
+    *total = sh[NT / 32];
     __syncthreads();
     return res;
 }
@@ -58,64 +64,97 @@ __device__ __forceinline__ uint64_t block_excl_scan_u64(uint64_t v, uint64_t* to
 __global__ void __launch_bounds__(kThr)
 threshold_kernel(const uint32_t* __restrict__ hist, int group, int packs, int64_t nchunks,
                  int64_t C, int32_t* __restrict__ thr, int32_t* __restrict__ cbase) {
-    __shared__ uint32_t part[4][NBINS];
-    __shared__ uint32_t tot[NBINS];
+    __shared__ uint32_t part[kThr / 32][NBINS];
     __shared__ int32_t sT, sE;
     __shared__ uint64_t scan_sh[kThr / 32 + 1];
+    __shared__ uint64_t cnt[kThr];
 
     const int head = blockIdx.x;
     const int unit = head / group, g = head % group;
     const int64_t up = static_cast<int64_t>(unit) * packs + g / PACK;
     const int h = g % PACK;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t* hb = hist + up * nchunks * (PACK * NBINS) + h * NBINS;
 
-    {
-        const int bin = threadIdx.x & (NBINS - 1), p = threadIdx.x / NBINS;
-        uint32_t s = 0;
-        for (int64_t c = p; c < nchunks; c += 4) s += hb[c * (PACK * NBINS) + bin];
-        part[p][bin] = s;
+    // total histogram: warp w sums chunks w, w + 8, ...; lane l owns bins l and l + 32
+    uint32_t a = 0, b = 0;
+    for (int64_t c = warp; c < nchunks; c += kThr / 32) {
+        a += hb[c * (PACK * NBINS) + lane];
+        b += hb[c * (PACK * NBINS) + lane + 32];
     }
+    part[warp][lane] = a;
+    part[warp][lane + 32] = b;
     __syncthreads();
-    if (threadIdx.x < NBINS)
-        tot[threadIdx.x] = part[0][threadIdx.x] + part[1][threadIdx.x] + part[2][threadIdx.x] +
-                           part[3][threadIdx.x];
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int64_t cum = 0;
-        int T = 0;
-        for (int t = NBINS - 1; t >= 0; --t) {
-            if (cum + tot[t] >= C) { T = t; break; }
-            cum += tot[t];
+    if (warp == 0) {
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int w = 0; w < kThr / 32; ++w) { lo += part[w][lane]; hi += part[w][lane + 32]; }
+        // count of scores >= t for t = lane and lane + 32 (suffix sums over the 64 bins)
+        uint32_t shi = hi;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_down_sync(0xffffffffu, shi, o);
+            if (lane + o < 32) shi += y;
         }
-        sT = T;
-        sE = static_cast<int32_t>(C - cum);
-        thr[head * 4 + 0] = T;
-        thr[head * 4 + 1] = sE;
-        thr[head * 4 + 2] = static_cast<int32_t>(C);
-        thr[head * 4 + 3] = static_cast<int32_t>(cum);
+        const uint32_t tot_hi = __shfl_sync(0xffffffffu, shi, 0);
+        uint32_t slo = lo;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_down_sync(0xffffffffu, slo, o);
+            if (lane + o < 32) slo += y;
+        }
+        slo += tot_hi;
+        // T = the largest t with #{score >= t} >= C
+        const uint32_t mhi = __ballot_sync(0xffffffffu, shi >= C);
+        const uint32_t mlo = __ballot_sync(0xffffffffu, slo >= C);
+        int T;
+        uint32_t ge_T, cnt_T;
+        if (mhi) {
+            T = 31 - __clz(mhi) + 32;
+            ge_T = __shfl_sync(0xffffffffu, shi, T - 32);
+            cnt_T = __shfl_sync(0xffffffffu, hi, T - 32);
+        } else {
+            T = 31 - __clz(mlo);
+            ge_T = __shfl_sync(0xffffffffu, slo, T);
+            cnt_T = __shfl_sync(0xffffffffu, lo, T);
+        }
+        if (lane == 0) {
+            const int64_t above = static_cast<int64_t>(ge_T) - cnt_T;  // #{score > T}
+            sT = T;
+            sE = static_cast<int32_t>(C - above);
+            thr[head * 4 + 0] = T;
+            thr[head * 4 + 1] = sE;
+            thr[head * 4 + 2] = static_cast<int32_t>(C);
+            thr[head * 4 + 3] = static_cast<int32_t>(above);
+        }
     }
     __syncthreads();
     const int T = sT;
     const int64_t E = sE;
+    // per chunk: candidates above T and ties at T, then exclusive scans over chunks
     uint64_t run_gt = 0, run_eq = 0;
     for (int64_t base = 0; base < nchunks; base += kThr) {
-        const int64_t c = base + threadIdx.x;
-        uint32_t gt = 0, eq = 0;
-        if (c < nchunks) {
-            const uint32_t* hc = hb + c * (PACK * NBINS);
-            for (int t = T + 1; t < NBINS; ++t) gt += hc[t];
-            eq = hc[T];
+        for (int i = warp; i < kThr; i += kThr / 32) {
+            const int64_t c = base + i;
+            uint32_t gt = 0, eq = 0;
+            if (c < nchunks) {
+                const uint32_t* hc = hb + c * (PACK * NBINS);
+                const uint32_t x = hc[lane], y = hc[lane + 32];
+                gt = __reduce_add_sync(0xffffffffu, (lane > T ? x : 0u) + (lane + 32 > T ? y : 0u));
+                eq = __shfl_sync(0xffffffffu, T < 32 ? x : y, T & 31);
+            }
+            if (lane == 0) cnt[i] = (static_cast<uint64_t>(eq) << 32) | gt;
         }
-        // two 32-bit counters packed in one 64-bit scan word (totals <= 2^31)
+        __syncthreads();
+        const int64_t c = base + threadIdx.x;
         uint64_t total;
-        const uint64_t pre = block_excl_scan_u64((static_cast<uint64_t>(eq) << 32) | gt, &total,
-                                                 scan_sh);
+        const uint64_t mine = cnt[threadIdx.x];
+        const uint64_t pre = block_excl_scan_u64<kThr>(mine, &total, scan_sh);
         if (c < nchunks) {
             const int64_t gt_before = run_gt + (pre & 0xffffffffu);
             const int64_t eq_before = run_eq + (pre >> 32);
-            const int64_t sel_before = gt_before + min(eq_before, E);
             cbase[(static_cast<int64_t>(head) * nchunks + c) * 2 + 0] =
-                static_cast<int32_t>(sel_before);
+                static_cast<int32_t>(gt_before + min64(eq_before, E));
             cbase[(static_cast<int64_t>(head) * nchunks + c) * 2 + 1] =
                 static_cast<int32_t>(eq_before);
         }
@@ -124,84 +163,103 @@ threshold_kernel(const uint32_t* __restrict__ hist, int group, int packs, int64_
     }
 }
 
-__global__ void __launch_bounds__(kThr)
+// Byte b of the result is 1 when byte b of x is non-zero (bytes <= 0x80).
+__device__ __forceinline__ uint32_t nonzero_bytes(uint32_t x) {
+    return ((x + 0x7F7F7F7Fu) >> 7) & 0x01010101u;
+}
+
+// Spreads 4 byte counters into 4 16-bit lanes of a 64-bit word.
+__device__ __forceinline__ uint64_t widen(uint32_t x) {
+    return static_cast<uint64_t>(x & 0xffu) | (static_cast<uint64_t>((x >> 8) & 0xffu) << 16) |
+           (static_cast<uint64_t>((x >> 16) & 0xffu) << 32) |
+           (static_cast<uint64_t>(x >> 24) << 48);
+}
+
+__global__ void __launch_bounds__(kCThr, 2)
 compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ thr,
                const int32_t* __restrict__ cbase, int32_t* __restrict__ cand, int64_t n,
                int64_t cap_pad, int group, int packs, int64_t nchunks, int64_t cmax,
                int* status) {
-    __shared__ uint64_t scan_sh[kThr / 32 + 1];
+    __shared__ uint64_t scan_sh[kCThr / 32 + 1];
     const int64_t c = blockIdx.x;
     const int64_t up = blockIdx.y;
     const int unit = static_cast<int>(up / packs), p = static_cast<int>(up % packs);
     const int hp = min(PACK, group - p * PACK);
-    const int64_t k0 = c * CHUNK, k1 = min(n, k0 + CHUNK);
-    const int64_t my0 = k0 + static_cast<int64_t>(threadIdx.x) * 32;
+    const int64_t k0 = c * CHUNK, k1 = min64(n, k0 + CHUNK);
+    const int64_t my0 = k0 + static_cast<int64_t>(threadIdx.x) * kKeysPerThread;
+    const int nvalid = static_cast<int>(max64(0, min64(kKeysPerThread, k1 - my0)));
 
-    int T[PACK], E[PACK], head[PACK], sel_base[PACK], eq_base[PACK];
+    // Per-head thresholds packed one per byte. A head outside the pack gets T = 127, which
+    // no score (< 64) reaches. Byte h of (s + gt_add) has bit 7 set iff score_h > T_h, and
+    // of (s + ge_add) iff score_h >= T_h; bytes never carry (score + 128 <= 191).
+    uint32_t gt_add = 0, ge_add = 0;
 #pragma unroll
     for (int h = 0; h < PACK; ++h) {
-        head[h] = unit * group + p * PACK + min(h, hp - 1);
-        T[h] = thr[head[h] * 4 + 0];
-        E[h] = thr[head[h] * 4 + 1];
-        sel_base[h] = cbase[(static_cast<int64_t>(head[h]) * nchunks + c) * 2 + 0];
-        eq_base[h] = cbase[(static_cast<int64_t>(head[h]) * nchunks + c) * 2 + 1];
+        const int T = h < hp ? thr[(unit * group + p * PACK + h) * 4 + 0] : 127;
+        gt_add |= static_cast<uint32_t>(127 - T) << (8 * h);
+        ge_add |= static_cast<uint32_t>(128 - T) << (8 * h);
     }
 
-    uint32_t s[32];
+    uint32_t s[kKeysPerThread];
     const uint32_t* src = scores + up * cap_pad + my0;
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-        if (my0 + j < k1) {
+    for (int j = 0; j < kKeysPerThread; j += 4) {
+        if (j < nvalid) {
             const uint4 v = *reinterpret_cast<const uint4*>(src + j);
             s[j] = v.x; s[j + 1] = v.y; s[j + 2] = v.z; s[j + 3] = v.w;
         } else {
             s[j] = s[j + 1] = s[j + 2] = s[j + 3] = 0;
         }
     }
-    const int nvalid = static_cast<int>(max64(0, min64(32, k1 - my0)));
-
-    uint32_t gt[PACK], eq[PACK];
-    uint64_t eq_pack = 0;
+    // byte counters per head: keys above T and keys equal to T among this thread's keys
+    uint32_t gcnt = 0, ecnt = 0;
 #pragma unroll
-    for (int h = 0; h < PACK; ++h) {
-        gt[h] = eq[h] = 0;
-        if (h < hp) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int sh = (s[j] >> (8 * h)) & 0xff;
-                gt[h] += (j < nvalid && sh > T[h]) ? 1u : 0u;
-                eq[h] += (j < nvalid && sh == T[h]) ? 1u : 0u;
-            }
-        }
-        eq_pack |= static_cast<uint64_t>(eq[h]) << (16 * h);
+    for (int j = 0; j < kKeysPerThread; ++j) {
+        const uint32_t m = j < nvalid ? 0x01010101u : 0u;
+        const uint32_t g = ((s[j] + gt_add) >> 7) & m;
+        const uint32_t ge = ((s[j] + ge_add) >> 7) & m;
+        gcnt += g;
+        ecnt += ge ^ g;
     }
     uint64_t tot;
-    const uint64_t eq_pre = block_excl_scan_u64(eq_pack, &tot, scan_sh);
-    uint32_t take_eq[PACK];
-    uint64_t sel_pack = 0;
-#pragma unroll
-    for (int h = 0; h < PACK; ++h) {
-        const int64_t before = eq_base[h] + static_cast<int64_t>((eq_pre >> (16 * h)) & 0xffff);
-        const int64_t room = max64(0, E[h] - before);
-        take_eq[h] = static_cast<uint32_t>(min64(room, eq[h]));
-        sel_pack |= static_cast<uint64_t>(gt[h] + take_eq[h]) << (16 * h);
-    }
-    const uint64_t sel_pre = block_excl_scan_u64(sel_pack, &tot, scan_sh);
+    const uint64_t eq_pre = block_excl_scan_u64<kCThr>(widen(ecnt), &tot, scan_sh);
+    uint32_t take = 0;  // ties this thread keeps, per head (one byte each)
 #pragma unroll
     for (int h = 0; h < PACK; ++h) {
         if (h >= hp) continue;
-        int64_t pos = sel_base[h] + static_cast<int64_t>((sel_pre >> (16 * h)) & 0xffff);
-        uint32_t eq_left = take_eq[h];
-        int32_t* out = cand + static_cast<int64_t>(head[h]) * cmax;
+        const int head = unit * group + p * PACK + h;
+        const int64_t before = cbase[(static_cast<int64_t>(head) * nchunks + c) * 2 + 1] +
+                               static_cast<int64_t>((eq_pre >> (16 * h)) & 0xffff);
+        const int64_t room = max64(0, thr[head * 4 + 1] - before);
+        take |= static_cast<uint32_t>(min64(room, (ecnt >> (8 * h)) & 0xffu)) << (8 * h);
+    }
+    const uint64_t sel_pre = block_excl_scan_u64<kCThr>(widen(gcnt + take), &tot, scan_sh);
+    uint32_t pos[PACK];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int sh = (s[j] >> (8 * h)) & 0xff;
-            bool sel = j < nvalid && sh > T[h];
-            if (j < nvalid && sh == T[h] && eq_left > 0) { sel = true; --eq_left; }
-            if (sel) {
-                if (pos < thr[head[h] * 4 + 2]) out[pos] = static_cast<int32_t>(my0 + j);
-                else atomicExch(status, ST_BADINDEX);
-                ++pos;
+    for (int h = 0; h < PACK; ++h) {
+        const int head = unit * group + p * PACK + min(h, hp - 1);
+        pos[h] = static_cast<uint32_t>(cbase[(static_cast<int64_t>(head) * nchunks + c) * 2]) +
+                 static_cast<uint32_t>((sel_pre >> (16 * h)) & 0xffff);
+    }
+#pragma unroll
+    for (int j = 0; j < kKeysPerThread; ++j) {
+        const uint32_t m = j < nvalid ? 0x01010101u : 0u;
+        const uint32_t g = ((s[j] + gt_add) >> 7) & m;
+        const uint32_t e = (((s[j] + ge_add) >> 7) & m) ^ g;
+        const uint32_t t = e & nonzero_bytes(take);
+        take -= t;
+        const uint32_t sel = g | t;
+        if (sel) {
+#pragma unroll
+            for (int h = 0; h < PACK; ++h) {
+                if ((sel >> (8 * h)) & 1u) {
+                    const int head = unit * group + p * PACK + h;
+                    if (pos[h] < static_cast<uint32_t>(thr[head * 4 + 2]))
+                        cand[head * cmax + pos[h]] = static_cast<int32_t>(my0 + j);
+                    else
+                        atomicExch(status, ST_BADINDEX);
+                    ++pos[h];
+                }
             }
         }
     }
@@ -220,7 +278,7 @@ cudaError_t launch_threshold(const pariskv_index* ix, int64_t C, cudaStream_t st
 cudaError_t launch_compact(const pariskv_index* ix, cudaStream_t st) {
     const int64_t nchunks = ceil_div(ix->n, CHUNK);
     dim3 grid(static_cast<unsigned>(nchunks), static_cast<unsigned>(ix->units * ix->packs));
-    compact_kernel<<<grid, kThr, 0, st>>>(ix->scores, ix->thr, ix->cbase, ix->cand, ix->n,
+    compact_kernel<<<grid, kCThr, 0, st>>>(ix->scores, ix->thr, ix->cbase, ix->cand, ix->n,
                                           ix->cap_pad, ix->cfg.group, ix->packs, nchunks,
                                           ix->cmax, ix->status);
     return cudaGetLastError();

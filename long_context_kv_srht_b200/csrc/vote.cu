@@ -39,11 +39,18 @@ constexpr int kStageKeys = 1024;
 constexpr int kStageBytes = kStageKeys * 16;
 constexpr int kStages = 4;
 constexpr int kTableBytes = 256 * 256;
-constexpr int kSmemBytes = kTableBytes + kStages * kStageBytes + 2 * kStages * 8 + 1024;
+constexpr int kSmemBytes = kTableBytes + kStages * kStageBytes + 2 * kStages * 8;
 static_assert(CHUNK % kStageKeys == 0, "chunks hold whole stages");
 
 __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" :: "r"(kConsumerWarps * 32) : "memory");
+}
+
+__device__ __forceinline__ uint32_t tab_ld(const uint8_t* tab, uint32_t off) {
+    return *reinterpret_cast<const uint32_t*>(tab + off);
+}
+__device__ __forceinline__ void tab_inc(uint8_t* tab, uint32_t off) {
+    atomicAdd(reinterpret_cast<uint32_t*>(tab + off), 1u);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -51,12 +58,13 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
             uint32_t* __restrict__ scores, uint32_t* __restrict__ hist, int64_t n,
             int64_t cap_pad, int packs, int group, int64_t nchunks, int64_t items,
             int* status) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // 1024-byte aligned base (the table rows must not straddle the alignment assumptions)
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const uint32_t tab = smem_addr(smem);
-    const uint32_t ring = tab + kTableBytes;
+    // Shared memory: [table + histograms: 256 rows x 256 B][ring of kStages id tiles][bars].
+    // Only 16-byte alignment is needed (bulk-copy destinations, 16-byte id loads); a row
+    // start need not sit on bank 0 because every row keeps the same bank permutation.
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint8_t* tab = smem;
+    const uint8_t* ringp = smem + kTableBytes;
+    const uint32_t ring = smem_addr(ringp);
     const uint32_t full_bar = ring + kStages * kStageBytes;
     const uint32_t empty_bar = full_bar + kStages * 8;
 
@@ -80,7 +88,7 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
             for (int64_t item = i0; item < i1; ++item) {
                 const int64_t up = item / nchunks, c = item % nchunks;
                 const int64_t unit = up / packs;
-                const int64_t k0 = c * CHUNK, k1 = min(n, k0 + CHUNK);
+                const int64_t k0 = c * CHUNK, k1 = min64(n, k0 + CHUNK);
                 for (int64_t s0 = k0; s0 < k1; s0 += kStageKeys, ++it) {
                     const int slot = it % kStages;
                     if (it >= kStages)
@@ -97,14 +105,15 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
     }
 
     // ---------------------------------------------------------------------- consumers
+    // Per-lane address parts: at step t lane L reads subspace (t + L) mod 16 (see the
+    // encoder's byte rotation), whose copy (L >> 4) owns bank column 2 * subspace + copy.
     uint32_t col[16];
 #pragma unroll
     for (int t = 0; t < 16; ++t) col[t] = 4u * (2u * ((t + lane) & 15) + (lane >> 4));
     const uint32_t hcol = 128u + 4u * lane;
 
-    // zero the histogram half of every row
     for (int r = warp; r < 256; r += kConsumerWarps)
-        asm volatile("st.shared.u32 [%0], %1;" :: "r"(tab + r * 256 + hcol), "r"(0u) : "memory");
+        *reinterpret_cast<uint32_t*>(tab + r * 256 + hcol) = 0u;
 
     int64_t cur_up = -1;
     uint32_t it = 0;
@@ -113,39 +122,43 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
         const int hp = min(PACK, group - static_cast<int>(up % packs) * PACK);
         if (up != cur_up) {
             consumer_sync();
-            // table: column 2b + k of row c holds W_b[c] (both copies k = 0, 1)
+            // row c, column 2b + k holds W_b[c] (copies k = 0, 1)
             const uint32_t* lsrc = lut + up * (NB * NC);
             const int b = lane >> 1;
-            for (int r = warp; r < NC; r += kConsumerWarps) {
-                const uint32_t v = __ldg(lsrc + b * NC + r);
-                asm volatile("st.shared.u32 [%0], %1;" :: "r"(tab + r * 256 + 4 * lane), "r"(v)
-                             : "memory");
-            }
+            for (int r = warp; r < NC; r += kConsumerWarps)
+                *reinterpret_cast<uint32_t*>(tab + r * 256 + 4 * lane) = __ldg(lsrc + b * NC + r);
             consumer_sync();
             cur_up = up;
         }
-        const int64_t k0 = c * CHUNK, k1 = min(n, k0 + CHUNK);
-        uint32_t* sc_out = scores + up * cap_pad;
+        const int64_t k0 = c * CHUNK, k1 = min64(n, k0 + CHUNK);
         for (int64_t s0 = k0; s0 < k1; s0 += kStageKeys, ++it) {
             const int slot = it % kStages;
             mbar_wait(full_bar + 8 * slot, (it / kStages) & 1, status);
-            const int ntiles = static_cast<int>(ceil_div(min64(kStageKeys, k1 - s0), 32));
-            const uint32_t sbase = ring + slot * kStageBytes + lane * 16;
-            for (int tile = warp; tile < ntiles; tile += kConsumerWarps) {
-                const uint4 idv = lds_u128(sbase + tile * 512);
+            const int nkeys = static_cast<int>(min64(kStageKeys, k1 - s0));
+            const uint8_t* stage = ringp + slot * kStageBytes + lane * 16;
+            uint32_t* sc_out = scores + up * cap_pad + s0;
+            for (int tile = warp; tile * 32 < nkeys; tile += kConsumerWarps) {
+                const uint4 idv = *reinterpret_cast<const uint4*>(stage + tile * 512);
                 const uint32_t wd[4] = {idv.x, idv.y, idv.z, idv.w};
+                uint32_t v[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t)
+                    v[t] = tab_ld(tab, prmt(wd[t >> 2], col[t], 0x5504u | ((t & 3u) << 4)));
                 uint32_t acc = 0;
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const uint32_t a = prmt(wd[t >> 2], col[t], 0x5504u | ((t & 3u) << 4));
-                    acc += lds_u32(tab + a);
-                }
-                const int64_t key = s0 + tile * 32 + lane;
-                if (key < k1) {
-                    sc_out[key] = acc;
+                for (int t = 0; t < 16; ++t) acc += v[t];
+                const int kk = tile * 32 + lane;
+                if (kk < nkeys) {
+                    sc_out[kk] = acc;
                     const uint32_t sc = acc + 0xC0804000u;  // byte h -> 64 h + score_h
-                    for (int h = 0; h < hp; ++h)
-                        red_shared_add(tab + prmt(sc, hcol, 0x5504u | (static_cast<uint32_t>(h) << 4)), 1u);
+                    if (hp == PACK) {
+#pragma unroll
+                        for (int h = 0; h < PACK; ++h)
+                            tab_inc(tab, prmt(sc, hcol, 0x5504u | (static_cast<uint32_t>(h) << 4)));
+                    } else {
+                        for (int h = 0; h < hp; ++h)
+                            tab_inc(tab, prmt(sc, hcol, 0x5504u | (static_cast<uint32_t>(h) << 4)));
+                    }
                 }
             }
             __syncwarp();
@@ -155,10 +168,9 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
         consumer_sync();
         uint32_t* hout = hist + (up * nchunks + c) * (PACK * NBINS);
         for (int r = warp; r < PACK * NBINS; r += kConsumerWarps) {
-            const uint32_t a = tab + r * 256 + hcol;
-            const uint32_t v = lds_u32(a);
-            const uint32_t tot = __reduce_add_sync(0xffffffffu, v);
-            asm volatile("st.shared.u32 [%0], %1;" :: "r"(a), "r"(0u) : "memory");
+            uint32_t* a = reinterpret_cast<uint32_t*>(tab + r * 256 + hcol);
+            const uint32_t tot = __reduce_add_sync(0xffffffffu, *a);
+            *a = 0u;
             if (lane == 0) hout[r] = tot;
         }
         consumer_sync();
