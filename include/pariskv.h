@@ -139,6 +139,29 @@ PARISKV_API pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, cons
                                                  float scale, void* out, int32_t out_dtype,
                                                  void* stream);
 
+/* Allocation-free variant of pariskv_sparse_attend (an addition of this library; the
+ * ParisKV pages have no counterpart). Same arguments, layouts and results (up to the
+ * summation order of the split-K partials), but the call never allocates: the partials live
+ * in a fixed 4 MiB device array inside the library. It is meant for callers that may not
+ * touch a device allocator on the decode path: a serving runtime whose memory manager
+ * reserves all of HBM up front, a process where stream-ordered memory pools are unavailable
+ * or disabled, or a latency-critical loop where an allocation could block.
+ *  - The first call on each device looks the array's device address up (once, with that
+ *    device current); make that first call before capturing any CUDA graph.
+ *  - Every device that loads the library keeps the array until the process exits.
+ *  - All calls on a device share the array: calls that can overlap on the GPU (different
+ *    streams without ordering) race and must be serialised by the caller. Nothing in it has
+ *    to start at zero; each call overwrites what it reads.
+ *  - batch * num_kv_heads * group may not exceed 7943 (one split per head); larger
+ *    requests are rejected with PARISKV_EINVAL before anything is enqueued.
+ * Errors: EINVAL, ECUDA. */
+PARISKV_API pariskv_status pariskv_sparse_attend_noalloc(const pariskv_config* cfg,
+                                                         const void* q, const void* K,
+                                                         const void* V, int64_t ld_tok,
+                                                         int64_t n, const int32_t* topk_idx,
+                                                         int32_t k, float scale, void* out,
+                                                         int32_t out_dtype, void* stream);
+
 /* Waits for the index's stream work and reports any asynchronous error or expired wait. */
 PARISKV_API pariskv_status pariskv_sync(pariskv_index* index, void* stream);
 

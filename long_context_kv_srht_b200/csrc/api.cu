@@ -355,6 +355,48 @@ pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, c
     return PARISKV_OK;
 }
 
+pariskv_status pariskv_sparse_attend_noalloc(const pariskv_config* cfg, const void* q,
+                                             const void* K, const void* V, int64_t ld_tok,
+                                             int64_t n, const int32_t* topk_idx, int32_t k,
+                                             float scale, void* out, int32_t out_dtype,
+                                             void* stream) {
+    pariskv_status s = check_config(cfg);
+    if (s != PARISKV_OK) return s;
+    const size_t al = cfg->dtype == PARISKV_BF16 ? 8 : 16;
+    if (k < 1 || k > n) return fail(PARISKV_EINVAL, "k=%d not in [1, n=%lld]", k,
+                                    static_cast<long long>(n));
+    if (ld_tok < n) return fail(PARISKV_EINVAL, "ld_tok < n");
+    if ((s = check_dev_ptr(q, al, "q")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(K, al, "K")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(V, al, "V")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(topk_idx, 4, "topk_idx")) != PARISKV_OK) return s;
+    if (out_dtype != PARISKV_F32 && out_dtype != PARISKV_BF16)
+        return fail(PARISKV_EINVAL, "out_dtype %d unknown", out_dtype);
+    if ((s = check_dev_ptr(out, out_dtype == PARISKV_BF16 ? 8 : 16, "out")) != PARISKV_OK)
+        return s;
+    if (!(scale == scale)) return fail(PARISKV_EINVAL, "scale is NaN");
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int heads = cfg->batch * cfg->num_kv_heads * cfg->group;
+    // the split count is capped so that the partials fit the fixed workspace
+    const size_t per_split = attend_workspace_floats(heads, 1);
+    const int fit = static_cast<int>(kAttendScratchFloats / per_split);
+    if (fit < 1)
+        return fail(PARISKV_EINVAL, "%d query heads exceed the fixed attention workspace "
+                    "(at most %zu heads)", heads, kAttendScratchFloats / attend_workspace_floats(1, 1));
+    const int nsplit = min(attend_splits(heads, k, sms), fit);
+    float* work = nullptr;
+    cudaError_t e = attend_static_scratch(&work);
+    if (e != cudaSuccess) return cuda_fail(e, "fixed attention workspace lookup");
+    g_launches = 0;
+    e = launch_attend(cfg, q, K, V, ld_tok, n, topk_idx, k, scale, out, out_dtype, work, nsplit,
+                      static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    g_launches = 2;
+    return PARISKV_OK;
+}
+
 pariskv_status pariskv_sync(pariskv_index* index, void* stream) {
     pariskv_status s = check_index(index);
     if (s != PARISKV_OK) return s;

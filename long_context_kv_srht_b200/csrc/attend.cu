@@ -13,12 +13,16 @@
 // for K/V in host memory, where a read crosses PCIe). The warps are merged in shared memory
 // and the CTA writes (128 accumulators, max, denominator) to the workspace; a second kernel
 // merges the splits with the log-sum-exp rule and writes the output in the input dtype.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.hpp"
 
 namespace pkv {
 
 namespace {
+
+constexpr int kMaxScratchDevices = 64;
 
 constexpr int kAW = 4;            // warps per CTA
 constexpr int kUnroll = 4;        // tokens in flight per warp
@@ -136,7 +140,33 @@ attend_combine_kernel(const float* __restrict__ work, int nsplit, T* __restrict_
     store4<T>(out + static_cast<int64_t>(head) * D + 4 * lane, o);
 }
 
+// Fixed workspace of the allocation-free attention entry point: split-K partials in a
+// file-scope device array, so a call needs no allocator. Every device that loads the library
+// holds these 4 MiB until the process exits; all calls on a device share them.
+static __device__ __align__(256) float g_attend_scratch[kAttendScratchFloats];
+
+std::mutex g_scratch_mu;
+float* g_scratch_addr[kMaxScratchDevices] = {};
+
 }  // namespace
+
+cudaError_t attend_static_scratch(float** ptr) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        // the array's host-side name is only a stand-in; its device address comes from the
+        // runtime, once per device, with that device current
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_attend_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_addr[dev] = static_cast<float*>(p);
+    }
+    *ptr = g_scratch_addr[dev];
+    return cudaSuccess;
+}
 
 int attend_splits(int heads, int32_t k, int num_sms) {
     const int want = static_cast<int>(ceil_div(4LL * num_sms, heads));

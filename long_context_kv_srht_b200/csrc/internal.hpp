@@ -79,6 +79,10 @@ cudaError_t launch_attend(const pariskv_config* cfg, const void* q, const void* 
                           int32_t k, float scale, void* out, int32_t out_dtype, float* work,
                           int nsplit, cudaStream_t st);
 int attend_splits(int heads, int32_t k, int num_sms);
+// Allocation-free attention: floats in the fixed per-device workspace and its address on the
+// current device (looked up on first use per device).
+constexpr size_t kAttendScratchFloats = size_t(1) << 20;
+cudaError_t attend_static_scratch(float** ptr);
 size_t attend_workspace_floats(int heads, int nsplit);
 
 }  // namespace pkv

@@ -61,6 +61,8 @@ _SIGS = {
     "pariskv_search": (_S, [_P, _P, _I32, _P, _P, _P]),
     "pariskv_sparse_attend": (_S, [ctypes.POINTER(Config), _P, _P, _P, _I64, _I64, _P, _I32,
                                    ctypes.c_float, _P, _I32, _P]),
+    "pariskv_sparse_attend_noalloc": (_S, [ctypes.POINTER(Config), _P, _P, _P, _I64, _I64, _P,
+                                           _I32, ctypes.c_float, _P, _I32, _P]),
     "pariskv_sync": (_S, [_P, _P]),
     "pariskv_destroy": (_S, [_P]),
     "pariskv_size": (_I64, [_P]),
@@ -277,6 +279,22 @@ def sparse_attend(cfg: Config, q, K, V, topk_idx, k: int, scale: float, n: Optio
     _check(lib.pariskv_sparse_attend(ctypes.byref(cfg), q.data_ptr(), K.data_ptr(), V.data_ptr(),
                                      _slab(K), n, topk_idx.data_ptr(), k, float(scale),
                                      out.data_ptr(), od, _stream(stream)), "pariskv_sparse_attend")
+    return out
+
+
+def sparse_attend_noalloc(cfg: Config, q, K, V, topk_idx, k: int, scale: float,
+                          n: Optional[int] = None, out=None, out_dtype=None, stream=None):
+    """pariskv_sparse_attend_noalloc: the attention above with its partials in the library's
+    fixed device workspace instead of a per-call allocation (``out`` is still the caller's)."""
+    import torch
+    n = K.shape[-2] if n is None else n
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    od = BF16 if out.dtype == torch.bfloat16 else F32
+    _check(lib.pariskv_sparse_attend_noalloc(ctypes.byref(cfg), q.data_ptr(), K.data_ptr(),
+                                             V.data_ptr(), _slab(K), n, topk_idx.data_ptr(), k,
+                                             float(scale), out.data_ptr(), od, _stream(stream)),
+           "pariskv_sparse_attend_noalloc")
     return out
 
 
