@@ -549,7 +549,7 @@ pariskv_status pariskv_debug_export_index(pariskv_index* ix, uint8_t* ids, uint8
         for (int64_t i = 0; i < n; ++i) {
             const int64_t o = static_cast<int64_t>(u) * n + i;
             for (int b = 0; b < NB; ++b) {
-                if (ids) ids[o * NB + b] = hid[i * 16 + ((b - i) & 15)];
+                if (ids) ids[o * NB + b] = hid[i * 16 + ((b - (i >> 1)) & 15)];
                 const int64_t at = i * REC + 32 * (b >> 2) + 4 * (b & 3);
                 uint32_t w;
                 memcpy(&w, &hrec[at], 4);

@@ -20,9 +20,9 @@
 // the even lane writes the id byte, the 32-bit code word and the factor.
 //
 // HBM layout written here (per unit = (sequence, KV head), per key i):
-//  ids: 16 bytes at (unit * cap_pad + i) * 16; subspace b is stored at byte (b - i) mod 16.
-//       The rotation by the key index lets the vote scan read, at each step, 32 different
-//       subspaces across a warp and so hit 32 different shared-memory banks.
+//  ids: 16 bytes at (unit * cap_pad + i) * 16; subspace b is stored at byte (b - i / 2) mod
+//       16. The rotation lets the vote scan (one lane per pair of keys) read, at each step,
+//       32 different subspaces across a warp and so hit 32 different shared-memory banks.
 //  rec: 128 bytes at (unit * cap_pad + i) * 128, four 32-byte chunks; chunk p serves
 //       subspaces 4p..4p+3: its first 16 bytes are their code words (subspace b's 8 codes in
 //       one 32-bit word, dim j in nibble j, sign in bit 3 of the nibble), its last 16 bytes
@@ -109,7 +109,7 @@ encode_kernel(const T* __restrict__ src, const float* __restrict__ knorm_in, int
         const int b = lane >> 1;
         const int64_t key = pos0 + r;
         const int64_t slot = unit * cap_pad + key;
-        ids[slot * 16 + ((b - key) & 15)] = static_cast<uint8_t>(id);
+        ids[slot * 16 + ((b - (key >> 1)) & 15)] = static_cast<uint8_t>(id);
         uint8_t* rr = rec + slot * REC + 32 * (b >> 2) + 4 * (b & 3);
         *reinterpret_cast<uint32_t*>(rr) = code;
         *reinterpret_cast<float*>(rr + 16) = f;

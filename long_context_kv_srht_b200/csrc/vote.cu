@@ -9,16 +9,17 @@
 // streamed once per KV head and scored for all query heads of its GQA group at once.
 //
 // Design (sm_100a, HBM-bound):
-//  - A producer warp streams id tiles (1024 keys = 16 KB) with cp.async.bulk into a 4-stage
-//    shared-memory ring guarded by mbarriers (no multicast); 16 consumer warps score them.
-//  - Lane L of a consumer warp scores key (tile base + L). The 32-bit table entry packs the
-//    vote weights of up to four query heads (one byte each; a byte sum never exceeds 48), so
-//    one lookup per (key, subspace) serves the whole pack of heads.
+//  - Each lane scores two consecutive keys of a 64-key warp-tile, reading their 32 bytes of
+//    ids with one 256-bit non-allocating load; the next tile's ids are loaded while the
+//    current one is scored. Measured on B200, 256-bit loads stream at full HBM bandwidth;
+//    a cp.async.bulk ring refilled only once all warps had released a stage stayed far below.
+//  - The 32-bit table entry packs the vote weights of up to four query heads (one byte each;
+//    a byte sum never exceeds 48), so one lookup per (key, subspace) serves the whole pack.
 //  - Conflict-free lookups: the table holds two copies of every subspace's 256 entries, and
 //    subspace b / copy k owns shared-memory bank 2b + k (entry c of it at row c, 256-byte
-//    rows). Because the encoder stores subspace b of key i at byte (b - i) mod 16, at step t
-//    lane L reads subspace (t + L) mod 16 from byte t of its own 16 bytes; the 32 lanes then
-//    touch 32 distinct banks. One PRMT builds the address (row = id byte, column from a
+//    rows). Because the encoder stores subspace b of key i at byte (b - i / 2) mod 16, at
+//    step t lane L reads subspace (t + L) mod 16 from byte t of each of its keys; the 32 lanes
+//    then touch 32 distinct banks. One PRMT builds the address (row = id byte, column from a
 //    per-lane constant), one LDS reads the entry, one add accumulates.
 //  - Histograms of the packed scores (64 bins per query head) are built in the upper half of
 //    the same rows, one private counter column per lane (so no intra-warp conflicts), and
@@ -33,147 +34,146 @@ namespace pkv {
 
 namespace {
 
-constexpr int kConsumerWarps = 16;
-constexpr int kThreads = 32 * (kConsumerWarps + 1);
-constexpr int kStageKeys = 1024;
-constexpr int kStageBytes = kStageKeys * 16;
-constexpr int kStages = 4;
+constexpr int kWarps = 16;                   // two CTAs per SM: 32 scoring warps
+constexpr int kThreads = 32 * kWarps;
+constexpr int kTileKeys = 64;                // a warp-tile: two keys per lane
 constexpr int kTableBytes = 256 * 256;
-constexpr int kSmemBytes = kTableBytes + kStages * kStageBytes + 2 * kStages * 8;
-static_assert(CHUNK % kStageKeys == 0, "chunks hold whole stages");
-
-__device__ __forceinline__ void consumer_sync() {
-    asm volatile("bar.sync 1, %0;" :: "r"(kConsumerWarps * 32) : "memory");
-}
+constexpr int kSmemBytes = kTableBytes;
+constexpr int kTilesPerChunk = CHUNK / kTileKeys;
+static_assert(kTilesPerChunk % kWarps == 0, "whole tiles per warp and chunk");
 
 __device__ __forceinline__ uint32_t tab_ld(const uint8_t* tab, uint32_t off) {
     return *reinterpret_cast<const uint32_t*>(tab + off);
 }
-__device__ __forceinline__ void tab_inc(uint8_t* tab, uint32_t off) {
-    atomicAdd(reinterpret_cast<uint32_t*>(tab + off), 1u);
+
+__device__ __forceinline__ u32x8 ldg_ids(const uint8_t* p) { return ldg_stream_u256(p); }
+
+// Table entry of step t: byte0 <- column (byte t % 3 of colp[t / 3]), byte1 <- id byte t % 4,
+// bytes 2, 3 <- the zero top byte of colp[t / 3].
+template <int T>
+__device__ __forceinline__ uint32_t look(const uint8_t* tab, const uint32_t* wd,
+                                         const uint32_t* colp) {
+    constexpr uint32_t sel = 0x7700u | ((T & 3u) << 4) | (4u + (T % 3));
+    return tab_ld(tab, prmt_i<sel>(wd[T >> 2], colp[T / 3]));
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// Packed coarse score of one key: the sum of its 16 table entries (byte h = query head h).
+__device__ __forceinline__ uint32_t score_key(const uint8_t* tab, const uint32_t* wd,
+                                              const uint32_t* colp) {
+    const uint32_t v0 = look<0>(tab, wd, colp), v1 = look<1>(tab, wd, colp);
+    const uint32_t v2 = look<2>(tab, wd, colp), v3 = look<3>(tab, wd, colp);
+    const uint32_t v4 = look<4>(tab, wd, colp), v5 = look<5>(tab, wd, colp);
+    const uint32_t v6 = look<6>(tab, wd, colp), v7 = look<7>(tab, wd, colp);
+    const uint32_t v8 = look<8>(tab, wd, colp), v9 = look<9>(tab, wd, colp);
+    const uint32_t v10 = look<10>(tab, wd, colp), v11 = look<11>(tab, wd, colp);
+    const uint32_t v12 = look<12>(tab, wd, colp), v13 = look<13>(tab, wd, colp);
+    const uint32_t v14 = look<14>(tab, wd, colp), v15 = look<15>(tab, wd, colp);
+    const uint32_t a = v0 + v1 + v2, b = v3 + v4 + v5, c = v6 + v7 + v8, d = v9 + v10 + v11;
+    const uint32_t e = v12 + v13 + v14;
+    return (a + b + c) + (d + e + v15);
+}
+
+template <int H>
+__device__ __forceinline__ void hist_inc(uint8_t* tab, uint32_t sc, uint32_t hcol) {
+    atomicAdd(reinterpret_cast<uint32_t*>(tab + prmt_i<0x5504u | (H << 4)>(sc, hcol)), 1u);
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
 vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
             uint32_t* __restrict__ scores, uint32_t* __restrict__ hist, int64_t n,
             int64_t cap_pad, int packs, int group, int64_t nchunks, int64_t items,
             int* status) {
-    // Shared memory: [table + histograms: 256 rows x 256 B][ring of kStages id tiles][bars].
-    // Only 16-byte alignment is needed (bulk-copy destinations, 16-byte id loads); a row
-    // start need not sit on bank 0 because every row keeps the same bank permutation.
+    // Shared memory: table + histograms, 256 rows x 256 B (see the file comment).
     extern __shared__ __align__(16) uint8_t smem[];
     uint8_t* tab = smem;
-    const uint8_t* ringp = smem + kTableBytes;
-    const uint32_t ring = smem_addr(ringp);
-    const uint32_t full_bar = ring + kStages * kStageBytes;
-    const uint32_t empty_bar = full_bar + kStages * 8;
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t i0 = items * blockIdx.x / gridDim.x;
     const int64_t i1 = items * (blockIdx.x + 1) / gridDim.x;
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(full_bar + 8 * s, 1);
-            mbar_init(empty_bar + 8 * s, kConsumerWarps);
-        }
-        mbar_fence_init();
-    }
-    __syncthreads();
-
-    if (warp == kConsumerWarps) {
-        // ------------------------------------------------------------------ producer
-        if (lane == 0) {
-            uint32_t it = 0;
-            for (int64_t item = i0; item < i1; ++item) {
-                const int64_t up = item / nchunks, c = item % nchunks;
-                const int64_t unit = up / packs;
-                const int64_t k0 = c * CHUNK, k1 = min64(n, k0 + CHUNK);
-                for (int64_t s0 = k0; s0 < k1; s0 += kStageKeys, ++it) {
-                    const int slot = it % kStages;
-                    if (it >= kStages)
-                        mbar_wait(empty_bar + 8 * slot, ((it / kStages) + 1) & 1, status);
-                    const int64_t nk = round_up(min64(kStageKeys, k1 - s0), 32);
-                    const uint32_t bytes = static_cast<uint32_t>(nk * 16);
-                    mbar_arrive_expect_tx(full_bar + 8 * slot, bytes);
-                    bulk_g2s(ring + slot * kStageBytes, ids + (unit * cap_pad + s0) * 16, bytes,
-                             full_bar + 8 * slot);
-                }
-            }
-        }
-        return;
-    }
-
-    // ---------------------------------------------------------------------- consumers
-    // Per-lane address parts: at step t lane L reads subspace (t + L) mod 16 (see the
-    // encoder's byte rotation), whose copy (L >> 4) owns bank column 2 * subspace + copy.
-    uint32_t col[16];
+    // Per-lane address parts: at step t lane L reads subspace (t + L) mod 16 of both its keys
+    // (the encoder rotates key i's bytes by (i / 2) mod 16), whose copy (L >> 4) owns bank
+    // column 2 * subspace + copy. Three columns per register with a zero top byte, so one
+    // PRMT builds an address.
+    uint32_t colp[6];
 #pragma unroll
-    for (int t = 0; t < 16; ++t) col[t] = 4u * (2u * ((t + lane) & 15) + (lane >> 4));
+    for (int r = 0; r < 6; ++r) {
+        uint32_t w = 0;
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            const int t = 3 * r + j;
+            if (t < 16) w |= (4u * (2u * ((t + lane) & 15) + (lane >> 4))) << (8 * j);
+        }
+        colp[r] = w;
+    }
     const uint32_t hcol = 128u + 4u * lane;
-
-    for (int r = warp; r < 256; r += kConsumerWarps)
+    for (int r = warp; r < 256; r += kWarps)
         *reinterpret_cast<uint32_t*>(tab + r * 256 + hcol) = 0u;
 
+    // warp w scores tiles w, w + kWarps, ... of each chunk; the next tile's ids are loaded
+    // while the current tile is scored
+    auto tile_ptr = [&](int64_t item, int tl) -> const uint8_t* {
+        const int64_t up = item / nchunks, c = item % nchunks;
+        const int64_t unit = up / packs;
+        return ids + (unit * cap_pad + c * CHUNK + static_cast<int64_t>(tl) * kTileKeys) * 16 +
+               lane * 32;
+    };
     int64_t cur_up = -1;
-    uint32_t it = 0;
+    u32x8 nxt;
+    if (i0 < i1) nxt = ldg_ids(tile_ptr(i0, warp));
     for (int64_t item = i0; item < i1; ++item) {
         const int64_t up = item / nchunks, c = item % nchunks;
         const int hp = min(PACK, group - static_cast<int>(up % packs) * PACK);
         if (up != cur_up) {
-            consumer_sync();
+            __syncthreads();
             // row c, column 2b + k holds W_b[c] (copies k = 0, 1)
             const uint32_t* lsrc = lut + up * (NB * NC);
             const int b = lane >> 1;
-            for (int r = warp; r < NC; r += kConsumerWarps)
+            for (int r = warp; r < NC; r += kWarps)
                 *reinterpret_cast<uint32_t*>(tab + r * 256 + 4 * lane) = __ldg(lsrc + b * NC + r);
-            consumer_sync();
+            __syncthreads();
             cur_up = up;
         }
-        const int64_t k0 = c * CHUNK, k1 = min64(n, k0 + CHUNK);
-        for (int64_t s0 = k0; s0 < k1; s0 += kStageKeys, ++it) {
-            const int slot = it % kStages;
-            mbar_wait(full_bar + 8 * slot, (it / kStages) & 1, status);
-            const int nkeys = static_cast<int>(min64(kStageKeys, k1 - s0));
-            const uint8_t* stage = ringp + slot * kStageBytes + lane * 16;
-            uint32_t* sc_out = scores + up * cap_pad + s0;
-            for (int tile = warp; tile * 32 < nkeys; tile += kConsumerWarps) {
-                const uint4 idv = *reinterpret_cast<const uint4*>(stage + tile * 512);
-                const uint32_t wd[4] = {idv.x, idv.y, idv.z, idv.w};
-                uint32_t v[16];
+        const int64_t k0 = c * CHUNK;
+        const int nkeys = static_cast<int>(min64(n - k0, CHUNK));
+        uint32_t* sc_out = scores + up * cap_pad + k0;
+#pragma unroll 1
+        for (int tl = warp; tl < kTilesPerChunk; tl += kWarps) {
+            const u32x8 cur = nxt;
+            // prefetch: the next tile of this chunk, else this warp's first of the next item
+            // (tiles past the last key read padding inside the capacity, never beyond it)
+            if (tl + kWarps < kTilesPerChunk) nxt = ldg_ids(tile_ptr(item, tl + kWarps));
+            else if (item + 1 < i1) nxt = ldg_ids(tile_ptr(item + 1, warp));
+            if (tl * kTileKeys >= nkeys) continue;
+            uint32_t acc[2];
 #pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    v[t] = tab_ld(tab, prmt(wd[t >> 2], col[t], 0x5504u | ((t & 3u) << 4)));
-                uint32_t acc = 0;
+            for (int j = 0; j < 2; ++j) acc[j] = score_key(tab, cur.w + 4 * j, colp);
+            const int kk = tl * kTileKeys + 2 * lane;
+            if (kk + 1 < nkeys) {
+                *reinterpret_cast<uint2*>(sc_out + kk) = make_uint2(acc[0], acc[1]);
+            } else if (kk < nkeys) {
+                sc_out[kk] = acc[0];
+            }
 #pragma unroll
-                for (int t = 0; t < 16; ++t) acc += v[t];
-                const int kk = tile * 32 + lane;
-                if (kk < nkeys) {
-                    sc_out[kk] = acc;
-                    const uint32_t sc = acc + 0xC0804000u;  // byte h -> 64 h + score_h
-                    if (hp == PACK) {
-#pragma unroll
-                        for (int h = 0; h < PACK; ++h)
-                            tab_inc(tab, prmt(sc, hcol, 0x5504u | (static_cast<uint32_t>(h) << 4)));
-                    } else {
-                        for (int h = 0; h < hp; ++h)
-                            tab_inc(tab, prmt(sc, hcol, 0x5504u | (static_cast<uint32_t>(h) << 4)));
-                    }
+            for (int j = 0; j < 2; ++j) {
+                if (kk + j < nkeys) {
+                    const uint32_t sc = acc[j] + 0xC0804000u;  // byte h -> 64 h + score_h
+                    hist_inc<0>(tab, sc, hcol);
+                    if (hp > 1) hist_inc<1>(tab, sc, hcol);
+                    if (hp > 2) hist_inc<2>(tab, sc, hcol);
+                    if (hp > 3) hist_inc<3>(tab, sc, hcol);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty_bar + 8 * slot);
         }
         // flush this chunk's histograms: row 64 h + s, one counter per lane
-        consumer_sync();
+        __syncthreads();
         uint32_t* hout = hist + (up * nchunks + c) * (PACK * NBINS);
-        for (int r = warp; r < PACK * NBINS; r += kConsumerWarps) {
+        for (int r = warp; r < PACK * NBINS; r += kWarps) {
             uint32_t* a = reinterpret_cast<uint32_t*>(tab + r * 256 + hcol);
             const uint32_t tot = __reduce_add_sync(0xffffffffu, *a);
             *a = 0u;
             if (lane == 0) hout[r] = tot;
         }
-        consumer_sync();
+        __syncthreads();
     }
 }
 
@@ -194,7 +194,7 @@ cudaError_t launch_vote(const pariskv_index* ix, cudaStream_t st) {
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int grid = static_cast<int>(min64(items, sms));
+    const int grid = static_cast<int>(min64(items, 2LL * sms));
     vote_kernel<<<grid, kThreads, kSmemBytes, st>>>(ix->ids, ix->lut, ix->scores, ix->hist,
                                                    ix->n, ix->cap_pad, ix->packs,
                                                    ix->cfg.group, nchunks, items, ix->status);
