@@ -161,6 +161,7 @@ pariskv_status create_index(const pariskv_config* cfg, const int8_t* signs, cuda
 
 pariskv_status ensure_candidates(pariskv_index* ix, int64_t C) {
     if (C <= ix->cmax) return PARISKV_OK;
+    C = round_up(C, 32);  // every head's slice starts on a 128-byte boundary
     const int64_t heads = static_cast<int64_t>(ix->units) * ix->cfg.group;
     int32_t* c2 = nullptr;
     float* s2 = nullptr;
@@ -549,12 +550,20 @@ pariskv_status pariskv_debug_export_index(pariskv_index* ix, uint8_t* ids, uint8
         for (int64_t i = 0; i < n; ++i) {
             const int64_t o = static_cast<int64_t>(u) * n + i;
             for (int b = 0; b < NB; ++b) {
-                if (ids) ids[o * NB + b] = hid[i * 16 + ((b - (i >> 1)) & 15)];
+                const uint8_t id = hid[i * 16 + ((b - (i >> 1)) & 15)];
+                if (ids) ids[o * NB + b] = id;
                 const int64_t at = i * REC + 32 * (b >> 2) + 4 * (b & 3);
                 uint32_t w;
                 memcpy(&w, &hrec[at], 4);
+                // stored offset binary u = vt + 8; canonical code = sign << 3 | magnitude,
+                // the sign being bit j of the bucket id
                 if (codes)
-                    for (int j = 0; j < M; ++j) codes[o * D + b * M + j] = (w >> (4 * j)) & 15u;
+                    for (int j = 0; j < M; ++j) {
+                        const int u = static_cast<int>((w >> (4 * j)) & 15u);
+                        const int mag = u >= 8 ? u - 8 : 8 - u;
+                        codes[o * D + b * M + j] =
+                            static_cast<uint8_t>((((id >> j) & 1u) << 3) | static_cast<uint32_t>(mag));
+                    }
                 if (factors) memcpy(&factors[o * NB + b], &hrec[at + 16], 4);
             }
         }

@@ -25,8 +25,10 @@
 //       32 different subspaces across a warp and so hit 32 different shared-memory banks.
 //  rec: 128 bytes at (unit * cap_pad + i) * 128, four 32-byte chunks; chunk p serves
 //       subspaces 4p..4p+3: its first 16 bytes are their code words (subspace b's 8 codes in
-//       one 32-bit word, dim j in nibble j, sign in bit 3 of the nibble), its last 16 bytes
-//       their factors f_b. The rerank reads one chunk per lane with a single 32-byte load.
+//       one 32-bit word, dim j in nibble j), its last 16 bytes their factors f_b. A code is
+//       stored in offset binary, u = vt + 8 in [1, 15], which the rerank turns into fp32 with
+//       two integer operations. Nothing is lost: the code's sign bit is the sign of y_j, which
+//       is bit j of the bucket id (for a zero level it is only there).
 #include "common.cuh"
 #include "internal.hpp"
 #include "rotate.cuh"
@@ -58,8 +60,9 @@ __device__ __forceinline__ void encode_subspace(const float w[8], float knorm, u
             t = __fadd_rn(t, 0.5f);
             q = min(static_cast<int>(floorf(t)), 7);
         }
-        const uint32_t sgn = w[j] < 0.0f ? 1u : 0u;
-        code |= ((sgn << 3) | static_cast<uint32_t>(q)) << (4 * j);
+        const bool sgn = w[j] < 0.0f;
+        const int lv = sgn ? -q : q;                               // signed level vt
+        code |= static_cast<uint32_t>(lv + 8) << (4 * j);           // offset binary
         const float vt = sgn ? -static_cast<float>(q) : static_cast<float>(q);
         n2 = __fmaf_rn(w[j], w[j], n2);
         dot = __fmaf_rn(vt, w[j], dot);

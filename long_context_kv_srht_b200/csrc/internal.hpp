@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "pariskv.h"
 
 struct pariskv_index {
@@ -43,6 +45,20 @@ struct pariskv_index {
 };
 
 namespace pkv {
+
+// Raises a kernel's dynamic shared-memory limit on the current device, once per device
+// (devices 0..63 are remembered in `done`; others set the attribute on every call).
+template <typename Kern>
+cudaError_t raise_smem_limit(Kern kernel, int bytes, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
 
 // status helpers (defined in api.cu)
 pariskv_status fail(pariskv_status s, const char* fmt, ...);

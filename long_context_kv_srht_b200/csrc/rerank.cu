@@ -12,20 +12,19 @@
 // Memory: the candidates' 128-byte records sit at random places in a 1 GiB array, and HBM
 // only delivers its bandwidth with far more bytes in flight than registers can hold. So the
 // records are gathered with asynchronous global->shared copies (cp.async, 16 bytes per lane;
-// eight lanes move one record, so a warp instruction moves four whole records): the kernel
-// is persistent (two CTAs per SM), every warp owns a ring of kSlots stages of 16 records in
-// shared memory (128 KB per SM), and a stage is refilled as soon as it has been scored. The
-// candidate indices of the refill are loaded while the stage is scored. (Measured on B200:
-// one 128-byte cp.async.bulk per record was several times slower than this.)
+// eight lanes move one record, so one warp instruction moves four whole records): the kernel
+// is persistent (two CTAs per SM), every warp owns a ring of kSlots stages of 32 records, and
+// a stage is refilled as soon as it has been scored. Piece c of the record in stage row r is
+// stored at 16-byte position c ^ (r mod 8), so that eight lanes reading the same piece of
+// eight different records touch all 32 banks once.
 //
-// Scoring: four lanes cooperate on a record, and each group of four scores two records at
-// once so that their dependency chains interleave; lane p owns subspaces 4p..4p+3 (one 32-byte
-// chunk: 4 code words + 4 factors) and keeps its 32 rotated-query coordinates in registers
-// as fp32 pairs. Decoding is exact integer arithmetic: 8 sign-magnitude nibbles become offset
-// nibbles u = vt + 8 with five SWAR instructions, a PRMT places u in the mantissa of 2^23 and
-// one packed subtraction of 2^23 + 8 gives vt exactly as fp32. Two subspaces advance
-// together in Blackwell's packed fp32x2 FMA (each half an ordinary IEEE fp32 FMA); the S
-// chain then runs across the four lanes in order, lane p continuing lane p - 1's sum.
+// Scoring: one lane per record. The warp's current query head has its rotated query in
+// shared memory as (subspace 2t, subspace 2t + 1) fp32 pairs, read with broadcast loads; a
+// lane walks the 8 subspace pairs in order, two p chains advancing together in Blackwell's
+// packed fp32x2 FMA (each half an ordinary IEEE fp32 FMA), and extends its S chain after
+// every pair. Decoding is exact integer arithmetic: the stored offset-binary nibbles
+// u = vt + 8 are split into even and odd dims with two masks, a PRMT places u in the
+// mantissa of 2^23, and one packed subtraction of 2^23 + 8 gives vt exactly as fp32.
 #include "common.cuh"
 #include "internal.hpp"
 
@@ -35,16 +34,16 @@ namespace {
 
 constexpr int kWarps = 8;               // two persistent CTAs per SM; every warp gathers and scores
 constexpr int kThr = 32 * kWarps;
-constexpr int kSlots = 4;               // stages in flight per warp
-constexpr int kStageRecs = 16;          // records per stage: two per four-lane group
+constexpr int kSlots = 3;               // stages in flight per warp
+constexpr int kStageRecs = 32;          // records per stage: one per lane
 constexpr int kStageBytes = kStageRecs * REC;
-constexpr int kSmem = kWarps * kSlots * kStageBytes;
+constexpr int kQBytes = D * 4;          // one head's rotated query
+constexpr int kWarpBytes = kSlots * kStageBytes + kQBytes;
+constexpr int kSmem = kWarps * kWarpBytes;
+static_assert(kWarpBytes % 128 == 0, "warp areas stay 128-byte aligned");
 
-__device__ __forceinline__ uint32_t offset_nibbles(uint32_t w) {
-    const uint32_t s = (w >> 3) & 0x11111111u;       // sign bit of each nibble as 0/1
-    const uint32_t sm = s * 7u;                        // 7 in every negative nibble
-    const uint32_t x = (w & 0x77777777u) ^ sm;         // mag, or 7 - mag when negative
-    return x + (0x88888888u - sm);                     // + 8 (positive) or + 1 (negative)
+__device__ __forceinline__ uint32_t piece_at(int row, int c) {
+    return static_cast<uint32_t>(row * REC + ((c ^ (row & 7)) << 4));
 }
 
 template <int K>
@@ -55,31 +54,55 @@ __device__ __forceinline__ uint64_t level_pair(uint32_t xa, uint32_t xb) {
                 kOff);
 }
 
-// p chains of the subspace pair (a, b): codes wa, wb; q pairs q[j] = (q~_{a,j}, q~_{b,j}).
-__device__ __forceinline__ float2 pair_dots(uint32_t wa, uint32_t wb, const uint64_t q[8]) {
-    const uint32_t ua = offset_nibbles(wa), ub = offset_nibbles(wb);
-    const uint32_t ea = ua & 0x0F0F0F0Fu, oa = (ua >> 4) & 0x0F0F0F0Fu;   // dims 0, 2, 4, 6
-    const uint32_t eb = ub & 0x0F0F0F0Fu, ob = (ub >> 4) & 0x0F0F0F0Fu;   // dims 1, 3, 5, 7
+// p chains of the subspace pair (a, b) from their code words; qp holds the pairs
+// (q~_{a,j}, q~_{b,j}) for j = 0..7 in shared memory.
+__device__ __forceinline__ float2 pair_dots(uint32_t wa, uint32_t wb, const uint64_t* qp) {
+    const uint32_t ea = wa & 0x0F0F0F0Fu, oa = (wa >> 4) & 0x0F0F0F0Fu;  // dims 0,2,4,6 | 1,3,5,7
+    const uint32_t eb = wb & 0x0F0F0F0Fu, ob = (wb >> 4) & 0x0F0F0F0Fu;
+    const ulonglong2 q01 = reinterpret_cast<const ulonglong2*>(qp)[0];
+    const ulonglong2 q23 = reinterpret_cast<const ulonglong2*>(qp)[1];
+    const ulonglong2 q45 = reinterpret_cast<const ulonglong2*>(qp)[2];
+    const ulonglong2 q67 = reinterpret_cast<const ulonglong2*>(qp)[3];
     uint64_t p = pack2(0.0f, 0.0f);
-    p = fma2(level_pair<0>(ea, eb), q[0], p);
-    p = fma2(level_pair<0>(oa, ob), q[1], p);
-    p = fma2(level_pair<1>(ea, eb), q[2], p);
-    p = fma2(level_pair<1>(oa, ob), q[3], p);
-    p = fma2(level_pair<2>(ea, eb), q[4], p);
-    p = fma2(level_pair<2>(oa, ob), q[5], p);
-    p = fma2(level_pair<3>(ea, eb), q[6], p);
-    p = fma2(level_pair<3>(oa, ob), q[7], p);
+    p = fma2(level_pair<0>(ea, eb), q01.x, p);
+    p = fma2(level_pair<0>(oa, ob), q01.y, p);
+    p = fma2(level_pair<1>(ea, eb), q23.x, p);
+    p = fma2(level_pair<1>(oa, ob), q23.y, p);
+    p = fma2(level_pair<2>(ea, eb), q45.x, p);
+    p = fma2(level_pair<2>(oa, ob), q45.y, p);
+    p = fma2(level_pair<3>(ea, eb), q67.x, p);
+    p = fma2(level_pair<3>(oa, ob), q67.y, p);
     return unpack2(p);
 }
 
-__device__ __forceinline__ void load_q(const float* __restrict__ qt, int64_t head, int p,
-                                       uint64_t qa[8], uint64_t qb[8]) {
-    const float* qh = qt + head * D + 32 * p;
+// S of the record in stage row `row`; qp = the head's 64 query pairs (pair t at qp + 8 t).
+__device__ __forceinline__ float score_record(const uint8_t* st, int row, const uint64_t* qp) {
+    float S = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        qa[j] = pack2(qh[j], qh[8 + j]);
-        qb[j] = pack2(qh[16 + j], qh[24 + j]);
+    for (int c = 0; c < 4; ++c) {   // chunk c: subspaces 4c..4c+3
+        const uint4 cw = *reinterpret_cast<const uint4*>(st + piece_at(row, 2 * c));
+        const uint4 fw = *reinterpret_cast<const uint4*>(st + piece_at(row, 2 * c + 1));
+        const float2 pa = pair_dots(cw.x, cw.y, qp + 16 * c);
+        S = __fmaf_rn(__uint_as_float(fw.x), pa.x, S);
+        S = __fmaf_rn(__uint_as_float(fw.y), pa.y, S);
+        const float2 pb = pair_dots(cw.z, cw.w, qp + 16 * c + 8);
+        S = __fmaf_rn(__uint_as_float(fw.z), pb.x, S);
+        S = __fmaf_rn(__uint_as_float(fw.w), pb.y, S);
     }
+    return S;
+}
+
+// Stages head h's rotated query into the warp's pair table: entry 8 t + j holds
+// (q~[16 t + j], q~[16 t + 8 + j]).
+__device__ __forceinline__ void stage_query(const float* __restrict__ qt, int64_t h,
+                                            float2* qs, int lane) {
+    const float* qh = qt + h * D;
+#pragma unroll
+    for (int e = lane; e < 64; e += 32) {
+        const int t = e >> 3, j = e & 7;
+        qs[e] = make_float2(qh[16 * t + j], qh[16 * t + 8 + j]);
+    }
+    __syncwarp();
 }
 
 __global__ void __launch_bounds__(kThr, 2)
@@ -88,16 +111,16 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
               int64_t cap_pad, int64_t n, int group, int64_t total, int* status) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int p = lane & 3;            // part: subspaces 4p..4p+3
-    const int slot_rec = lane >> 2;    // four-lane group: scores records slot_rec, slot_rec + 8
-    uint8_t* ring = smem + warp * kSlots * kStageBytes;
+    uint8_t* ring = smem + warp * kWarpBytes;
+    float2* qs = reinterpret_cast<float2*>(ring + kSlots * kStageBytes);
+    const uint64_t* qp = reinterpret_cast<const uint64_t*>(qs);
 
     // this CTA's slice of the flattened (head, candidate) sequence, cut in 32-record stages;
     // the warp takes CTA stages warp, warp + kWarps, warp + 2 kWarps, ...
     const int64_t r0 = total * blockIdx.x / gridDim.x, r1 = total * (blockIdx.x + 1) / gridDim.x;
     const int64_t nstage = ceil_div(r1 - r0, kStageRecs);
 
-    // stage refill: lane l < 16 holds the record number of the stage's l-th record; for copy
+    // stage refill: lane l holds the record number of the stage's l-th record; for copy
     // instruction j, lanes 8g..8g+7 move the 8 16-byte pieces of record 4j + g
     auto issue = [&](int slot, int64_t ridx, bool valid) {
         uint8_t* dst0 = ring + slot * kStageBytes;
@@ -108,7 +131,7 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
             const int64_t ri = __shfl_sync(0xffffffffu, ridx, rr);
             const bool v = __shfl_sync(0xffffffffu, valid, rr);
             if (v) {
-                const uint32_t dst = smem_addr(dst0 + rr * REC + piece * 16);
+                const uint32_t dst = smem_addr(dst0 + piece_at(rr, piece));
                 const uint8_t* src = rec + ri * REC + piece * 16;
                 asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(src)
                              : "memory");
@@ -117,7 +140,7 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
     // (head, candidate) positions advance incrementally: one division at the start, then
-    // an add and at most one wrap per step when C >= 32 (several for tiny candidate sets)
+    // an add and at most one wrap per step when C >= 256 (several for small candidate sets)
     auto wrap = [&](int64_t& h, int64_t& c) {
         while (c >= C) { c -= C; ++h; }
     };
@@ -144,15 +167,14 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
     for (int g = 0; g < kSlots; ++g) {
         const int64_t cs = warp + static_cast<int64_t>(kWarps) * g;
         const int64_t rs = r0 + cs * kStageRecs;
-        bool valid = cs < nstage && lane < kStageRecs && rs + lane < r1;
+        bool valid = cs < nstage && rs + lane < r1;
         const int64_t ri = locate(ih, ic, valid);
         issue(g, ri, valid);
         ic += kStep;
         wrap(ih, ic);
     }
 
-    int64_t cur_head = -1;
-    uint64_t qa[8], qb[8];
+    int64_t staged = -1;   // head whose query is in qs
 #pragma unroll 1
     for (int64_t g = 0;; ++g) {
         const int64_t cs = warp + static_cast<int64_t>(kWarps) * g;
@@ -161,60 +183,36 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
         // indices of the stage that will refill this slot (their load overlaps the scoring)
         const int64_t cs_next = cs + static_cast<int64_t>(kWarps) * kSlots;
         const int64_t rs_next = r0 + cs_next * kStageRecs;
-        bool valid_next = cs_next < nstage && lane < kStageRecs && rs_next + lane < r1;
+        bool valid_next = cs_next < nstage && rs_next + lane < r1;
         const int64_t ri_next = locate(ih, ic, valid_next);
         ic += kStep;
         wrap(ih, ic);
+
+        // this lane's record: head and candidate position (the valid lanes are a prefix)
+        const int64_t rs = r0 + cs * kStageRecs;
+        const bool ok = rs + lane < r1;
+        int64_t head = hh, cc = hc + lane;
+        wrap(head, cc);
+        const int last = static_cast<int>(min64(31, r1 - rs - 1));
+        const int64_t hlast = __shfl_sync(0xffffffffu, head, last);
 
         // the oldest committed group is this stage's; each lane waits for its own pieces and
         // the warp barrier makes every lane's pieces visible
         asm volatile("cp.async.wait_group %0;" :: "n"(kSlots - 1) : "memory");
         __syncwarp();
         const uint8_t* st = ring + slot * kStageBytes;
-        const int64_t rs = r0 + cs * kStageRecs;
-        // group slot_rec scores records slot_rec and slot_rec + 8 of the stage together
-        bool ok[2];
-        int64_t head[2], cc[2];
-        uint4 w0[2], w1[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int rr = slot_rec + 8 * u;
-            ok[u] = rs + rr < r1;
-            head[u] = hh;
-            cc[u] = hc + rr;
-            wrap(head[u], cc[u]);
-            w0[u] = *reinterpret_cast<const uint4*>(st + rr * REC + 32 * p);
-            w1[u] = *reinterpret_cast<const uint4*>(st + rr * REC + 32 * p + 16);
-        }
-        float s[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            if (ok[u] && head[u] != cur_head) {
-                load_q(qt, head[u], p, qa, qb);
-                cur_head = head[u];
+        // one pass per query head present in the stage (one, except where a head's
+        // candidates end inside the stage)
+        float s = 0.0f;
+        for (int64_t h = hh; h <= hlast; ++h) {
+            if (h != staged) {
+                __syncwarp();
+                stage_query(qt, h, qs, lane);
+                staged = h;
             }
-            const float2 pa = pair_dots(w0[u].x, w0[u].y, qa);
-            const float2 pb = pair_dots(w0[u].z, w0[u].w, qb);
-            const float f0 = __uint_as_float(w1[u].x), f1 = __uint_as_float(w1[u].y);
-            const float f2 = __uint_as_float(w1[u].z), f3 = __uint_as_float(w1[u].w);
-            float t = 0.0f;
-#pragma unroll
-            for (int step = 0; step < 4; ++step) {
-                const float prev = __shfl_up_sync(0xffffffffu, t, 1, 4);
-                if (p == step) {
-                    float x = step == 0 ? 0.0f : prev;
-                    x = __fmaf_rn(f0, pa.x, x);
-                    x = __fmaf_rn(f1, pa.y, x);
-                    x = __fmaf_rn(f2, pb.x, x);
-                    x = __fmaf_rn(f3, pb.y, x);
-                    t = x;
-                }
-            }
-            s[u] = t;
+            if (ok && head == h) s = score_record(st, lane, qp);
         }
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-            if (p == 3 && ok[u]) S[head[u] * cmax + cc[u]] = s[u];
+        if (ok) S[head * cmax + cc] = s;
         hc += kStep;
         wrap(hh, hc);
         __syncwarp();                        // every lane has read the slot before its refill
@@ -227,13 +225,9 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
 
 cudaError_t launch_rerank(const pariskv_index* ix, int64_t C, cudaStream_t st) {
     if (C <= 0) return cudaSuccess;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(rerank_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<uint64_t> smem_raised{0};
+    if (cudaError_t e = raise_smem_limit(rerank_kernel, kSmem, smem_raised); e != cudaSuccess)
+        return e;
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

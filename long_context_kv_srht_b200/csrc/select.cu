@@ -14,11 +14,12 @@
 //    vote scan (warp per chunk, lane per pair of bins), finds T and E with suffix sums and
 //    ballots, and writes for every 8192-key chunk how many candidates and how many score-T
 //    keys precede it (exclusive scans over chunks).
-//  compact_kernel (one CTA per chunk and vote pack): each thread owns 16 consecutive keys.
-//    SWAR byte arithmetic tests the four packed scores of a key against the four heads'
-//    thresholds at once (two adds and masks); byte counters count keys above T and ties;
-//    two block-wide scans (four heads in 16-bit lanes of a 64-bit word) give every
-//    candidate its output position, and the ties each thread may keep follow from E.
+//  compact_kernel (one CTA per chunk and vote pack): each thread owns 32 consecutive keys
+//    (read coalesced and transposed through shared memory). SWAR byte arithmetic tests the
+//    four packed scores of a key against the four heads' thresholds at once. A counting pass
+//    and one block-wide scan of the per-head counts give every thread where its candidates
+//    start and how many of its ties it keeps (all, none, or -- in the one thread where the
+//    E-th tie falls -- the first few); the write pass then stores its candidates in key order.
 #include "common.cuh"
 #include "internal.hpp"
 
@@ -27,8 +28,6 @@ namespace pkv {
 namespace {
 
 constexpr int kThr = 256;                  // threshold kernel
-constexpr int kKeysPerThread = 16;         // compaction: keys per thread
-constexpr int kCThr = CHUNK / kKeysPerThread;  // compaction: one chunk per block
 
 // Block-wide exclusive scan of a 64-bit value (4 packed 16-bit counters in the compaction,
 // none of which overflows because a block's total per counter is at most CHUNK = 8192).
@@ -163,31 +162,64 @@ threshold_kernel(const uint32_t* __restrict__ hist, int group, int packs, int64_
     }
 }
 
-// Byte b of the result is 1 when byte b of x is non-zero (bytes <= 0x80).
-__device__ __forceinline__ uint32_t nonzero_bytes(uint32_t x) {
-    return ((x + 0x7F7F7F7Fu) >> 7) & 0x01010101u;
+constexpr int kCW = 8;                          // compaction: warps per block
+constexpr int kCThr = 32 * kCW;
+constexpr int kKeys = CHUNK / kCThr;            // 32 consecutive keys per thread
+static_assert(kKeys == 32, "one 32-key run per thread");
+
+// Bytes 0,1 / 2,3 of a word spread into the 16-bit lanes of a 32-bit word.
+__device__ __forceinline__ uint64_t spread_bytes(uint32_t x) {
+    return (static_cast<uint64_t>(prmt_i<0x5352u>(x, 0u)) << 32) | prmt_i<0x5150u>(x, 0u);
 }
 
-// Spreads 4 byte counters into 4 16-bit lanes of a 64-bit word.
-__device__ __forceinline__ uint64_t widen(uint32_t x) {
-    return static_cast<uint64_t>(x & 0xffu) | (static_cast<uint64_t>((x >> 8) & 0xffu) << 16) |
-           (static_cast<uint64_t>((x >> 16) & 0xffu) << 32) |
-           (static_cast<uint64_t>(x >> 24) << 48);
+// Block-wide exclusive scan of two 64-bit values at once (4 packed 16-bit counters each,
+// none of which overflows: a block's total per counter is at most CHUNK = 8192).
+__device__ __forceinline__ void block_excl_scan2(uint64_t& a, uint64_t& b,
+                                                 uint64_t (*sh)[2] /* [kCW + 1][2] */) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint64_t x = a, y = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t xo = __shfl_up_sync(0xffffffffu, x, o);
+        const uint64_t yo = __shfl_up_sync(0xffffffffu, y, o);
+        if (lane >= o) { x += xo; y += yo; }
+    }
+    if (lane == 31) { sh[warp][0] = x; sh[warp][1] = y; }
+    __syncthreads();
+    uint64_t bx = 0, by = 0;
+    for (int w = 0; w < warp; ++w) { bx += sh[w][0]; by += sh[w][1]; }
+    a = bx + x - a;
+    b = by + y - b;
 }
 
-__global__ void __launch_bounds__(kCThr, 2)
+__global__ void __launch_bounds__(kCThr)
 compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ thr,
                const int32_t* __restrict__ cbase, int32_t* __restrict__ cand, int64_t n,
                int64_t cap_pad, int group, int packs, int64_t nchunks, int64_t cmax,
                int* status) {
-    __shared__ uint64_t scan_sh[kCThr / 32 + 1];
+    __shared__ uint32_t tr[kCW][32 * 33];
+    __shared__ uint64_t scan_sh[kCW + 1][2];
     const int64_t c = blockIdx.x;
     const int64_t up = blockIdx.y;
     const int unit = static_cast<int>(up / packs), p = static_cast<int>(up % packs);
     const int hp = min(PACK, group - p * PACK);
-    const int64_t k0 = c * CHUNK, k1 = min64(n, k0 + CHUNK);
-    const int64_t my0 = k0 + static_cast<int64_t>(threadIdx.x) * kKeysPerThread;
-    const int nvalid = static_cast<int>(max64(0, min64(kKeysPerThread, k1 - my0)));
+    const int head0 = unit * group + p * PACK;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t kw = c * CHUNK + static_cast<int64_t>(warp) * (32 * kKeys);  // warp's first key
+    const int64_t k0 = kw + static_cast<int64_t>(lane) * kKeys;                // thread's first key
+    const int nv = static_cast<int>(max64(0, min64(kKeys, n - k0)));          // its valid keys
+
+    // coalesced load of the warp's 1024 packed scores, transposed so that lane l then reads
+    // keys 32 l .. 32 l + 31 (row stride 33 words: both directions are conflict-free)
+    {
+        const uint32_t* src = scores + up * cap_pad + kw + lane;
+        const int nw = static_cast<int>(max64(0, min64(32 * kKeys, n - kw)));
+#pragma unroll 8
+        for (int t = 0; t < kKeys; ++t)
+            tr[warp][t * 33 + lane] = (32 * t + lane < nw) ? src[32 * t] : 0u;
+        __syncwarp();
+    }
+    const uint32_t* s = &tr[warp][lane * 33];
 
     // Per-head thresholds packed one per byte. A head outside the pack gets T = 127, which
     // no score (< 64) reaches. Byte h of (s + gt_add) has bit 7 set iff score_h > T_h, and
@@ -195,72 +227,72 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
     uint32_t gt_add = 0, ge_add = 0;
 #pragma unroll
     for (int h = 0; h < PACK; ++h) {
-        const int T = h < hp ? thr[(unit * group + p * PACK + h) * 4 + 0] : 127;
+        const int T = h < hp ? thr[(head0 + h) * 4 + 0] : 127;
         gt_add |= static_cast<uint32_t>(127 - T) << (8 * h);
         ge_add |= static_cast<uint32_t>(128 - T) << (8 * h);
     }
-
-    uint32_t s[kKeysPerThread];
-    const uint32_t* src = scores + up * cap_pad + my0;
-#pragma unroll
-    for (int j = 0; j < kKeysPerThread; j += 4) {
-        if (j < nvalid) {
-            const uint4 v = *reinterpret_cast<const uint4*>(src + j);
-            s[j] = v.x; s[j + 1] = v.y; s[j + 2] = v.z; s[j + 3] = v.w;
-        } else {
-            s[j] = s[j + 1] = s[j + 2] = s[j + 3] = 0;
-        }
-    }
-    // byte counters per head: keys above T and keys equal to T among this thread's keys
+    // counting pass: keys above T and ties, per head in byte counters (at most 32 each)
     uint32_t gcnt = 0, ecnt = 0;
-#pragma unroll
-    for (int j = 0; j < kKeysPerThread; ++j) {
-        const uint32_t m = j < nvalid ? 0x01010101u : 0u;
+#pragma unroll 8
+    for (int j = 0; j < kKeys; ++j) {
+        const uint32_t m = j < nv ? 0x01010101u : 0u;
         const uint32_t g = ((s[j] + gt_add) >> 7) & m;
-        const uint32_t ge = ((s[j] + ge_add) >> 7) & m;
         gcnt += g;
-        ecnt += ge ^ g;
+        ecnt += (((s[j] + ge_add) >> 7) & m) ^ g;
     }
-    uint64_t tot;
-    const uint64_t eq_pre = block_excl_scan_u64<kCThr>(widen(ecnt), &tot, scan_sh);
-    uint32_t take = 0;  // ties this thread keeps, per head (one byte each)
+    uint64_t gb = spread_bytes(gcnt), eb = spread_bytes(ecnt);
+    block_excl_scan2(gb, eb, scan_sh);   // keys above T / ties in this chunk before this thread
+
+    // where this thread's candidates start, and how many of its ties it keeps: the chunk
+    // keeps the first B = max(0, E - ties before the chunk) of its ties, in key order
+    int32_t* out[PACK];
+    uint32_t run[PACK], budget[PACK];
+    uint32_t all_ties = 0, partial = 0;
+    const int32_t C = thr[head0 * 4 + 2];
 #pragma unroll
     for (int h = 0; h < PACK; ++h) {
+        out[h] = cand + static_cast<int64_t>(head0 + min(h, hp - 1)) * cmax;
+        run[h] = 0;
+        budget[h] = 0;
         if (h >= hp) continue;
-        const int head = unit * group + p * PACK + h;
-        const int64_t before = cbase[(static_cast<int64_t>(head) * nchunks + c) * 2 + 1] +
-                               static_cast<int64_t>((eq_pre >> (16 * h)) & 0xffff);
-        const int64_t room = max64(0, thr[head * 4 + 1] - before);
-        take |= static_cast<uint32_t>(min64(room, (ecnt >> (8 * h)) & 0xffu)) << (8 * h);
+        const int64_t hb = (static_cast<int64_t>(head0 + h) * nchunks + c) * 2;
+        const int64_t E = thr[(head0 + h) * 4 + 1];
+        const int64_t B = max64(0, E - cbase[hb + 1]);
+        const int64_t gbefore = (gb >> (16 * h)) & 0xffffu, ebefore = (eb >> (16 * h)) & 0xffffu;
+        const int64_t mine_g = (gcnt >> (8 * h)) & 0xffu, mine_e = (ecnt >> (8 * h)) & 0xffu;
+        const int64_t take = min64(max64(B - ebefore, 0), mine_e);
+        const int64_t start = cbase[hb + 0] + gbefore + min64(B, ebefore);
+        if (start + mine_g + take > C) {   // never taken when the histograms are consistent
+            atomicExch(status, ST_BADINDEX);
+            return;
+        }
+        run[h] = static_cast<uint32_t>(start);
+        budget[h] = static_cast<uint32_t>(take);
+        if (take == mine_e) all_ties |= 1u << (8 * h);
+        else if (take > 0) partial |= 1u << (8 * h);
     }
-    const uint64_t sel_pre = block_excl_scan_u64<kCThr>(widen(gcnt + take), &tot, scan_sh);
-    uint32_t pos[PACK];
-#pragma unroll
-    for (int h = 0; h < PACK; ++h) {
-        const int head = unit * group + p * PACK + min(h, hp - 1);
-        pos[h] = static_cast<uint32_t>(cbase[(static_cast<int64_t>(head) * nchunks + c) * 2]) +
-                 static_cast<uint32_t>((sel_pre >> (16 * h)) & 0xffff);
-    }
-#pragma unroll
-    for (int j = 0; j < kKeysPerThread; ++j) {
-        const uint32_t m = j < nvalid ? 0x01010101u : 0u;
+
+    // write pass, in key order
+#pragma unroll 4
+    for (int j = 0; j < kKeys; ++j) {
+        const uint32_t m = j < nv ? 0x01010101u : 0u;
         const uint32_t g = ((s[j] + gt_add) >> 7) & m;
         const uint32_t e = (((s[j] + ge_add) >> 7) & m) ^ g;
-        const uint32_t t = e & nonzero_bytes(take);
-        take -= t;
-        const uint32_t sel = g | t;
-        if (sel) {
+        uint32_t sel = g | (e & all_ties);
+        if (partial) {                       // the one thread per head where the E-th tie falls
 #pragma unroll
             for (int h = 0; h < PACK; ++h) {
-                if ((sel >> (8 * h)) & 1u) {
-                    const int head = unit * group + p * PACK + h;
-                    if (pos[h] < static_cast<uint32_t>(thr[head * 4 + 2]))
-                        cand[head * cmax + pos[h]] = static_cast<int32_t>(my0 + j);
-                    else
-                        atomicExch(status, ST_BADINDEX);
-                    ++pos[h];
+                if (((partial & e) >> (8 * h)) & 1u) {
+                    if (budget[h] > 0) { sel |= 1u << (8 * h); --budget[h]; }
                 }
             }
+        }
+        const int32_t key = static_cast<int32_t>(k0 + j);
+#pragma unroll
+        for (int h = 0; h < PACK; ++h) {
+            const uint32_t b = (sel >> (8 * h)) & 1u;
+            if (b) out[h][run[h]] = key;
+            run[h] += b;
         }
     }
 }

@@ -180,14 +180,8 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
 }  // namespace
 
 cudaError_t launch_vote(const pariskv_index* ix, cudaStream_t st) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(vote_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<uint64_t> smem_raised{0};
+    if (cudaError_t e = raise_smem_limit(vote_kernel, kSmemBytes, smem_raised); e != cudaSuccess) return e;
     if (ix->n <= 0) return cudaSuccess;
     const int64_t nchunks = ceil_div(ix->n, CHUNK);
     const int64_t items = static_cast<int64_t>(ix->units) * ix->packs * nchunks;
