@@ -19,7 +19,8 @@
 //    four packed scores of a key against the four heads' thresholds at once. A counting pass
 //    and one block-wide scan of the per-head counts give every thread where its candidates
 //    start and how many of its ties it keeps (all, none, or -- in the one thread where the
-//    E-th tie falls -- the first few); the write pass then stores its candidates in key order.
+//    E-th tie falls -- the first few); the write pass then visits, in key order, only the
+//    keys that reach some head's T (a bit mask from the counting pass) and stores them.
 #include "common.cuh"
 #include "internal.hpp"
 
@@ -231,14 +232,17 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
         gt_add |= static_cast<uint32_t>(127 - T) << (8 * h);
         ge_add |= static_cast<uint32_t>(128 - T) << (8 * h);
     }
-    // counting pass: keys above T and ties, per head in byte counters (at most 32 each)
-    uint32_t gcnt = 0, ecnt = 0;
+    // counting pass: keys above T and ties, per head in byte counters (at most 32 each),
+    // and the mask of keys that reach T for some head (the only ones the write pass visits)
+    uint32_t gcnt = 0, ecnt = 0, reach = 0;
 #pragma unroll 8
     for (int j = 0; j < kKeys; ++j) {
         const uint32_t m = j < nv ? 0x01010101u : 0u;
         const uint32_t g = ((s[j] + gt_add) >> 7) & m;
+        const uint32_t ge = ((s[j] + ge_add) >> 7) & m;
         gcnt += g;
-        ecnt += (((s[j] + ge_add) >> 7) & m) ^ g;
+        ecnt += ge ^ g;
+        reach |= (ge != 0u ? 1u : 0u) << j;
     }
     uint64_t gb = spread_bytes(gcnt), eb = spread_bytes(ecnt);
     block_excl_scan2(gb, eb, scan_sh);   // keys above T / ties in this chunk before this thread
@@ -272,12 +276,13 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
         else if (take > 0) partial |= 1u << (8 * h);
     }
 
-    // write pass, in key order
-#pragma unroll 4
-    for (int j = 0; j < kKeys; ++j) {
-        const uint32_t m = j < nv ? 0x01010101u : 0u;
-        const uint32_t g = ((s[j] + gt_add) >> 7) & m;
-        const uint32_t e = (((s[j] + ge_add) >> 7) & m) ^ g;
+    // write pass over the keys that reach T, in key order
+    while (reach) {
+        const int j = __ffs(reach) - 1;
+        reach &= reach - 1u;
+        const uint32_t sv = s[j];
+        const uint32_t g = (sv + gt_add) >> 7 & 0x01010101u;
+        const uint32_t e = ((sv + ge_add) >> 7 & 0x01010101u) ^ g;
         uint32_t sel = g | (e & all_ties);
         if (partial) {                       // the one thread per head where the E-th tie falls
 #pragma unroll

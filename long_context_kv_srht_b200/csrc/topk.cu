@@ -7,31 +7,37 @@
 // index, and returned in ascending key order with est = ||q|| * S.
 //
 // Exact selection on the order-preserving 32-bit image u of S (flip all bits of negative
-// values, set the sign bit of the others), one 1024-thread CTA per query head:
-//  - one bulk copy brings the head's S values into shared memory (up to kResident of them;
-//    larger candidate sets are read from global memory on every pass), where they are turned
-//    into u in place while the block finds min and max;
+// values, set the sign bit of the others), by a cluster of four CTAs per query head:
+//  - CTA r loads the r-th quarter of the head's S values (as u) and candidate indices into
+//    shared memory with coalesced loads (quarters longer than kSlice stay in global memory
+//    and are re-read on every pass);
+//  - the cluster agrees on [min, max] of u through distributed shared memory;
 //  - range-adaptive radix levels: the current interval [lo, hi] is cut into at most 2048
-//    power-of-two-wide bins, a shared histogram is built over the values in the interval, a
-//    suffix scan finds the bin holding the k-th largest, and the interval shrinks to that
-//    bin. Because the first interval is [min, max] of the data, one level usually settles
-//    all but a few values; every level shrinks the interval 2048-fold, so at most three run;
-//  - with T the k-th largest value and E the number of T-valued candidates to keep, a ballot
-//    pass over warp-contiguous ranges writes every candidate above T and the first E equal to
-//    T, in ascending key order (the candidates are stored in key order). est comes from the
-//    value image itself; the candidate indices of eight tiles are fetched at once, so a warp
-//    waits for global memory a few times rather than once per tile.
+//    power-of-two-wide bins, every CTA histograms its quarter, and every CTA sums the four
+//    histograms bin by bin over DSMEM and runs the same suffix scan, so all four pick the
+//    same bin (the one holding the k-th largest) without further exchange. Histograms
+//    alternate between two buffers, so one cluster barrier per level suffices; every level
+//    shrinks the interval 2048-fold, so at most three run;
+//  - with T the k-th largest value and E the number of T-valued candidates to keep, each
+//    warp counts its contiguous range, the counts are scanned over warps and over the
+//    cluster, and a ballot pass writes every candidate above T and the first E equal to T in
+//    ascending key order (the candidates are stored in key order); est comes from u itself.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "internal.hpp"
 
 namespace pkv {
 
+namespace cg = cooperative_groups;
+
 namespace {
 
+constexpr int kCL = 4;             // CTAs per query head
 constexpr int kT = 1024;
 constexpr int kWarps = kT / 32;
 constexpr int kBins = 2048;
-constexpr int kResident = 53248;   // candidates kept in shared memory (208 KB)
+constexpr int kSlice = 16384;      // values per CTA kept in shared memory (u and index)
 
 __device__ __forceinline__ uint32_t order_key(float s) {
     const uint32_t u = __float_as_uint(s);
@@ -43,39 +49,40 @@ __device__ __forceinline__ float value_of(uint32_t key) {
 }
 
 template <bool RES>
-__global__ void __launch_bounds__(kT, 1)
+__global__ void __cluster_dims__(kCL, 1, 1) __launch_bounds__(kT, 1)
 topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
             const float* __restrict__ qnorm, int32_t C, int64_t cmax, int32_t k,
             int32_t* __restrict__ out_idx, float* __restrict__ out_est, int* status) {
-    extern __shared__ __align__(16) uint32_t keys[];
-    __shared__ uint32_t hist[kBins];
-    __shared__ uint32_t wa[kWarps], wb[kWarps], wsel0[kWarps], weq0[kWarps];
+    extern __shared__ __align__(16) uint32_t dyn[];
+    __shared__ uint32_t hist[2][kBins];
+    __shared__ uint32_t wa[kWarps], wb[kWarps];
+    __shared__ uint32_t ctot[2];       // this CTA's candidates above T / ties at T
+    __shared__ uint32_t cmm[2];        // this CTA's min / max of u
     __shared__ uint32_t pick[2];
-    __shared__ __align__(8) uint64_t bar;
 
-    const int head = blockIdx.x;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = static_cast<int>(cluster.block_rank());
+    const int head = blockIdx.x / kCL;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const float* Sh = S + head * cmax;
-    const int32_t* ch = cand + head * cmax;
+    const int s0 = static_cast<int>(static_cast<int64_t>(C) * rank / kCL);
+    const int s1 = static_cast<int>(static_cast<int64_t>(C) * (rank + 1) / kCL);
+    const int L = s1 - s0;
+    const float* Sh = S + head * cmax + s0;
+    const int32_t* ch = cand + head * cmax + s0;
+    uint32_t* keys = dyn;                                   // [kSlice] u
+    int32_t* idx = reinterpret_cast<int32_t*>(dyn + kSlice);  // [kSlice] candidate index
     auto key_at = [&](int i) -> uint32_t { return RES ? keys[i] : order_key(Sh[i]); };
+    auto idx_at = [&](int i) -> int32_t { return RES ? idx[i] : ch[i]; };
 
-    // 1. S -> shared memory in one bulk copy (16-byte granules; the array is padded)
-    if (RES) {
-        const uint32_t b = smem_addr(&bar);
-        const uint32_t bytes = static_cast<uint32_t>(round_up(C, 4) * 4);
-        if (threadIdx.x == 0) {
-            mbar_init(b, 1);
-            mbar_fence_init();
-            mbar_arrive_expect_tx(b, bytes);
-            bulk_g2s(smem_addr(keys), Sh, bytes, b);
-        }
-        __syncthreads();
-        mbar_wait(b, 0, status);
-    }
+    // 1. the quarter into shared memory; local min / max
     uint32_t mn = 0xffffffffu, mx = 0u;
-    for (int i = threadIdx.x; i < C; i += kT) {
-        const uint32_t u = RES ? order_key(__uint_as_float(keys[i])) : order_key(Sh[i]);
-        if (RES) keys[i] = u;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < L; i += kT) {
+        const uint32_t u = order_key(Sh[i]);
+        if (RES) {
+            keys[i] = u;
+            idx[i] = ch[i];
+        }
         mn = min(mn, u);
         mx = max(mx, u);
     }
@@ -83,43 +90,57 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
     mx = __reduce_max_sync(0xffffffffu, mx);
     if (lane == 0) { wa[warp] = mn; wb[warp] = mx; }
     __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t a = 0xffffffffu, b = 0u;
+        for (int w = 0; w < kWarps; ++w) { a = min(a, wa[w]); b = max(b, wb[w]); }
+        cmm[0] = a;
+        cmm[1] = b;
+    }
+    cluster.sync();
     uint32_t lo = 0xffffffffu, hi = 0u;
-#pragma unroll 8
-    for (int w = 0; w < kWarps; ++w) { lo = min(lo, wa[w]); hi = max(hi, wb[w]); }
-    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < kCL; ++q) {
+        const uint32_t* r = cluster.map_shared_rank(cmm, q);
+        lo = min(lo, r[0]);
+        hi = max(hi, r[1]);
+    }
 
-    // 2. range-adaptive radix levels
+    // 2. range-adaptive radix levels over the cluster
     uint32_t krem = static_cast<uint32_t>(k);
+    int level = 0;
     while (lo != hi) {
+        uint32_t* hb = hist[level & 1];
         const uint32_t span = hi - lo;
         const int bitlen = 32 - __clz(span);
         const int sh = bitlen > 11 ? bitlen - 11 : 0;   // (span >> sh) < 2048
-        hist[threadIdx.x] = 0u;
-        hist[threadIdx.x + kT] = 0u;
+        hb[threadIdx.x] = 0u;
+        hb[threadIdx.x + kT] = 0u;
         __syncthreads();
-        if (RES) {
+        if (RES && (L & 3) == 0) {
             const uint4* k4 = reinterpret_cast<const uint4*>(keys);
-            const int C4 = C >> 2;
-            for (int i = threadIdx.x; i < C4; i += kT) {
+            for (int i = threadIdx.x; i < (L >> 2); i += kT) {
                 const uint4 v = k4[i];
                 const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    if (u[j] >= lo && u[j] <= hi) atomicAdd(&hist[(u[j] - lo) >> sh], 1u);
-            }
-            for (int i = (C4 << 2) + threadIdx.x; i < C; i += kT) {
-                const uint32_t u = keys[i];
-                if (u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> sh], 1u);
+                    if (u[j] >= lo && u[j] <= hi) atomicAdd(&hb[(u[j] - lo) >> sh], 1u);
             }
         } else {
-            for (int i = threadIdx.x; i < C; i += kT) {
+            for (int i = threadIdx.x; i < L; i += kT) {
                 const uint32_t u = key_at(i);
-                if (u >= lo && u <= hi) atomicAdd(&hist[(u - lo) >> sh], 1u);
+                if (u >= lo && u <= hi) atomicAdd(&hb[(u - lo) >> sh], 1u);
             }
         }
-        __syncthreads();
-        // suffix counts: thread t owns bins 2t, 2t + 1
-        const uint32_t h0 = hist[2 * threadIdx.x], h1 = hist[2 * threadIdx.x + 1];
+        cluster.sync();   // every quarter's histogram is complete
+        // thread t sums bins 2t, 2t + 1 over the cluster; suffix counts over the bins
+        uint32_t h0 = 0, h1 = 0;
+#pragma unroll
+        for (int q = 0; q < kCL; ++q) {
+            const uint2 v = *reinterpret_cast<const uint2*>(cluster.map_shared_rank(hb, q) +
+                                                             2 * threadIdx.x);
+            h0 += v.x;
+            h1 += v.y;
+        }
         uint32_t x = h0 + h1;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -138,92 +159,89 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
         const uint32_t b = pick[0];
         krem -= pick[1];
         const uint32_t nlo = lo + (b << sh);
-        lo = nlo;
         const uint64_t bin_hi = static_cast<uint64_t>(nlo) + ((uint64_t{1} << sh) - 1u);
+        lo = nlo;
         hi = static_cast<uint32_t>(min(static_cast<uint64_t>(hi), bin_hi));
-        __syncthreads();
+        ++level;
+        __syncthreads();   // pick[] and wa[] are rewritten by the next level
     }
     const uint32_t T = lo;
     const uint32_t E = krem;   // ties at T to keep, in key order
 
-    // 3. compaction over warp-contiguous ranges, ascending key order
-    const int w0 = static_cast<int>(static_cast<int64_t>(C) * warp / kWarps);
-    const int w1 = static_cast<int>(static_cast<int64_t>(C) * (warp + 1) / kWarps);
+    // 3. counts per warp-contiguous range, then offsets over warps and over the cluster
+    const int w0 = static_cast<int>(static_cast<int64_t>(L) * warp / kWarps);
+    const int w1 = static_cast<int>(static_cast<int64_t>(L) * (warp + 1) / kWarps);
     uint32_t ngt = 0, neq = 0;
-    for (int pbase = w0; pbase < w1; pbase += 32) {
-        const int pp = pbase + lane;
-        const bool valid = pp < w1;
-        const uint32_t u = valid ? key_at(pp) : 0u;
-        ngt += __popc(__ballot_sync(0xffffffffu, valid && u > T));
-        neq += __popc(__ballot_sync(0xffffffffu, valid && u == T));
+    for (int pp = w0 + lane; pp < w1; pp += 32) {
+        const uint32_t u = key_at(pp);
+        ngt += u > T;
+        neq += u == T;
     }
+    ngt = __reduce_add_sync(0xffffffffu, ngt);
+    neq = __reduce_add_sync(0xffffffffu, neq);
     if (lane == 0) { wa[warp] = ngt; wb[warp] = neq; }
     __syncthreads();
     if (threadIdx.x == 0) {
-        uint32_t sel = 0, eqb = 0;
-        for (int w = 0; w < kWarps; ++w) {
-            wsel0[w] = sel;
-            weq0[w] = eqb;
-            sel += wa[w] + (eqb >= E ? 0u : min(E - eqb, wb[w]));
-            eqb += wb[w];
-        }
+        uint32_t g = 0, e = 0;
+        for (int w = 0; w < kWarps; ++w) { g += wa[w]; e += wb[w]; }
+        ctot[0] = g;
+        ctot[1] = e;
     }
-    __syncthreads();
-    uint32_t sel_run = wsel0[warp], eq_run = weq0[warp];
+    cluster.sync();
+    uint32_t gt_run = 0, eq_run = 0;   // above T / ties before this warp's range
+    for (int q = 0; q < rank; ++q) {
+        const uint32_t* r = cluster.map_shared_rank(ctot, q);
+        gt_run += r[0];
+        eq_run += r[1];
+    }
+    for (int w = 0; w < warp; ++w) { gt_run += wa[w]; eq_run += wb[w]; }
+    cluster.barrier_arrive();          // no remote read of this CTA's memory follows
+
+    // 4. ballot pass in key order
     const float qn = qnorm[head];
     const uint32_t lt = (1u << lane) - 1u;
-    // the candidate indices of kBatch tiles are loaded together, so their latencies overlap
-    constexpr int kBatch = 8;
-    for (int pb = w0; pb < w1; pb += 32 * kBatch) {
-        int32_t ci[kBatch];
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int pp = pb + 32 * b + lane;
-            ci[b] = pp < w1 ? ch[pp] : 0;
-        }
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int pp = pb + 32 * b + lane;
-            const bool valid = pp < w1;
-            const uint32_t u = valid ? key_at(pp) : 0u;
-            const uint32_t eqm = __ballot_sync(0xffffffffu, valid && u == T);
-            const bool take = valid && u == T && (eq_run + __popc(eqm & lt)) < E;
-            const bool sel = (valid && u > T) || take;
-            const uint32_t selm = __ballot_sync(0xffffffffu, sel);
-            if (sel) {
-                const uint32_t r = sel_run + __popc(selm & lt);
-                if (r < static_cast<uint32_t>(k)) {
-                    const int64_t pos = static_cast<int64_t>(head) * k + r;
-                    out_idx[pos] = ci[b];
-                    if (out_est) out_est[pos] = __fmul_rn(qn, value_of(u));
-                } else {
-                    atomicExch(status, ST_BADINDEX);
-                }
+    for (int pb = w0; pb < w1; pb += 32) {
+        const int pp = pb + lane;
+        const bool valid = pp < w1;
+        const uint32_t u = valid ? key_at(pp) : 0u;
+        const bool eq = valid && u == T;
+        const bool gt = valid && u > T;
+        const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+        const bool sel = gt || (eq && (eq_run + __popc(eqm & lt)) < E);
+        const uint32_t selm = __ballot_sync(0xffffffffu, sel);
+        if (sel) {
+            const uint32_t r = gt_run + min(eq_run, E) + __popc(selm & lt);
+            if (r < static_cast<uint32_t>(k)) {
+                const int64_t pos = static_cast<int64_t>(head) * k + r;
+                out_idx[pos] = idx_at(pp);
+                if (out_est) out_est[pos] = __fmul_rn(qn, value_of(u));
+            } else {
+                atomicExch(status, ST_BADINDEX);
             }
-            sel_run += __popc(selm);
-            eq_run += __popc(eqm);
         }
+        gt_run += __popc(__ballot_sync(0xffffffffu, gt));
+        eq_run += __popc(eqm);
     }
+    cluster.barrier_wait();
 }
 
 }  // namespace
 
 cudaError_t launch_topk(const pariskv_index* ix, int64_t C, int32_t k, int32_t* topk_idx,
                         float* topk_est, cudaStream_t st) {
+    constexpr int kDyn = 2 * kSlice * 4;
     static std::atomic<uint64_t> smem_raised{0};
-    if (cudaError_t e = raise_smem_limit(topk_kernel<true>, kResident * 4, smem_raised);
-        e != cudaSuccess)
+    if (cudaError_t e = raise_smem_limit(topk_kernel<true>, kDyn, smem_raised); e != cudaSuccess)
         return e;
     const int heads = ix->units * ix->cfg.group;
-    if (C <= kResident) {
-        const size_t smem = static_cast<size_t>(round_up(C, 4)) * 4;
-        topk_kernel<true><<<heads, kT, smem, st>>>(ix->S, ix->cand, ix->qnorm,
-                                                   static_cast<int32_t>(C), ix->cmax, k,
-                                                   topk_idx, topk_est, ix->status);
+    if (ceil_div(C, kCL) <= kSlice) {
+        topk_kernel<true><<<heads * kCL, kT, kDyn, st>>>(ix->S, ix->cand, ix->qnorm,
+                                                         static_cast<int32_t>(C), ix->cmax, k,
+                                                         topk_idx, topk_est, ix->status);
     } else {
-        topk_kernel<false><<<heads, kT, 0, st>>>(ix->S, ix->cand, ix->qnorm,
-                                                 static_cast<int32_t>(C), ix->cmax, k, topk_idx,
-                                                 topk_est, ix->status);
+        topk_kernel<false><<<heads * kCL, kT, 0, st>>>(ix->S, ix->cand, ix->qnorm,
+                                                       static_cast<int32_t>(C), ix->cmax, k,
+                                                       topk_idx, topk_est, ix->status);
     }
     return cudaGetLastError();
 }

@@ -110,19 +110,21 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
         *reinterpret_cast<uint32_t*>(tab + r * 256 + hcol) = 0u;
 
     // warp w scores tiles w, w + kWarps, ... of each chunk; the next tile's ids are loaded
-    // while the current tile is scored
-    auto tile_ptr = [&](int64_t item, int tl) -> const uint8_t* {
-        const int64_t up = item / nchunks, c = item % nchunks;
+    // while the current tile is scored. Item -> ids address: the divisions run once per item.
+    auto item_ids = [&](int64_t item) -> const uint8_t* {
+        const int64_t up = item / nchunks, c = item - (item / nchunks) * nchunks;
         const int64_t unit = up / packs;
-        return ids + (unit * cap_pad + c * CHUNK + static_cast<int64_t>(tl) * kTileKeys) * 16 +
-               lane * 32;
+        return ids + (unit * cap_pad + c * CHUNK) * 16 + lane * 32;
     };
+    constexpr int kTileBytes = kTileKeys * 16;
     int64_t cur_up = -1;
     u32x8 nxt;
-    if (i0 < i1) nxt = ldg_ids(tile_ptr(i0, warp));
+    const uint8_t* base = i0 < i1 ? item_ids(i0) : ids;
+    if (i0 < i1) nxt = ldg_ids(base + warp * kTileBytes);
     for (int64_t item = i0; item < i1; ++item) {
-        const int64_t up = item / nchunks, c = item % nchunks;
+        const int64_t up = item / nchunks, c = item - up * nchunks;
         const int hp = min(PACK, group - static_cast<int>(up % packs) * PACK);
+        const uint8_t* next_base = item + 1 < i1 ? item_ids(item + 1) : base;
         if (up != cur_up) {
             __syncthreads();
             // row c, column 2b + k holds W_b[c] (copies k = 0, 1)
@@ -141,9 +143,9 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
             const u32x8 cur = nxt;
             // prefetch: the next tile of this chunk, else this warp's first of the next item
             // (tiles past the last key read padding inside the capacity, never beyond it)
-            if (tl + kWarps < kTilesPerChunk) nxt = ldg_ids(tile_ptr(item, tl + kWarps));
-            else if (item + 1 < i1) nxt = ldg_ids(tile_ptr(item + 1, warp));
-            if (tl * kTileKeys >= nkeys) continue;
+            if (tl + kWarps < kTilesPerChunk) nxt = ldg_ids(base + (tl + kWarps) * kTileBytes);
+            else if (item + 1 < i1) nxt = ldg_ids(next_base + warp * kTileBytes);
+        if (tl * kTileKeys >= nkeys) continue;
             uint32_t acc[2];
 #pragma unroll
             for (int j = 0; j < 2; ++j) acc[j] = score_key(tab, cur.w + 4 * j, colp);
@@ -174,6 +176,7 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
             if (lane == 0) hout[r] = tot;
         }
         __syncthreads();
+        base = next_base;
     }
 }
 
