@@ -105,118 +105,101 @@ __device__ __forceinline__ void stage_query(const float* __restrict__ qt, int64_
     __syncwarp();
 }
 
+// Work is cut into items of kItem consecutive candidates of one query head; warp g of the
+// grid takes items g, g + W, g + 2 W, ... (W warps in all), so within a stage the head, its
+// unit's record base and its rotated query are the same for every lane.
+constexpr int kItem = 256;
+constexpr uint32_t kNoRec = 0xffffffffu;
+
+struct StreamPos {
+    int64_t it;            // item
+    int s, nst;            // stage within the item, stages in the item
+    int head, c0, cend;    // query head, first candidate, one past the item's last
+    const uint8_t* ubase;  // records of the head's unit
+};
+
 __global__ void __launch_bounds__(kThr, 2)
 rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
-              const float* __restrict__ qt, float* __restrict__ S, int64_t C, int64_t cmax,
-              int64_t cap_pad, int64_t n, int group, int64_t total, int* status) {
+              const float* __restrict__ qt, float* __restrict__ S, int32_t C, int64_t cmax,
+              int64_t cap_pad, int64_t n, int group, int iph, int64_t items, int* status) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* ring = smem + warp * kWarpBytes;
     float2* qs = reinterpret_cast<float2*>(ring + kSlots * kStageBytes);
     const uint64_t* qp = reinterpret_cast<const uint64_t*>(qs);
+    const int64_t W = static_cast<int64_t>(gridDim.x) * kWarps;
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
 
-    // this CTA's slice of the flattened (head, candidate) sequence, cut in 32-record stages;
-    // the warp takes CTA stages warp, warp + kWarps, warp + 2 kWarps, ...
-    const int64_t r0 = total * blockIdx.x / gridDim.x, r1 = total * (blockIdx.x + 1) / gridDim.x;
-    const int64_t nstage = ceil_div(r1 - r0, kStageRecs);
-
-    // stage refill: lane l holds the record number of the stage's l-th record; for copy
+    auto start_item = [&](StreamPos& p) {
+        if (p.it >= items) return;
+        p.head = static_cast<int>(p.it / iph);
+        p.c0 = static_cast<int>(p.it - static_cast<int64_t>(p.head) * iph) * kItem;
+        p.cend = min(C, p.c0 + kItem);
+        p.nst = (p.cend - p.c0 + 31) >> 5;
+        p.s = 0;
+        p.ubase = rec + static_cast<int64_t>(p.head / group) * cap_pad * REC;
+    };
+    auto advance = [&](StreamPos& p) {
+        if (++p.s == p.nst) {
+            p.it += W;
+            start_item(p);
+        }
+    };
+    // stage refill: lane l looks up the record of candidate c0 + 32 s + l; for copy
     // instruction j, lanes 8g..8g+7 move the 8 16-byte pieces of record 4j + g
-    auto issue = [&](int slot, int64_t ridx, bool valid) {
-        uint8_t* dst0 = ring + slot * kStageBytes;
-        const int piece = lane & 7, sub = lane >> 3;
+    auto issue = [&](int slot, const StreamPos& p) {
+        if (p.it < items) {
+            const int c = p.c0 + 32 * p.s + lane;
+            uint32_t idx = kNoRec;
+            if (c < p.cend) {
+                const int32_t i = cand[p.head * cmax + c];
+                if (i >= 0 && i < n) idx = static_cast<uint32_t>(i);
+                else atomicExch(status, ST_BADINDEX);  // never taken when the selection is consistent
+            }
+            uint8_t* dst0 = ring + slot * kStageBytes;
+            const int piece = lane & 7, sub = lane >> 3;
 #pragma unroll
-        for (int j = 0; j < kStageRecs / 4; ++j) {
-            const int rr = 4 * j + sub;
-            const int64_t ri = __shfl_sync(0xffffffffu, ridx, rr);
-            const bool v = __shfl_sync(0xffffffffu, valid, rr);
-            if (v) {
-                const uint32_t dst = smem_addr(dst0 + piece_at(rr, piece));
-                const uint8_t* src = rec + ri * REC + piece * 16;
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(src)
-                             : "memory");
+            for (int j = 0; j < kStageRecs / 4; ++j) {
+                const int rr = 4 * j + sub;
+                const uint32_t ri = __shfl_sync(0xffffffffu, idx, rr);
+                if (ri != kNoRec) {
+                    const uint32_t dst = smem_addr(dst0 + piece_at(rr, piece));
+                    const uint8_t* src = p.ubase + static_cast<uint64_t>(ri) * REC + piece * 16;
+                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(src)
+                                 : "memory");
+                }
             }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    // (head, candidate) positions advance incrementally: one division at the start, then
-    // an add and at most one wrap per step when C >= 256 (several for small candidate sets)
-    auto wrap = [&](int64_t& h, int64_t& c) {
-        while (c >= C) { c -= C; ++h; }
-    };
-    // record number of the stage's lane-th record, with its bounds check
-    auto locate = [&](int64_t sh, int64_t sc, bool& valid) -> int64_t {
-        if (!valid) return 0;
-        int64_t head = sh, c = sc + lane;
-        wrap(head, c);
-        const int64_t i = cand[head * cmax + c];
-        if (i < 0 || i >= n) {  // never taken when the selection is consistent
-            atomicExch(status, ST_BADINDEX);
-            valid = false;
-            return 0;
-        }
-        const int64_t unit = static_cast<uint32_t>(head) / static_cast<uint32_t>(group);
-        return unit * cap_pad + i;
-    };
-    constexpr int64_t kStep = static_cast<int64_t>(kWarps) * kStageRecs;
-    const int64_t first = r0 + static_cast<int64_t>(warp) * kStageRecs;
-    int64_t ih = first / C, ic = first - ih * C;    // issue stream: stage start (head, cand)
-    int64_t hh = ih, hc = ic;                       // scoring stream
 
+    StreamPos iss{gw, 0, 0, 0, 0, 0, rec}, sc{gw, 0, 0, 0, 0, 0, rec};
+    start_item(iss);
+    start_item(sc);
     // prologue: fill the ring
     for (int g = 0; g < kSlots; ++g) {
-        const int64_t cs = warp + static_cast<int64_t>(kWarps) * g;
-        const int64_t rs = r0 + cs * kStageRecs;
-        bool valid = cs < nstage && rs + lane < r1;
-        const int64_t ri = locate(ih, ic, valid);
-        issue(g, ri, valid);
-        ic += kStep;
-        wrap(ih, ic);
+        issue(g, iss);
+        if (iss.it < items) advance(iss);
     }
 
-    int64_t staged = -1;   // head whose query is in qs
+    int staged = -1;   // head whose query is in qs
 #pragma unroll 1
-    for (int64_t g = 0;; ++g) {
-        const int64_t cs = warp + static_cast<int64_t>(kWarps) * g;
-        if (cs >= nstage) break;
-        const int slot = static_cast<int>(g % kSlots);
-        // indices of the stage that will refill this slot (their load overlaps the scoring)
-        const int64_t cs_next = cs + static_cast<int64_t>(kWarps) * kSlots;
-        const int64_t rs_next = r0 + cs_next * kStageRecs;
-        bool valid_next = cs_next < nstage && rs_next + lane < r1;
-        const int64_t ri_next = locate(ih, ic, valid_next);
-        ic += kStep;
-        wrap(ih, ic);
-
-        // this lane's record: head and candidate position (the valid lanes are a prefix)
-        const int64_t rs = r0 + cs * kStageRecs;
-        const bool ok = rs + lane < r1;
-        int64_t head = hh, cc = hc + lane;
-        wrap(head, cc);
-        const int last = static_cast<int>(min64(31, r1 - rs - 1));
-        const int64_t hlast = __shfl_sync(0xffffffffu, head, last);
-
+    for (int g = 0; sc.it < items; ++g) {
+        const int slot = g % kSlots;
         // the oldest committed group is this stage's; each lane waits for its own pieces and
         // the warp barrier makes every lane's pieces visible
         asm volatile("cp.async.wait_group %0;" :: "n"(kSlots - 1) : "memory");
         __syncwarp();
-        const uint8_t* st = ring + slot * kStageBytes;
-        // one pass per query head present in the stage (one, except where a head's
-        // candidates end inside the stage)
-        float s = 0.0f;
-        for (int64_t h = hh; h <= hlast; ++h) {
-            if (h != staged) {
-                __syncwarp();
-                stage_query(qt, h, qs, lane);
-                staged = h;
-            }
-            if (ok && head == h) s = score_record(st, lane, qp);
+        if (sc.head != staged) {
+            stage_query(qt, sc.head, qs, lane);
+            staged = sc.head;
         }
-        if (ok) S[head * cmax + cc] = s;
-        hc += kStep;
-        wrap(hh, hc);
-        __syncwarp();                        // every lane has read the slot before its refill
-        issue(slot, ri_next, valid_next);
+        const int c = sc.c0 + 32 * sc.s + lane;
+        if (c < sc.cend) S[sc.head * cmax + c] = score_record(ring + slot * kStageBytes, lane, qp);
+        __syncwarp();                        // every lane has read the slot and the query
+        issue(slot, iss);
+        if (iss.it < items) advance(iss);
+        advance(sc);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");   // no copy in flight at exit
 }
@@ -232,12 +215,12 @@ cudaError_t launch_rerank(const pariskv_index* ix, int64_t C, cudaStream_t st) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int heads = ix->units * ix->cfg.group;
-    const int64_t total = static_cast<int64_t>(heads) * C;
-    const int64_t stages = ceil_div(total, kStageRecs);
-    const int grid = static_cast<int>(max64(1, min64(2LL * sms, ceil_div(stages, kWarps))));
-    rerank_kernel<<<grid, kThr, kSmem, st>>>(ix->rec, ix->cand, ix->qt, ix->S, C, ix->cmax,
-                                             ix->cap_pad, ix->n, ix->cfg.group, total,
-                                             ix->status);
+    const int iph = static_cast<int>(ceil_div(C, kItem));
+    const int64_t items = static_cast<int64_t>(heads) * iph;
+    const int grid = static_cast<int>(max64(1, min64(2LL * sms, ceil_div(items, kWarps))));
+    rerank_kernel<<<grid, kThr, kSmem, st>>>(ix->rec, ix->cand, ix->qt, ix->S,
+                                             static_cast<int32_t>(C), ix->cmax, ix->cap_pad,
+                                             ix->n, ix->cfg.group, iph, items, ix->status);
     return cudaGetLastError();
 }
 

@@ -11,16 +11,17 @@
 // score == T.
 //
 //  threshold_kernel (one CTA per query head): sums the per-chunk histograms written by the
-//    vote scan (warp per chunk, lane per pair of bins), finds T and E with suffix sums and
-//    ballots, and writes for every 8192-key chunk how many candidates and how many score-T
-//    keys precede it (exclusive scans over chunks).
+//    vote scan (all loads in flight at once), finds T and E with suffix sums and ballots, and
+//    writes for every 8192-key chunk how many candidates and how many score-T keys precede
+//    it (one thread per chunk reads its 64 bins with vector loads; exclusive scans over
+//    chunks).
 //  compact_kernel (one CTA per chunk and vote pack): each thread owns 32 consecutive keys
 //    (read coalesced and transposed through shared memory). SWAR byte arithmetic tests the
-//    four packed scores of a key against the four heads' thresholds at once. A counting pass
-//    and one block-wide scan of the per-head counts give every thread where its candidates
-//    start and how many of its ties it keeps (all, none, or -- in the one thread where the
-//    E-th tie falls -- the first few); the write pass then visits, in key order, only the
-//    keys that reach some head's T (a bit mask from the counting pass) and stores them.
+//    four packed scores of a key against the four heads' thresholds at once, and the test
+//    bits are sliced into one 32-bit mask per head (above T, at T) over the thread's keys.
+//    POPC gives the counts; one block-wide scan of them gives every thread where its
+//    candidates start and how many of its ties it keeps (all, none, or -- in the one thread
+//    where the E-th tie falls -- the first few); the set bits are then written in key order.
 #include "common.cuh"
 #include "internal.hpp"
 
@@ -64,10 +65,9 @@ __device__ __forceinline__ uint64_t block_excl_scan_u64(uint64_t v, uint64_t* to
 __global__ void __launch_bounds__(kThr)
 threshold_kernel(const uint32_t* __restrict__ hist, int group, int packs, int64_t nchunks,
                  int64_t C, int32_t* __restrict__ thr, int32_t* __restrict__ cbase) {
-    __shared__ uint32_t part[kThr / 32][NBINS];
+    __shared__ uint32_t part[kThr / NBINS][NBINS];
     __shared__ int32_t sT, sE;
     __shared__ uint64_t scan_sh[kThr / 32 + 1];
-    __shared__ uint64_t cnt[kThr];
 
     const int head = blockIdx.x;
     const int unit = head / group, g = head % group;
@@ -76,19 +76,21 @@ threshold_kernel(const uint32_t* __restrict__ hist, int group, int packs, int64_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t* hb = hist + up * nchunks * (PACK * NBINS) + h * NBINS;
 
-    // total histogram: warp w sums chunks w, w + 8, ...; lane l owns bins l and l + 32
-    uint32_t a = 0, b = 0;
-    for (int64_t c = warp; c < nchunks; c += kThr / 32) {
-        a += hb[c * (PACK * NBINS) + lane];
-        b += hb[c * (PACK * NBINS) + lane + 32];
+    // total histogram: thread t sums bin t % 64 over chunks t / 64, t / 64 + 4, ... (the
+    // loads are independent, so they are all in flight together)
+    {
+        constexpr int kRows = kThr / NBINS;
+        const int bin = threadIdx.x % NBINS, r0 = threadIdx.x / NBINS;
+        uint32_t a = 0;
+#pragma unroll 8
+        for (int64_t c = r0; c < nchunks; c += kRows) a += hb[c * (PACK * NBINS) + bin];
+        part[r0][bin] = a;
     }
-    part[warp][lane] = a;
-    part[warp][lane + 32] = b;
     __syncthreads();
     if (warp == 0) {
         uint32_t lo = 0, hi = 0;
 #pragma unroll
-        for (int w = 0; w < kThr / 32; ++w) { lo += part[w][lane]; hi += part[w][lane + 32]; }
+        for (int r = 0; r < kThr / NBINS; ++r) { lo += part[r][lane]; hi += part[r][lane + 32]; }
         // count of scores >= t for t = lane and lane + 32 (suffix sums over the 64 bins)
         uint32_t shi = hi;
 #pragma unroll
@@ -131,24 +133,30 @@ threshold_kernel(const uint32_t* __restrict__ hist, int group, int packs, int64_
     __syncthreads();
     const int T = sT;
     const int64_t E = sE;
-    // per chunk: candidates above T and ties at T, then exclusive scans over chunks
+    // per chunk (one per thread, its 64 bins in 16 vector loads): keys above T and ties at T,
+    // then exclusive scans over chunks
     uint64_t run_gt = 0, run_eq = 0;
     for (int64_t base = 0; base < nchunks; base += kThr) {
-        for (int i = warp; i < kThr; i += kThr / 32) {
-            const int64_t c = base + i;
-            uint32_t gt = 0, eq = 0;
-            if (c < nchunks) {
-                const uint32_t* hc = hb + c * (PACK * NBINS);
-                const uint32_t x = hc[lane], y = hc[lane + 32];
-                gt = __reduce_add_sync(0xffffffffu, (lane > T ? x : 0u) + (lane + 32 > T ? y : 0u));
-                eq = __shfl_sync(0xffffffffu, T < 32 ? x : y, T & 31);
-            }
-            if (lane == 0) cnt[i] = (static_cast<uint64_t>(eq) << 32) | gt;
-        }
-        __syncthreads();
         const int64_t c = base + threadIdx.x;
+        uint32_t gt = 0, eq = 0;
+        if (c < nchunks) {
+            const uint4* hc = reinterpret_cast<const uint4*>(hb + c * (PACK * NBINS));
+            uint4 v[NBINS / 4];
+#pragma unroll
+            for (int i = 0; i < NBINS / 4; ++i) v[i] = hc[i];
+#pragma unroll
+            for (int i = 0; i < NBINS / 4; ++i) {
+                const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int bin = 4 * i + j;
+                    gt += bin > T ? w[j] : 0u;
+                    eq += bin == T ? w[j] : 0u;
+                }
+            }
+        }
+        const uint64_t mine = (static_cast<uint64_t>(eq) << 32) | gt;
         uint64_t total;
-        const uint64_t mine = cnt[threadIdx.x];
         const uint64_t pre = block_excl_scan_u64<kThr>(mine, &total, scan_sh);
         if (c < nchunks) {
             const int64_t gt_before = run_gt + (pre & 0xffffffffu);
@@ -167,11 +175,6 @@ constexpr int kCW = 8;                          // compaction: warps per block
 constexpr int kCThr = 32 * kCW;
 constexpr int kKeys = CHUNK / kCThr;            // 32 consecutive keys per thread
 static_assert(kKeys == 32, "one 32-key run per thread");
-
-// Bytes 0,1 / 2,3 of a word spread into the 16-bit lanes of a 32-bit word.
-__device__ __forceinline__ uint64_t spread_bytes(uint32_t x) {
-    return (static_cast<uint64_t>(prmt_i<0x5352u>(x, 0u)) << 32) | prmt_i<0x5150u>(x, 0u);
-}
 
 // Block-wide exclusive scan of two 64-bit values at once (4 packed 16-bit counters each,
 // none of which overflows: a block's total per counter is at most CHUNK = 8192).
@@ -232,72 +235,74 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
         gt_add |= static_cast<uint32_t>(127 - T) << (8 * h);
         ge_add |= static_cast<uint32_t>(128 - T) << (8 * h);
     }
-    // counting pass: keys above T and ties, per head in byte counters (at most 32 each),
-    // and the mask of keys that reach T for some head (the only ones the write pass visits)
-    uint32_t gcnt = 0, ecnt = 0, reach = 0;
-#pragma unroll 8
-    for (int j = 0; j < kKeys; ++j) {
-        const uint32_t m = j < nv ? 0x01010101u : 0u;
-        const uint32_t g = ((s[j] + gt_add) >> 7) & m;
-        const uint32_t ge = ((s[j] + ge_add) >> 7) & m;
-        gcnt += g;
-        ecnt += ge ^ g;
-        reach |= (ge != 0u ? 1u : 0u) << j;
+    // Bit-sliced tests: word q of G (GE) holds, in byte h, bit i = key 8 q + i has
+    // score_h > T_h (>= T_h). Then per head a 32-bit mask over the thread's keys.
+    uint32_t G[4], GE[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t a = 0, b = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t sv = s[8 * q + i];
+            a |= (((sv + gt_add) >> 7) & 0x01010101u) << i;
+            b |= (((sv + ge_add) >> 7) & 0x01010101u) << i;
+        }
+        G[q] = a;
+        GE[q] = b;
     }
-    uint64_t gb = spread_bytes(gcnt), eb = spread_bytes(ecnt);
+    const uint32_t vbits = nv >= 32 ? 0xffffffffu : ((1u << nv) - 1u);
+    uint32_t gm[PACK], em[PACK];
+#define PKV_HEAD_MASK(W, H)                                                              \
+    (prmt_i<0x5410u>(prmt_i<((4u + (H)) << 4) | (H)>(W[0], W[1]),                      \
+                     prmt_i<((4u + (H)) << 4) | (H)>(W[2], W[3])))
+    gm[0] = PKV_HEAD_MASK(G, 0) & vbits;  em[0] = PKV_HEAD_MASK(GE, 0) & vbits & ~gm[0];
+    gm[1] = PKV_HEAD_MASK(G, 1) & vbits;  em[1] = PKV_HEAD_MASK(GE, 1) & vbits & ~gm[1];
+    gm[2] = PKV_HEAD_MASK(G, 2) & vbits;  em[2] = PKV_HEAD_MASK(GE, 2) & vbits & ~gm[2];
+    gm[3] = PKV_HEAD_MASK(G, 3) & vbits;  em[3] = PKV_HEAD_MASK(GE, 3) & vbits & ~gm[3];
+#undef PKV_HEAD_MASK
+    uint64_t gb = 0, eb = 0;
+#pragma unroll
+    for (int h = 0; h < PACK; ++h) {
+        gb |= static_cast<uint64_t>(__popc(gm[h])) << (16 * h);
+        eb |= static_cast<uint64_t>(__popc(em[h])) << (16 * h);
+    }
     block_excl_scan2(gb, eb, scan_sh);   // keys above T / ties in this chunk before this thread
 
-    // where this thread's candidates start, and how many of its ties it keeps: the chunk
-    // keeps the first B = max(0, E - ties before the chunk) of its ties, in key order
-    int32_t* out[PACK];
-    uint32_t run[PACK], budget[PACK];
-    uint32_t all_ties = 0, partial = 0;
+    // Per head: where this thread's candidates start, and which of its ties it keeps: the
+    // chunk keeps the first B = max(0, E - ties before the chunk) of its ties, in key order.
+    // Then its candidates are written in key order.
     const int32_t C = thr[head0 * 4 + 2];
 #pragma unroll
     for (int h = 0; h < PACK; ++h) {
-        out[h] = cand + static_cast<int64_t>(head0 + min(h, hp - 1)) * cmax;
-        run[h] = 0;
-        budget[h] = 0;
-        if (h >= hp) continue;
+        if (h >= hp) break;
         const int64_t hb = (static_cast<int64_t>(head0 + h) * nchunks + c) * 2;
         const int64_t E = thr[(head0 + h) * 4 + 1];
         const int64_t B = max64(0, E - cbase[hb + 1]);
         const int64_t gbefore = (gb >> (16 * h)) & 0xffffu, ebefore = (eb >> (16 * h)) & 0xffffu;
-        const int64_t mine_g = (gcnt >> (8 * h)) & 0xffu, mine_e = (ecnt >> (8 * h)) & 0xffu;
-        const int64_t take = min64(max64(B - ebefore, 0), mine_e);
-        const int64_t start = cbase[hb + 0] + gbefore + min64(B, ebefore);
-        if (start + mine_g + take > C) {   // never taken when the histograms are consistent
-            atomicExch(status, ST_BADINDEX);
-            return;
-        }
-        run[h] = static_cast<uint32_t>(start);
-        budget[h] = static_cast<uint32_t>(take);
-        if (take == mine_e) all_ties |= 1u << (8 * h);
-        else if (take > 0) partial |= 1u << (8 * h);
-    }
-
-    // write pass over the keys that reach T, in key order
-    while (reach) {
-        const int j = __ffs(reach) - 1;
-        reach &= reach - 1u;
-        const uint32_t sv = s[j];
-        const uint32_t g = (sv + gt_add) >> 7 & 0x01010101u;
-        const uint32_t e = ((sv + ge_add) >> 7 & 0x01010101u) ^ g;
-        uint32_t sel = g | (e & all_ties);
-        if (partial) {                       // the one thread per head where the E-th tie falls
-#pragma unroll
-            for (int h = 0; h < PACK; ++h) {
-                if (((partial & e) >> (8 * h)) & 1u) {
-                    if (budget[h] > 0) { sel |= 1u << (8 * h); --budget[h]; }
-                }
+        const int mine_e = __popc(em[h]);
+        const int take = static_cast<int>(min64(max64(B - ebefore, 0), mine_e));
+        uint32_t sel = gm[h];
+        if (take == mine_e) {
+            sel |= em[h];
+        } else {                              // the one thread where the E-th tie falls
+            uint32_t m = em[h];
+            for (int t = 0; t < take; ++t) {
+                const uint32_t low = m & (0u - m);
+                sel |= low;
+                m ^= low;
             }
         }
-        const int32_t key = static_cast<int32_t>(k0 + j);
-#pragma unroll
-        for (int h = 0; h < PACK; ++h) {
-            const uint32_t b = (sel >> (8 * h)) & 1u;
-            if (b) out[h][run[h]] = key;
-            run[h] += b;
+        const int64_t start = cbase[hb + 0] + gbefore + min64(B, ebefore);
+        if (start + __popc(sel) > C) {       // never taken when the histograms are consistent
+            atomicExch(status, ST_BADINDEX);
+            continue;
+        }
+        int32_t* out = cand + static_cast<int64_t>(head0 + h) * cmax + start;
+        const int32_t kbase = static_cast<int32_t>(k0);
+        while (sel) {
+            const int j = __ffs(sel) - 1;
+            sel &= sel - 1u;
+            *out++ = kbase + j;
         }
     }
 }

@@ -149,8 +149,18 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
         }
         if (lane == 0) wa[warp] = x;   // warp totals
         __syncthreads();
-        uint32_t later = 0;            // bins of later warps
-        for (int w = warp + 1; w < kWarps; ++w) later += wa[w];
+        if (warp == 0) {               // exclusive suffix sums of the warp totals
+            const uint32_t t = wa[lane];
+            uint32_t y = t;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t z = __shfl_down_sync(0xffffffffu, y, o);
+                if (lane + o < 32) y += z;
+            }
+            wb[lane] = y - t;
+        }
+        __syncthreads();
+        const uint32_t later = wb[warp];                // bins of later warps
         const uint32_t above1 = later + x - (h0 + h1);  // strictly above bin 2t + 1
         const uint32_t above0 = above1 + h1;             // strictly above bin 2t
         if (above1 < krem && krem <= above1 + h1) { pick[0] = 2 * threadIdx.x + 1; pick[1] = above1; }
