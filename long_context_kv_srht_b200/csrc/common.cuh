@@ -15,7 +15,7 @@ constexpr int NB = D / M;       // subspaces (16)
 constexpr int NC = 1 << M;      // sign centroids per subspace (256)
 constexpr int REC = 128;        // bytes per key record: 64 B of 4-bit codes + 16 fp32 factors
 constexpr int NBINS = 64;       // coarse scores are < 64 (B * w_rank1 <= 48)
-constexpr int CHUNK = 8192;     // keys per coarse-score histogram chunk
+constexpr int CHUNK = 8192;     // keys per coarse-score histogram chunk (a vote work item)
 constexpr int PACK = 4;         // query heads whose vote weights share one 32-bit table entry
 
 enum : int { ST_OK = 0, ST_TIMEOUT = 5, ST_BADINDEX = 6 };
@@ -62,6 +62,17 @@ __device__ __forceinline__ uint32_t prmt_i(uint32_t a, uint32_t b) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "n"(SEL));
     return r;
+}
+
+// Programmatic dependent launch. A search kernel is launched so that it may start while
+// the previous kernel of the stream is finishing; pdl_wait() blocks until that kernel has
+// completed and its writes are visible (every kernel calls it before reading the previous
+// kernel's results and before any global write), and pdl_launch_dependents() then lets the
+// next kernel begin launching. Because every kernel triggers only after its own wait, a
+// kernel that has started may read anything written before its immediate predecessor.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {

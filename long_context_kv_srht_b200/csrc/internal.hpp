@@ -60,6 +60,23 @@ cudaError_t raise_smem_limit(Kern kernel, int bytes, std::atomic<uint64_t>& done
     return e;
 }
 
+// Launches a search kernel with programmatic stream serialization (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // status helpers (defined in api.cu)
 pariskv_status fail(pariskv_status s, const char* fmt, ...);
 pariskv_status cuda_fail(cudaError_t e, const char* what);

@@ -36,6 +36,8 @@ query_prep_kernel(const T* __restrict__ q, const float* __restrict__ qt_in,
     const int unit = head / group, g = head % group;
     const int pack = g / PACK, slot = g % PACK;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_launch_dependents();
 
     if (warp == 0) {
         float v[4];
@@ -129,18 +131,18 @@ cudaError_t launch_query_prep(const pariskv_index* ix, const void* q, const floa
     const int heads = ix->units * c.group;
     uint8_t* lut8 = reinterpret_cast<uint8_t*>(ix->lut);
     if (rotated)
-        query_prep_kernel<float, true><<<heads, 256, 0, st>>>(
-            nullptr, qt_in, qn_in, ix->signs, c.group, ix->packs, c.rho, c.w_rank1, c.w_rest,
-            ix->qt, ix->qnorm, lut8);
+        return launch_pdl(query_prep_kernel<float, true>, heads, 256, 0, st, nullptr, qt_in,
+                          qn_in, ix->signs, c.group, ix->packs, c.rho, c.w_rank1, c.w_rest,
+                          ix->qt, ix->qnorm, lut8);
     else if (c.dtype == PARISKV_BF16)
-        query_prep_kernel<__nv_bfloat16, false><<<heads, 256, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(q), nullptr, nullptr, ix->signs, c.group,
-            ix->packs, c.rho, c.w_rank1, c.w_rest, ix->qt, ix->qnorm, lut8);
+        return launch_pdl(query_prep_kernel<__nv_bfloat16, false>, heads, 256, 0, st,
+                          static_cast<const __nv_bfloat16*>(q), nullptr, nullptr, ix->signs,
+                          c.group, ix->packs, c.rho, c.w_rank1, c.w_rest, ix->qt, ix->qnorm,
+                          lut8);
     else
-        query_prep_kernel<float, false><<<heads, 256, 0, st>>>(
-            static_cast<const float*>(q), nullptr, nullptr, ix->signs, c.group, ix->packs,
-            c.rho, c.w_rank1, c.w_rest, ix->qt, ix->qnorm, lut8);
-    return cudaGetLastError();
+        return launch_pdl(query_prep_kernel<float, false>, heads, 256, 0, st,
+                          static_cast<const float*>(q), nullptr, nullptr, ix->signs, c.group,
+                          ix->packs, c.rho, c.w_rank1, c.w_rest, ix->qt, ix->qnorm, lut8);
 }
 
 }  // namespace pkv

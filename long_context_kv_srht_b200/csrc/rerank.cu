@@ -13,7 +13,7 @@
 // only delivers its bandwidth with far more bytes in flight than registers can hold. So the
 // records are gathered with asynchronous global->shared copies (cp.async, 16 bytes per lane;
 // eight lanes move one record, so one warp instruction moves four whole records): the kernel
-// is persistent (two CTAs per SM), every warp owns a ring of kSlots stages of 32 records, and
+// is persistent (kCtasPerSm CTAs per SM), every warp owns a ring of kSlots stages of 32 records, and
 // a stage is refilled as soon as it has been scored. Piece c of the record in stage row r is
 // stored at 16-byte position c ^ (r mod 8), so that eight lanes reading the same piece of
 // eight different records touch all 32 banks once.
@@ -32,9 +32,10 @@ namespace pkv {
 
 namespace {
 
-constexpr int kWarps = 8;               // two persistent CTAs per SM; every warp gathers and scores
+constexpr int kWarps = 8;               // every warp gathers and scores
+constexpr int kCtasPerSm = 3;           // persistent CTAs per SM
 constexpr int kThr = 32 * kWarps;
-constexpr int kSlots = 3;               // stages in flight per warp
+constexpr int kSlots = 2;               // stages in flight per warp
 constexpr int kStageRecs = 32;          // records per stage: one per lane
 constexpr int kStageBytes = kStageRecs * REC;
 constexpr int kQBytes = D * 4;          // one head's rotated query
@@ -118,7 +119,7 @@ struct StreamPos {
     const uint8_t* ubase;  // records of the head's unit
 };
 
-__global__ void __launch_bounds__(kThr, 2)
+__global__ void __launch_bounds__(kThr, kCtasPerSm)
 rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
               const float* __restrict__ qt, float* __restrict__ S, int32_t C, int64_t cmax,
               int64_t cap_pad, int64_t n, int group, int iph, int64_t items, int* status) {
@@ -145,16 +146,20 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
             start_item(p);
         }
     };
-    // stage refill: lane l looks up the record of candidate c0 + 32 s + l; for copy
-    // instruction j, lanes 8g..8g+7 move the 8 16-byte pieces of record 4j + g
-    auto issue = [&](int slot, const StreamPos& p) {
+    // candidate index of this lane's record in the stage at p (loaded one stage ahead of its
+    // use, so the load overlaps the scoring of a stage)
+    auto load_idx = [&](const StreamPos& p) -> uint32_t {
+        if (p.it >= items) return kNoRec;
+        const int c = p.c0 + 32 * p.s + lane;
+        return c < p.cend ? static_cast<uint32_t>(cand[p.head * cmax + c]) : kNoRec;
+    };
+    // stage refill: lane l holds the index of the stage's l-th record; for copy instruction
+    // j, lanes 8g..8g+7 move the 8 16-byte pieces of record 4j + g
+    auto issue = [&](int slot, const StreamPos& p, uint32_t idx) {
         if (p.it < items) {
-            const int c = p.c0 + 32 * p.s + lane;
-            uint32_t idx = kNoRec;
-            if (c < p.cend) {
-                const int32_t i = cand[p.head * cmax + c];
-                if (i >= 0 && i < n) idx = static_cast<uint32_t>(i);
-                else atomicExch(status, ST_BADINDEX);  // never taken when the selection is consistent
+            if (idx != kNoRec && idx >= static_cast<uint64_t>(n)) {
+                atomicExch(status, ST_BADINDEX);  // never taken when the selection is consistent
+                idx = kNoRec;
             }
             uint8_t* dst0 = ring + slot * kStageBytes;
             const int piece = lane & 7, sub = lane >> 3;
@@ -173,13 +178,17 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
+    pdl_wait();
+    pdl_launch_dependents();
     StreamPos iss{gw, 0, 0, 0, 0, 0, rec}, sc{gw, 0, 0, 0, 0, 0, rec};
     start_item(iss);
     start_item(sc);
     // prologue: fill the ring
+    uint32_t pend = load_idx(iss);
     for (int g = 0; g < kSlots; ++g) {
-        issue(g, iss);
+        issue(g, iss, pend);
         if (iss.it < items) advance(iss);
+        pend = load_idx(iss);
     }
 
     int staged = -1;   // head whose query is in qs
@@ -197,8 +206,9 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
         const int c = sc.c0 + 32 * sc.s + lane;
         if (c < sc.cend) S[sc.head * cmax + c] = score_record(ring + slot * kStageBytes, lane, qp);
         __syncwarp();                        // every lane has read the slot and the query
-        issue(slot, iss);
+        issue(slot, iss, pend);
         if (iss.it < items) advance(iss);
+        pend = load_idx(iss);
         advance(sc);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");   // no copy in flight at exit
@@ -217,11 +227,11 @@ cudaError_t launch_rerank(const pariskv_index* ix, int64_t C, cudaStream_t st) {
     const int heads = ix->units * ix->cfg.group;
     const int iph = static_cast<int>(ceil_div(C, kItem));
     const int64_t items = static_cast<int64_t>(heads) * iph;
-    const int grid = static_cast<int>(max64(1, min64(2LL * sms, ceil_div(items, kWarps))));
-    rerank_kernel<<<grid, kThr, kSmem, st>>>(ix->rec, ix->cand, ix->qt, ix->S,
-                                             static_cast<int32_t>(C), ix->cmax, ix->cap_pad,
-                                             ix->n, ix->cfg.group, iph, items, ix->status);
-    return cudaGetLastError();
+    const int grid =
+        static_cast<int>(max64(1, min64(int64_t{kCtasPerSm} * sms, ceil_div(items, kWarps))));
+    return launch_pdl(rerank_kernel, grid, kThr, kSmem, st, ix->rec, ix->cand, ix->qt, ix->S,
+                      static_cast<int32_t>(C), ix->cmax, ix->cap_pad, ix->n, ix->cfg.group, iph,
+                      items, ix->status);
 }
 
 }  // namespace pkv

@@ -32,7 +32,7 @@ namespace {
 constexpr int kThr = 256;                  // threshold kernel
 
 // Block-wide exclusive scan of a 64-bit value (4 packed 16-bit counters in the compaction,
-// none of which overflows because a block's total per counter is at most CHUNK = 8192).
+// none of which overflows because a block's total per counter is at most CHUNK).
 // Returns the exclusive prefix; *total receives the block total. All threads must call it.
 template <int NT>
 __device__ __forceinline__ uint64_t block_excl_scan_u64(uint64_t v, uint64_t* total,
@@ -75,6 +75,8 @@ threshold_kernel(const uint32_t* __restrict__ hist, int group, int packs, int64_
     const int h = g % PACK;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t* hb = hist + up * nchunks * (PACK * NBINS) + h * NBINS;
+    pdl_wait();
+    pdl_launch_dependents();
 
     // total histogram: thread t sums bin t % 64 over chunks t / 64, t / 64 + 4, ... (the
     // loads are independent, so they are all in flight together)
@@ -171,13 +173,13 @@ threshold_kernel(const uint32_t* __restrict__ hist, int group, int packs, int64_
     }
 }
 
-constexpr int kCW = 8;                          // compaction: warps per block
+constexpr int kCW = CHUNK / (32 * 32);          // compaction: warps per block (one chunk)
 constexpr int kCThr = 32 * kCW;
 constexpr int kKeys = CHUNK / kCThr;            // 32 consecutive keys per thread
 static_assert(kKeys == 32, "one 32-key run per thread");
 
 // Block-wide exclusive scan of two 64-bit values at once (4 packed 16-bit counters each,
-// none of which overflows: a block's total per counter is at most CHUNK = 8192).
+// none of which overflows: a block's total per counter is at most CHUNK).
 __device__ __forceinline__ void block_excl_scan2(uint64_t& a, uint64_t& b,
                                                  uint64_t (*sh)[2] /* [kCW + 1][2] */) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -224,6 +226,10 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
         __syncwarp();
     }
     const uint32_t* s = &tr[warp][lane * 33];
+    // the scores above were written two kernels back; thresholds and offsets come from the
+    // threshold kernel just before this one
+    pdl_wait();
+    pdl_launch_dependents();
 
     // Per-head thresholds packed one per byte. A head outside the pack gets T = 127, which
     // no score (< 64) reaches. Byte h of (s + gt_add) has bit 7 set iff score_h > T_h, and
@@ -312,18 +318,16 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
 cudaError_t launch_threshold(const pariskv_index* ix, int64_t C, cudaStream_t st) {
     const int64_t nchunks = ceil_div(ix->n, CHUNK);
     const int heads = ix->units * ix->cfg.group;
-    threshold_kernel<<<heads, kThr, 0, st>>>(ix->hist, ix->cfg.group, ix->packs, nchunks, C,
-                                             ix->thr, ix->cbase);
-    return cudaGetLastError();
+    return launch_pdl(threshold_kernel, heads, kThr, 0, st, ix->hist, ix->cfg.group, ix->packs,
+                      nchunks, C, ix->thr, ix->cbase);
 }
 
 cudaError_t launch_compact(const pariskv_index* ix, cudaStream_t st) {
     const int64_t nchunks = ceil_div(ix->n, CHUNK);
     dim3 grid(static_cast<unsigned>(nchunks), static_cast<unsigned>(ix->units * ix->packs));
-    compact_kernel<<<grid, kCThr, 0, st>>>(ix->scores, ix->thr, ix->cbase, ix->cand, ix->n,
-                                          ix->cap_pad, ix->cfg.group, ix->packs, nchunks,
-                                          ix->cmax, ix->status);
-    return cudaGetLastError();
+    return launch_pdl(compact_kernel, grid, kCThr, 0, st, ix->scores, ix->thr, ix->cbase,
+                      ix->cand, ix->n, ix->cap_pad, ix->cfg.group, ix->packs, nchunks, ix->cmax,
+                      ix->status);
 }
 
 }  // namespace pkv

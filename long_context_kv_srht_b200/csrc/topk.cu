@@ -8,9 +8,9 @@
 //
 // Exact selection on the order-preserving 32-bit image u of S (flip all bits of negative
 // values, set the sign bit of the others), by a cluster of four CTAs per query head:
-//  - CTA r loads the r-th quarter of the head's S values (as u) and candidate indices into
-//    shared memory with coalesced loads (quarters longer than kSlice stay in global memory
-//    and are re-read on every pass);
+//  - CTA r copies the r-th quarter of the head's S values and candidate indices into shared
+//    memory with asynchronous copies, all in flight at once, and turns S into u in place
+//    (quarters longer than kSlice stay in global memory and are re-read on every pass);
 //  - the cluster agrees on [min, max] of u through distributed shared memory;
 //  - range-adaptive radix levels: the current interval [lo, hi] is cut into at most 2048
 //    power-of-two-wide bins, every CTA histograms its quarter, and every CTA sums the four
@@ -73,16 +73,26 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
     int32_t* idx = reinterpret_cast<int32_t*>(dyn + kSlice);  // [kSlice] candidate index
     auto key_at = [&](int i) -> uint32_t { return RES ? keys[i] : order_key(Sh[i]); };
     auto idx_at = [&](int i) -> int32_t { return RES ? idx[i] : ch[i]; };
+    pdl_wait();
+    pdl_launch_dependents();
 
-    // 1. the quarter into shared memory; local min / max
+    // 1. the quarter into shared memory (asynchronous 4-byte copies, all in flight at once);
+    //    then u in place and the local min / max
+    if (RES) {
+        for (int i = threadIdx.x; i < L; i += kT) {
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(keys + i)),
+                         "l"(Sh + i) : "memory");
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(idx + i)),
+                         "l"(ch + i) : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_all;" ::: "memory");
+    }
     uint32_t mn = 0xffffffffu, mx = 0u;
 #pragma unroll 4
     for (int i = threadIdx.x; i < L; i += kT) {
-        const uint32_t u = order_key(Sh[i]);
-        if (RES) {
-            keys[i] = u;
-            idx[i] = ch[i];
-        }
+        const uint32_t u = RES ? order_key(__uint_as_float(keys[i])) : order_key(Sh[i]);
+        if (RES) keys[i] = u;   // each thread converts the entries it copied itself
         mn = min(mn, u);
         mx = max(mx, u);
     }
@@ -245,15 +255,14 @@ cudaError_t launch_topk(const pariskv_index* ix, int64_t C, int32_t k, int32_t* 
         return e;
     const int heads = ix->units * ix->cfg.group;
     if (ceil_div(C, kCL) <= kSlice) {
-        topk_kernel<true><<<heads * kCL, kT, kDyn, st>>>(ix->S, ix->cand, ix->qnorm,
-                                                         static_cast<int32_t>(C), ix->cmax, k,
-                                                         topk_idx, topk_est, ix->status);
+        return launch_pdl(topk_kernel<true>, heads * kCL, kT, kDyn, st, ix->S, ix->cand,
+                          ix->qnorm, static_cast<int32_t>(C), ix->cmax, k, topk_idx, topk_est,
+                          ix->status);
     } else {
-        topk_kernel<false><<<heads * kCL, kT, 0, st>>>(ix->S, ix->cand, ix->qnorm,
-                                                       static_cast<int32_t>(C), ix->cmax, k,
-                                                       topk_idx, topk_est, ix->status);
+        return launch_pdl(topk_kernel<false>, heads * kCL, kT, 0, st, ix->S, ix->cand,
+                          ix->qnorm, static_cast<int32_t>(C), ix->cmax, k, topk_idx, topk_est,
+                          ix->status);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace pkv

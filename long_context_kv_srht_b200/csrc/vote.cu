@@ -9,16 +9,18 @@
 // streamed once per KV head and scored for all query heads of its GQA group at once.
 //
 // Design (sm_100a, HBM-bound):
-//  - Each lane scores two consecutive keys of a 64-key warp-tile, reading their 32 bytes of
-//    ids with one 256-bit non-allocating load; the next tile's ids are loaded while the
-//    current one is scored. Measured on B200, 256-bit loads stream at full HBM bandwidth;
-//    a cp.async.bulk ring refilled only once all warps had released a stage stayed far below.
+//  - Lane L scores keys L and L + 32 of a 64-key warp-tile, reading their ids with two
+//    128-bit non-allocating loads (each a fully coalesced 512-byte warp access, the fewest L1
+//    wavefronts per byte); the next tile's ids are loaded while the current one is scored.
+//    (Measured on B200: a cp.async.bulk ring refilled only once all warps had released a
+//    stage stayed far below HBM bandwidth.)
 //  - The 32-bit table entry packs the vote weights of up to four query heads (one byte each;
 //    a byte sum never exceeds 48), so one lookup per (key, subspace) serves the whole pack.
 //  - Conflict-free lookups: the table holds two copies of every subspace's 256 entries, and
 //    subspace b / copy k owns shared-memory bank 2b + k (entry c of it at row c, 256-byte
-//    rows). Because the encoder stores subspace b of key i at byte (b - i / 2) mod 16, at
-//    step t lane L reads subspace (t + L) mod 16 from byte t of each of its keys; the 32 lanes
+//    rows). Because the encoder stores subspace b of key i at byte (b - i / 2) mod 16, and
+//    keys L and L + 32 of a tile share (i / 2) mod 16 = L / 2, at step t lane L reads
+//    subspace (t + L / 2) mod 16 from byte t of both its keys, in copy L mod 2; the 32 lanes
 //    then touch 32 distinct banks. One PRMT builds the address (row = id byte, column from a
 //    per-lane constant), one LDS reads the entry, one add accumulates.
 //  - Histograms of the packed scores (64 bins per query head) are built in the upper half of
@@ -46,7 +48,16 @@ __device__ __forceinline__ uint32_t tab_ld(const uint8_t* tab, uint32_t off) {
     return *reinterpret_cast<const uint32_t*>(tab + off);
 }
 
-__device__ __forceinline__ u32x8 ldg_ids(const uint8_t* p) { return ldg_stream_u256(p); }
+// The ids of keys L and L + 32 of a 64-key tile (lane L): two 128-bit non-allocating loads,
+// each a fully coalesced 512-byte warp access.
+__device__ __forceinline__ u32x8 ldg_ids(const uint8_t* p) {
+    u32x8 v;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]) : "l"(p));
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(v.w[4]), "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7]) : "l"(p + 512));
+    return v;
+}
 
 // Table entry of step t: byte0 <- column (byte t % 3 of colp[t / 3]), byte1 <- id byte t % 4,
 // bytes 2, 3 <- the zero top byte of colp[t / 3].
@@ -90,10 +101,10 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
     const int64_t i0 = items * blockIdx.x / gridDim.x;
     const int64_t i1 = items * (blockIdx.x + 1) / gridDim.x;
 
-    // Per-lane address parts: at step t lane L reads subspace (t + L) mod 16 of both its keys
-    // (the encoder rotates key i's bytes by (i / 2) mod 16), whose copy (L >> 4) owns bank
-    // column 2 * subspace + copy. Three columns per register with a zero top byte, so one
-    // PRMT builds an address.
+    // Per-lane address parts: at step t lane L reads subspace (t + L / 2) mod 16 of both its
+    // keys (the encoder rotates key i's bytes by (i / 2) mod 16), in copy L mod 2, which owns
+    // bank column 2 * subspace + copy. Three columns per register with a zero top byte, so
+    // one PRMT builds an address.
     uint32_t colp[6];
 #pragma unroll
     for (int r = 0; r < 6; ++r) {
@@ -101,7 +112,7 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
             const int t = 3 * r + j;
-            if (t < 16) w |= (4u * (2u * ((t + lane) & 15) + (lane >> 4))) << (8 * j);
+            if (t < 16) w |= (4u * (2u * ((t + (lane >> 1)) & 15) + (lane & 1))) << (8 * j);
         }
         colp[r] = w;
     }
@@ -114,13 +125,16 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
     auto item_ids = [&](int64_t item) -> const uint8_t* {
         const int64_t up = item / nchunks, c = item - (item / nchunks) * nchunks;
         const int64_t unit = up / packs;
-        return ids + (unit * cap_pad + c * CHUNK) * 16 + lane * 32;
+        return ids + (unit * cap_pad + c * CHUNK) * 16 + lane * 16;
     };
     constexpr int kTileBytes = kTileKeys * 16;
     int64_t cur_up = -1;
     u32x8 nxt;
     const uint8_t* base = i0 < i1 ? item_ids(i0) : ids;
     if (i0 < i1) nxt = ldg_ids(base + warp * kTileBytes);
+    // the ids were written before the query kernel; its table is read only after the wait
+    pdl_wait();
+    pdl_launch_dependents();
     for (int64_t item = i0; item < i1; ++item) {
         const int64_t up = item / nchunks, c = item - up * nchunks;
         const int hp = min(PACK, group - static_cast<int>(up % packs) * PACK);
@@ -149,15 +163,13 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
             uint32_t acc[2];
 #pragma unroll
             for (int j = 0; j < 2; ++j) acc[j] = score_key(tab, cur.w + 4 * j, colp);
-            const int kk = tl * kTileKeys + 2 * lane;
-            if (kk + 1 < nkeys) {
-                *reinterpret_cast<uint2*>(sc_out + kk) = make_uint2(acc[0], acc[1]);
-            } else if (kk < nkeys) {
-                sc_out[kk] = acc[0];
-            }
+            const int kk = tl * kTileKeys + lane;    // keys kk and kk + 32
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+                if (kk + 32 * j < nkeys) sc_out[kk + 32 * j] = acc[j];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                if (kk + j < nkeys) {
+                if (kk + 32 * j < nkeys) {
                     const uint32_t sc = acc[j] + 0xC0804000u;  // byte h -> 64 h + score_h
                     hist_inc<0>(tab, sc, hcol);
                     if (hp > 1) hist_inc<1>(tab, sc, hcol);
@@ -192,10 +204,9 @@ cudaError_t launch_vote(const pariskv_index* ix, cudaStream_t st) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = static_cast<int>(min64(items, 2LL * sms));
-    vote_kernel<<<grid, kThreads, kSmemBytes, st>>>(ix->ids, ix->lut, ix->scores, ix->hist,
-                                                   ix->n, ix->cap_pad, ix->packs,
-                                                   ix->cfg.group, nchunks, items, ix->status);
-    return cudaGetLastError();
+    return launch_pdl(vote_kernel, grid, kThreads, kSmemBytes, st, ix->ids, ix->lut, ix->scores,
+                      ix->hist, ix->n, ix->cap_pad, ix->packs, ix->cfg.group, nchunks, items,
+                      ix->status);
 }
 
 }  // namespace pkv
