@@ -136,20 +136,22 @@ def measured_peaks():
 
 
 def kernel_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, only while the kernel source is
-    unchanged since the capture (its sha256 is stored next to the figure)."""
+    """DRAM bytes per launch from the committed ncu summary, only while the kernel's source
+    and the shared device headers are unchanged since the capture (their sha256 is stored
+    next to the figure)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    e = d.get(kernel, {}).get(workload)
+    e = d.get("kernels", {}).get(kernel, {}).get(workload)
     if not e:
         return None
-    src = os.path.join(ROOT, "long_context_kv_srht_b200", "csrc", e["source"])
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
-    return e["dram_bytes_per_launch"] if sha == e["sha256"] else None
+    h = hashlib.sha256()
+    for name in e["sources"]:
+        with open(os.path.join(ROOT, "long_context_kv_srht_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return e["dram_bytes_per_launch"] if h.hexdigest() == e["sha256"] else None
 
 
 def algorithmic_bytes(stage: str, sp, C: int) -> int:
