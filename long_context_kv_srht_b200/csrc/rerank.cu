@@ -13,12 +13,13 @@
 // only delivers its bandwidth with far more bytes in flight than registers can hold. So the
 // records are gathered with asynchronous global->shared copies (cp.async, 16 bytes per lane;
 // eight lanes move one record, so one warp instruction moves four whole records): the kernel
-// is persistent (kCtasPerSm CTAs per SM), every warp owns a ring of kSlots stages of 32 records, and
-// a stage is refilled as soon as it has been scored. Piece c of the record in stage row r is
+// is persistent (kCtasPerSm CTAs per SM), every warp owns a ring of kSlots stages of 64
+// records, and a stage is refilled as soon as it has been scored. Piece c of the record in stage row r is
 // stored at 16-byte position c ^ (r mod 8), so that eight lanes reading the same piece of
 // eight different records touch all 32 banks once.
 //
-// Scoring: one lane per record. The warp's current query head has its rotated query in
+// Scoring: each lane scores two records of a stage (rows lane and lane + 32, whose chains
+// interleave). The warp's current query head has its rotated query in
 // shared memory as (subspace 2t, subspace 2t + 1) fp32 pairs, read with broadcast loads; a
 // lane walks the 8 subspace pairs in order, two p chains advancing together in Blackwell's
 // packed fp32x2 FMA (each half an ordinary IEEE fp32 FMA), and extends its S chain after
@@ -32,11 +33,12 @@ namespace pkv {
 
 namespace {
 
-constexpr int kWarps = 8;               // every warp gathers and scores
+constexpr int kWarps = 4;               // every warp gathers and scores
 constexpr int kCtasPerSm = 3;           // persistent CTAs per SM
 constexpr int kThr = 32 * kWarps;
 constexpr int kSlots = 2;               // stages in flight per warp
-constexpr int kStageRecs = 32;          // records per stage: one per lane
+constexpr int kPerLane = 2;             // records scored per lane and stage
+constexpr int kStageRecs = 32 * kPerLane;
 constexpr int kStageBytes = kStageRecs * REC;
 constexpr int kQBytes = D * 4;          // one head's rotated query
 constexpr int kWarpBytes = kSlots * kStageBytes + kQBytes;
@@ -136,7 +138,7 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
         p.head = static_cast<int>(p.it / iph);
         p.c0 = static_cast<int>(p.it - static_cast<int64_t>(p.head) * iph) * kItem;
         p.cend = min(C, p.c0 + kItem);
-        p.nst = (p.cend - p.c0 + 31) >> 5;
+        p.nst = (p.cend - p.c0 + kStageRecs - 1) / kStageRecs;
         p.s = 0;
         p.ubase = rec + static_cast<int64_t>(p.head / group) * cap_pad * REC;
     };
@@ -146,27 +148,36 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
             start_item(p);
         }
     };
-    // candidate index of this lane's record in the stage at p (loaded one stage ahead of its
-    // use, so the load overlaps the scoring of a stage)
-    auto load_idx = [&](const StreamPos& p) -> uint32_t {
-        if (p.it >= items) return kNoRec;
-        const int c = p.c0 + 32 * p.s + lane;
-        return c < p.cend ? static_cast<uint32_t>(cand[p.head * cmax + c]) : kNoRec;
+    // candidate indices of this lane's records (rows lane, lane + 32) in the stage at p,
+    // loaded one stage ahead of their use so the loads overlap the scoring of a stage
+    struct Idx { uint32_t v[kPerLane]; };
+    auto load_idx = [&](const StreamPos& p) -> Idx {
+        Idx r;
+#pragma unroll
+        for (int u = 0; u < kPerLane; ++u) {
+            const int c = p.c0 + kStageRecs * p.s + 32 * u + lane;
+            r.v[u] = (p.it < items && c < p.cend) ? static_cast<uint32_t>(cand[p.head * cmax + c])
+                                                  : kNoRec;
+        }
+        return r;
     };
-    // stage refill: lane l holds the index of the stage's l-th record; for copy instruction
-    // j, lanes 8g..8g+7 move the 8 16-byte pieces of record 4j + g
-    auto issue = [&](int slot, const StreamPos& p, uint32_t idx) {
+    // stage refill: for copy instruction j, lanes 8g..8g+7 move the 8 16-byte pieces of
+    // record 4j + g (whose index lane (4j + g) mod 32 holds)
+    auto issue = [&](int slot, const StreamPos& p, Idx idx) {
         if (p.it < items) {
-            if (idx != kNoRec && idx >= static_cast<uint64_t>(n)) {
-                atomicExch(status, ST_BADINDEX);  // never taken when the selection is consistent
-                idx = kNoRec;
+#pragma unroll
+            for (int u = 0; u < kPerLane; ++u) {
+                if (idx.v[u] != kNoRec && idx.v[u] >= static_cast<uint64_t>(n)) {
+                    atomicExch(status, ST_BADINDEX);  // never taken when the selection is consistent
+                    idx.v[u] = kNoRec;
+                }
             }
             uint8_t* dst0 = ring + slot * kStageBytes;
             const int piece = lane & 7, sub = lane >> 3;
 #pragma unroll
             for (int j = 0; j < kStageRecs / 4; ++j) {
                 const int rr = 4 * j + sub;
-                const uint32_t ri = __shfl_sync(0xffffffffu, idx, rr);
+                const uint32_t ri = __shfl_sync(0xffffffffu, idx.v[j / 8], rr & 31);
                 if (ri != kNoRec) {
                     const uint32_t dst = smem_addr(dst0 + piece_at(rr, piece));
                     const uint8_t* src = p.ubase + static_cast<uint64_t>(ri) * REC + piece * 16;
@@ -184,7 +195,7 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
     start_item(iss);
     start_item(sc);
     // prologue: fill the ring
-    uint32_t pend = load_idx(iss);
+    Idx pend = load_idx(iss);
     for (int g = 0; g < kSlots; ++g) {
         issue(g, iss, pend);
         if (iss.it < items) advance(iss);
@@ -203,8 +214,15 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
             stage_query(qt, sc.head, qs, lane);
             staged = sc.head;
         }
-        const int c = sc.c0 + 32 * sc.s + lane;
-        if (c < sc.cend) S[sc.head * cmax + c] = score_record(ring + slot * kStageBytes, lane, qp);
+        const uint8_t* st = ring + slot * kStageBytes;
+        float sv[kPerLane];
+#pragma unroll
+        for (int u = 0; u < kPerLane; ++u) sv[u] = score_record(st, 32 * u + lane, qp);
+#pragma unroll
+        for (int u = 0; u < kPerLane; ++u) {
+            const int c = sc.c0 + kStageRecs * sc.s + 32 * u + lane;
+            if (c < sc.cend) S[sc.head * cmax + c] = sv[u];
+        }
         __syncwarp();                        // every lane has read the slot and the query
         issue(slot, iss, pend);
         if (iss.it < items) advance(iss);
