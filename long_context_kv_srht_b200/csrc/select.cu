@@ -218,11 +218,19 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
     // coalesced load of the warp's 1024 packed scores, transposed so that lane l then reads
     // keys 32 l .. 32 l + 31 (row stride 33 words: both directions are conflict-free)
     {
+        // asynchronous 4-byte copies, all in flight at once; keys at or past n read as 0
+        // (zero fill, src-size 0); their address stays inside the padded capacity
         const uint32_t* src = scores + up * cap_pad + kw + lane;
         const int nw = static_cast<int>(max64(0, min64(32 * kKeys, n - kw)));
-#pragma unroll 8
-        for (int t = 0; t < kKeys; ++t)
-            tr[warp][t * 33 + lane] = (32 * t + lane < nw) ? src[32 * t] : 0u;
+#pragma unroll
+        for (int t = 0; t < kKeys; ++t) {
+            const uint32_t dst = smem_addr(&tr[warp][t * 33 + lane]);
+            const uint32_t bytes = (32 * t + lane < nw) ? 4u : 0u;
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst),
+                         "l"(src + 32 * t), "r"(bytes) : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_all;" ::: "memory");
         __syncwarp();
     }
     const uint32_t* s = &tr[warp][lane * 33];

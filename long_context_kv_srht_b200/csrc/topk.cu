@@ -19,9 +19,10 @@
 //    alternate between two buffers, so one cluster barrier per level suffices; every level
 //    shrinks the interval 2048-fold, so at most three run;
 //  - with T the k-th largest value and E the number of T-valued candidates to keep, each
-//    warp counts its contiguous range, the counts are scanned over warps and over the
-//    cluster, and a ballot pass writes every candidate above T and the first E equal to T in
-//    ascending key order (the candidates are stored in key order); est comes from u itself.
+//    thread counts a contiguous run of values, the counts are scanned over the CTA and the
+//    cluster, and each thread then writes its run's values above T and its ties at T while
+//    fewer than E ties precede them, in ascending key order (the candidates are stored in
+//    key order); est comes from u itself.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -188,18 +189,25 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
     const uint32_t T = lo;
     const uint32_t E = krem;   // ties at T to keep, in key order
 
-    // 3. counts per warp-contiguous range, then offsets over warps and over the cluster
-    const int w0 = static_cast<int>(static_cast<int64_t>(L) * warp / kWarps);
-    const int w1 = static_cast<int>(static_cast<int64_t>(L) * (warp + 1) / kWarps);
+    // 3. counts per thread-contiguous run, then offsets over the CTA (block scan) and over
+    //    the cluster
+    const int a = static_cast<int>(static_cast<int64_t>(L) * threadIdx.x / kT);
+    const int b = static_cast<int>(static_cast<int64_t>(L) * (threadIdx.x + 1) / kT);
     uint32_t ngt = 0, neq = 0;
-    for (int pp = w0 + lane; pp < w1; pp += 32) {
-        const uint32_t u = key_at(pp);
+    for (int i = a; i < b; ++i) {
+        const uint32_t u = key_at(i);
         ngt += u > T;
         neq += u == T;
     }
-    ngt = __reduce_add_sync(0xffffffffu, ngt);
-    neq = __reduce_add_sync(0xffffffffu, neq);
-    if (lane == 0) { wa[warp] = ngt; wb[warp] = neq; }
+    // inclusive warp scans of (gt, eq), then warp totals
+    uint32_t xg = ngt, xe = neq;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t yg = __shfl_up_sync(0xffffffffu, xg, o);
+        const uint32_t ye = __shfl_up_sync(0xffffffffu, xe, o);
+        if (lane >= o) { xg += yg; xe += ye; }
+    }
+    if (lane == 31) { wa[warp] = xg; wb[warp] = xe; }
     __syncthreads();
     if (threadIdx.x == 0) {
         uint32_t g = 0, e = 0;
@@ -208,7 +216,7 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
         ctot[1] = e;
     }
     cluster.sync();
-    uint32_t gt_run = 0, eq_run = 0;   // above T / ties before this warp's range
+    uint32_t gt_run = xg - ngt, eq_run = xe - neq;   // above T / ties before this thread
     for (int q = 0; q < rank; ++q) {
         const uint32_t* r = cluster.map_shared_rank(ctot, q);
         gt_run += r[0];
@@ -217,30 +225,25 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
     for (int w = 0; w < warp; ++w) { gt_run += wa[w]; eq_run += wb[w]; }
     cluster.barrier_arrive();          // no remote read of this CTA's memory follows
 
-    // 4. ballot pass in key order
+    // 4. this thread's winners in key order: every value above T, and the ties at T while
+    //    fewer than E ties precede them
     const float qn = qnorm[head];
-    const uint32_t lt = (1u << lane) - 1u;
-    for (int pb = w0; pb < w1; pb += 32) {
-        const int pp = pb + lane;
-        const bool valid = pp < w1;
-        const uint32_t u = valid ? key_at(pp) : 0u;
-        const bool eq = valid && u == T;
-        const bool gt = valid && u > T;
-        const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-        const bool sel = gt || (eq && (eq_run + __popc(eqm & lt)) < E);
-        const uint32_t selm = __ballot_sync(0xffffffffu, sel);
-        if (sel) {
-            const uint32_t r = gt_run + min(eq_run, E) + __popc(selm & lt);
-            if (r < static_cast<uint32_t>(k)) {
-                const int64_t pos = static_cast<int64_t>(head) * k + r;
-                out_idx[pos] = idx_at(pp);
-                if (out_est) out_est[pos] = __fmul_rn(qn, value_of(u));
-            } else {
-                atomicExch(status, ST_BADINDEX);
+    uint32_t pos = gt_run + min(eq_run, E);
+    if (pos + ngt + (E > eq_run ? min(E - eq_run, neq) : 0u) > static_cast<uint32_t>(k)) {
+        atomicExch(status, ST_BADINDEX);   // never taken when the counts are consistent
+    } else {
+        int32_t* oi = out_idx + static_cast<int64_t>(head) * k;
+        float* oe = out_est ? out_est + static_cast<int64_t>(head) * k : nullptr;
+        for (int i = a; i < b; ++i) {
+            const uint32_t u = key_at(i);
+            bool take = u > T;
+            if (u == T) take = eq_run++ < E;
+            if (take) {
+                oi[pos] = idx_at(i);
+                if (oe) oe[pos] = __fmul_rn(qn, value_of(u));
+                ++pos;
             }
         }
-        gt_run += __popc(__ballot_sync(0xffffffffu, gt));
-        eq_run += __popc(eqm);
     }
     cluster.barrier_wait();
 }
