@@ -6,6 +6,7 @@ select + RSQ-IP rerank + top-k), i.e. batch * query heads * cached keys / search
 the achieved fraction of the HBM roofline of the dominant kernel.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload million_offload]
+    python bench.py --workload drift_32k    # long-generation drift: append + search per step
     python bench.py --impl reference ...   # the CPU oracle on a bounded sample
 
 Default workload: the million-token offload decode step (batch 1, 32 query / 8 KV heads,
@@ -268,11 +269,111 @@ def decode_step(args, ix, cfg, sp, keys, vals, qs, idx, est, k, H, dev, kv_host)
 
 
 # ------------------------------------------------------------------------------------ main
+def run_drift(args, ws, rank, local):
+    """Long-generation drift (8 KV heads, 32768 prefill keys, then one appended key per KV
+    head per decode step while the keys' mean vector drifts; k = 1024). Every timed step
+    appends one key per KV head and searches once over the grown index; L2 is flushed between
+    steps. Recall of the returned top-k against the exact inner-product top-k (computed on
+    the device, outside the timed region) is tracked at sampled steps. The warm-up steps are
+    the first decode steps of the sequence; all remaining steps are timed."""
+    import numpy as np
+    import torch
+    from long_context_kv_srht_b200 import pariskv as pk
+    from long_context_kv_srht_b200 import workload
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    base = workload.spec("drift_32k")
+    sp = workload.spec("drift_32k", seed=base.seed + 1000 * rank)
+    T, H, n0, k = sp.decode_steps, sp.num_kv_heads, sp.n, sp.k
+    w = workload.generate_drift(sp)
+    bf = lambda a: torch.from_numpy(workload.bf16_bits(a)).view(torch.bfloat16).to(dev)
+    pre, app, qs = bf(w.prefill[None]), bf(w.appended), bf(w.queries)
+    cfg = pk.config(batch=1, num_kv_heads=H, group=1, capacity=n0 + T, dtype=sp.dtype,
+                    rho=sp.rho, cand_bp=sp.cand_bp)
+    ix = pk.build_index(cfg, w.signs, pre)
+    idx = torch.empty((H, k), dtype=torch.int32, device=dev)
+    est = torch.empty((H, k), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    W = max(0, min(args.warmup, T - 1))
+    for t in range(W):
+        ix.append(app[t].view(1, H, 1, 128))
+        ix.search(qs[t].view(1, H, 128), k, idx, est)
+    torch.cuda.synchronize()
+
+    steps = T - W
+    sample = set(range(W, T, 4096)) | {T - 1}
+    kept = {}
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    dist_barrier(ws)
+    torch.cuda.synchronize()
+    launches = 0
+    for i, t in enumerate(range(W, T)):
+        flush.fill_(t & 255)
+        ev[i][0].record()
+        ix.append(app[t].view(1, H, 1, 128))
+        ev[i][1].record()
+        ix.search(qs[t].view(1, H, 128), k, idx, est)
+        ev[i][2].record()
+        launches += pk.last_launch_count() + 1
+        if t in sample:
+            kept[t] = idx.clone()
+    torch.cuda.synchronize()
+    dist_barrier(ws)
+    clk = clocks.stop()
+    app_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    srch_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
+    step_ms = dist_max(app_ms + srch_ms, ws)
+    keys_searched = sum(H * (n0 + t + 1) for t in range(W, T))
+    value = ws * keys_searched / (step_ms * steps / 1e3)
+
+    # recall against the exact top-k by <q, k> over the keys present at each sampled step
+    allk = torch.cat([pre[0], app.permute(1, 0, 2)], dim=1).float()   # [H, n0 + T, d]
+    rec = {}
+    for t, got in sorted(kept.items()):
+        sc = torch.einsum("hnd,hd->hn", allk[:, : n0 + t + 1], qs[t].float())
+        ex = torch.topk(sc, k, dim=1).indices
+        hit = 0
+        for h in range(H):
+            hit += np.intersect1d(got[h].cpu().numpy(), ex[h].cpu().numpy()).size
+        rec[str(t)] = hit / (H * k)
+
+    if rank == 0:
+        line = {
+            "metric": "keys searched/s per decode step (vote+rerank+top-k)",
+            "value": value, "unit": "keys/s", "n_gpus": ws, "steps": steps,
+            "warmup": W, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": sp.name, "kv_heads": H, "q_heads_per_kv": 1, "d": sp.d,
+                       "n_prefill": n0, "decode_steps": T, "k": k, "B": sp.B, "m": sp.m,
+                       "rho": sp.rho, "cand_bp": sp.cand_bp, "key_dtype": sp.dtype,
+                       "step": "append one key per KV head + one search",
+                       "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"},
+            "decode_step": {"append_ms": app_ms, "search_ms": srch_ms},
+            "recall_vs_exact_topk": rec,
+            "roofline": None,
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    ix.sync()
+    ix.destroy()
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     ws, rank, local = dist_setup(args)
     if args.impl == "reference":
         run_reference(args, ws, rank)
+        return
+    if args.workload == "drift_32k":
+        run_drift(args, ws, rank, local)
         return
     import numpy as np
     import torch

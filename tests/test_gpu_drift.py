@@ -1,0 +1,67 @@
+"""Long-generation drift through the C ABI ("ParisKV: Fast and Drift-Robust KV-Cache
+Retrieval for Long-Context LLMs", abstract: retrieval under distribution drift; "Technical
+Summary: ParisKV", Key Contributions 1 and Core Algorithmic Innovations 1: the index is kept
+current as keys are generated).
+
+Workload: 8 KV heads, a 32768-key prefill, then one appended key per KV head per decode step
+while the keys' mean vector moves linearly to a fresh random direction; one query head per
+KV head searches after every append with k = 1024. The index only ever grows by append.
+
+Gates: at sampled steps the top-k from raw bf16 inputs matches the oracle's search over the
+same keys with recall >= 0.999 (the GPU rotates in fp32, the oracle in fp64); after the last
+step the appended index is bit-identical to one built from all keys in a single call."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_kv_srht_b200 import pariskv as pk
+from long_context_kv_srht_b200 import workload
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+STEPS = 4096          # decode steps run here (the benchmark's drift mode runs all 32768)
+
+
+def _bf16(a):
+    return torch.from_numpy(workload.bf16_bits(a)).view(torch.bfloat16)
+
+
+def test_drift_append_and_search():
+    sp = workload.spec("drift_32k")
+    w = workload.generate_drift(sp, steps=STEPS)
+    H, n0, k = sp.num_kv_heads, sp.n, sp.k
+    cfg = pk.config(batch=1, num_kv_heads=H, group=1, capacity=n0 + STEPS, dtype=sp.dtype,
+                    rho=sp.rho, cand_bp=sp.cand_bp)
+    pre = _bf16(w.prefill[None]).to(DEV)               # [1, H, n0, d]
+    app = _bf16(w.appended).to(DEV)                    # [steps, H, d]
+    qs = _bf16(w.queries).to(DEV)                      # [steps, H, d]
+    ix = pk.build_index(cfg, w.signs, pre)
+    check = sorted(set(range(0, STEPS, 1365)) | {STEPS - 1})
+    got = {}
+    for t in range(STEPS):
+        ix.append(app[t].view(1, H, 1, 128))
+        idx, _ = ix.search(qs[t].view(1, H, 128), k)
+        if t in check:
+            got[t] = idx.cpu().numpy()
+    ix.sync()
+    assert ix.size == n0 + STEPS
+
+    p = oracle.SearchParams(m=8, rho=sp.rho, cand_bp=sp.cand_bp)
+    for t in check:
+        hits = 0
+        for h in range(H):
+            keys = np.concatenate([w.prefill[h], w.appended[: t + 1, h]], axis=0)
+            enc = oracle.build_unit(keys, w.signs, 8)
+            o_idx, *_ = oracle.search(enc, w.queries[t, h], w.signs, k, p)
+            g_idx = got[t][h]
+            assert np.all(np.diff(g_idx) > 0)
+            assert g_idx.max() <= n0 + t      # only keys present at step t
+            hits += len(set(g_idx.tolist()) & set(o_idx.tolist()))
+        assert hits / (H * k) >= 0.999, (t, hits / (H * k))
+
+    # append-only growth leaves the same index as one build over all keys
+    allk = torch.cat([pre, app.permute(1, 0, 2).unsqueeze(0)], dim=2).contiguous()
+    ref = pk.build_index(cfg, w.signs, allk)
+    for a, b in zip(ix.export_index(), ref.export_index()):
+        np.testing.assert_array_equal(a, b)
