@@ -57,42 +57,63 @@ __device__ __forceinline__ uint64_t level_pair(uint32_t xa, uint32_t xb) {
                 kOff);
 }
 
-// p chains of the subspace pair (a, b) from their code words; qp holds the pairs
-// (q~_{a,j}, q~_{b,j}) for j = 0..7 in shared memory.
-__device__ __forceinline__ float2 pair_dots(uint32_t wa, uint32_t wb, const uint64_t* qp) {
+// p chains of the subspace pair (a, b) from their code words, with the query pairs
+// q[j] = (q~_{a,j}, q~_{b,j}) for j = 0..7.
+__device__ __forceinline__ float2 pair_dots(uint32_t wa, uint32_t wb, const uint64_t q[8]) {
     const uint32_t ea = wa & 0x0F0F0F0Fu, oa = (wa >> 4) & 0x0F0F0F0Fu;  // dims 0,2,4,6 | 1,3,5,7
     const uint32_t eb = wb & 0x0F0F0F0Fu, ob = (wb >> 4) & 0x0F0F0F0Fu;
-    const ulonglong2 q01 = reinterpret_cast<const ulonglong2*>(qp)[0];
-    const ulonglong2 q23 = reinterpret_cast<const ulonglong2*>(qp)[1];
-    const ulonglong2 q45 = reinterpret_cast<const ulonglong2*>(qp)[2];
-    const ulonglong2 q67 = reinterpret_cast<const ulonglong2*>(qp)[3];
     uint64_t p = pack2(0.0f, 0.0f);
-    p = fma2(level_pair<0>(ea, eb), q01.x, p);
-    p = fma2(level_pair<0>(oa, ob), q01.y, p);
-    p = fma2(level_pair<1>(ea, eb), q23.x, p);
-    p = fma2(level_pair<1>(oa, ob), q23.y, p);
-    p = fma2(level_pair<2>(ea, eb), q45.x, p);
-    p = fma2(level_pair<2>(oa, ob), q45.y, p);
-    p = fma2(level_pair<3>(ea, eb), q67.x, p);
-    p = fma2(level_pair<3>(oa, ob), q67.y, p);
+    p = fma2(level_pair<0>(ea, eb), q[0], p);
+    p = fma2(level_pair<0>(oa, ob), q[1], p);
+    p = fma2(level_pair<1>(ea, eb), q[2], p);
+    p = fma2(level_pair<1>(oa, ob), q[3], p);
+    p = fma2(level_pair<2>(ea, eb), q[4], p);
+    p = fma2(level_pair<2>(oa, ob), q[5], p);
+    p = fma2(level_pair<3>(ea, eb), q[6], p);
+    p = fma2(level_pair<3>(oa, ob), q[7], p);
     return unpack2(p);
 }
 
-// S of the record in stage row `row`; qp = the head's 64 query pairs (pair t at qp + 8 t).
-__device__ __forceinline__ float score_record(const uint8_t* st, int row, const uint64_t* qp) {
-    float S = 0.0f;
+__device__ __forceinline__ void load_qpairs(const uint64_t* qp, uint64_t q[8]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const ulonglong2 v = reinterpret_cast<const ulonglong2*>(qp)[i];
+        q[2 * i] = v.x;
+        q[2 * i + 1] = v.y;
+    }
+}
+
+// S of the kPerLane records in stage rows row0 + 32 u; qp = the head's 64 query pairs (pair
+// t at qp + 8 t). Each query pair is read once for all the lane's records; every record
+// keeps its own p and S chains in the defined order.
+__device__ __forceinline__ void score_records(const uint8_t* st, int row0, const uint64_t* qp,
+                                              float S[kPerLane]) {
+#pragma unroll
+    for (int u = 0; u < kPerLane; ++u) S[u] = 0.0f;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {   // chunk c: subspaces 4c..4c+3
-        const uint4 cw = *reinterpret_cast<const uint4*>(st + piece_at(row, 2 * c));
-        const uint4 fw = *reinterpret_cast<const uint4*>(st + piece_at(row, 2 * c + 1));
-        const float2 pa = pair_dots(cw.x, cw.y, qp + 16 * c);
-        S = __fmaf_rn(__uint_as_float(fw.x), pa.x, S);
-        S = __fmaf_rn(__uint_as_float(fw.y), pa.y, S);
-        const float2 pb = pair_dots(cw.z, cw.w, qp + 16 * c + 8);
-        S = __fmaf_rn(__uint_as_float(fw.z), pb.x, S);
-        S = __fmaf_rn(__uint_as_float(fw.w), pb.y, S);
+        uint4 cw[kPerLane], fw[kPerLane];
+#pragma unroll
+        for (int u = 0; u < kPerLane; ++u) {
+            cw[u] = *reinterpret_cast<const uint4*>(st + piece_at(row0 + 32 * u, 2 * c));
+            fw[u] = *reinterpret_cast<const uint4*>(st + piece_at(row0 + 32 * u, 2 * c + 1));
+        }
+        uint64_t q[8];
+        load_qpairs(qp + 16 * c, q);
+#pragma unroll
+        for (int u = 0; u < kPerLane; ++u) {
+            const float2 pa = pair_dots(cw[u].x, cw[u].y, q);
+            S[u] = __fmaf_rn(__uint_as_float(fw[u].x), pa.x, S[u]);
+            S[u] = __fmaf_rn(__uint_as_float(fw[u].y), pa.y, S[u]);
+        }
+        load_qpairs(qp + 16 * c + 8, q);
+#pragma unroll
+        for (int u = 0; u < kPerLane; ++u) {
+            const float2 pb = pair_dots(cw[u].z, cw[u].w, q);
+            S[u] = __fmaf_rn(__uint_as_float(fw[u].z), pb.x, S[u]);
+            S[u] = __fmaf_rn(__uint_as_float(fw[u].w), pb.y, S[u]);
+        }
     }
-    return S;
 }
 
 // Stages head h's rotated query into the warp's pair table: entry 8 t + j holds
@@ -216,8 +237,7 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
         }
         const uint8_t* st = ring + slot * kStageBytes;
         float sv[kPerLane];
-#pragma unroll
-        for (int u = 0; u < kPerLane; ++u) sv[u] = score_record(st, 32 * u + lane, qp);
+        score_records(st, lane, qp, sv);
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
             const int c = sc.c0 + kStageRecs * sc.s + 32 * u + lane;
