@@ -131,7 +131,9 @@ PARISKV_API pariskv_status pariskv_search(pariskv_index* index, const void* q, i
  *   out:      device pointer [batch][Hq][d] of element type out_dtype (PARISKV_F32 keeps the
  *             fp32 accumulator precision; PARISKV_BF16 rounds to nearest even).
  * q, K and V have element type cfg->dtype; accumulation is fp32. The split-K partials live in
- * a stream-ordered workspace (cudaMallocAsync / cudaFreeAsync on `stream`).
+ * a stream-ordered workspace allocated and freed on `stream` from a memory pool the library
+ * keeps per device (it keeps its memory mapped between calls; it holds at most the largest
+ * workspaces in flight at once).
  * Errors: EINVAL, ENOMEM, ECUDA. */
 PARISKV_API pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q,
                                                  const void* K, const void* V, int64_t ld_tok,

@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -317,10 +318,46 @@ pariskv_status pariskv_search(pariskv_index* index, const void* q, int32_t k, in
                       static_cast<cudaStream_t>(stream));
 }
 
+// Stream-ordered workspaces of the allocating attention call come from a library-owned pool
+// per device that keeps its memory mapped (release threshold: unlimited). Freed workspaces
+// are reused by later calls, so a call never maps or unmaps device memory once the pool has
+// grown to its working size; with the default pool, memory released at every synchronisation
+// and mapped again by the next call was measured to slow the following host-memory gathers
+// (first-touch and TLB costs) by up to 4x.
+static cudaError_t workspace_pool(cudaMemPool_t* out) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!pools[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t p = nullptr;
+        e = cudaMemPoolCreate(&p, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = ~uint64_t{0};
+        e = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) {
+            cudaMemPoolDestroy(p);
+            return e;
+        }
+        pools[dev] = p;
+    }
+    *out = pools[dev];
+    return cudaSuccess;
+}
+
 pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, const void* K,
                                      const void* V, int64_t ld_tok, int64_t n,
                                      const int32_t* topk_idx, int32_t k, float scale, void* out,
                                      int32_t out_dtype, void* stream) {
+
+
     pariskv_status s = check_config(cfg);
     if (s != PARISKV_OK) return s;
     const size_t al = cfg->dtype == PARISKV_BF16 ? 8 : 16;
@@ -344,8 +381,12 @@ pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, c
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float* work = nullptr;
     if (fault_alloc()) return fail(PARISKV_ENOMEM, "attention workspace");
-    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&work),
-                                    attend_workspace_floats(heads, nsplit) * sizeof(float), st);
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = workspace_pool(&pool);
+    if (e == cudaSuccess)
+        e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&work),
+                                    attend_workspace_floats(heads, nsplit) * sizeof(float), pool,
+                                    st);
     if (e != cudaSuccess) return cuda_fail(e, "attention workspace");
     g_launches = 0;
     e = launch_attend(cfg, q, K, V, ld_tok, n, topk_idx, k, scale, out, out_dtype, work, nsplit,
