@@ -113,7 +113,7 @@ void free_index(pariskv_index* ix) {
     if (!ix) return;
     dfree(ix->signs); dfree(ix->ids); dfree(ix->rec); dfree(ix->lut); dfree(ix->qt);
     dfree(ix->qnorm); dfree(ix->scores); dfree(ix->hist); dfree(ix->thr); dfree(ix->cbase);
-    dfree(ix->cand); dfree(ix->S); dfree(ix->status);
+    dfree(ix->cand); dfree(ix->S); dfree(ix->shist); dfree(ix->status);
     for (auto& e : ix->ev)
         if (e) cudaEventDestroy(e);
     delete ix;
@@ -141,7 +141,8 @@ pariskv_status create_index(const pariskv_config* cfg, const int8_t* signs, cuda
               dalloc(&ix->lut, up * NB * NC) && dalloc(&ix->qt, heads * D) &&
               dalloc(&ix->qnorm, heads) && dalloc(&ix->scores, up * ix->cap_pad) &&
               dalloc(&ix->hist, up * nch * PACK * NBINS) && dalloc(&ix->thr, heads * 4) &&
-              dalloc(&ix->cbase, heads * nch * 2) && dalloc(&ix->status, 1);
+              dalloc(&ix->cbase, heads * nch * 2) && dalloc(&ix->shist, heads * SBINS) &&
+              dalloc(&ix->status, 1);
     if (!ok) {
         free_index(ix);
         return fail(PARISKV_ENOMEM, "device allocation for the index failed");

@@ -15,6 +15,8 @@ constexpr int NB = D / M;       // subspaces (16)
 constexpr int NC = 1 << M;      // sign centroids per subspace (256)
 constexpr int REC = 128;        // bytes per key record: 64 B of 4-bit codes + 16 fp32 factors
 constexpr int NBINS = 64;       // coarse scores are < 64 (B * w_rank1 <= 48)
+constexpr int SBINS_BITS = 11;  // first radix level of the top-k, counted by the rerank
+constexpr int SBINS = 1 << SBINS_BITS;
 constexpr int CHUNK = 8192;     // keys per coarse-score histogram chunk (a vote work item)
 constexpr int PACK = 4;         // query heads whose vote weights share one 32-bit table entry
 
@@ -73,6 +75,16 @@ __device__ __forceinline__ uint32_t prmt_i(uint32_t a, uint32_t b) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Order-preserving 32-bit image of an fp32 value (flip all bits of negative values, set the
+// sign bit of the others) and its exact inverse.
+__device__ __forceinline__ uint32_t order_key(float s) {
+    const uint32_t u = __float_as_uint(s);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float value_of(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {

@@ -18,6 +18,11 @@
 // stored at 16-byte position c ^ (r mod 8), so that eight lanes reading the same piece of
 // eight different records touch all 32 banks once.
 //
+// Each value is also counted, by the top bits of its order-preserving image, into a per-head
+// histogram, which is the top-k's first radix level: lanes holding the same bin are grouped
+// with a warp match and one of them adds the group's count (one global reduction per value
+// piled onto the few hot bins and doubled the kernel's time).
+//
 // Scoring: each lane scores two records of a stage (rows lane and lane + 32, whose chains
 // interleave). The warp's current query head has its rotated query in
 // shared memory as (subspace 2t, subspace 2t + 1) fp32 pairs, read with broadcast loads; a
@@ -145,7 +150,8 @@ struct StreamPos {
 __global__ void __launch_bounds__(kThr, kCtasPerSm)
 rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
               const float* __restrict__ qt, float* __restrict__ S, int32_t C, int64_t cmax,
-              int64_t cap_pad, int64_t n, int group, int iph, int64_t items, int* status) {
+              int64_t cap_pad, int64_t n, int group, int iph, int64_t items,
+              uint32_t* __restrict__ shist, int* status) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* ring = smem + warp * kWarpBytes;
@@ -241,7 +247,14 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
             const int c = sc.c0 + kStageRecs * sc.s + 32 * u + lane;
-            if (c < sc.cend) S[sc.head * cmax + c] = sv[u];
+            const bool ok = c < sc.cend;
+            if (ok) S[sc.head * cmax + c] = sv[u];
+            // the top-k's first radix level: count the values by their top order-key bits,
+            // one global reduction per distinct bin in the warp (values cluster in few bins)
+            const uint32_t bin = ok ? order_key(sv[u]) >> (32 - SBINS_BITS) : 0xffffffffu;
+            const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+            if (ok && lane == __ffs(peers) - 1)
+                atomicAdd(&shist[sc.head * SBINS + bin], static_cast<uint32_t>(__popc(peers)));
         }
         __syncwarp();                        // every lane has read the slot and the query
         issue(slot, iss, pend);
@@ -269,7 +282,7 @@ cudaError_t launch_rerank(const pariskv_index* ix, int64_t C, cudaStream_t st) {
         static_cast<int>(max64(1, min64(int64_t{kCtasPerSm} * sms, ceil_div(items, kWarps))));
     return launch_pdl(rerank_kernel, grid, kThr, kSmem, st, ix->rec, ix->cand, ix->qt, ix->S,
                       static_cast<int32_t>(C), ix->cmax, ix->cap_pad, ix->n, ix->cfg.group, iph,
-                      items, ix->status);
+                      items, ix->shist, ix->status);
 }
 
 }  // namespace pkv

@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(kCThr)
 compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ thr,
                const int32_t* __restrict__ cbase, int32_t* __restrict__ cand, int64_t n,
                int64_t cap_pad, int group, int packs, int64_t nchunks, int64_t cmax,
-               int* status) {
+               uint32_t* __restrict__ shist, int* status) {
     __shared__ uint32_t tr[kCW][32 * 33];
     __shared__ uint64_t scan_sh[kCW + 1][2];
     const int64_t c = blockIdx.x;
@@ -238,6 +238,10 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
     // threshold kernel just before this one
     pdl_wait();
     pdl_launch_dependents();
+    // the rerank that follows counts its values per head into shist: start it at zero
+    if (c == 0)
+        for (int i = threadIdx.x; i < hp * SBINS; i += kCThr)
+            shist[static_cast<int64_t>(head0) * SBINS + i] = 0u;
 
     // Per-head thresholds packed one per byte. A head outside the pack gets T = 127, which
     // no score (< 64) reaches. Byte h of (s + gt_add) has bit 7 set iff score_h > T_h, and
@@ -335,7 +339,7 @@ cudaError_t launch_compact(const pariskv_index* ix, cudaStream_t st) {
     dim3 grid(static_cast<unsigned>(nchunks), static_cast<unsigned>(ix->units * ix->packs));
     return launch_pdl(compact_kernel, grid, kCThr, 0, st, ix->scores, ix->thr, ix->cbase,
                       ix->cand, ix->n, ix->cap_pad, ix->cfg.group, ix->packs, nchunks, ix->cmax,
-                      ix->status);
+                      ix->shist, ix->status);
 }
 
 }  // namespace pkv

@@ -11,13 +11,14 @@
 //  - CTA r copies the r-th quarter of the head's S values and candidate indices into shared
 //    memory with asynchronous copies, all in flight at once, and turns S into u in place
 //    (quarters longer than kSlice stay in global memory and are re-read on every pass);
-//  - the cluster agrees on [min, max] of u through distributed shared memory;
-//  - range-adaptive radix levels: the current interval [lo, hi] is cut into at most 2048
+//  - the first radix level, the top 11 bits of u, was counted by the rerank as it wrote S
+//    (a per-head 2048-bin histogram in global memory), so it costs one read here;
+//  - then range-adaptive radix levels: the current interval [lo, hi] is cut into at most 2048
 //    power-of-two-wide bins, every CTA histograms its quarter, and every CTA sums the four
 //    histograms bin by bin over DSMEM and runs the same suffix scan, so all four pick the
 //    same bin (the one holding the k-th largest) without further exchange. Histograms
-//    alternate between two buffers, so one cluster barrier per level suffices; every level
-//    shrinks the interval 2048-fold, so at most three run;
+//    alternate between two buffers, so one cluster barrier per level suffices; the 21 bits
+//    left after the first level take at most two more levels;
 //  - with T the k-th largest value and E the number of T-valued candidates to keep, each
 //    thread counts a contiguous run of values, the counts are scanned over the CTA and the
 //    cluster, and each thread then writes its run's values above T and its ties at T while
@@ -40,25 +41,16 @@ constexpr int kWarps = kT / 32;
 constexpr int kBins = 2048;
 constexpr int kSlice = 16384;      // values per CTA kept in shared memory (u and index)
 
-__device__ __forceinline__ uint32_t order_key(float s) {
-    const uint32_t u = __float_as_uint(s);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-// the inverse map (exact)
-__device__ __forceinline__ float value_of(uint32_t key) {
-    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
-}
-
 template <bool RES>
 __global__ void __cluster_dims__(kCL, 1, 1) __launch_bounds__(kT, 1)
 topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
-            const float* __restrict__ qnorm, int32_t C, int64_t cmax, int32_t k,
-            int32_t* __restrict__ out_idx, float* __restrict__ out_est, int* status) {
+            const float* __restrict__ qnorm, const uint32_t* __restrict__ shist, int32_t C,
+            int64_t cmax, int32_t k, int32_t* __restrict__ out_idx, float* __restrict__ out_est,
+            int* status) {
     extern __shared__ __align__(16) uint32_t dyn[];
     __shared__ uint32_t hist[2][kBins];
     __shared__ uint32_t wa[kWarps], wb[kWarps];
     __shared__ uint32_t ctot[2];       // this CTA's candidates above T / ties at T
-    __shared__ uint32_t cmm[2];        // this CTA's min / max of u
     __shared__ uint32_t pick[2];
 
     cg::cluster_group cluster = cg::this_cluster();
@@ -89,70 +81,19 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
         asm volatile("cp.async.commit_group;" ::: "memory");
         asm volatile("cp.async.wait_all;" ::: "memory");
     }
-    uint32_t mn = 0xffffffffu, mx = 0u;
-#pragma unroll 4
-    for (int i = threadIdx.x; i < L; i += kT) {
-        const uint32_t u = RES ? order_key(__uint_as_float(keys[i])) : order_key(Sh[i]);
-        if (RES) keys[i] = u;   // each thread converts the entries it copied itself
-        mn = min(mn, u);
-        mx = max(mx, u);
-    }
-    mn = __reduce_min_sync(0xffffffffu, mn);
-    mx = __reduce_max_sync(0xffffffffu, mx);
-    if (lane == 0) { wa[warp] = mn; wb[warp] = mx; }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t a = 0xffffffffu, b = 0u;
-        for (int w = 0; w < kWarps; ++w) { a = min(a, wa[w]); b = max(b, wb[w]); }
-        cmm[0] = a;
-        cmm[1] = b;
-    }
-    cluster.sync();
-    uint32_t lo = 0xffffffffu, hi = 0u;
-#pragma unroll
-    for (int q = 0; q < kCL; ++q) {
-        const uint32_t* r = cluster.map_shared_rank(cmm, q);
-        lo = min(lo, r[0]);
-        hi = max(hi, r[1]);
-    }
+    if (RES)
+        for (int i = threadIdx.x; i < L; i += kT)   // each thread converts what it copied
+            keys[i] = order_key(__uint_as_float(keys[i]));
 
-    // 2. range-adaptive radix levels over the cluster
+    // 2. radix levels. The first (the top SBINS_BITS bits of u) was counted by the rerank;
+    //    the following ones are range-adaptive histograms over the cluster. choose() finds,
+    //    from each thread's two bins (2t, 2t + 1), the bin holding the krem-th largest value
+    //    and narrows [lo, hi] to it; every CTA of the cluster sees the same counts and so
+    //    makes the same choice.
     uint32_t krem = static_cast<uint32_t>(k);
-    int level = 0;
-    while (lo != hi) {
-        uint32_t* hb = hist[level & 1];
-        const uint32_t span = hi - lo;
-        const int bitlen = 32 - __clz(span);
-        const int sh = bitlen > 11 ? bitlen - 11 : 0;   // (span >> sh) < 2048
-        hb[threadIdx.x] = 0u;
-        hb[threadIdx.x + kT] = 0u;
-        __syncthreads();
-        if (RES && (L & 3) == 0) {
-            const uint4* k4 = reinterpret_cast<const uint4*>(keys);
-            for (int i = threadIdx.x; i < (L >> 2); i += kT) {
-                const uint4 v = k4[i];
-                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (u[j] >= lo && u[j] <= hi) atomicAdd(&hb[(u[j] - lo) >> sh], 1u);
-            }
-        } else {
-            for (int i = threadIdx.x; i < L; i += kT) {
-                const uint32_t u = key_at(i);
-                if (u >= lo && u <= hi) atomicAdd(&hb[(u - lo) >> sh], 1u);
-            }
-        }
-        cluster.sync();   // every quarter's histogram is complete
-        // thread t sums bins 2t, 2t + 1 over the cluster; suffix counts over the bins
-        uint32_t h0 = 0, h1 = 0;
-#pragma unroll
-        for (int q = 0; q < kCL; ++q) {
-            const uint2 v = *reinterpret_cast<const uint2*>(cluster.map_shared_rank(hb, q) +
-                                                             2 * threadIdx.x);
-            h0 += v.x;
-            h1 += v.y;
-        }
-        uint32_t x = h0 + h1;
+    uint32_t lo = 0u, hi = 0xffffffffu;
+    auto choose = [&](uint32_t h0, uint32_t h1, int sh) {
+        uint32_t x = h0 + h1;   // suffix counts over the bins
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
@@ -183,8 +124,49 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
         const uint64_t bin_hi = static_cast<uint64_t>(nlo) + ((uint64_t{1} << sh) - 1u);
         lo = nlo;
         hi = static_cast<uint32_t>(min(static_cast<uint64_t>(hi), bin_hi));
+        __syncthreads();   // pick[], wa[] and wb[] are rewritten by the next level
+    };
+    static_assert(SBINS == kBins, "the first level has one bin pair per thread");
+    {
+        const uint2 v = reinterpret_cast<const uint2*>(shist + static_cast<int64_t>(head) * SBINS)[threadIdx.x];
+        choose(v.x, v.y, 32 - SBINS_BITS);
+    }
+    int level = 0;
+    while (lo != hi) {
+        uint32_t* hb = hist[level & 1];
+        const uint32_t span = hi - lo;
+        const int bitlen = 32 - __clz(span);
+        const int sh = bitlen > 11 ? bitlen - 11 : 0;   // (span >> sh) < 2048
+        hb[threadIdx.x] = 0u;
+        hb[threadIdx.x + kT] = 0u;
+        __syncthreads();
+        if (RES && (L & 3) == 0) {
+            const uint4* k4 = reinterpret_cast<const uint4*>(keys);
+            for (int i = threadIdx.x; i < (L >> 2); i += kT) {
+                const uint4 v = k4[i];
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (u[j] >= lo && u[j] <= hi) atomicAdd(&hb[(u[j] - lo) >> sh], 1u);
+            }
+        } else {
+            for (int i = threadIdx.x; i < L; i += kT) {
+                const uint32_t u = key_at(i);
+                if (u >= lo && u <= hi) atomicAdd(&hb[(u - lo) >> sh], 1u);
+            }
+        }
+        cluster.sync();   // every quarter's histogram is complete
+        // thread t sums bins 2t, 2t + 1 over the cluster
+        uint32_t h0 = 0, h1 = 0;
+#pragma unroll
+        for (int q = 0; q < kCL; ++q) {
+            const uint2 v = *reinterpret_cast<const uint2*>(cluster.map_shared_rank(hb, q) +
+                                                             2 * threadIdx.x);
+            h0 += v.x;
+            h1 += v.y;
+        }
+        choose(h0, h1, sh);
         ++level;
-        __syncthreads();   // pick[] and wa[] are rewritten by the next level
     }
     const uint32_t T = lo;
     const uint32_t E = krem;   // ties at T to keep, in key order
@@ -259,12 +241,12 @@ cudaError_t launch_topk(const pariskv_index* ix, int64_t C, int32_t k, int32_t* 
     const int heads = ix->units * ix->cfg.group;
     if (ceil_div(C, kCL) <= kSlice) {
         return launch_pdl(topk_kernel<true>, heads * kCL, kT, kDyn, st, ix->S, ix->cand,
-                          ix->qnorm, static_cast<int32_t>(C), ix->cmax, k, topk_idx, topk_est,
-                          ix->status);
+                          ix->qnorm, ix->shist, static_cast<int32_t>(C), ix->cmax, k, topk_idx,
+                          topk_est, ix->status);
     } else {
         return launch_pdl(topk_kernel<false>, heads * kCL, kT, 0, st, ix->S, ix->cand,
-                          ix->qnorm, static_cast<int32_t>(C), ix->cmax, k, topk_idx, topk_est,
-                          ix->status);
+                          ix->qnorm, ix->shist, static_cast<int32_t>(C), ix->cmax, k, topk_idx,
+                          topk_est, ix->status);
     }
 }
 
