@@ -10,8 +10,8 @@
 // by similarity with ties to the lower id; pen is an fp32 sum over j ascending. The first
 // rho centroids get vote weights w_rank1 (rank 1) and w_rest (ranks 2..rho); all others 0.
 //
-// One CTA per query head. Warp 0 rotates the query; then each of the 8 warps ranks the 256
-// centroids of two subspaces, 8 per lane, as 64-bit keys (pen bits << 32 | id): rho rounds
+// One CTA per query head. Warp 0 rotates the query; then each of the 16 warps ranks the 256
+// centroids of one subspace, 8 per lane, as 64-bit keys (pen bits << 32 | id): rho rounds
 // of a warp-wide minimum for small rho, an all-pairs rank count for large rho.
 //
 // Output table layout: u8 [unit * packs + pack][b][c][4]; byte (g mod 4) of each 32-bit
@@ -25,8 +25,10 @@ namespace pkv {
 
 namespace {
 
+constexpr int kQWarps = NB;   // one warp per subspace
+
 template <typename T, bool ROTATED>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(32 * kQWarps)
 query_prep_kernel(const T* __restrict__ q, const float* __restrict__ qt_in,
                   const float* __restrict__ qn_in, const float* __restrict__ signs, int group,
                   int packs, int rho, int w1, int wr, float* __restrict__ qt_out,
@@ -59,7 +61,7 @@ query_prep_kernel(const T* __restrict__ q, const float* __restrict__ qt_in,
     }
     __syncthreads();
 
-    for (int b = warp; b < NB; b += 8) {
+    for (int b = warp; b < NB; b += kQWarps) {
         float a[8];
         uint32_t c1 = 0;
 #pragma unroll
@@ -131,16 +133,16 @@ cudaError_t launch_query_prep(const pariskv_index* ix, const void* q, const floa
     const int heads = ix->units * c.group;
     uint8_t* lut8 = reinterpret_cast<uint8_t*>(ix->lut);
     if (rotated)
-        return launch_pdl(query_prep_kernel<float, true>, heads, 256, 0, st, nullptr, qt_in,
+        return launch_pdl(query_prep_kernel<float, true>, heads, 32 * kQWarps, 0, st, nullptr, qt_in,
                           qn_in, ix->signs, c.group, ix->packs, c.rho, c.w_rank1, c.w_rest,
                           ix->qt, ix->qnorm, lut8);
     else if (c.dtype == PARISKV_BF16)
-        return launch_pdl(query_prep_kernel<__nv_bfloat16, false>, heads, 256, 0, st,
+        return launch_pdl(query_prep_kernel<__nv_bfloat16, false>, heads, 32 * kQWarps, 0, st,
                           static_cast<const __nv_bfloat16*>(q), nullptr, nullptr, ix->signs,
                           c.group, ix->packs, c.rho, c.w_rank1, c.w_rest, ix->qt, ix->qnorm,
                           lut8);
     else
-        return launch_pdl(query_prep_kernel<float, false>, heads, 256, 0, st,
+        return launch_pdl(query_prep_kernel<float, false>, heads, 32 * kQWarps, 0, st,
                           static_cast<const float*>(q), nullptr, nullptr, ix->signs, c.group,
                           ix->packs, c.rho, c.w_rank1, c.w_rest, ix->qt, ix->qnorm, lut8);
 }

@@ -84,7 +84,7 @@ threshold_kernel(const uint32_t* __restrict__ hist, int group, int packs, int64_
         constexpr int kRows = kThr / NBINS;
         const int bin = threadIdx.x % NBINS, r0 = threadIdx.x / NBINS;
         uint32_t a = 0;
-#pragma unroll 8
+#pragma unroll 32
         for (int64_t c = r0; c < nchunks; c += kRows) a += hb[c * (PACK * NBINS) + bin];
         part[r0][bin] = a;
     }
