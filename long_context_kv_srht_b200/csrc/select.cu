@@ -15,10 +15,10 @@
 //    writes for every 8192-key chunk how many candidates and how many score-T keys precede
 //    it (one thread per chunk reads its 64 bins with vector loads; exclusive scans over
 //    chunks).
-//  compact_kernel (one CTA per chunk and vote pack): each thread owns 32 consecutive keys
+//  compact_kernel (one CTA per chunk and vote pack): each thread owns 64 consecutive keys
 //    (read coalesced and transposed through shared memory). SWAR byte arithmetic tests the
 //    four packed scores of a key against the four heads' thresholds at once, and the test
-//    bits are sliced into one 32-bit mask per head (above T, at T) over the thread's keys.
+//    bits are sliced into 32-bit masks per head (above T, at T) over the thread's keys.
 //    POPC gives the counts; one block-wide scan of them gives every thread where its
 //    candidates start and how many of its ties it keeps (all, none, or -- in the one thread
 //    where the E-th tie falls -- the first few); the set bits are then written in key order.
@@ -173,10 +173,12 @@ threshold_kernel(const uint32_t* __restrict__ hist, int group, int packs, int64_
     }
 }
 
-constexpr int kCW = CHUNK / (32 * 32);          // compaction: warps per block (one chunk)
+constexpr int kKeys = 64;                       // consecutive keys per thread
+constexpr int kWords = kKeys / 32;              // 32-bit key masks per head and kind
+constexpr int kCW = CHUNK / (32 * kKeys);       // compaction: warps per block (one chunk)
 constexpr int kCThr = 32 * kCW;
-constexpr int kKeys = CHUNK / kCThr;            // 32 consecutive keys per thread
-static_assert(kKeys == 32, "one 32-key run per thread");
+constexpr int kRow = kKeys + 1;                 // transposed row stride (conflict-free)
+static_assert(kCW * 32 * kKeys == CHUNK, "one chunk per block");
 
 // Block-wide exclusive scan of two 64-bit values at once (4 packed 16-bit counters each,
 // none of which overflows: a block's total per counter is at most CHUNK).
@@ -203,7 +205,7 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
                const int32_t* __restrict__ cbase, int32_t* __restrict__ cand, int64_t n,
                int64_t cap_pad, int group, int packs, int64_t nchunks, int64_t cmax,
                uint32_t* __restrict__ shist, int* status) {
-    __shared__ uint32_t tr[kCW][32 * 33];
+    __shared__ uint32_t tr[kCW][32 * kRow];
     __shared__ uint64_t scan_sh[kCW + 1][2];
     const int64_t c = blockIdx.x;
     const int64_t up = blockIdx.y;
@@ -215,17 +217,18 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
     const int64_t k0 = kw + static_cast<int64_t>(lane) * kKeys;                // thread's first key
     const int nv = static_cast<int>(max64(0, min64(kKeys, n - k0)));          // its valid keys
 
-    // coalesced load of the warp's 1024 packed scores, transposed so that lane l then reads
-    // keys 32 l .. 32 l + 31 (row stride 33 words: both directions are conflict-free)
+    // coalesced load of the warp's 32 x kKeys packed scores, transposed so that lane l then
+    // reads keys kKeys l .. kKeys l + kKeys - 1 (row stride kKeys + 1 words: both directions
+    // are conflict-free). Asynchronous 4-byte copies, all in flight at once; keys at or past
+    // n read as 0 (zero fill, src-size 0); their address stays inside the padded capacity.
     {
-        // asynchronous 4-byte copies, all in flight at once; keys at or past n read as 0
-        // (zero fill, src-size 0); their address stays inside the padded capacity
         const uint32_t* src = scores + up * cap_pad + kw + lane;
         const int nw = static_cast<int>(max64(0, min64(32 * kKeys, n - kw)));
 #pragma unroll
         for (int t = 0; t < kKeys; ++t) {
-            const uint32_t dst = smem_addr(&tr[warp][t * 33 + lane]);
-            const uint32_t bytes = (32 * t + lane < nw) ? 4u : 0u;
+            const int key = 32 * t + lane;                 // within the warp's range
+            const uint32_t dst = smem_addr(&tr[warp][(key / kKeys) * kRow + key % kKeys]);
+            const uint32_t bytes = key < nw ? 4u : 0u;
             asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst),
                          "l"(src + 32 * t), "r"(bytes) : "memory");
         }
@@ -233,7 +236,7 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
         asm volatile("cp.async.wait_all;" ::: "memory");
         __syncwarp();
     }
-    const uint32_t* s = &tr[warp][lane * 33];
+    const uint32_t* s = &tr[warp][lane * kRow];
     // the scores above were written two kernels back; thresholds and offsets come from the
     // threshold kernel just before this one
     pdl_wait();
@@ -253,36 +256,43 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
         gt_add |= static_cast<uint32_t>(127 - T) << (8 * h);
         ge_add |= static_cast<uint32_t>(128 - T) << (8 * h);
     }
-    // Bit-sliced tests: word q of G (GE) holds, in byte h, bit i = key 8 q + i has
-    // score_h > T_h (>= T_h). Then per head a 32-bit mask over the thread's keys.
-    uint32_t G[4], GE[4];
+    // Bit-sliced tests: for mask word w, word q of G (GE) holds, in byte h, bit i = key
+    // 32 w + 8 q + i has score_h > T_h (>= T_h). Then per head and word a 32-bit key mask.
+    uint32_t gm[PACK][kWords], em[PACK][kWords];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint32_t a = 0, b = 0;
+    for (int w = 0; w < kWords; ++w) {
+        uint32_t G[4], GE[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t sv = s[8 * q + i];
-            a |= (((sv + gt_add) >> 7) & 0x01010101u) << i;
-            b |= (((sv + ge_add) >> 7) & 0x01010101u) << i;
+        for (int q = 0; q < 4; ++q) {
+            uint32_t a = 0, b = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t sv = s[32 * w + 8 * q + i];
+                a |= (((sv + gt_add) >> 7) & 0x01010101u) << i;
+                b |= (((sv + ge_add) >> 7) & 0x01010101u) << i;
+            }
+            G[q] = a;
+            GE[q] = b;
         }
-        G[q] = a;
-        GE[q] = b;
-    }
-    const uint32_t vbits = nv >= 32 ? 0xffffffffu : ((1u << nv) - 1u);
-    uint32_t gm[PACK], em[PACK];
+        const int vw = nv - 32 * w;                         // valid keys in this word
+        const uint32_t vbits = vw >= 32 ? 0xffffffffu : (vw <= 0 ? 0u : ((1u << vw) - 1u));
 #define PKV_HEAD_MASK(W, H)                                                              \
     (prmt_i<0x5410u>(prmt_i<((4u + (H)) << 4) | (H)>(W[0], W[1]),                      \
                      prmt_i<((4u + (H)) << 4) | (H)>(W[2], W[3])))
-    gm[0] = PKV_HEAD_MASK(G, 0) & vbits;  em[0] = PKV_HEAD_MASK(GE, 0) & vbits & ~gm[0];
-    gm[1] = PKV_HEAD_MASK(G, 1) & vbits;  em[1] = PKV_HEAD_MASK(GE, 1) & vbits & ~gm[1];
-    gm[2] = PKV_HEAD_MASK(G, 2) & vbits;  em[2] = PKV_HEAD_MASK(GE, 2) & vbits & ~gm[2];
-    gm[3] = PKV_HEAD_MASK(G, 3) & vbits;  em[3] = PKV_HEAD_MASK(GE, 3) & vbits & ~gm[3];
+        gm[0][w] = PKV_HEAD_MASK(G, 0) & vbits;  em[0][w] = PKV_HEAD_MASK(GE, 0) & vbits & ~gm[0][w];
+        gm[1][w] = PKV_HEAD_MASK(G, 1) & vbits;  em[1][w] = PKV_HEAD_MASK(GE, 1) & vbits & ~gm[1][w];
+        gm[2][w] = PKV_HEAD_MASK(G, 2) & vbits;  em[2][w] = PKV_HEAD_MASK(GE, 2) & vbits & ~gm[2][w];
+        gm[3][w] = PKV_HEAD_MASK(G, 3) & vbits;  em[3][w] = PKV_HEAD_MASK(GE, 3) & vbits & ~gm[3][w];
 #undef PKV_HEAD_MASK
+    }
     uint64_t gb = 0, eb = 0;
 #pragma unroll
     for (int h = 0; h < PACK; ++h) {
-        gb |= static_cast<uint64_t>(__popc(gm[h])) << (16 * h);
-        eb |= static_cast<uint64_t>(__popc(em[h])) << (16 * h);
+        uint32_t ng = 0, ne = 0;
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) { ng += __popc(gm[h][w]); ne += __popc(em[h][w]); }
+        gb |= static_cast<uint64_t>(ng) << (16 * h);
+        eb |= static_cast<uint64_t>(ne) << (16 * h);
     }
     block_excl_scan2(gb, eb, scan_sh);   // keys above T / ties in this chunk before this thread
 
@@ -290,37 +300,50 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
     // chunk keeps the first B = max(0, E - ties before the chunk) of its ties, in key order.
     // Then its candidates are written in key order.
     const int32_t C = thr[head0 * 4 + 2];
+    const int32_t kbase = static_cast<int32_t>(k0);
 #pragma unroll
     for (int h = 0; h < PACK; ++h) {
         if (h >= hp) break;
         const int64_t hb = (static_cast<int64_t>(head0 + h) * nchunks + c) * 2;
-        const int64_t E = thr[(head0 + h) * 4 + 1];
-        const int64_t B = max64(0, E - cbase[hb + 1]);
-        const int64_t gbefore = (gb >> (16 * h)) & 0xffffu, ebefore = (eb >> (16 * h)) & 0xffffu;
-        const int mine_e = __popc(em[h]);
-        const int take = static_cast<int>(min64(max64(B - ebefore, 0), mine_e));
-        uint32_t sel = gm[h];
-        if (take == mine_e) {
-            sel |= em[h];
-        } else {                              // the one thread where the E-th tie falls
-            uint32_t m = em[h];
-            for (int t = 0; t < take; ++t) {
-                const uint32_t low = m & (0u - m);
-                sel |= low;
-                m ^= low;
+        const int32_t E = thr[(head0 + h) * 4 + 1];
+        const int32_t B = max(0, E - cbase[hb + 1]);
+        const int32_t gbefore = static_cast<int32_t>((gb >> (16 * h)) & 0xffffu);
+        const int32_t ebefore = static_cast<int32_t>((eb >> (16 * h)) & 0xffffu);
+        uint32_t sel[kWords];
+        int mine_e = 0, nsel = 0;
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) mine_e += __popc(em[h][w]);
+        const int take = min(max(B - ebefore, 0), mine_e);
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) sel[w] = gm[h][w] | (take == mine_e ? em[h][w] : 0u);
+        if (take != mine_e) {                 // the one thread where the E-th tie falls
+            int left = take;
+#pragma unroll
+            for (int w = 0; w < kWords; ++w) {
+                uint32_t m = em[h][w];
+                for (; left > 0 && m; --left) {
+                    const uint32_t low = m & (0u - m);
+                    sel[w] |= low;
+                    m ^= low;
+                }
             }
         }
-        const int64_t start = cbase[hb + 0] + gbefore + min64(B, ebefore);
-        if (start + __popc(sel) > C) {       // never taken when the histograms are consistent
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) nsel += __popc(sel[w]);
+        const int32_t start = cbase[hb + 0] + gbefore + min(B, ebefore);
+        if (start + nsel > C) {               // never taken when the histograms are consistent
             atomicExch(status, ST_BADINDEX);
             continue;
         }
         int32_t* out = cand + static_cast<int64_t>(head0 + h) * cmax + start;
-        const int32_t kbase = static_cast<int32_t>(k0);
-        while (sel) {
-            const int j = __ffs(sel) - 1;
-            sel &= sel - 1u;
-            *out++ = kbase + j;
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) {
+            uint32_t m = sel[w];
+            while (m) {
+                const int j = __ffs(m) - 1;
+                m &= m - 1u;
+                *out++ = kbase + 32 * w + j;
+            }
         }
     }
 }

@@ -142,10 +142,14 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
         if (up != cur_up) {
             __syncthreads();
             // row c, column 2b + k holds W_b[c] (copies k = 0, 1)
-            const uint32_t* lsrc = lut + up * (NB * NC);
-            const int b = lane >> 1;
-            for (int r = warp; r < NC; r += kWarps)
-                *reinterpret_cast<uint32_t*>(tab + r * 256 + 4 * lane) = __ldg(lsrc + b * NC + r);
+            // (all of a warp's loads are issued before its stores: one round trip)
+            const uint32_t* lsrc = lut + up * (NB * NC) + (lane >> 1) * NC + warp;
+            uint32_t v[NC / kWarps];
+#pragma unroll
+            for (int i = 0; i < NC / kWarps; ++i) v[i] = __ldg(lsrc + kWarps * i);
+#pragma unroll
+            for (int i = 0; i < NC / kWarps; ++i)
+                *reinterpret_cast<uint32_t*>(tab + (warp + kWarps * i) * 256 + 4 * lane) = v[i];
             __syncthreads();
             cur_up = up;
         }
@@ -181,11 +185,20 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
         // flush this chunk's histograms: row 64 h + s, one counter per lane
         __syncthreads();
         uint32_t* hout = hist + (up * nchunks + c) * (PACK * NBINS);
-        for (int r = warp; r < PACK * NBINS; r += kWarps) {
-            uint32_t* a = reinterpret_cast<uint32_t*>(tab + r * 256 + hcol);
-            const uint32_t tot = __reduce_add_sync(0xffffffffu, *a);
-            *a = 0u;
-            if (lane == 0) hout[r] = tot;
+        {
+            constexpr int kRows = PACK * NBINS / kWarps;   // rows warp, warp + kWarps, ...
+            uint32_t v[kRows];
+#pragma unroll
+            for (int i = 0; i < kRows; ++i) {
+                uint32_t* a = reinterpret_cast<uint32_t*>(tab + (warp + kWarps * i) * 256 + hcol);
+                v[i] = *a;
+                *a = 0u;
+            }
+#pragma unroll
+            for (int i = 0; i < kRows; ++i) v[i] = __reduce_add_sync(0xffffffffu, v[i]);
+            if (lane == 0)
+#pragma unroll
+                for (int i = 0; i < kRows; ++i) hout[warp + kWarps * i] = v[i];
         }
         __syncthreads();
         base = next_base;
