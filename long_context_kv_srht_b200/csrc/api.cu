@@ -141,7 +141,7 @@ pariskv_status create_index(const pariskv_config* cfg, const int8_t* signs, cuda
               dalloc(&ix->lut, up * NB * NC) && dalloc(&ix->qt, heads * D) &&
               dalloc(&ix->qnorm, heads) && dalloc(&ix->scores, up * ix->cap_pad) &&
               dalloc(&ix->hist, up * nch * PACK * NBINS) && dalloc(&ix->thr, heads * 4) &&
-              dalloc(&ix->cbase, heads * nch * 2) && dalloc(&ix->shist, heads * SBINS) &&
+              dalloc(&ix->cbase, heads * nch * 2) && dalloc(&ix->shist, heads * SCOPIES * SBINS) &&
               dalloc(&ix->status, 1);
     if (!ok) {
         free_index(ix);

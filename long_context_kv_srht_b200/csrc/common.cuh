@@ -17,6 +17,7 @@ constexpr int REC = 128;        // bytes per key record: 64 B of 4-bit codes + 1
 constexpr int NBINS = 64;       // coarse scores are < 64 (B * w_rank1 <= 48)
 constexpr int SBINS_BITS = 11;  // first radix level of the top-k, counted by the rerank
 constexpr int SBINS = 1 << SBINS_BITS;
+constexpr int SCOPIES = 1;      // copies of that histogram (one copy per warp group spreads the reductions)
 constexpr int CHUNK = 8192;     // keys per coarse-score histogram chunk (a vote work item)
 constexpr int PACK = 4;         // query heads whose vote weights share one 32-bit table entry
 

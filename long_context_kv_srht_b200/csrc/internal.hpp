@@ -31,7 +31,7 @@ struct pariskv_index {
     int32_t* cbase = nullptr;   // [units*group][chunks][2] selected/ties before each chunk
     int32_t* cand = nullptr;    // [units*group][cmax] candidate indices (ascending)
     float* S = nullptr;         // [units*group][cmax] rerank values
-    uint32_t* shist = nullptr;  // [units*group][kSBins] counts of S by the top bits of its order key
+    uint32_t* shist = nullptr;  // [units*group][SCOPIES][SBINS] counts of S by its top order-key bits
     int64_t cmax = 0;
     int* status = nullptr;      // device status word (ST_OK / ST_TIMEOUT)
 

@@ -20,8 +20,9 @@
 //
 // Each value is also counted, by the top bits of its order-preserving image, into a per-head
 // histogram, which is the top-k's first radix level: lanes holding the same bin are grouped
-// with a warp match and one of them adds the group's count (one global reduction per value
-// piled onto the few hot bins and doubled the kernel's time).
+// with a warp match and one of them adds the group's count, into one of SCOPIES copies chosen
+// by the warp. (One global reduction per value piled onto the few hot bins and doubled the
+// kernel's time; with the match, eight copies measured no faster than one.)
 //
 // Scoring: each lane scores two records of a stage (rows lane and lane + 32, whose chains
 // interleave). The warp's current query head has its rotated query in
@@ -254,7 +255,9 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
             const uint32_t bin = ok ? order_key(sv[u]) >> (32 - SBINS_BITS) : 0xffffffffu;
             const uint32_t peers = __match_any_sync(0xffffffffu, bin);
             if (ok && lane == __ffs(peers) - 1)
-                atomicAdd(&shist[sc.head * SBINS + bin], static_cast<uint32_t>(__popc(peers)));
+                atomicAdd(&shist[(static_cast<int64_t>(sc.head) * SCOPIES + (gw & (SCOPIES - 1))) *
+                                     SBINS + bin],
+                          static_cast<uint32_t>(__popc(peers)));
         }
         __syncwarp();                        // every lane has read the slot and the query
         issue(slot, iss, pend);

@@ -242,9 +242,10 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
     pdl_wait();
     pdl_launch_dependents();
     // the rerank that follows counts its values per head into shist: start it at zero
-    if (c == 0)
-        for (int i = threadIdx.x; i < hp * SBINS; i += kCThr)
-            shist[static_cast<int64_t>(head0) * SBINS + i] = 0u;
+    // (the pack's CTAs share the work: CTA c clears words c * kCThr + t, stepping by all)
+    for (int64_t i = c * kCThr + threadIdx.x; i < static_cast<int64_t>(hp) * SCOPIES * SBINS;
+         i += nchunks * kCThr)
+        shist[static_cast<int64_t>(head0) * SCOPIES * SBINS + i] = 0u;
 
     // Per-head thresholds packed one per byte. A head outside the pack gets T = 127, which
     // no score (< 64) reaches. Byte h of (s + gt_add) has bit 7 set iff score_h > T_h, and

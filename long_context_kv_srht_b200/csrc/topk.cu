@@ -12,7 +12,8 @@
 //    memory with asynchronous copies, all in flight at once, and turns S into u in place
 //    (quarters longer than kSlice stay in global memory and are re-read on every pass);
 //  - the first radix level, the top 11 bits of u, was counted by the rerank as it wrote S
-//    (a per-head 2048-bin histogram in global memory), so it costs one read here;
+//    (per head, SCOPIES copies of a 2048-bin histogram in global memory), so it costs one
+//    round of reads here;
 //  - then range-adaptive radix levels: the current interval [lo, hi] is cut into at most 2048
 //    power-of-two-wide bins, every CTA histograms its quarter, and every CTA sums the four
 //    histograms bin by bin over DSMEM and runs the same suffix scan, so all four pick the
@@ -128,8 +129,14 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
     };
     static_assert(SBINS == kBins, "the first level has one bin pair per thread");
     {
-        const uint2 v = reinterpret_cast<const uint2*>(shist + static_cast<int64_t>(head) * SBINS)[threadIdx.x];
-        choose(v.x, v.y, 32 - SBINS_BITS);
+        uint2 v[SCOPIES];
+        const uint2* hs = reinterpret_cast<const uint2*>(shist + static_cast<int64_t>(head) * SCOPIES * SBINS);
+#pragma unroll
+        for (int r = 0; r < SCOPIES; ++r) v[r] = hs[r * (SBINS / 2) + threadIdx.x];
+        uint32_t h0 = 0, h1 = 0;
+#pragma unroll
+        for (int r = 0; r < SCOPIES; ++r) { h0 += v[r].x; h1 += v[r].y; }
+        choose(h0, h1, 32 - SBINS_BITS);
     }
     int level = 0;
     while (lo != hi) {

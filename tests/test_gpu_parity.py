@@ -84,6 +84,7 @@ def test_rotation_within_tolerance(dtype):
     (1, 1, 2, 31, 31, 500),        # k = n
     (1, 1, 1, 33, 5, 10000),       # every key is a candidate
     (1, 1, 4, 8193, 700, 300),     # one key past a chunk boundary
+    (1, 1, 2, 70000, 3000, 10000), # > 65536 candidates per head: top-k reads them from memory
 ])
 def test_stages_bit_exact(batch, hkv, G, n, k, bp):
     sp = workload.spec("tiny", batch=batch, num_kv_heads=hkv, group=G, n=n, dtype="f32",
