@@ -14,9 +14,9 @@
 // records are gathered with asynchronous global->shared copies (cp.async, 16 bytes per lane;
 // eight lanes move one record, so one warp instruction moves four whole records): the kernel
 // is persistent (kCtasPerSm CTAs per SM), every warp owns a ring of kSlots stages of 64
-// records, and a stage is refilled as soon as it has been scored. Piece c of the record in stage row r is
-// stored at 16-byte position c ^ (r mod 8), so that eight lanes reading the same piece of
-// eight different records touch all 32 banks once.
+// records, and a stage is refilled as soon as it has been scored. Piece c of the record in
+// stage row r is stored at 16-byte position c ^ (r mod 8), so that eight lanes reading the
+// same piece of eight different records touch all 32 banks once.
 //
 // Each value is also counted, by the top bits of its order-preserving image, into a per-head
 // histogram, which is the top-k's first radix level: lanes holding the same bin are grouped
@@ -25,11 +25,11 @@
 // kernel's time; with the match, eight copies measured no faster than one.)
 //
 // Scoring: each lane scores two records of a stage (rows lane and lane + 32, whose chains
-// interleave). The warp's current query head has its rotated query in
-// shared memory as (subspace 2t, subspace 2t + 1) fp32 pairs, read with broadcast loads; a
+// interleave). The warp's current query head has its rotated query in shared memory as
+// (subspace 2t, subspace 2t + 1) fp32 pairs, each read once by broadcast for both records; a
 // lane walks the 8 subspace pairs in order, two p chains advancing together in Blackwell's
-// packed fp32x2 FMA (each half an ordinary IEEE fp32 FMA), and extends its S chain after
-// every pair. Decoding is exact integer arithmetic: the stored offset-binary nibbles
+// packed fp32x2 FMA (each half an ordinary IEEE fp32 FMA), and extends each record's S chain
+// after every pair. Decoding is exact integer arithmetic: the stored offset-binary nibbles
 // u = vt + 8 are split into even and odd dims with two masks, a PRMT places u in the
 // mantissa of 2^23, and one packed subtraction of 2^23 + 8 gives vt exactly as fp32.
 #include "common.cuh"

@@ -8,12 +8,16 @@
 // This is the N-proportional part of the decode step: 16 bytes of bucket ids per key are
 // streamed once per KV head and scored for all query heads of its GQA group at once.
 //
-// Design (sm_100a, HBM-bound):
+// Design (sm_100a; measured bound: the L1/shared-memory pipe, about 84 % busy, with DRAM at
+// a third of its bandwidth):
 //  - Lane L scores keys L and L + 32 of a 64-key warp-tile, reading their ids with two
-//    128-bit non-allocating loads (each a fully coalesced 512-byte warp access, the fewest L1
-//    wavefronts per byte); the next tile's ids are loaded while the current one is scored.
-//    (Measured on B200: a cp.async.bulk ring refilled only once all warps had released a
-//    stage stayed far below HBM bandwidth.)
+//    128-bit non-allocating loads (each a fully coalesced 512-byte warp access); the next
+//    tile's ids are loaded while the current one is scored. Measured on B200, staging the ids
+//    in shared memory costs more than it hides, because every staged byte is read again
+//    through the same pipe: a per-warp ring of 1 KB tiles filled by TMA bulk copies
+//    (cp.async.bulk on per-slot mbarriers) ran 51 us against 46 us, the same ring filled by
+//    16-byte cp.async 50 us, and a CTA-wide bulk-copy ring refilled only once all warps had
+//    released a stage stayed far below HBM bandwidth.
 //  - The 32-bit table entry packs the vote weights of up to four query heads (one byte each;
 //    a byte sum never exceeds 48), so one lookup per (key, subspace) serves the whole pack.
 //  - Conflict-free lookups: the table holds two copies of every subspace's 256 entries, and
