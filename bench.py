@@ -172,6 +172,17 @@ def candidate_count(n, k, bp):
 
 
 # ------------------------------------------------------------------------------------ oracle
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def oracle_sample(sp, data, reps: int, heads: int = 4):
     """Times the CPU oracle (as it stands) on one (sequence, KV head) unit of the workload:
     index build untimed, then `reps` searches of `heads` query heads over all n keys."""
@@ -221,7 +232,7 @@ def run_reference(args, ws, rank):
         "config": {"workload": sp.name, "sample": "1 query head x 1 (sequence, KV head) unit",
                    "n": sp.n, "k": sp.k, "cand_bp": sp.cand_bp},
         "cpu_baseline": {"value": value, "unit": "keys/s", "cores": oracle.num_threads(),
-                         "kind": "oracle",
+                         "kind": "oracle", "cpu_model": cpu_model(),
                          "sample": f"each step: one query head over one unit's {sp.n} keys"},
         "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -267,6 +278,23 @@ def decode_step(args, ix, cfg, sp, keys, vals, qs, idx, est, k, H, dev, kv_host)
               "total_ms": app_ms + srch_ms + att_ms,
               "kv_source": "pinned host (UVA)" if kv_host else "HBM",
               "attend_gbs": kv_bytes / (att_ms / 1e3) / 1e9}
+    if kv_host:
+        # the PCIe roofline of the attention: one coalesced pass over 256 MiB of the pinned K
+        # array, read by the device the same way (UVA)
+        nb = min(256 << 20, keys.numel() * keys.element_size()) // 16 * 16
+        sink = torch.zeros(1, dtype=torch.int32, device=dev)
+        pk.read_stream(keys, nb, sink)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(3):
+            e0.record()
+            pk.read_stream(keys, nb, sink)
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        pcie = nb / (min(ts) / 1e3) / 1e9
+        decode["pcie_read_gbs"] = pcie
+        decode["attend_pcie_frac"] = decode["attend_gbs"] / pcie
     decode["search_stage_ms"] = stage
     return decode
 
@@ -425,8 +453,10 @@ def main():
     torch.cuda.synchronize()
     dist_barrier(ws)
     clk = clocks.stop()
-    step_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev0, ev1)]))
+    step_times = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
+    step_ms = float(np.mean(step_times))
     step_ms_max = dist_max(step_ms, ws)
+    step_median = dist_max(float(np.median(step_times)), ws)
     keys_per_step = sp.batch * sp.num_q_heads * sp.n
     value = ws * keys_per_step / (step_ms_max / 1e3)
 
@@ -454,7 +484,8 @@ def main():
                 "peak_kind": peak_kind, "algorithmic_bytes_per_launch": abytes,
                 "traffic": kernel_traffic(dom, sp.name),
                 "step_algorithmic_bytes": step_bytes,
-                "step_frac": step_bytes / (step_ms_max / 1e3) / 1e9 / peak}
+                "step_frac": step_bytes / (step_ms_max / 1e3) / 1e9 / peak,
+                "step_frac_of_nominal_8tbs": step_bytes / (step_ms_max / 1e3) / 8e12}
 
     # host cost of enqueueing one search (the device is kept busy meanwhile), and the same
     # search replayed as a CUDA graph (one launch per step, no host work between kernels)
@@ -531,6 +562,7 @@ def main():
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         v, dt, cores = oracle_sample(sp, data, reps=1)
         cpu = {"value": v, "unit": "keys/s", "cores": cores, "kind": "oracle",
+               "cpu_model": cpu_model(),
                "sample": f"one (sequence, KV head) unit: 4 query heads x {sp.n} keys, "
                          f"index build untimed ({dt:.1f} s timed)"}
 
@@ -538,7 +570,8 @@ def main():
         line = {
             "metric": "keys searched/s per decode step (vote+rerank+top-k)",
             "value": value, "unit": "keys/s", "n_gpus": ws, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": step_ms_max, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": step_ms_max, "ms_per_step_median": step_median,
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": sp.name, "batch": sp.batch, "q_heads": sp.num_q_heads,
                        "kv_heads": sp.num_kv_heads, "d": sp.d, "n": sp.n, "k": k,

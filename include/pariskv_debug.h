@@ -66,6 +66,16 @@ PARISKV_API pariskv_status pariskv_debug_profile(pariskv_index* index, int32_t e
 PARISKV_API pariskv_status pariskv_debug_stage_ms(pariskv_index* index, float* ms,
                                                   int32_t* nstages);
 
+/* Reads `bytes` from `src` once, with coalesced 16-byte loads spread over every SM, and
+ * folds the data into one word that may be written to `sink` (a device pointer to 4 bytes),
+ * on `stream`. Timed with CUDA events around the call it measures how fast the device reads
+ * that memory: for pinned host memory (mapped into the device address space) this is the
+ * PCIe read bandwidth that bounds sparse attention over host K/V. No counterpart on the
+ * pages (a measurement aid). src must be 16-byte aligned and bytes a positive multiple of
+ * 16. Errors: EINVAL, ECUDA. */
+PARISKV_API pariskv_status pariskv_debug_read_stream(const void* src, int64_t bytes,
+                                                     uint32_t* sink, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

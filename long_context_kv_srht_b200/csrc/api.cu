@@ -552,6 +552,21 @@ pariskv_status pariskv_debug_profile(pariskv_index* ix, int32_t enable) {
     return PARISKV_OK;
 }
 
+pariskv_status pariskv_debug_read_stream(const void* src, int64_t bytes, uint32_t* sink,
+                                        void* stream) {
+    if (bytes <= 0 || bytes % 16 != 0)
+        return fail(PARISKV_EINVAL, "bytes=%lld is not a positive multiple of 16",
+                    static_cast<long long>(bytes));
+    pariskv_status s;
+    if ((s = check_dev_ptr(src, 16, "src")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(sink, 4, "sink")) != PARISKV_OK) return s;
+    g_launches = 0;
+    cudaError_t e = launch_read_stream(src, bytes, sink, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "read stream");
+    g_launches = 1;
+    return PARISKV_OK;
+}
+
 pariskv_status pariskv_debug_stage_ms(pariskv_index* ix, float* ms, int32_t* nstages) {
     pariskv_status s = check_index(ix);
     if (s != PARISKV_OK) return s;

@@ -183,7 +183,31 @@ static __device__ __align__(256) float g_attend_scratch[kAttendScratchFloats];
 std::mutex g_scratch_mu;
 float* g_scratch_addr[kMaxScratchDevices] = {};
 
+// One pass over `n16` 16-byte words, four independent loads in flight per thread.
+__global__ void __launch_bounds__(256)
+read_stream_kernel(const uint4* __restrict__ p, int64_t n16, uint32_t* __restrict__ sink) {
+    uint32_t acc = 0;
+    int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (; i + 3 * stride < n16; i += 4 * stride) {
+        const uint4 a = p[i], b = p[i + stride], c = p[i + 2 * stride], d = p[i + 3 * stride];
+        acc ^= a.x ^ b.y ^ c.z ^ d.w;
+    }
+    for (; i < n16; i += stride) acc ^= p[i].x;
+    if (acc == 0x9E3779B9u) *sink = acc;   // keeps the loads; almost never stores
+}
+
 }  // namespace
+
+cudaError_t launch_read_stream(const void* src, int64_t bytes, uint32_t* sink,
+                               cudaStream_t st) {
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    read_stream_kernel<<<4 * sms, 256, 0, st>>>(static_cast<const uint4*>(src), bytes / 16,
+                                                 sink);
+    return cudaGetLastError();
+}
 
 cudaError_t attend_static_scratch(float** ptr) {
     int dev = -1;

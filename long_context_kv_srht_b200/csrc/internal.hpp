@@ -108,6 +108,8 @@ cudaError_t launch_topk(const pariskv_index* ix, int64_t C, int32_t k, int32_t* 
                         float* topk_est, cudaStream_t st);
 
 // attend.cu
+cudaError_t launch_read_stream(const void* src, int64_t bytes, uint32_t* sink,
+                               cudaStream_t st);
 cudaError_t launch_attend(const pariskv_config* cfg, const void* q, const void* K,
                           const void* V, int64_t ld_tok, int64_t n, const int32_t* topk_idx,
                           int32_t k, float scale, void* out, int32_t out_dtype, float* work,

@@ -78,6 +78,7 @@ _SIGS = {
     "pariskv_debug_export_search": (_S, [_P, _P, _P, ctypes.POINTER(_I64), _P, _P]),
     "pariskv_debug_profile": (_S, [_P, _I32]),
     "pariskv_debug_stage_ms": (_S, [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_I32)]),
+    "pariskv_debug_read_stream": (_S, [_P, _I64, _P, _P]),
 }
 
 STAGES = ("query_prep", "vote", "threshold", "compact", "rerank", "topk")
@@ -300,3 +301,10 @@ def sparse_attend_noalloc(cfg: Config, q, K, V, topk_idx, k: int, scale: float,
 
 def last_launch_count() -> int:
     return int(lib.pariskv_last_launch_count())
+
+
+def read_stream(src, nbytes: int, sink, stream=None) -> None:
+    """pariskv_debug_read_stream: one coalesced pass over nbytes of ``src`` (a device tensor
+    or a pinned host tensor); ``sink`` is a device tensor of at least 4 bytes."""
+    _check(lib.pariskv_debug_read_stream(src.data_ptr(), int(nbytes), sink.data_ptr(),
+                                         _stream(stream)), "pariskv_debug_read_stream")
