@@ -7,10 +7,11 @@
 // index, and returned in ascending key order with est = ||q|| * S.
 //
 // Exact selection on the order-preserving 32-bit image u of S (flip all bits of negative
-// values, set the sign bit of the others). A head's candidates are split over CL CTAs: a
-// single 256-thread CTA when they fit its shared memory (up to 8192, with a smaller slice up
-// to 4096 so four CTAs share an SM; with many heads this keeps the launch in about one
-// wave), else a cluster of four 1024-thread CTAs:
+// values, set the sign bit of the others). A head's candidates are split over CL CTAs: one
+// CTA when they fit its shared memory (up to 8192) -- 1024 threads when there are no more
+// heads than SMs, else 256 threads (with a 4096-value slice when it suffices, so four CTAs
+// share an SM and even many heads run in about one wave) -- and otherwise a cluster of four
+// 1024-thread CTAs:
 //  - CTA r copies the r-th part of the head's S values and candidate indices into shared
 //    memory with asynchronous copies, all in flight at once, and turns S into u in place
 //    (parts longer than the slice stay in global memory and are re-read on every pass);
@@ -281,6 +282,12 @@ cudaError_t launch_cfg(const pariskv_index* ix, int64_t C, int32_t k, int32_t* t
 
 cudaError_t launch_topk(const pariskv_index* ix, int64_t C, int32_t k, int32_t* topk_idx,
                         float* topk_est, cudaStream_t st) {
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int heads = ix->units * ix->cfg.group;
+    if (C <= 8192 && heads <= sms)   // at most one head per SM: use all of its threads
+        return launch_cfg<1, 1024, 8192, true>(ix, C, k, topk_idx, topk_est, st);
     if (C <= 4096) return launch_cfg<1, 256, 4096, true>(ix, C, k, topk_idx, topk_est, st);
     if (C <= 8192) return launch_cfg<1, 256, 8192, true>(ix, C, k, topk_idx, topk_est, st);
     if (C <= 4 * 16384)
