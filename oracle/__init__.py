@@ -246,3 +246,61 @@ def search(enc: Encoded, q: np.ndarray, signs: np.ndarray, k: int, p: SearchPara
     """One query head from its raw query vector [d]."""
     qt, qn = normalize_rotate(q[None, :], signs)
     return search_rotated(enc, qt[0], float(qn[0]), k, p)
+
+
+# ---------------------------------------------------------------------------------------
+# Four-region KV cache ("Technical Summary: ParisKV", System-Level Innovations 2,
+# "Sliding-Window Update Mechanism"): Sink and Local stay on the GPU, older tokens go to
+# the Retrieval zone, new tokens collect in an Update Buffer; a full buffer evicts the oldest
+# Local tokens to Retrieval and joins Local. Token positions are tracked as plain lists.
+# Readings where the page is silent: a token enters Sink while Sink is short, else the
+# buffer; a promotion evicts the max(0, |Local| + |buffer| - n_local) oldest Local tokens;
+# prefill fills Sink first, then the last n_local tokens go to Local and the rest between
+# the two to Retrieval.
+# ---------------------------------------------------------------------------------------
+class CacheRegions:
+    def __init__(self, n_sink: int, n_local: int, n_buffer: int):
+        assert n_sink >= 0 and 1 <= n_buffer <= n_local
+        self.n_sink, self.n_local, self.n_buffer = n_sink, n_local, n_buffer
+        self.sink, self.local, self.buffer, self.retrieval = [], [], [], []
+        self.total = 0
+
+    def prefill(self, n: int) -> None:
+        assert self.total == 0
+        toks = list(range(n))
+        self.sink = toks[: self.n_sink]
+        rest = toks[self.n_sink:]
+        n_loc = min(len(rest), self.n_local)
+        self.local = rest[len(rest) - n_loc:]
+        self.retrieval = rest[: len(rest) - n_loc]
+        self.total = n
+
+    def append(self) -> None:
+        t = self.total
+        self.total += 1
+        if len(self.sink) < self.n_sink:
+            self.sink.append(t)
+            return
+        self.buffer.append(t)
+        if len(self.buffer) == self.n_buffer:
+            drop = max(0, len(self.local) + len(self.buffer) - self.n_local)
+            self.retrieval += self.local[:drop]
+            self.local = self.local[drop:] + self.buffer
+            self.buffer = []
+
+    def dense(self) -> list:
+        """Tokens every step attends to exactly: Sink, Local and buffer."""
+        return self.sink + self.local + self.buffer
+
+
+def cache_step_attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, regions: CacheRegions,
+                      enc: Encoded, signs: np.ndarray, k: int, scale: float, p: SearchParams):
+    """One decode step's attention for one query head: a ParisKV search over the Retrieval
+    zone's index (enc holds the Retrieval tokens in order), then one softmax over the dense
+    tokens plus the retrieved ones. K, V: [total, d] indexed by token position. Returns
+    (out, retrieved Retrieval rows)."""
+    rows = np.empty((0,), np.int32)
+    if regions.retrieval:
+        rows, *_ = search(enc, q, signs, min(k, len(regions.retrieval)), p)
+    toks = np.asarray(regions.dense() + [regions.retrieval[r] for r in rows], np.int32)
+    return attend(q, K, V, toks, scale), rows

@@ -343,3 +343,62 @@ def test_tiny_workload_retrieves_planted_keys():
     true_top = set(np.argsort(-exact, kind="stable")[:sp.k].tolist())
     recall = len(true_top & set(idx.tolist())) / sp.k
     assert recall >= 0.5, recall
+
+
+# ----------------------------------------------------------------------------- four-region cache
+def test_cache_regions_worked_example():
+    """Hand-traced against the Sliding-Window Update Mechanism ("Technical Summary: ParisKV",
+    System-Level Innovations 2): n_sink=2, n_local=4, n_buffer=2, prefill of 9 tokens."""
+    r = oracle.CacheRegions(2, 4, 2)
+    r.prefill(9)
+    assert (r.sink, r.local, r.buffer, r.retrieval) == ([0, 1], [5, 6, 7, 8], [], [2, 3, 4])
+    r.append()                                    # token 9 waits in the buffer
+    assert (r.local, r.buffer, r.retrieval) == ([5, 6, 7, 8], [9], [2, 3, 4])
+    r.append()                                    # buffer full: 5, 6 evicted, 9, 10 join Local
+    assert (r.local, r.buffer, r.retrieval) == ([7, 8, 9, 10], [], [2, 3, 4, 5, 6])
+    short = oracle.CacheRegions(3, 4, 2)          # a short prefill leaves Sink to fill first
+    short.prefill(1)
+    short.append(); short.append()
+    assert (short.sink, short.local, short.buffer) == ([0, 1, 2], [], [])
+    short.append(); short.append()                # Local not yet full: nothing evicted
+    assert (short.local, short.buffer, short.retrieval) == ([3, 4], [], [])
+
+
+@pytest.mark.parametrize("cfg", [(0, 8, 8, 0), (4, 16, 4, 100), (4, 16, 16, 3), (1, 5, 2, 40)])
+def test_cache_regions_invariants(cfg):
+    """Over a long run: the regions partition the tokens seen so far, each region keeps token
+    order, Retrieval row r holds token n_sink + r, Local never exceeds n_local and the buffer
+    stays below n_buffer, and the newest token is always in a dense region."""
+    n_sink, n_local, n_buffer, n0 = cfg
+    r = oracle.CacheRegions(n_sink, n_local, n_buffer)
+    r.prefill(n0)
+    for _ in range(300):
+        r.append()
+        allt = r.sink + r.retrieval + r.local + r.buffer
+        assert allt == list(range(r.total))
+        assert len(r.local) <= n_local and len(r.buffer) < n_buffer
+        assert r.retrieval == list(range(n_sink, n_sink + len(r.retrieval)))
+        assert r.total - 1 in r.dense()
+        if r.retrieval:                            # Local is full once anything was evicted
+            assert len(r.local) + len(r.buffer) >= n_local
+
+
+def test_cache_step_attend_is_dense_softmax_when_k_covers_retrieval():
+    """With k at least the Retrieval size every token is attended: the result equals plain
+    softmax attention over all tokens (numpy, fp64)."""
+    rng = np.random.default_rng(5)
+    s = _signs(D, 3)
+    r = oracle.CacheRegions(2, 8, 4)
+    r.prefill(30)
+    for _ in range(7):
+        r.append()
+    K = rng.standard_normal((r.total, D)).astype(np.float32)
+    V = rng.standard_normal((r.total, D)).astype(np.float32)
+    q = rng.standard_normal(D).astype(np.float32)
+    enc = oracle.build_unit(K[r.retrieval], s, M)
+    out, rows = oracle.cache_step_attend(q, K, V, r, enc, s, 64, 0.09,
+                                         oracle.SearchParams(m=M, cand_bp=10000))
+    assert sorted(rows.tolist()) == list(range(len(r.retrieval)))
+    z = K.astype(np.float64) @ q.astype(np.float64) * 0.09
+    w = np.exp(z - z.max())
+    np.testing.assert_allclose(out, (w / w.sum()) @ V.astype(np.float64), rtol=1e-10, atol=1e-12)
