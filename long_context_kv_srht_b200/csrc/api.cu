@@ -99,6 +99,19 @@ pariskv_status check_dev_ptr(const void* p, size_t align, const char* name) {
     return PARISKV_OK;
 }
 
+}  // namespace
+
+namespace pkv {
+bool alloc_fault_injected() { return fault_alloc(); }
+pariskv_status check_device_pointer(const void* p, size_t align, const char* name) {
+    return check_dev_ptr(p, align, name);
+}
+void set_last_launches(int32_t n) { g_launches = n; }
+int32_t last_launches() { return g_launches; }
+}  // namespace pkv
+
+namespace {
+
 pariskv_status check_index(const pariskv_index* ix) {
     if (!ix) return fail(PARISKV_EINVAL, "index is NULL");
     int dev = -1;

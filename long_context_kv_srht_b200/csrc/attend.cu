@@ -70,7 +70,8 @@ template <typename T>
 __global__ void __launch_bounds__(kAW * 32)
 attend_partial_kernel(const T* __restrict__ q, const T* __restrict__ K, const T* __restrict__ V,
                       int64_t ld_tok, int64_t n, const int32_t* __restrict__ topk, int32_t k,
-                      float scale, int group, int nsplit, float* __restrict__ work) {
+                      int32_t k_stride, float scale, int group, int nsplit, int split_base,
+                      int split_total, float* __restrict__ work) {
     __shared__ __align__(16) float sm[kAW][kPart];
     const int head = blockIdx.y, split = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -82,7 +83,7 @@ attend_partial_kernel(const T* __restrict__ q, const T* __restrict__ K, const T*
     Elem<T>::load4(q + static_cast<int64_t>(head) * D + 4 * lane, qv);
     const T* Kb = K + unit * ld_tok * D + 4 * lane;
     const T* Vb = V + unit * ld_tok * D + 4 * lane;
-    const int32_t* idx = topk + static_cast<int64_t>(head) * k;
+    const int32_t* idx = topk + static_cast<int64_t>(head) * k_stride;
 
     float mx = -INFINITY, den = 0.0f, acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     // this warp's tokens: t0 + warp, t0 + warp + kAW, ...; their indices are fetched 64 at a
@@ -147,7 +148,7 @@ attend_partial_kernel(const T* __restrict__ q, const T* __restrict__ K, const T*
 #pragma unroll
             for (int i = 0; i < 4; ++i) a[i] += sm[w][4 * lane + i] * f;
         }
-        float* out = work + (static_cast<int64_t>(head) * nsplit + split) * kPart;
+        float* out = work + (static_cast<int64_t>(head) * split_total + split_base + split) * kPart;
         *reinterpret_cast<float4*>(out + 4 * lane) = make_float4(a[0], a[1], a[2], a[3]);
         if (lane == 0) { out[kMax] = M; out[kDen] = dsum; }
     }
@@ -238,29 +239,48 @@ size_t attend_workspace_floats(int heads, int nsplit) {
     return static_cast<size_t>(heads) * nsplit * kPart;
 }
 
-cudaError_t launch_attend(const pariskv_config* cfg, const void* q, const void* K,
-                          const void* V, int64_t ld_tok, int64_t n, const int32_t* topk_idx,
-                          int32_t k, float scale, void* out, int32_t out_dtype, float* work,
-                          int nsplit, cudaStream_t st) {
+cudaError_t launch_attend_partial(const pariskv_config* cfg, const void* q, const void* K,
+                                  const void* V, int64_t ld_tok, int64_t n,
+                                  const int32_t* idx, int32_t k, int32_t k_stride, float scale,
+                                  float* work, int nsplit, int split_base, int split_total,
+                                  cudaStream_t st) {
     const int heads = cfg->batch * cfg->num_kv_heads * cfg->group;
     dim3 grid(nsplit, heads);
     if (cfg->dtype == PARISKV_BF16) {
         using T = __nv_bfloat16;
         attend_partial_kernel<T><<<grid, kAW * 32, 0, st>>>(
             static_cast<const T*>(q), static_cast<const T*>(K), static_cast<const T*>(V),
-            ld_tok, n, topk_idx, k, scale, cfg->group, nsplit, work);
+            ld_tok, n, idx, k, k_stride, scale, cfg->group, nsplit, split_base, split_total,
+            work);
     } else {
         attend_partial_kernel<float><<<grid, kAW * 32, 0, st>>>(
             static_cast<const float*>(q), static_cast<const float*>(K),
-            static_cast<const float*>(V), ld_tok, n, topk_idx, k, scale, cfg->group, nsplit,
-            work);
+            static_cast<const float*>(V), ld_tok, n, idx, k, k_stride, scale, cfg->group, nsplit,
+            split_base, split_total, work);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attend_combine(int heads, const float* work, int split_total, void* out,
+                                  int32_t out_dtype, cudaStream_t st) {
     if (out_dtype == PARISKV_BF16)
         attend_combine_kernel<__nv_bfloat16><<<heads, 32, 0, st>>>(
-            work, nsplit, static_cast<__nv_bfloat16*>(out));
+            work, split_total, static_cast<__nv_bfloat16*>(out));
     else
-        attend_combine_kernel<float><<<heads, 32, 0, st>>>(work, nsplit, static_cast<float*>(out));
+        attend_combine_kernel<float><<<heads, 32, 0, st>>>(work, split_total,
+                                                           static_cast<float*>(out));
     return cudaGetLastError();
+}
+
+cudaError_t launch_attend(const pariskv_config* cfg, const void* q, const void* K,
+                          const void* V, int64_t ld_tok, int64_t n, const int32_t* topk_idx,
+                          int32_t k, float scale, void* out, int32_t out_dtype, float* work,
+                          int nsplit, cudaStream_t st) {
+    cudaError_t e = launch_attend_partial(cfg, q, K, V, ld_tok, n, topk_idx, k, k, scale, work,
+                                          nsplit, 0, nsplit, st);
+    if (e != cudaSuccess) return e;
+    const int heads = cfg->batch * cfg->num_kv_heads * cfg->group;
+    return launch_attend_combine(heads, work, nsplit, out, out_dtype, st);
 }
 
 }  // namespace pkv

@@ -1,0 +1,357 @@
+// cache.cu -- four-region KV cache for unbounded decoding (pariskv_cache.h).
+//
+// "Technical Summary: ParisKV", System-Level Innovations 2 ("Sliding-Window Update
+// Mechanism"): Sink and Local tokens stay on the GPU, older tokens are offloaded to the
+// Retrieval zone and found through the index, and an Update Buffer collects new tokens;
+// when it fills, the oldest Local tokens are evicted to Retrieval and the buffer becomes
+// Local. System-Level Innovations 1 (UVA offloading): the attention reads the offloaded
+// K/V rows of the retrieved tokens directly from pinned host memory.
+//
+// Region bookkeeping is host-side (the counts are the same for every (sequence, KV head)),
+// and every data movement is stream-ordered:
+//  - the new token's K/V row goes to the end of the device pool (one 2-D copy per tensor);
+//  - a promotion copies the evicted rows to the host Retrieval arrays (2-D copies, device
+//    to pinned host), appends their keys to the index (the encode kernel reads them from
+//    the pool), then slides the remaining Local and buffer rows down over them through a
+//    scratch buffer, so Sink, Local and buffer always occupy pool rows [0, n_dense);
+//  - the search runs on the index of the Retrieval zone; the attention writes split-K
+//    partials for the dense rows (every head reads rows 0..n_dense-1 of its unit's pool)
+//    and for the retrieved rows (pinned host memory) into one workspace, and one merge
+//    (log-sum-exp) gives a single softmax over the union.
+#include <cuda_runtime.h>
+
+#include <new>
+
+#include "common.cuh"
+#include "internal.hpp"
+#include "pariskv_cache.h"
+
+using namespace pkv;
+
+struct pariskv_cache {
+    pariskv_config cfg;           // capacity = retrieval_capacity
+    pariskv_cache_config cc;
+    int device = 0;
+    int units = 0, heads = 0;
+    int64_t P = 0;                // pool rows per unit: n_sink + n_local + n_buffer
+    size_t row = 0;               // bytes per K or V row
+    uint8_t* poolK = nullptr;     // device [units][P][d]
+    uint8_t* poolV = nullptr;
+    uint8_t* tmp = nullptr;       // device [units][n_local + n_buffer][d] (one tensor at a time)
+    uint8_t* hostK = nullptr;     // pinned host [units][R][d]
+    uint8_t* hostV = nullptr;
+    int32_t* dense_idx = nullptr; // device [P]: 0, 1, ..., P - 1 (every head reads it)
+    int32_t* topk = nullptr;      // device [heads][k]
+    float* work = nullptr;        // device [heads][max_splits][partial]
+    int max_splits = 0;           // per source (dense, retrieved)
+    int sms = 0;
+    pariskv_index* ix = nullptr;
+    int64_t sink = 0, local = 0, buffer = 0, retr = 0;
+};
+
+namespace {
+
+__global__ void iota_kernel(int32_t* p, int64_t n) {
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i < n) p[i] = static_cast<int32_t>(i);
+}
+
+void free_cache(pariskv_cache* c) {
+    if (!c) return;
+    if (c->ix) pariskv_destroy(c->ix);
+    cudaFree(c->poolK);
+    cudaFree(c->poolV);
+    cudaFree(c->tmp);
+    cudaFree(c->dense_idx);
+    cudaFree(c->topk);
+    cudaFree(c->work);
+    if (c->hostK) cudaFreeHost(c->hostK);
+    if (c->hostV) cudaFreeHost(c->hostV);
+    delete c;
+}
+
+template <typename T>
+bool dev_alloc(T** p, size_t bytes) {
+    *p = nullptr;
+    if (alloc_fault_injected()) return false;
+    if (cudaMalloc(reinterpret_cast<void**>(p), bytes) != cudaSuccess) {
+        cudaGetLastError();
+        *p = nullptr;
+        return false;
+    }
+    return true;
+}
+
+bool host_alloc(uint8_t** p, size_t bytes) {
+    *p = nullptr;
+    if (alloc_fault_injected()) return false;
+    if (cudaHostAlloc(reinterpret_cast<void**>(p), bytes, cudaHostAllocMapped) != cudaSuccess) {
+        cudaGetLastError();
+        *p = nullptr;
+        return false;
+    }
+    return true;
+}
+
+pariskv_status check_cache(const pariskv_cache* c) {
+    if (!c) return fail(PARISKV_EINVAL, "cache is NULL");
+    int dev = -1;
+    cudaGetDevice(&dev);
+    if (dev != c->device)
+        return fail(PARISKV_EINVAL, "cache lives on device %d but device %d is current",
+                    c->device, dev);
+    return PARISKV_OK;
+}
+
+// rows [r0, r0 + nr) of every unit: src (pitch src_rows rows) -> dst (pitch dst_rows rows)
+cudaError_t copy_rows(void* dst, int64_t dst_rows, int64_t dst_r0, const void* src,
+                      int64_t src_rows, int64_t src_r0, int64_t nr, int units, size_t row,
+                      cudaStream_t st) {
+    if (nr <= 0) return cudaSuccess;
+    return cudaMemcpy2DAsync(static_cast<uint8_t*>(dst) + dst_r0 * row, dst_rows * row,
+                             static_cast<const uint8_t*>(src) + src_r0 * row, src_rows * row,
+                             nr * row, units, cudaMemcpyDefault, st);
+}
+
+// Evicts the oldest `move` Local rows to the Retrieval zone and slides the rest of Local
+// and the buffer down over them.
+pariskv_status evict(pariskv_cache* c, int64_t move, cudaStream_t st) {
+    const int64_t R = c->cc.retrieval_capacity;
+    const int64_t rest = c->local + c->buffer - move;   // rows that stay after Sink
+    cudaError_t e = copy_rows(c->hostK, R, c->retr, c->poolK, c->P, c->sink, move, c->units,
+                              c->row, st);
+    if (e == cudaSuccess)
+        e = copy_rows(c->hostV, R, c->retr, c->poolV, c->P, c->sink, move, c->units, c->row,
+                      st);
+    if (e != cudaSuccess) return cuda_fail(e, "eviction copy");
+    pariskv_status s = pariskv_append(c->ix, c->poolK + c->sink * c->row, c->P, move, st);
+    if (s != PARISKV_OK) return s;
+    for (uint8_t* pool : {c->poolK, c->poolV}) {
+        const int64_t tr = c->cc.n_local + c->cc.n_buffer;
+        e = copy_rows(c->tmp, tr, 0, pool, c->P, c->sink + move, rest, c->units, c->row, st);
+        if (e == cudaSuccess)
+            e = copy_rows(pool, c->P, c->sink, c->tmp, tr, 0, rest, c->units, c->row, st);
+        if (e != cudaSuccess) return cuda_fail(e, "pool compaction");
+    }
+    c->retr += move;
+    return PARISKV_OK;
+}
+
+// Partials of the dense rows and of the retrieved rows, merged into `out`.
+pariskv_status attend(pariskv_cache* c, const void* q, float scale, int32_t k_eff, void* out,
+                      int32_t out_dtype, cudaStream_t st, int32_t* launches) {
+    const int64_t n_dense = c->sink + c->local + c->buffer;
+    const int nd = min(attend_splits(c->heads, static_cast<int32_t>(n_dense), c->sms),
+                       c->max_splits);
+    const int nr = k_eff > 0 ? min(attend_splits(c->heads, k_eff, c->sms), c->max_splits) : 0;
+    cudaError_t e = launch_attend_partial(&c->cfg, q, c->poolK, c->poolV, c->P, n_dense,
+                                          c->dense_idx, static_cast<int32_t>(n_dense), 0,
+                                          scale, c->work, nd, 0, nd + nr, st);
+    *launches += 1;
+    if (e == cudaSuccess && nr > 0) {
+        e = launch_attend_partial(&c->cfg, q, c->hostK, c->hostV, c->cc.retrieval_capacity,
+                                  c->retr, c->topk, k_eff, k_eff, scale, c->work, nr, nd,
+                                  nd + nr, st);
+        *launches += 1;
+    }
+    if (e == cudaSuccess) {
+        e = launch_attend_combine(c->heads, c->work, nd + nr, out, out_dtype, st);
+        *launches += 1;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    return PARISKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pariskv_status pariskv_cache_create(const pariskv_config* cfg, const pariskv_cache_config* cc,
+                                    const int8_t* srht_signs, void* stream,
+                                    pariskv_cache** out) {
+    if (!out) return fail(PARISKV_EINVAL, "out is NULL");
+    *out = nullptr;
+    if (!cfg || !cc) return fail(PARISKV_EINVAL, "config is NULL");
+    if (cc->n_sink < 0 || cc->n_buffer < 1 || cc->n_local < cc->n_buffer || cc->k < 1 ||
+        cc->retrieval_capacity < 1)
+        return fail(PARISKV_EINVAL, "cache config needs n_sink >= 0, n_buffer >= 1, "
+                    "n_local >= n_buffer, k >= 1, retrieval_capacity >= 1");
+    pariskv_config icfg = *cfg;
+    icfg.capacity = cc->retrieval_capacity;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    pariskv_index* ix = nullptr;
+    // an empty index validates the configuration and the signs
+    pariskv_status s = pariskv_build_index(&icfg, srht_signs, nullptr, 0, 0, stream, &ix);
+    if (s != PARISKV_OK) return s;
+    pariskv_cache* c = new (std::nothrow) pariskv_cache();
+    if (!c) {
+        pariskv_destroy(ix);
+        return fail(PARISKV_ENOMEM, "host allocation failed");
+    }
+    c->cfg = icfg;
+    c->cc = *cc;
+    c->ix = ix;
+    cudaGetDevice(&c->device);
+    cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, c->device);
+    c->units = icfg.batch * icfg.num_kv_heads;
+    c->heads = c->units * icfg.group;
+    c->P = static_cast<int64_t>(cc->n_sink) + cc->n_local + cc->n_buffer;
+    c->row = static_cast<size_t>(D) * (icfg.dtype == PARISKV_BF16 ? 2 : 4);
+    c->max_splits = max(1, 2 * c->sms / c->heads) + 1;
+    const size_t pool = static_cast<size_t>(c->units) * c->P * c->row;
+    const size_t host = static_cast<size_t>(c->units) * cc->retrieval_capacity * c->row;
+    const bool ok =
+        dev_alloc(&c->poolK, pool) && dev_alloc(&c->poolV, pool) &&
+        dev_alloc(&c->tmp, static_cast<size_t>(c->units) * (cc->n_local + cc->n_buffer) *
+                               c->row) &&
+        dev_alloc(&c->dense_idx, static_cast<size_t>(c->P) * 4) &&
+        dev_alloc(&c->topk, static_cast<size_t>(c->heads) * cc->k * 4) &&
+        dev_alloc(&c->work, attend_workspace_floats(c->heads, 2 * c->max_splits) * 4) &&
+        host_alloc(&c->hostK, host) && host_alloc(&c->hostV, host);
+    if (!ok) {
+        free_cache(c);
+        return fail(PARISKV_ENOMEM, "cache allocation failed");
+    }
+    iota_kernel<<<static_cast<unsigned>(ceil_div(c->P, 256)), 256, 0, st>>>(c->dense_idx, c->P);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        free_cache(c);
+        return cuda_fail(e, "cache initialisation");
+    }
+    *out = c;
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_cache_prefill(pariskv_cache* c, const void* K, const void* V,
+                                     int64_t ld_tok, int64_t n, void* stream) {
+    pariskv_status s = check_cache(c);
+    if (s != PARISKV_OK) return s;
+    if (c->sink + c->local + c->buffer + c->retr != 0)
+        return fail(PARISKV_EINVAL, "prefill needs an empty cache");
+    if (n < 0 || (n > 0 && ld_tok < n)) return fail(PARISKV_EINVAL, "n < 0 or ld_tok < n");
+    if (n == 0) return PARISKV_OK;
+    const size_t al = c->cfg.dtype == PARISKV_BF16 ? 8 : 16;
+    if ((s = check_device_pointer(K, al, "K")) != PARISKV_OK) return s;
+    if ((s = check_device_pointer(V, al, "V")) != PARISKV_OK) return s;
+    const int64_t ns = min64(n, c->cc.n_sink), rest = n - ns;
+    const int64_t nl = min64(rest, c->cc.n_local), nr = rest - nl;
+    if (nr > c->cc.retrieval_capacity)
+        return fail(PARISKV_ECAPACITY, "prefill puts %lld tokens in a Retrieval zone of %lld",
+                    static_cast<long long>(nr),
+                    static_cast<long long>(c->cc.retrieval_capacity));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t R = c->cc.retrieval_capacity;
+    cudaError_t e = cudaSuccess;
+    for (int t = 0; t < 2 && e == cudaSuccess; ++t) {
+        const void* src = t ? V : K;
+        uint8_t* pool = t ? c->poolV : c->poolK;
+        uint8_t* hostz = t ? c->hostV : c->hostK;
+        e = copy_rows(pool, c->P, 0, src, ld_tok, 0, ns, c->units, c->row, st);
+        if (e == cudaSuccess)
+            e = copy_rows(pool, c->P, ns, src, ld_tok, ns + nr, nl, c->units, c->row, st);
+        if (e == cudaSuccess)
+            e = copy_rows(hostz, R, 0, src, ld_tok, ns, nr, c->units, c->row, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "prefill copy");
+    if (nr > 0) {
+        s = pariskv_append(c->ix, static_cast<const uint8_t*>(K) + ns * c->row, ld_tok, nr,
+                           stream);
+        if (s != PARISKV_OK) return s;
+    }
+    c->sink = ns;
+    c->local = nl;
+    c->buffer = 0;
+    c->retr = nr;
+    set_last_launches(nr > 0 ? 1 : 0);
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_cache_step(pariskv_cache* c, const void* q, const void* k_new,
+                                  const void* v_new, float scale, void* out, int32_t out_dtype,
+                                  int32_t* topk_idx, void* stream) {
+    pariskv_status s = check_cache(c);
+    if (s != PARISKV_OK) return s;
+    const size_t al = c->cfg.dtype == PARISKV_BF16 ? 8 : 16;
+    if ((s = check_device_pointer(q, al, "q")) != PARISKV_OK) return s;
+    if ((s = check_device_pointer(k_new, al, "k_new")) != PARISKV_OK) return s;
+    if ((s = check_device_pointer(v_new, al, "v_new")) != PARISKV_OK) return s;
+    if ((s = check_device_pointer(out, out_dtype == PARISKV_BF16 ? 8 : 16, "out")) != PARISKV_OK)
+        return s;
+    if (out_dtype != PARISKV_F32 && out_dtype != PARISKV_BF16)
+        return fail(PARISKV_EINVAL, "out_dtype %d unknown", out_dtype);
+    if (topk_idx && (s = check_device_pointer(topk_idx, 4, "topk_idx")) != PARISKV_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // where the new token goes, and whether this step promotes the buffer
+    const bool to_sink = c->sink < c->cc.n_sink;
+    const int64_t nb = c->buffer + (to_sink ? 0 : 1);
+    const bool promote = !to_sink && nb == c->cc.n_buffer;
+    const int64_t move = promote ? max64(0, c->local + nb - c->cc.n_local) : 0;
+    if (c->retr + move > c->cc.retrieval_capacity)
+        return fail(PARISKV_ECAPACITY, "the Retrieval zone (%lld tokens) is full",
+                    static_cast<long long>(c->cc.retrieval_capacity));
+
+    int32_t launches = 0;
+    const int64_t at = c->sink + c->local + c->buffer;   // first free pool row
+    cudaError_t e = copy_rows(c->poolK, c->P, at, k_new, 1, 0, 1, c->units, c->row, st);
+    if (e == cudaSuccess) e = copy_rows(c->poolV, c->P, at, v_new, 1, 0, 1, c->units, c->row, st);
+    if (e != cudaSuccess) return cuda_fail(e, "token copy");
+    if (to_sink) {
+        ++c->sink;
+    } else {
+        c->buffer = nb;
+        if (promote) {
+            if (move > 0) {
+                if ((s = evict(c, move, st)) != PARISKV_OK) return s;
+                launches += 1;
+            }
+            c->local = c->local + c->buffer - move;
+            c->buffer = 0;
+        }
+    }
+
+    int32_t k_eff = 0;
+    if (c->retr > 0) {
+        k_eff = static_cast<int32_t>(min64(c->cc.k, c->retr));
+        s = pariskv_search(c->ix, q, k_eff, c->topk, nullptr, stream);
+        if (s != PARISKV_OK) return s;
+        launches += last_launches();
+    }
+    if ((s = attend(c, q, scale, k_eff, out, out_dtype, st, &launches)) != PARISKV_OK) return s;
+    if (topk_idx) {
+        const size_t bytes = static_cast<size_t>(c->heads) * c->cc.k * 4;
+        e = cudaMemsetAsync(topk_idx, 0xff, bytes, st);
+        if (e == cudaSuccess && k_eff > 0)
+            e = cudaMemcpy2DAsync(topk_idx, static_cast<size_t>(c->cc.k) * 4, c->topk,
+                                  static_cast<size_t>(k_eff) * 4,
+                                  static_cast<size_t>(k_eff) * 4, c->heads,
+                                  cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return cuda_fail(e, "top-k copy");
+    }
+    set_last_launches(launches);
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_cache_counts(const pariskv_cache* c, int64_t* counts) {
+    if (!c || !counts) return fail(PARISKV_EINVAL, "NULL argument");
+    counts[0] = c->sink;
+    counts[1] = c->local;
+    counts[2] = c->buffer;
+    counts[3] = c->retr;
+    return PARISKV_OK;
+}
+
+pariskv_index* pariskv_cache_index(pariskv_cache* c) { return c ? c->ix : nullptr; }
+
+pariskv_status pariskv_cache_destroy(pariskv_cache* c) {
+    if (!c) return PARISKV_OK;
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(c->device);
+    cudaDeviceSynchronize();
+    free_cache(c);
+    cudaSetDevice(prev);
+    return PARISKV_OK;
+}
+
+}  // extern "C"

@@ -97,6 +97,10 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // status helpers (defined in api.cu)
 pariskv_status fail(pariskv_status s, const char* fmt, ...);
 pariskv_status cuda_fail(cudaError_t e, const char* what);
+bool alloc_fault_injected();   // PARISKV_FAULT=alloc: every device allocation fails
+pariskv_status check_device_pointer(const void* p, size_t align, const char* name);
+void set_last_launches(int32_t n);   // what pariskv_last_launch_count reports
+int32_t last_launches();
 
 // encode.cu
 cudaError_t launch_encode(const pariskv_index* ix, const void* keys, const float* knorm,
@@ -130,6 +134,16 @@ cudaError_t launch_attend(const pariskv_config* cfg, const void* q, const void* 
                           const void* V, int64_t ld_tok, int64_t n, const int32_t* topk_idx,
                           int32_t k, float scale, void* out, int32_t out_dtype, float* work,
                           int nsplit, cudaStream_t st);
+// the two halves of launch_attend: split-K partials of `k` indices per head (row `head` of
+// idx starts at head * k_stride) written to splits [split_base, split_base + nsplit) of
+// split_total per head, and the log-sum-exp merge of split_total splits per head
+cudaError_t launch_attend_partial(const pariskv_config* cfg, const void* q, const void* K,
+                                  const void* V, int64_t ld_tok, int64_t n,
+                                  const int32_t* idx, int32_t k, int32_t k_stride, float scale,
+                                  float* work, int nsplit, int split_base, int split_total,
+                                  cudaStream_t st);
+cudaError_t launch_attend_combine(int heads, const float* work, int split_total, void* out,
+                                  int32_t out_dtype, cudaStream_t st);
 int attend_splits(int heads, int32_t k, int num_sms);
 // Allocation-free attention: floats in the fixed per-device workspace and its address on the
 // current device (looked up on first use per device).

@@ -1,5 +1,5 @@
-"""Thin ctypes binding over libpariskv.so (the C ABI declared in include/pariskv.h and
-include/pariskv_debug.h).
+"""Thin ctypes binding over libpariskv.so (the C ABI declared in include/pariskv.h,
+include/pariskv_cache.h and include/pariskv_debug.h).
 
 Only argument marshalling happens here: tensors become data pointers and strides become the
 library's slab strides; every step of the retrieval path runs in the library's CUDA kernels.
@@ -17,7 +17,7 @@ import numpy as np
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "_lib", "libpariskv.so")
 HEADERS = [os.path.join(os.path.dirname(_PKG), "include", h)
-           for h in ("pariskv.h", "pariskv_debug.h")]
+           for h in ("pariskv.h", "pariskv_cache.h", "pariskv_debug.h")]
 
 OK, EINVAL, ENOMEM, ECUDA, ECAPACITY, ETIMEOUT = range(6)
 F32, BF16 = 0, 1
@@ -44,6 +44,12 @@ class Config(ctypes.Structure):
     @property
     def num_q_heads(self) -> int:
         return self.num_kv_heads * self.group
+
+
+class CacheConfig(ctypes.Structure):
+    _fields_ = [("n_sink", ctypes.c_int32), ("n_local", ctypes.c_int32),
+                ("n_buffer", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("retrieval_capacity", ctypes.c_int64)]
 
 
 if not os.path.exists(LIB_PATH):
@@ -79,6 +85,13 @@ _SIGS = {
     "pariskv_debug_profile": (_S, [_P, _I32]),
     "pariskv_debug_stage_ms": (_S, [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_I32)]),
     "pariskv_debug_read_stream": (_S, [_P, _I64, _P, _P]),
+    "pariskv_cache_create": (_S, [ctypes.POINTER(Config), ctypes.POINTER(CacheConfig), _P, _P,
+                                  ctypes.POINTER(_P)]),
+    "pariskv_cache_prefill": (_S, [_P, _P, _P, _I64, _I64, _P]),
+    "pariskv_cache_step": (_S, [_P, _P, _P, _P, ctypes.c_float, _P, _I32, _P, _P]),
+    "pariskv_cache_counts": (_S, [_P, ctypes.POINTER(_I64)]),
+    "pariskv_cache_index": (_P, [_P]),
+    "pariskv_cache_destroy": (_S, [_P]),
 }
 
 STAGES = ("query_prep", "vote", "threshold", "compact", "rerank", "topk")
@@ -140,9 +153,10 @@ def _slab(t, d: int = 128) -> int:
 class Index:
     """Owner of a ``pariskv_index*``; methods map one-to-one onto the C calls."""
 
-    def __init__(self, handle: int, cfg: Config):
+    def __init__(self, handle: int, cfg: Config, owned: bool = True):
         self.handle = ctypes.c_void_p(handle)
         self.cfg = cfg
+        self.owned = owned          # False for a view of an index some other object owns
 
     # -- product calls ------------------------------------------------------------------
     def append(self, keys, t: Optional[int] = None, stream=None) -> None:
@@ -171,9 +185,9 @@ class Index:
         return int(lib.pariskv_size(self.handle))
 
     def destroy(self) -> None:
-        if self.handle:
+        if self.handle and self.owned:
             lib.pariskv_destroy(self.handle)
-            self.handle = ctypes.c_void_p(0)
+        self.handle = ctypes.c_void_p(0)
 
     def __del__(self):
         try:
@@ -308,3 +322,67 @@ def read_stream(src, nbytes: int, sink, stream=None) -> None:
     or a pinned host tensor); ``sink`` is a device tensor of at least 4 bytes."""
     _check(lib.pariskv_debug_read_stream(src.data_ptr(), int(nbytes), sink.data_ptr(),
                                          _stream(stream)), "pariskv_debug_read_stream")
+
+
+class Cache:
+    """Owner of a ``pariskv_cache*`` (include/pariskv_cache.h): Sink, Local and Update Buffer
+    on the GPU, the Retrieval zone in pinned host memory behind a ParisKV index."""
+
+    REGIONS = ("sink", "local", "buffer", "retrieval")
+
+    def __init__(self, cfg: Config, signs, n_sink: int, n_local: int, n_buffer: int, k: int,
+                 retrieval_capacity: int, stream=None):
+        self.cfg = cfg
+        self.cc = CacheConfig(n_sink, n_local, n_buffer, k, retrieval_capacity)
+        sa, sp = _signs_ptr(signs)
+        h = _P()
+        self.handle = ctypes.c_void_p(0)
+        _check(lib.pariskv_cache_create(ctypes.byref(cfg), ctypes.byref(self.cc), sp,
+                                        _stream(stream), ctypes.byref(h)),
+               "pariskv_cache_create")
+        self.handle = ctypes.c_void_p(h.value)
+
+    def prefill(self, K, V, n: Optional[int] = None, stream=None) -> None:
+        """K, V: [batch, num_kv_heads, L, d] (device or pinned host); n <= L tokens used."""
+        n = K.shape[-2] if n is None else n
+        assert _slab(K) == _slab(V)
+        _check(lib.pariskv_cache_prefill(self.handle, K.data_ptr(), V.data_ptr(), _slab(K), n,
+                                         _stream(stream)), "pariskv_cache_prefill")
+
+    def step(self, q, k_new, v_new, scale: float, out=None, out_dtype=None,
+             topk_idx=None, want_topk: bool = False, stream=None):
+        """q [batch, Hq, d]; k_new, v_new [batch, Hkv, d] (device). Returns (out, topk_idx)."""
+        import torch
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+        if topk_idx is None and want_topk:
+            topk_idx = torch.empty((self.cfg.batch * self.cfg.num_q_heads, self.cc.k),
+                                   dtype=torch.int32, device=q.device)
+        od = BF16 if out.dtype == torch.bfloat16 else F32
+        _check(lib.pariskv_cache_step(self.handle, q.data_ptr(), k_new.data_ptr(),
+                                      v_new.data_ptr(), float(scale), out.data_ptr(), od,
+                                      topk_idx.data_ptr() if topk_idx is not None else None,
+                                      _stream(stream)), "pariskv_cache_step")
+        return out, topk_idx
+
+    def counts(self) -> dict:
+        c = (_I64 * 4)()
+        _check(lib.pariskv_cache_counts(self.handle, c), "pariskv_cache_counts")
+        return dict(zip(self.REGIONS, (int(x) for x in c)))
+
+    def index(self) -> Index:
+        """A non-owning view of the Retrieval zone's index."""
+        cfg = Config.from_buffer_copy(self.cfg)
+        cfg.capacity = self.cc.retrieval_capacity
+        return Index(lib.pariskv_cache_index(self.handle), cfg, owned=False)
+
+    def destroy(self) -> None:
+        if self.handle:
+            lib.pariskv_cache_destroy(self.handle)
+            self.handle = ctypes.c_void_p(0)
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
