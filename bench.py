@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cache", action="store_true")
     return ap.parse_args()
 
 
@@ -300,6 +301,68 @@ def decode_step(args, ix, cfg, sp, keys, vals, qs, idx, est, k, H, dev, kv_host)
 
 
 # ------------------------------------------------------------------------------------ main
+# Region sizes of the four-region cache measurement (the pages give none; 64 sink tokens as in
+# the sink-token convention of the P4 page, a 2048-token local window, a 256-token buffer).
+CACHE_REGIONS = dict(n_sink=64, n_local=2048, n_buffer=256)
+
+
+def cache_decode(cfg, sp, data, k, dev):
+    """Decode steps through the four-region cache (pariskv_cache_step): prefill of all but the
+    last T_WARM + T tokens of the workload, then one token per step; each step appends the
+    token, promotes a full buffer (evicting the oldest Local tokens to the Retrieval zone in
+    pinned host memory and to its index), searches the Retrieval zone and attends over
+    Sink + Local + buffer + the top-k. Every step is timed with events on the stream."""
+    import numpy as np
+    import torch
+    from long_context_kv_srht_b200 import pariskv as pk
+    t_warm, T = 8, 512
+    r = CACHE_REGIONS
+    n0 = sp.n - t_warm - T
+    if n0 < r["n_sink"] + r["n_local"] + k:
+        return None
+    keys, vals, qs = data["keys"], data["values"], data["queries"]
+    H = sp.batch * sp.num_q_heads
+    cache = pk.Cache(cfg, data["signs"], r["n_sink"], r["n_local"], r["n_buffer"], k,
+                     retrieval_capacity=sp.n)
+    t0 = time.perf_counter()
+    cache.prefill(keys, vals, n=n0)
+    torch.cuda.synchronize()
+    prefill_s = time.perf_counter() - t0
+    kn = keys[:, :, n0:sp.n].to(dev)
+    vn = vals[:, :, n0:sp.n].to(dev)
+    kn = [kn[:, :, s].contiguous() for s in range(t_warm + T)]
+    vn = [vn[:, :, s].contiguous() for s in range(t_warm + T)]
+    out = torch.empty((sp.batch, sp.num_q_heads, sp.d), dtype=torch.float32, device=dev)
+    scale = 1.0 / float(np.sqrt(sp.d))
+    for s in range(t_warm):
+        cache.step(qs, kn[s], vn[s], scale, out=out)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(T + 1)]
+    promo, launches, before = [], 0, cache.counts()["retrieval"]
+    ev[0].record()
+    for s in range(T):
+        cache.step(qs, kn[t_warm + s], vn[t_warm + s], scale, out=out)
+        ev[s + 1].record()
+        launches += pk.last_launch_count()
+        now = cache.counts()["retrieval"]
+        if now != before:
+            promo.append(s)
+        before = now
+    torch.cuda.synchronize()
+    ts = np.array([ev[s].elapsed_time(ev[s + 1]) for s in range(T)])
+    plain = np.delete(ts, promo)
+    counts = cache.counts()
+    cache.destroy()
+    return {"regions": r, "k": k, "prefill_tokens": n0, "prefill_s": prefill_s,
+            "steps": T, "ms_per_step": float(ts.mean()), "ms_per_step_median": float(np.median(ts)),
+            "promotion_steps": len(promo),
+            "promotion_step_ms": float(ts[promo].mean()) if promo else None,
+            "other_step_ms": float(plain.mean()),
+            "counts_after": counts, "gpu_launches_per_step": launches / T,
+            "tokens_attended_per_head": counts["sink"] + counts["local"] + counts["buffer"] + k,
+            "retrieval_kv": "pinned host (UVA)", "heads": H}
+
+
 def run_drift(args, ws, rank, local):
     """Long-generation drift (8 KV heads, 32768 prefill keys, then one appended key per KV
     head per decode step while the keys' mean vector drifts; k = 1024). Every timed step
@@ -557,6 +620,12 @@ def main():
     if not args.no_decode:
         decode = decode_step(args, ix, cfg, sp, keys, vals, qs, idx, est, k, H, dev, kv_host)
 
+    # the same decode step through the four-region cache (Sink / Local / buffer in HBM, the
+    # Retrieval zone in pinned host memory)
+    cache_step = None
+    if not args.no_cache:
+        cache_step = cache_decode(cfg, sp, data, k, dev)
+
     cpu = None
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -585,6 +654,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": e2e,
             "decode_step": decode,
+            "cache_step": cache_step,
             "gpu_launches": launches,
             "clocks": clk,
         }

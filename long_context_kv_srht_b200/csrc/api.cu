@@ -132,6 +132,8 @@ void free_index(pariskv_index* ix) {
     delete ix;
 }
 
+pariskv_status ensure_candidates(pariskv_index* ix, int64_t C);
+
 pariskv_status create_index(const pariskv_config* cfg, const int8_t* signs, cudaStream_t st,
                             pariskv_index** out) {
     *out = nullptr;
@@ -159,6 +161,13 @@ pariskv_status create_index(const pariskv_config* cfg, const int8_t* signs, cuda
     if (!ok) {
         free_index(ix);
         return fail(PARISKV_ENOMEM, "device allocation for the index failed");
+    }
+    // candidate buffers for a full index up front, so a search on a growing index never
+    // reallocates them (a cudaFree synchronises the device) unless k exceeds the pruned count
+    pariskv_status s = ensure_candidates(ix, candidate_count(cfg->capacity, 1, cfg->cand_bp));
+    if (s != PARISKV_OK) {
+        free_index(ix);
+        return s;
     }
     float hs[D];
     for (int j = 0; j < D; ++j) hs[j] = static_cast<float>(signs[j]);

@@ -8,12 +8,13 @@
 // K/V rows of the retrieved tokens directly from pinned host memory.
 //
 // Region bookkeeping is host-side (the counts are the same for every (sequence, KV head)),
-// and every data movement is stream-ordered:
-//  - the new token's K/V row goes to the end of the device pool (one 2-D copy per tensor);
-//  - a promotion copies the evicted rows to the host Retrieval arrays (2-D copies, device
-//    to pinned host), appends their keys to the index (the encode kernel reads them from
-//    the pool), then slides the remaining Local and buffer rows down over them through a
-//    scratch buffer, so Sink, Local and buffer always occupy pool rows [0, n_dense);
+// and every data movement is a kernel on the caller's stream (no copy-engine calls while
+// decoding):
+//  - put_token_kernel writes the new token's K/V row at the end of the device pool;
+//  - a promotion that evicts runs spill_kernel (evicted rows -> the host Retrieval arrays,
+//    written over UVA; the rows that stay -> a scratch buffer), the index's encode kernel
+//    (which reads the evicted keys from the pool) and slide_kernel (scratch -> pool rows right
+//    after Sink), so Sink, Local and buffer always occupy pool rows [0, n_dense);
 //  - the search runs on the index of the Retrieval zone; the attention writes split-K
 //    partials for the dense rows (every head reads rows 0..n_dense-1 of its unit's pool)
 //    and for the retrieved rows (pinned host memory) into one workspace, and one merge
@@ -37,7 +38,7 @@ struct pariskv_cache {
     size_t row = 0;               // bytes per K or V row
     uint8_t* poolK = nullptr;     // device [units][P][d]
     uint8_t* poolV = nullptr;
-    uint8_t* tmp = nullptr;       // device [units][n_local + n_buffer][d] (one tensor at a time)
+    uint8_t* tmp = nullptr;       // device [2][units][n_local + n_buffer][d] (K, then V)
     uint8_t* hostK = nullptr;     // pinned host [units][R][d]
     uint8_t* hostV = nullptr;
     int32_t* dense_idx = nullptr; // device [P]: 0, 1, ..., P - 1 (every head reads it)
@@ -54,6 +55,55 @@ namespace {
 __global__ void iota_kernel(int32_t* p, int64_t n) {
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i < n) p[i] = static_cast<int32_t>(i);
+}
+
+// Row copies in 16-byte words (every buffer here is allocation-aligned and a row is 256 or 512
+// bytes). blockIdx.z picks the tensor (0: K, 1: V), blockIdx.y the unit.
+struct Rows {
+    uint4* pool[2];   // [units][P][vpr]
+    uint4* host[2];   // [units][R][vpr]
+    uint4* tmp[2];    // [units][L][vpr]
+    int64_t P, R, L;
+    int vpr;          // 16-byte words per row
+};
+
+// Rows sink + j, j in [0, move + rest): the first `move` go to host rows retr + j, the others
+// to scratch rows j - move.
+__global__ void __launch_bounds__(256)
+spill_kernel(Rows r, int64_t sink, int64_t move, int64_t rest, int64_t retr) {
+    const int t = blockIdx.z;
+    const int64_t u = blockIdx.y;
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= (move + rest) * r.vpr) return;
+    const int64_t j = i / r.vpr, c = i - j * r.vpr;
+    const uint4 v = r.pool[t][(u * r.P + sink + j) * r.vpr + c];
+    if (j < move)
+        r.host[t][(u * r.R + retr + j) * r.vpr + c] = v;
+    else
+        r.tmp[t][(u * r.L + j - move) * r.vpr + c] = v;
+}
+
+// Scratch rows [0, rest) -> pool rows sink + j.
+__global__ void __launch_bounds__(256)
+slide_kernel(Rows r, int64_t sink, int64_t rest) {
+    const int t = blockIdx.z;
+    const int64_t u = blockIdx.y;
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= rest * r.vpr) return;
+    const int64_t j = i / r.vpr, c = i - j * r.vpr;
+    r.pool[t][(u * r.P + sink + j) * r.vpr + c] = r.tmp[t][(u * r.L + j) * r.vpr + c];
+}
+
+// The new token's rows ([units][vpr8] 8-byte words each; the caller's pointers are 8-byte
+// aligned) -> pool row `at`.
+__global__ void __launch_bounds__(256)
+put_token_kernel(const uint2* __restrict__ kn, const uint2* __restrict__ vn, uint2* poolK,
+                 uint2* poolV, int64_t P, int64_t at, int units, int vpr8) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= 2 * units * vpr8) return;
+    const int t = i / (units * vpr8), r = i - t * units * vpr8;
+    const int u = r / vpr8, c = r - u * vpr8;
+    (t ? poolV : poolK)[(static_cast<int64_t>(u) * P + at) * vpr8 + c] = (t ? vn : kn)[r];
 }
 
 void free_cache(pariskv_cache* c) {
@@ -113,25 +163,40 @@ cudaError_t copy_rows(void* dst, int64_t dst_rows, int64_t dst_r0, const void* s
                              nr * row, units, cudaMemcpyDefault, st);
 }
 
-// Evicts the oldest `move` Local rows to the Retrieval zone and slides the rest of Local
-// and the buffer down over them.
+Rows rows_of(const pariskv_cache* c) {
+    Rows r;
+    const int64_t L = c->cc.n_local + c->cc.n_buffer;
+    const size_t tmp_bytes = static_cast<size_t>(c->units) * L * c->row;
+    r.pool[0] = reinterpret_cast<uint4*>(c->poolK);
+    r.pool[1] = reinterpret_cast<uint4*>(c->poolV);
+    r.host[0] = reinterpret_cast<uint4*>(c->hostK);
+    r.host[1] = reinterpret_cast<uint4*>(c->hostV);
+    r.tmp[0] = reinterpret_cast<uint4*>(c->tmp);
+    r.tmp[1] = reinterpret_cast<uint4*>(c->tmp + tmp_bytes);
+    r.P = c->P;
+    r.R = c->cc.retrieval_capacity;
+    r.L = L;
+    r.vpr = static_cast<int>(c->row / 16);
+    return r;
+}
+
+// Evicts the oldest `move` Local rows to the Retrieval zone (host rows and index) and slides
+// the rest of Local and the buffer down over them. Three launches.
 pariskv_status evict(pariskv_cache* c, int64_t move, cudaStream_t st) {
-    const int64_t R = c->cc.retrieval_capacity;
     const int64_t rest = c->local + c->buffer - move;   // rows that stay after Sink
-    cudaError_t e = copy_rows(c->hostK, R, c->retr, c->poolK, c->P, c->sink, move, c->units,
-                              c->row, st);
-    if (e == cudaSuccess)
-        e = copy_rows(c->hostV, R, c->retr, c->poolV, c->P, c->sink, move, c->units, c->row,
-                      st);
-    if (e != cudaSuccess) return cuda_fail(e, "eviction copy");
+    const Rows r = rows_of(c);
+    const dim3 g1(static_cast<unsigned>(ceil_div((move + rest) * r.vpr, 256)),
+                  static_cast<unsigned>(c->units), 2);
+    spill_kernel<<<g1, 256, 0, st>>>(r, c->sink, move, rest, c->retr);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "eviction launch");
     pariskv_status s = pariskv_append(c->ix, c->poolK + c->sink * c->row, c->P, move, st);
     if (s != PARISKV_OK) return s;
-    for (uint8_t* pool : {c->poolK, c->poolV}) {
-        const int64_t tr = c->cc.n_local + c->cc.n_buffer;
-        e = copy_rows(c->tmp, tr, 0, pool, c->P, c->sink + move, rest, c->units, c->row, st);
-        if (e == cudaSuccess)
-            e = copy_rows(pool, c->P, c->sink, c->tmp, tr, 0, rest, c->units, c->row, st);
-        if (e != cudaSuccess) return cuda_fail(e, "pool compaction");
+    if (rest > 0) {
+        const dim3 g2(static_cast<unsigned>(ceil_div(rest * r.vpr, 256)),
+                      static_cast<unsigned>(c->units), 2);
+        slide_kernel<<<g2, 256, 0, st>>>(r, c->sink, rest);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "compaction launch");
     }
     c->retr += move;
     return PARISKV_OK;
@@ -202,7 +267,7 @@ pariskv_status pariskv_cache_create(const pariskv_config* cfg, const pariskv_cac
     const size_t host = static_cast<size_t>(c->units) * cc->retrieval_capacity * c->row;
     const bool ok =
         dev_alloc(&c->poolK, pool) && dev_alloc(&c->poolV, pool) &&
-        dev_alloc(&c->tmp, static_cast<size_t>(c->units) * (cc->n_local + cc->n_buffer) *
+        dev_alloc(&c->tmp, 2 * static_cast<size_t>(c->units) * (cc->n_local + cc->n_buffer) *
                                c->row) &&
         dev_alloc(&c->dense_idx, static_cast<size_t>(c->P) * 4) &&
         dev_alloc(&c->topk, static_cast<size_t>(c->heads) * cc->k * 4) &&
@@ -291,10 +356,14 @@ pariskv_status pariskv_cache_step(pariskv_cache* c, const void* q, const void* k
         return fail(PARISKV_ECAPACITY, "the Retrieval zone (%lld tokens) is full",
                     static_cast<long long>(c->cc.retrieval_capacity));
 
-    int32_t launches = 0;
+    int32_t launches = 1;
     const int64_t at = c->sink + c->local + c->buffer;   // first free pool row
-    cudaError_t e = copy_rows(c->poolK, c->P, at, k_new, 1, 0, 1, c->units, c->row, st);
-    if (e == cudaSuccess) e = copy_rows(c->poolV, c->P, at, v_new, 1, 0, 1, c->units, c->row, st);
+    const int vpr8 = static_cast<int>(c->row / 8);
+    put_token_kernel<<<static_cast<unsigned>(ceil_div(2 * c->units * vpr8, 256)), 256, 0, st>>>(
+        static_cast<const uint2*>(k_new), static_cast<const uint2*>(v_new),
+        reinterpret_cast<uint2*>(c->poolK), reinterpret_cast<uint2*>(c->poolV), c->P, at,
+        c->units, vpr8);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "token copy");
     if (to_sink) {
         ++c->sink;
@@ -303,7 +372,7 @@ pariskv_status pariskv_cache_step(pariskv_cache* c, const void* q, const void* k
         if (promote) {
             if (move > 0) {
                 if ((s = evict(c, move, st)) != PARISKV_OK) return s;
-                launches += 1;
+                launches += c->local + c->buffer - move > 0 ? 3 : 2;
             }
             c->local = c->local + c->buffer - move;
             c->buffer = 0;

@@ -155,8 +155,8 @@ def test_cache_capacity_and_errors():
 
 
 def test_cache_step_launch_count():
-    """A step is the search's launches, two attention partials and one merge, plus one
-    encode launch on a step that evicts to the Retrieval zone."""
+    """A step is one token-copy kernel, the search's launches, two attention partials and one
+    merge; a step that evicts to the Retrieval zone adds the spill, encode and slide kernels."""
     K, V, q = _data(2, 2, 2, 600, "bf16")
     signs = random_signs(2)
     cfg = pk.config(batch=1, num_kv_heads=2, group=2, capacity=1, dtype="bf16")
@@ -172,5 +172,5 @@ def test_cache_step_launch_count():
         cache.step(qd[t].view(1, 4, 128), Kd[:, :, t].contiguous(), Vd[:, :, t].contiguous(),
                    SCALE)
         seen.append(pk.last_launch_count())
-    assert seen.count(search_launches + 3) == 14 and seen.count(search_launches + 4) == 2
+    assert seen.count(search_launches + 4) == 14 and seen.count(search_launches + 7) == 2
     cache.destroy()
