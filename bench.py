@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cache", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
     return ap.parse_args()
 
 
@@ -301,6 +302,60 @@ def decode_step(args, ix, cfg, sp, keys, vals, qs, idx, est, k, H, dev, kv_host)
 
 
 # ------------------------------------------------------------------------------------ main
+def dense_comparator(cfg, sp, data, ix, k, dev, peak_gbs):
+    """Full attention over all n tokens (pariskv_dense_attend, K/V in HBM) against ParisKV's
+    retrieval + sparse attention over the top-k with the same K/V in HBM (the one-key append,
+    about 0.02 ms, is in the decode-step figures): the synthetic analogue of the pages'
+    comparison with full attention. Both are
+    timed with CUDA events over 10 steps after 3 warm-up steps; K/V (4 GiB at the
+    million-token workload) exceed L2, so no flush is needed between steps."""
+    import numpy as np
+    import torch
+    from long_context_kv_srht_b200 import pariskv as pk
+    if sp.dtype != "bf16" or sp.group > 8:
+        return None
+    keys, vals, qs = data["keys"], data["values"], data["queries"]
+    Kd = keys if keys.is_cuda else keys.to(dev)
+    Vd = vals if vals.is_cuda else vals.to(dev)
+    n = sp.n
+    scale = 1.0 / float(np.sqrt(sp.d))
+    out = torch.empty(qs.shape, dtype=torch.float32, device=dev)
+    H = sp.batch * sp.num_q_heads
+    idx = torch.empty((H, k), dtype=torch.int32, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn, reps=10, warm=3):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return float(np.mean(ts)), float(np.min(ts))
+
+    dense_ms, dense_min = timed(lambda: pk.dense_attend(cfg, qs, Kd, Vd, scale, n=n, out=out))
+    # the ParisKV retrieval and sparse attention on the same K/V in HBM (the index as it is;
+    # this measurement does not grow it)
+    size = ix.size
+
+    def paris():
+        ix.search(qs, k, idx)
+        pk.sparse_attend(cfg, qs, Kd, Vd, idx, k, scale, n=size, out=out)
+    paris_ms, _ = timed(paris)
+    kv_bytes = 2 * sp.batch * sp.num_kv_heads * n * sp.d * 2
+    del Kd, Vd
+    return {"dense_ms": dense_ms, "dense_ms_min": dense_min,
+            "dense_gbs": kv_bytes / (dense_ms / 1e3) / 1e9,
+            "dense_frac_of_measured_hbm": kv_bytes / (dense_ms / 1e3) / 1e9 / peak_gbs,
+            "dense_bytes_per_step": kv_bytes,
+            "paris_hbm_ms": paris_ms, "speedup_vs_dense_hbm": dense_ms / paris_ms,
+            "kv": "HBM (both)", "n": n, "k": k}
+
+
 # Region sizes of the four-region cache measurement (the pages give none; 64 sink tokens as in
 # the sink-token convention of the P4 page, a 2048-token local window, a 256-token buffer).
 CACHE_REGIONS = dict(n_sink=64, n_local=2048, n_buffer=256)
@@ -620,6 +675,13 @@ def main():
     if not args.no_decode:
         decode = decode_step(args, ix, cfg, sp, keys, vals, qs, idx, est, k, H, dev, kv_host)
 
+    # full attention over every token, the baseline the pages compare against
+    dense = None
+    if not args.no_dense:
+        dense = dense_comparator(cfg, sp, data, ix, k, dev, measured_peaks()[0])
+        if dense and decode:
+            dense["speedup_vs_dense_offloaded_step"] = dense["dense_ms"] / decode["total_ms"]
+
     # the same decode step through the four-region cache (Sink / Local / buffer in HBM, the
     # Retrieval zone in pinned host memory)
     cache_step = None
@@ -655,6 +717,7 @@ def main():
             "e2e": e2e,
             "decode_step": decode,
             "cache_step": cache_step,
+            "dense_comparator": dense,
             "gpu_launches": launches,
             "clocks": clk,
         }

@@ -115,8 +115,9 @@ PARISKV_API pariskv_status pariskv_append(pariskv_index* index, const void* keys
  *   topk_idx:  device pointer [batch][num_kv_heads * group][k] int32: the selected key
  *              indices in ascending index order.
  *   topk_est:  device pointer with the same shape (fp32 estimates of <k, q>), or NULL.
- * Scratch memory is owned by the index; the first search with a larger candidate count
- * allocates (so run one search before capturing a CUDA graph).
+ * Scratch memory is owned by the index and sized for a full index when it is created; a
+ * search allocates only when k exceeds ceil(capacity * cand_bp / 10000) and k is larger than
+ * any earlier search's (so run one search with the largest k before capturing a CUDA graph).
  * Errors: EINVAL, ENOMEM, ECUDA, ETIMEOUT. */
 PARISKV_API pariskv_status pariskv_search(pariskv_index* index, const void* q, int32_t k, int32_t* topk_idx,
                               float* topk_est, void* stream);
@@ -163,6 +164,28 @@ PARISKV_API pariskv_status pariskv_sparse_attend_noalloc(const pariskv_config* c
                                                          int64_t n, const int32_t* topk_idx,
                                                          int32_t k, float scale, void* out,
                                                          int32_t out_dtype, void* stream);
+
+/* Index images, for checkpoint and resume (the index is derived from the keys, so an image
+ * only saves re-encoding them). An image is a self-describing byte string: a 256-byte header
+ * (magic "PARISKV", format version, the pariskv_config, the SRHT signs, the size n and the
+ * number of units) followed by the bucket ids and the code records of every unit in the
+ * library's storage layout, units * n * (16 + 128) bytes. Images are read only by the same
+ * format version.
+ *   pariskv_export_bytes: the image size of the index as it is now.
+ *   pariskv_export: writes the image of `index` into `buf` (host memory, pinned or pageable,
+ *     at least pariskv_export_bytes bytes), after all work queued on `stream`; returns when
+ *     the image is complete.
+ *   pariskv_import: creates an index on the current device from an image, with capacity
+ *     `capacity` (0: the image's size; it must be >= the image's size); returns when `buf` is
+ *     no longer needed. The imported index searches and appends exactly like the exported one.
+ * Errors: EINVAL (NULL pointers, too small a buffer, a malformed, truncated or foreign image,
+ * capacity below the image's size), ENOMEM, ECUDA. The import checks the image's header and
+ * sizes on the host before it touches the device. */
+PARISKV_API pariskv_status pariskv_export_bytes(const pariskv_index* index, size_t* bytes);
+PARISKV_API pariskv_status pariskv_export(pariskv_index* index, void* buf, size_t bytes,
+                                          void* stream);
+PARISKV_API pariskv_status pariskv_import(const void* buf, size_t bytes, int64_t capacity,
+                                          void* stream, pariskv_index** out);
 
 /* Waits for the index's stream work and reports any asynchronous error or expired wait. */
 PARISKV_API pariskv_status pariskv_sync(pariskv_index* index, void* stream);

@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "internal.hpp"
+#include "pariskv_dense.h"
 #include "pariskv_debug.h"
 
 using namespace pkv;
@@ -143,6 +144,7 @@ pariskv_status create_index(const pariskv_config* cfg, const int8_t* signs, cuda
     pariskv_index* ix = new (std::nothrow) pariskv_index();
     if (!ix) return fail(PARISKV_ENOMEM, "host allocation failed");
     ix->cfg = *cfg;
+    memcpy(ix->hsigns, signs, sizeof(ix->hsigns));
     cudaGetDevice(&ix->device);
     ix->units = cfg->batch * cfg->num_kv_heads;
     ix->hq = cfg->num_kv_heads * cfg->group;
@@ -420,6 +422,47 @@ pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, c
     return PARISKV_OK;
 }
 
+pariskv_status pariskv_dense_attend(const pariskv_config* cfg, const void* q, const void* K,
+                                    const void* V, int64_t ld_tok, int64_t n, float scale,
+                                    void* out, int32_t out_dtype, void* stream) {
+    pariskv_status s = check_config(cfg);
+    if (s != PARISKV_OK) return s;
+    if (cfg->dtype != PARISKV_BF16) return fail(PARISKV_EINVAL, "dense attention reads bf16 K/V");
+    if (cfg->group > 8) return fail(PARISKV_EINVAL, "group %d > 8", cfg->group);
+    if (n < 1 || ld_tok < n) return fail(PARISKV_EINVAL, "need 1 <= n <= ld_tok");
+    if ((s = check_dev_ptr(q, 4, "q")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(K, 16, "K")) != PARISKV_OK) return s;
+    if ((s = check_dev_ptr(V, 16, "V")) != PARISKV_OK) return s;
+    if (out_dtype != PARISKV_F32 && out_dtype != PARISKV_BF16)
+        return fail(PARISKV_EINVAL, "out_dtype %d unknown", out_dtype);
+    if ((s = check_dev_ptr(out, out_dtype == PARISKV_BF16 ? 8 : 16, "out")) != PARISKV_OK)
+        return s;
+    if (!(scale == scale)) return fail(PARISKV_EINVAL, "scale is NaN");
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int units = cfg->batch * cfg->num_kv_heads;
+    const int heads = units * cfg->group;
+    const int nsplit = dense_splits(units, n, sms);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* work = nullptr;
+    if (fault_alloc()) return fail(PARISKV_ENOMEM, "attention workspace");
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = workspace_pool(&pool);
+    if (e == cudaSuccess)
+        e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&work),
+                                    attend_workspace_floats(heads, nsplit) * sizeof(float), pool,
+                                    st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention workspace");
+    g_launches = 0;
+    e = launch_dense_partial(cfg, q, K, V, ld_tok, n, scale, work, nsplit, st);
+    if (e == cudaSuccess) e = launch_attend_combine(heads, work, nsplit, out, out_dtype, st);
+    if (e == cudaSuccess) g_launches = 2;
+    cudaFreeAsync(work, st);
+    if (e != cudaSuccess) return cuda_fail(e, "dense attention launch");
+    return PARISKV_OK;
+}
+
 pariskv_status pariskv_sparse_attend_noalloc(const pariskv_config* cfg, const void* q,
                                              const void* K, const void* V, int64_t ld_tok,
                                              int64_t n, const int32_t* topk_idx, int32_t k,
@@ -459,6 +502,124 @@ pariskv_status pariskv_sparse_attend_noalloc(const pariskv_config* cfg, const vo
                       static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
     g_launches = 2;
+    return PARISKV_OK;
+}
+
+// ------------------------------------------------------------------------- index images
+namespace {
+
+constexpr char kMagic[8] = {'P', 'A', 'R', 'I', 'S', 'K', 'V', '\0'};
+constexpr uint32_t kImageVersion = 1;
+
+struct ImageHeader {
+    char magic[8];
+    uint32_t version;
+    uint32_t header_bytes;
+    pariskv_config cfg;
+    int64_t n;
+    int32_t units;
+    int32_t reserved;
+    int8_t signs[D];
+    uint8_t pad[256 - 88 - D];
+};
+static_assert(sizeof(pariskv_config) == 56, "image header layout");
+static_assert(sizeof(ImageHeader) == 256, "image header layout");
+
+constexpr size_t kKeyBytes = 16 + REC;   // bucket ids + code record per key
+
+}  // namespace
+
+pariskv_status pariskv_export_bytes(const pariskv_index* ix, size_t* bytes) {
+    if (!ix || !bytes) return fail(PARISKV_EINVAL, "NULL argument");
+    *bytes = sizeof(ImageHeader) + static_cast<size_t>(ix->units) * ix->n * kKeyBytes;
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_export(pariskv_index* ix, void* buf, size_t bytes, void* stream) {
+    pariskv_status s = check_index(ix);
+    if (s != PARISKV_OK) return s;
+    size_t need = 0;
+    pariskv_export_bytes(ix, &need);
+    if (!buf) return fail(PARISKV_EINVAL, "buf is NULL");
+    if (bytes < need)
+        return fail(PARISKV_EINVAL, "buffer of %zu bytes; the image needs %zu", bytes, need);
+    ImageHeader h;
+    memset(&h, 0, sizeof(h));
+    memcpy(h.magic, kMagic, sizeof(kMagic));
+    h.version = kImageVersion;
+    h.header_bytes = sizeof(ImageHeader);
+    h.cfg = ix->cfg;
+    h.n = ix->n;
+    h.units = ix->units;
+    memcpy(h.signs, ix->hsigns, sizeof(h.signs));
+    uint8_t* out = static_cast<uint8_t*>(buf);
+    memcpy(out, &h, sizeof(h));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t nid = static_cast<size_t>(ix->n) * 16, nrec = static_cast<size_t>(ix->n) * REC;
+    uint8_t* ids = out + sizeof(h);
+    uint8_t* rec = ids + static_cast<size_t>(ix->units) * nid;
+    cudaError_t e = cudaSuccess;
+    for (int u = 0; u < ix->units && ix->n > 0 && e == cudaSuccess; ++u) {
+        e = cudaMemcpyAsync(ids + u * nid, ix->ids + u * ix->cap_pad * 16, nid,
+                            cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(rec + u * nrec, ix->rec + u * ix->cap_pad * REC, nrec,
+                                cudaMemcpyDeviceToHost, st);
+    }
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "export copy");
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_import(const void* buf, size_t bytes, int64_t capacity, void* stream,
+                              pariskv_index** out) {
+    if (!out) return fail(PARISKV_EINVAL, "out is NULL");
+    *out = nullptr;
+    if (!buf) return fail(PARISKV_EINVAL, "buf is NULL");
+    if (bytes < sizeof(ImageHeader))
+        return fail(PARISKV_EINVAL, "%zu bytes cannot hold an image header", bytes);
+    ImageHeader h;
+    memcpy(&h, buf, sizeof(h));
+    if (memcmp(h.magic, kMagic, sizeof(kMagic)) != 0)
+        return fail(PARISKV_EINVAL, "not a ParisKV index image");
+    if (h.version != kImageVersion || h.header_bytes != sizeof(ImageHeader))
+        return fail(PARISKV_EINVAL, "image format version %u (this library reads %u)",
+                    h.version, kImageVersion);
+    if (h.n < 0 || h.units < 1 || h.cfg.batch < 1 || h.cfg.num_kv_heads < 1 ||
+        static_cast<int64_t>(h.cfg.batch) * h.cfg.num_kv_heads != h.units)
+        return fail(PARISKV_EINVAL, "inconsistent image header");
+    if (capacity == 0) capacity = h.n > 0 ? h.n : 1;
+    if (capacity < h.n)
+        return fail(PARISKV_EINVAL, "capacity %lld below the image's size %lld",
+                    static_cast<long long>(capacity), static_cast<long long>(h.n));
+    pariskv_config cfg = h.cfg;
+    cfg.capacity = capacity;
+    pariskv_status s = check_config(&cfg);
+    if (s != PARISKV_OK) return s;
+    const size_t nid = static_cast<size_t>(h.n) * 16, nrec = static_cast<size_t>(h.n) * REC;
+    if ((bytes - sizeof(h)) / kKeyBytes / h.units < static_cast<size_t>(h.n))
+        return fail(PARISKV_EINVAL, "image truncated: %zu bytes for %d units of %lld keys",
+                    bytes, h.units, static_cast<long long>(h.n));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    pariskv_index* ix = nullptr;
+    if ((s = create_index(&cfg, h.signs, st, &ix)) != PARISKV_OK) return s;
+    const uint8_t* ids = static_cast<const uint8_t*>(buf) + sizeof(h);
+    const uint8_t* rec = ids + static_cast<size_t>(h.units) * nid;
+    cudaError_t e = cudaSuccess;
+    for (int u = 0; u < ix->units && h.n > 0 && e == cudaSuccess; ++u) {
+        e = cudaMemcpyAsync(ix->ids + u * ix->cap_pad * 16, ids + u * nid, nid,
+                            cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(ix->rec + u * ix->cap_pad * REC, rec + u * nrec, nrec,
+                                cudaMemcpyHostToDevice, st);
+    }
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) {
+        free_index(ix);
+        return cuda_fail(e, "import copy");
+    }
+    ix->n = h.n;
+    *out = ix;
     return PARISKV_OK;
 }
 

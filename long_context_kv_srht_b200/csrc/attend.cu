@@ -32,7 +32,7 @@ constexpr int kAW = 8;            // warps per CTA
 constexpr int kUnroll = 4;        // tokens in flight per warp
 // floats per partial: 128 accumulators, then max and denominator, padded to a multiple of 4
 // so that every partial (and its accumulators) starts on a 16-byte boundary
-constexpr int kPart = D + 4;
+constexpr int kPart = kAttendPart;
 constexpr int kMax = D, kDen = D + 1;
 static_assert((kPart * sizeof(float)) % 16 == 0, "partials must stay 16-byte aligned");
 

@@ -18,6 +18,7 @@ struct pariskv_index {
     int hq = 0;           // query heads per sequence
     int packs = 0;        // ceil(group / 4): vote-table packs per KV head
 
+    int8_t hsigns[128] = {};    // the SRHT signs as given (host copy, for index images)
     float* signs = nullptr;     // [128] +-1.0f
     uint8_t* ids = nullptr;     // [units][cap_pad][16] bucket ids, byte-rotated per key
     uint8_t* rec = nullptr;     // [units][cap_pad][128] codes (64 B) + factors (16 x f32)
@@ -145,6 +146,16 @@ cudaError_t launch_attend_partial(const pariskv_config* cfg, const void* q, cons
 cudaError_t launch_attend_combine(int heads, const float* work, int split_total, void* out,
                                   int32_t out_dtype, cudaStream_t st);
 int attend_splits(int heads, int32_t k, int num_sms);
+// floats per split partial in the attention workspace: 128 accumulators, the running max
+// (natural-log units) and the denominator, padded so every partial starts 16-byte aligned
+constexpr int kAttendPart = 128 + 4;
+
+// dense.cu: split-K partials of dense attention over tokens [0, n) of every unit (bf16 K/V,
+// group <= 8), written like launch_attend_partial's with split_total = nsplit
+int dense_splits(int units, int64_t n, int num_sms);
+cudaError_t launch_dense_partial(const pariskv_config* cfg, const void* q, const void* K,
+                                 const void* V, int64_t ld_tok, int64_t n, float scale,
+                                 float* work, int nsplit, cudaStream_t st);
 // Allocation-free attention: floats in the fixed per-device workspace and its address on the
 // current device (looked up on first use per device).
 constexpr size_t kAttendScratchFloats = size_t(1) << 20;

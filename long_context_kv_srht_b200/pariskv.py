@@ -1,5 +1,5 @@
 """Thin ctypes binding over libpariskv.so (the C ABI declared in include/pariskv.h,
-include/pariskv_cache.h and include/pariskv_debug.h).
+include/pariskv_cache.h, include/pariskv_dense.h and include/pariskv_debug.h).
 
 Only argument marshalling happens here: tensors become data pointers and strides become the
 library's slab strides; every step of the retrieval path runs in the library's CUDA kernels.
@@ -17,7 +17,7 @@ import numpy as np
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "_lib", "libpariskv.so")
 HEADERS = [os.path.join(os.path.dirname(_PKG), "include", h)
-           for h in ("pariskv.h", "pariskv_cache.h", "pariskv_debug.h")]
+           for h in ("pariskv.h", "pariskv_cache.h", "pariskv_dense.h", "pariskv_debug.h")]
 
 OK, EINVAL, ENOMEM, ECUDA, ECAPACITY, ETIMEOUT = range(6)
 F32, BF16 = 0, 1
@@ -69,6 +69,11 @@ _SIGS = {
                                    ctypes.c_float, _P, _I32, _P]),
     "pariskv_sparse_attend_noalloc": (_S, [ctypes.POINTER(Config), _P, _P, _P, _I64, _I64, _P,
                                            _I32, ctypes.c_float, _P, _I32, _P]),
+    "pariskv_export_bytes": (_S, [_P, ctypes.POINTER(ctypes.c_size_t)]),
+    "pariskv_export": (_S, [_P, _P, ctypes.c_size_t, _P]),
+    "pariskv_import": (_S, [_P, ctypes.c_size_t, _I64, _P, ctypes.POINTER(_P)]),
+    "pariskv_dense_attend": (_S, [ctypes.POINTER(Config), _P, _P, _P, _I64, _I64, ctypes.c_float,
+                                  _P, _I32, _P]),
     "pariskv_sync": (_S, [_P, _P]),
     "pariskv_destroy": (_S, [_P]),
     "pariskv_size": (_I64, [_P]),
@@ -180,6 +185,15 @@ class Index:
     def sync(self, stream=None) -> None:
         _check(lib.pariskv_sync(self.handle, _stream(stream)), "pariskv_sync")
 
+    def export_image(self, stream=None) -> np.ndarray:
+        """pariskv_export: the index image as a uint8 array (host memory)."""
+        nb = ctypes.c_size_t(0)
+        _check(lib.pariskv_export_bytes(self.handle, ctypes.byref(nb)), "pariskv_export_bytes")
+        buf = np.empty((nb.value,), np.uint8)
+        _check(lib.pariskv_export(self.handle, buf.ctypes.data, nb.value, _stream(stream)),
+               "pariskv_export")
+        return buf
+
     @property
     def size(self) -> int:
         return int(lib.pariskv_size(self.handle))
@@ -258,6 +272,26 @@ def build_index(cfg: Config, signs, keys, n: Optional[int] = None, stream=None) 
     return Index(h.value, cfg)
 
 
+def import_index(image, capacity: int = 0, stream=None) -> Index:
+    """pariskv_import: an index from an image (a uint8 numpy array or bytes)."""
+    buf = np.ascontiguousarray(np.frombuffer(image, np.uint8) if isinstance(image, bytes)
+                               else image, dtype=np.uint8)
+    h = _P()
+    if stream is None:
+        import torch
+        # the legacy default stream when no device is visible (the call then fails in the
+        # library with ECUDA, after it has checked the image on the host)
+        st = torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else 0
+    else:
+        st = _stream(stream)
+    _check(lib.pariskv_import(buf.ctypes.data, buf.nbytes, capacity, st, ctypes.byref(h)),
+           "pariskv_import")
+    cfg = Config.from_buffer_copy(bytes(buf[16:16 + ctypes.sizeof(Config)]))
+    cfg.capacity = capacity if capacity else max(1, int(np.frombuffer(
+        bytes(buf[72:80]), np.int64)[0]))
+    return Index(h.value, cfg)
+
+
 def build_index_rotated(cfg: Config, signs, y, knorm, n: Optional[int] = None,
                         stream=None) -> Index:
     n = y.shape[-2] if n is None else n
@@ -310,6 +344,21 @@ def sparse_attend_noalloc(cfg: Config, q, K, V, topk_idx, k: int, scale: float,
                                              V.data_ptr(), _slab(K), n, topk_idx.data_ptr(), k,
                                              float(scale), out.data_ptr(), od, _stream(stream)),
            "pariskv_sparse_attend_noalloc")
+    return out
+
+
+def dense_attend(cfg: Config, q, K, V, scale: float, n: Optional[int] = None, out=None,
+                 out_dtype=None, stream=None):
+    """pariskv_dense_attend: softmax attention over all n tokens (bf16 q, K, V; K/V
+    [batch, Hkv, L, d]); the full-attention baseline."""
+    import torch
+    n = K.shape[-2] if n is None else n
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    od = BF16 if out.dtype == torch.bfloat16 else F32
+    _check(lib.pariskv_dense_attend(ctypes.byref(cfg), q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                    _slab(K), n, float(scale), out.data_ptr(), od,
+                                    _stream(stream)), "pariskv_dense_attend")
     return out
 
 

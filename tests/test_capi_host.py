@@ -56,3 +56,58 @@ def test_status_strings_and_null_handles():
     assert pk.lib.pariskv_size(None) == -1
     assert pk.lib.pariskv_destroy(None) == pk.OK
     assert pk.lib.pariskv_search(None, None, 1, None, None, None) == pk.EINVAL
+
+
+# ------------------------------------------------------------------ index images (host checks)
+def _header(n=5, units=2, version=1, magic=b"PARISKV\0", **cfg_kw):
+    """A 256-byte image header laid out as include/pariskv.h describes it."""
+    import numpy as np
+    cfg = pk.config(batch=1, num_kv_heads=units, capacity=max(n, 1), **cfg_kw)
+    h = bytearray(256)
+    h[0:8] = magic
+    h[8:12] = int(version).to_bytes(4, "little")
+    h[12:16] = (256).to_bytes(4, "little")
+    h[16:72] = bytes(cfg)
+    h[72:80] = int(n).to_bytes(8, "little", signed=True)
+    h[80:84] = int(units).to_bytes(4, "little", signed=True)
+    h[88:216] = np.ones(128, np.int8).tobytes()
+    return bytes(h)
+
+
+@pytest.mark.parametrize("case", ["short", "magic", "version", "units", "truncated",
+                                  "capacity", "config"])
+def test_import_rejects_bad_images_on_the_host(case):
+    """pariskv_import validates the image before any device work, so these run without a GPU."""
+    n, units = 5, 2
+    body = bytes(units * n * 144)
+    img, cap = _header(n, units) + body, 0
+    if case == "short":
+        img = img[:100]
+    elif case == "magic":
+        img = _header(n, units, magic=b"PARISKW\0") + body
+    elif case == "version":
+        img = _header(n, units, version=2) + body
+    elif case == "units":
+        img = _header(n, 3) + body          # header says 3 units, config says 3 KV heads
+        img = img[:16] + bytes(pk.config(batch=1, num_kv_heads=2, capacity=5)) + img[72:]
+    elif case == "truncated":
+        img = img[:-1]
+    elif case == "capacity":
+        cap = n - 1
+    elif case == "config":
+        img = _header(n, units, rho=0) + body
+    h = ctypes.c_void_p()
+    st = pk.lib.pariskv_import(img, len(img), cap, None, ctypes.byref(h))
+    assert st == pk.EINVAL and not h.value, pk.last_error()
+
+
+def test_import_accepts_a_well_formed_image_up_to_the_device():
+    """A well-formed image passes every host check; without a GPU the call then fails in the
+    device allocation (ECUDA or ENOMEM), not in validation."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is visible: the import would succeed (covered by the GPU tests)")
+    img = _header(5, 2) + bytes(2 * 5 * 144)
+    h = ctypes.c_void_p()
+    st = pk.lib.pariskv_import(img, len(img), 0, None, ctypes.byref(h))
+    assert st in (pk.ECUDA, pk.ENOMEM) and not h.value, (st, pk.last_error())
