@@ -307,8 +307,8 @@ def dense_comparator(cfg, sp, data, ix, k, dev, peak_gbs):
     retrieval + sparse attention over the top-k with the same K/V in HBM (the one-key append,
     about 0.02 ms, is in the decode-step figures): the synthetic analogue of the pages'
     comparison with full attention. Both are
-    timed with CUDA events over 10 steps after 3 warm-up steps; K/V (4 GiB at the
-    million-token workload) exceed L2, so no flush is needed between steps."""
+    timed with CUDA events around 20 steps enqueued back to back after 3 warm-up steps; K/V
+    (4 GiB at the million-token workload) exceed L2, so no flush is needed between steps."""
     import numpy as np
     import torch
     from long_context_kv_srht_b200 import pariskv as pk
@@ -324,20 +324,20 @@ def dense_comparator(cfg, sp, data, ix, k, dev, peak_gbs):
     idx = torch.empty((H, k), dtype=torch.int32, device=dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-    def timed(fn, reps=10, warm=3):
+    def timed(fn, reps=20, warm=3):
+        # steps enqueued back to back (no host synchronisation between them), so the time is
+        # the device's, not the host's launch latency; mean over the reps
         for _ in range(warm):
             fn()
         torch.cuda.synchronize()
-        ts = []
+        e0.record()
         for _ in range(reps):
-            e0.record()
             fn()
-            e1.record()
-            e1.synchronize()
-            ts.append(e0.elapsed_time(e1))
-        return float(np.mean(ts)), float(np.min(ts))
+        e1.record()
+        e1.synchronize()
+        return e0.elapsed_time(e1) / reps
 
-    dense_ms, dense_min = timed(lambda: pk.dense_attend(cfg, qs, Kd, Vd, scale, n=n, out=out))
+    dense_ms = timed(lambda: pk.dense_attend(cfg, qs, Kd, Vd, scale, n=n, out=out))
     # the ParisKV retrieval and sparse attention on the same K/V in HBM (the index as it is;
     # this measurement does not grow it)
     size = ix.size
@@ -345,14 +345,16 @@ def dense_comparator(cfg, sp, data, ix, k, dev, peak_gbs):
     def paris():
         ix.search(qs, k, idx)
         pk.sparse_attend(cfg, qs, Kd, Vd, idx, k, scale, n=size, out=out)
-    paris_ms, _ = timed(paris)
+    paris_ms = timed(paris)
     kv_bytes = 2 * sp.batch * sp.num_kv_heads * n * sp.d * 2
     del Kd, Vd
-    return {"dense_ms": dense_ms, "dense_ms_min": dense_min,
+    return {"dense_ms": dense_ms,
             "dense_gbs": kv_bytes / (dense_ms / 1e3) / 1e9,
             "dense_frac_of_measured_hbm": kv_bytes / (dense_ms / 1e3) / 1e9 / peak_gbs,
             "dense_bytes_per_step": kv_bytes,
+            "dense_roofline_ms": kv_bytes / (peak_gbs * 1e9) * 1e3,
             "paris_hbm_ms": paris_ms, "speedup_vs_dense_hbm": dense_ms / paris_ms,
+            "speedup_vs_dense_roofline": kv_bytes / (peak_gbs * 1e9) * 1e3 / paris_ms,
             "kv": "HBM (both)", "n": n, "k": k}
 
 

@@ -100,6 +100,16 @@ pariskv_status check_dev_ptr(const void* p, size_t align, const char* name) {
     return PARISKV_OK;
 }
 
+// true for device (or managed) memory, false for pinned host memory
+bool device_memory(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
 }  // namespace
 
 namespace pkv {
@@ -402,7 +412,8 @@ pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, c
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int heads = cfg->batch * cfg->num_kv_heads * cfg->group;
-    const int nsplit = attend_splits(heads, k, sms);
+    const bool mma = attend_uses_mma(cfg, device_memory(K) && device_memory(V));
+    const int nsplit = attend_splits(heads, k, sms, mma);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float* work = nullptr;
     if (fault_alloc()) return fail(PARISKV_ENOMEM, "attention workspace");
@@ -415,7 +426,7 @@ pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, c
     if (e != cudaSuccess) return cuda_fail(e, "attention workspace");
     g_launches = 0;
     e = launch_attend(cfg, q, K, V, ld_tok, n, topk_idx, k, scale, out, out_dtype, work, nsplit,
-                      st);
+                      mma, st);
     if (e == cudaSuccess) g_launches = 2;
     cudaFreeAsync(work, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
@@ -455,7 +466,7 @@ pariskv_status pariskv_dense_attend(const pariskv_config* cfg, const void* q, co
                                     st);
     if (e != cudaSuccess) return cuda_fail(e, "attention workspace");
     g_launches = 0;
-    e = launch_dense_partial(cfg, q, K, V, ld_tok, n, scale, work, nsplit, st);
+    e = launch_dense_partial(cfg, q, K, V, ld_tok, n, scale, work, nsplit, 0, nsplit, st);
     if (e == cudaSuccess) e = launch_attend_combine(heads, work, nsplit, out, out_dtype, st);
     if (e == cudaSuccess) g_launches = 2;
     cudaFreeAsync(work, st);
@@ -493,13 +504,14 @@ pariskv_status pariskv_sparse_attend_noalloc(const pariskv_config* cfg, const vo
     if (fit < 1)
         return fail(PARISKV_EINVAL, "%d query heads exceed the fixed attention workspace "
                     "(at most %zu heads)", heads, kAttendScratchFloats / attend_workspace_floats(1, 1));
-    const int nsplit = min(attend_splits(heads, k, sms), fit);
+    const bool mma = attend_uses_mma(cfg, device_memory(K) && device_memory(V));
+    const int nsplit = min(attend_splits(heads, k, sms, mma), fit);
     float* work = nullptr;
     cudaError_t e = attend_static_scratch(&work);
     if (e != cudaSuccess) return cuda_fail(e, "fixed attention workspace lookup");
     g_launches = 0;
     e = launch_attend(cfg, q, K, V, ld_tok, n, topk_idx, k, scale, out, out_dtype, work, nsplit,
-                      static_cast<cudaStream_t>(stream));
+                      mma, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
     g_launches = 2;
     return PARISKV_OK;

@@ -228,7 +228,8 @@ cudaError_t attend_static_scratch(float** ptr) {
     return cudaSuccess;
 }
 
-int attend_splits(int heads, int32_t k, int num_sms) {
+int attend_splits(int heads, int32_t k, int num_sms, bool mma) {
+    if (mma) return gather_splits(heads, k, num_sms);
     // one wave: two 8-warp CTAs per SM
     const int want = static_cast<int>(2LL * num_sms / heads);
     const int most = static_cast<int>(ceil_div(k, 64));
@@ -239,11 +240,18 @@ size_t attend_workspace_floats(int heads, int nsplit) {
     return static_cast<size_t>(heads) * nsplit * kPart;
 }
 
+bool attend_uses_mma(const pariskv_config* cfg, bool kv_device) {
+    return kv_device && cfg->dtype == PARISKV_BF16;
+}
+
 cudaError_t launch_attend_partial(const pariskv_config* cfg, const void* q, const void* K,
                                   const void* V, int64_t ld_tok, int64_t n,
                                   const int32_t* idx, int32_t k, int32_t k_stride, float scale,
                                   float* work, int nsplit, int split_base, int split_total,
-                                  cudaStream_t st) {
+                                  bool mma, cudaStream_t st) {
+    if (mma)
+        return launch_gather_partial(cfg, q, K, V, ld_tok, n, idx, k, k_stride, scale, work,
+                                     nsplit, split_base, split_total, st);
     const int heads = cfg->batch * cfg->num_kv_heads * cfg->group;
     dim3 grid(nsplit, heads);
     if (cfg->dtype == PARISKV_BF16) {
@@ -275,9 +283,9 @@ cudaError_t launch_attend_combine(int heads, const float* work, int split_total,
 cudaError_t launch_attend(const pariskv_config* cfg, const void* q, const void* K,
                           const void* V, int64_t ld_tok, int64_t n, const int32_t* topk_idx,
                           int32_t k, float scale, void* out, int32_t out_dtype, float* work,
-                          int nsplit, cudaStream_t st) {
+                          int nsplit, bool mma, cudaStream_t st) {
     cudaError_t e = launch_attend_partial(cfg, q, K, V, ld_tok, n, topk_idx, k, k, scale, work,
-                                          nsplit, 0, nsplit, st);
+                                          nsplit, 0, nsplit, mma, st);
     if (e != cudaSuccess) return e;
     const int heads = cfg->batch * cfg->num_kv_heads * cfg->group;
     return launch_attend_combine(heads, work, nsplit, out, out_dtype, st);

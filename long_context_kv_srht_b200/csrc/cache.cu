@@ -202,21 +202,30 @@ pariskv_status evict(pariskv_cache* c, int64_t move, cudaStream_t st) {
     return PARISKV_OK;
 }
 
-// Partials of the dense rows and of the retrieved rows, merged into `out`.
+// Partials of the dense rows and of the retrieved rows, merged into `out`. The dense rows are
+// pool rows [0, n_dense) of every unit: with bf16 K/V one tensor-core pass per unit serves
+// all query heads of the group; fp32 caches use the row-gather kernel over an iota index list.
 pariskv_status attend(pariskv_cache* c, const void* q, float scale, int32_t k_eff, void* out,
                       int32_t out_dtype, cudaStream_t st, int32_t* launches) {
     const int64_t n_dense = c->sink + c->local + c->buffer;
-    const int nd = min(attend_splits(c->heads, static_cast<int32_t>(n_dense), c->sms),
-                       c->max_splits);
-    const int nr = k_eff > 0 ? min(attend_splits(c->heads, k_eff, c->sms), c->max_splits) : 0;
-    cudaError_t e = launch_attend_partial(&c->cfg, q, c->poolK, c->poolV, c->P, n_dense,
-                                          c->dense_idx, static_cast<int32_t>(n_dense), 0,
-                                          scale, c->work, nd, 0, nd + nr, st);
+    const bool dense_mma = c->cfg.dtype == PARISKV_BF16 && c->cfg.group <= 8;
+    const int nd = dense_mma ? min(dense_splits(c->units, n_dense, c->sms), c->max_splits)
+                             : min(attend_splits(c->heads, static_cast<int32_t>(n_dense), c->sms,
+                                                 false),
+                                   c->max_splits);
+    const int nr = k_eff > 0 ? min(attend_splits(c->heads, k_eff, c->sms, false), c->max_splits)
+                             : 0;
+    cudaError_t e =
+        dense_mma ? launch_dense_partial(&c->cfg, q, c->poolK, c->poolV, c->P, n_dense, scale,
+                                         c->work, nd, 0, nd + nr, st)
+                  : launch_attend_partial(&c->cfg, q, c->poolK, c->poolV, c->P, n_dense,
+                                          c->dense_idx, static_cast<int32_t>(n_dense), 0, scale,
+                                          c->work, nd, 0, nd + nr, false, st);
     *launches += 1;
     if (e == cudaSuccess && nr > 0) {
         e = launch_attend_partial(&c->cfg, q, c->hostK, c->hostV, c->cc.retrieval_capacity,
                                   c->retr, c->topk, k_eff, k_eff, scale, c->work, nr, nd,
-                                  nd + nr, st);
+                                  nd + nr, false, st);
         *launches += 1;
     }
     if (e == cudaSuccess) {
@@ -262,7 +271,10 @@ pariskv_status pariskv_cache_create(const pariskv_config* cfg, const pariskv_cac
     c->heads = c->units * icfg.group;
     c->P = static_cast<int64_t>(cc->n_sink) + cc->n_local + cc->n_buffer;
     c->row = static_cast<size_t>(D) * (icfg.dtype == PARISKV_BF16 ? 2 : 4);
-    c->max_splits = max(1, 2 * c->sms / c->heads) + 1;
+    // per source: the row-gather kernel takes up to 2*sms/heads splits, the dense pass
+    // ceil(2*sms/units)
+    c->max_splits = max(max(1, 2 * c->sms / c->heads) + 1,
+                        static_cast<int>(ceil_div(2 * c->sms, c->units)));
     const size_t pool = static_cast<size_t>(c->units) * c->P * c->row;
     const size_t host = static_cast<size_t>(c->units) * cc->retrieval_capacity * c->row;
     const bool ok =

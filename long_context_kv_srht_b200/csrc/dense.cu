@@ -26,6 +26,12 @@
 //  - the 4 warps merge in shared memory and each head's split partial (128 accumulators, max,
 //    denominator) goes to the workspace format of the sparse attention, whose log-sum-exp
 //    combine kernel finishes the job.
+//
+// The same kernel in gather mode is the sparse attention over the retrieved tokens when K/V
+// are in device memory ("Technical Summary: ParisKV", Problem Statement: attend to the Top-k
+// subset): CTA (split, query head) streams the rows named by that head's top-k indices
+// through the same ring (the gathered rows are whole 256-byte lines), and the MMAs use one
+// column of N (the head itself).
 #include "common.cuh"
 #include "internal.hpp"
 
@@ -78,34 +84,60 @@ __device__ __forceinline__ float2 bf2_f(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
+struct MmaAttendArgs {
+    const __nv_bfloat16* q;     // [heads][128]
+    const uint8_t* K;           // [units][ld_tok][128] bf16
+    const uint8_t* V;
+    int64_t ld_tok, n;          // rows [0, n) exist
+    const int32_t* idx;         // gather mode: row j of head h at idx[h * k_stride + j]
+    int32_t k, k_stride;        // gather mode: indices per head
+    float scale;
+    int group;
+    int nsplit, split_base, split_total;
+    float* work;                // partials [heads][split_total][kAttendPart]
+};
+
+// kGather = false: CTA (split, unit) over rows [0, n) for all `group` heads of the unit.
+// kGather = true: CTA (split, head) over the rows its k indices name (outside [0, n): skipped).
+template <bool kGather>
 __global__ void __launch_bounds__(kDW * 32, 2)
-dense_attend_kernel(const __nv_bfloat16* __restrict__ q, const uint8_t* __restrict__ K,
-                    const uint8_t* __restrict__ V, int64_t ld_tok, int64_t n, float scale,
-                    int group, int nsplit, float* __restrict__ work) {
+attend_mma_kernel(const MmaAttendArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint8_t s_ok[kStages][kTile];   // gather mode: row holds a valid token
     uint8_t* sK = smem;
     uint8_t* sV = smem + kStages * kTileB;
-    const int64_t u = blockIdx.y;
     const int split = blockIdx.x;
+    const int64_t head0 = kGather ? static_cast<int64_t>(blockIdx.y) : 0;
+    const int64_t u = kGather ? head0 / a.group : static_cast<int64_t>(blockIdx.y);
+    const int ncols = kGather ? 1 : a.group;  // N columns in use
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;     // fragment row / column pair of this lane
+    const int64_t n = a.n;
+    const int64_t len = kGather ? a.k : n;     // positions to attend
+    const int32_t* hidx = kGather ? a.idx + head0 * a.k_stride : nullptr;
 
-    const int64_t tiles = ceil_div(n, kTile);
-    const int64_t tb0 = tiles * split / nsplit;
-    const int64_t ntile = tiles * (split + 1) / nsplit - tb0;
-    const uint8_t* Kb = K + u * ld_tok * kRowB;
-    const uint8_t* Vb = V + u * ld_tok * kRowB;
+    const int64_t tiles = ceil_div(len, kTile);
+    const int64_t tb0 = tiles * split / a.nsplit;
+    const int64_t ntile = tiles * (split + 1) / a.nsplit - tb0;
+    const uint8_t* Kb = a.K + u * a.ld_tok * kRowB;
+    const uint8_t* Vb = a.V + u * a.ld_tok * kRowB;
 
-    // stage a tile: 2 tensors x 64 rows x 16 chunks of 16 bytes; rows past n are zero-filled
-    // (and masked below)
+    // stage a tile: 2 tensors x 64 rows x 16 chunks of 16 bytes; missing rows are
+    // zero-filled (and masked below)
     auto load_tile = [&](int64_t tile, int stage) {
         const int64_t t0 = (tb0 + tile) * kTile;
 #pragma unroll
         for (int j = 0; j < kLoadsPerThread; ++j) {
             const int id = tid + kDW * 32 * j;
             const int tensor = id / (kTile * 16), row = (id >> 4) & (kTile - 1), c = id & 15;
-            const int64_t tok = t0 + row;
-            const bool ok = tok < n;
+            const int64_t pos = t0 + row;
+            int64_t tok = pos;
+            bool ok = pos < len;
+            if (kGather) {
+                tok = ok ? hidx[pos] : -1;
+                ok = tok >= 0 && tok < n;
+                if (tensor == 0 && c == 0) s_ok[stage][row] = ok;
+            }
             const uint8_t* src = (tensor ? Vb : Kb) + (ok ? tok : 0) * kRowB + c * 16;
             const uint32_t dst = smem_addr((tensor ? sV : sK) + stage * kTileB + row * kRowB +
                                            ((c ^ (row & 7)) << 4));
@@ -119,18 +151,19 @@ dense_attend_kernel(const __nv_bfloat16* __restrict__ q, const uint8_t* __restri
         asm volatile("cp.async.commit_group;" ::: "memory");
     }
 
-    // B fragments of Q^T (k = dims, n = heads): head g, dims 16s + 2t (+1) and 16s + 8 + 2t
-    // (+1); heads past the group are zero
+    // B fragments of Q^T (k = dims, n = heads): column g, dims 16s + 2t (+1) and
+    // 16s + 8 + 2t (+1); unused columns are zero
     uint32_t qb[8][2];
     {
-        const uint32_t* qh = reinterpret_cast<const uint32_t*>(q + (u * group + g) * D);
+        const int64_t qhead = kGather ? head0 : u * a.group + g;
+        const uint32_t* qh = reinterpret_cast<const uint32_t*>(a.q + qhead * D);
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
-            qb[s][0] = g < group ? qh[8 * s + t] : 0u;
-            qb[s][1] = g < group ? qh[8 * s + 4 + t] : 0u;
+            qb[s][0] = g < ncols ? qh[8 * s + t] : 0u;
+            qb[s][1] = g < ncols ? qh[8 * s + 4 + t] : 0u;
         }
     }
-    const float qs = scale * kLog2e;
+    const float qs = a.scale * kLog2e;
 
     // this lane's state: heads 2t and 2t+1 (base-2 max, denominator); O^T accumulators of
     // dim tile i: (dim 16i+g, heads 2t, 2t+1), (dim 16i+g+8, heads 2t, 2t+1)
@@ -164,10 +197,18 @@ dense_attend_kernel(const __nv_bfloat16* __restrict__ q, const uint8_t* __restri
             mma_bf16(sacc, a, qb[s][0], qb[s][1]);
         }
         // sacc[0..1]: token g, heads 2t, 2t+1; sacc[2..3]: token g+8
-        const int64_t tok = (tb0 + it) * kTile + 16 * warp + g;
         float s0 = sacc[0] * qs, s1 = sacc[1] * qs, s2 = sacc[2] * qs, s3 = sacc[3] * qs;
-        if (tok >= n) s0 = s1 = -INFINITY;
-        if (tok + 8 >= n) s2 = s3 = -INFINITY;
+        bool ok_a, ok_b;
+        if (kGather) {
+            ok_a = s_ok[st][16 * warp + g];
+            ok_b = s_ok[st][16 * warp + g + 8];
+        } else {
+            const int64_t tok = (tb0 + it) * kTile + 16 * warp + g;
+            ok_a = tok < n;
+            ok_b = tok + 8 < n;
+        }
+        if (!ok_a) s0 = s1 = -INFINITY;
+        if (!ok_b) s2 = s3 = -INFINITY;
         float b0 = fmaxf(s0, s2), b1 = fmaxf(s1, s3);
 #pragma unroll
         for (int x = 4; x < 32; x <<= 1) {
@@ -233,21 +274,22 @@ dense_attend_kernel(const __nv_bfloat16* __restrict__ q, const uint8_t* __restri
         }
     }
     __syncthreads();
-    for (int h = warp; h < group; h += kDW) {
+    for (int h = warp; h < ncols; h += kDW) {
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kDW; ++w) M = fmaxf(M, sc[(w * kHeadsN + h) * kAttendPart + D]);
-        float den = 0.0f, a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        float den = 0.0f, r[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
         for (int w = 0; w < kDW; ++w) {
             const float* src = sc + (w * kHeadsN + h) * kAttendPart;
             const float f = src[D] == -INFINITY ? 0.0f : exp2f(src[D] - M);
             den += src[D + 1] * f;
             const float4 v = *reinterpret_cast<const float4*>(src + 4 * lane);
-            a[0] += v.x * f; a[1] += v.y * f; a[2] += v.z * f; a[3] += v.w * f;
+            r[0] += v.x * f; r[1] += v.y * f; r[2] += v.z * f; r[3] += v.w * f;
         }
-        float* out = work + ((u * group + h) * nsplit + split) * kAttendPart;
-        *reinterpret_cast<float4*>(out + 4 * lane) = make_float4(a[0], a[1], a[2], a[3]);
+        const int64_t head = kGather ? head0 : u * a.group + h;
+        float* out = a.work + (head * a.split_total + a.split_base + split) * kAttendPart;
+        *reinterpret_cast<float4*>(out + 4 * lane) = make_float4(r[0], r[1], r[2], r[3]);
         if (lane == 0) {
             out[D] = M == -INFINITY ? M : M * kLn2;   // natural-log units, as the combine expects
             out[D + 1] = den;
@@ -263,18 +305,41 @@ int dense_splits(int units, int64_t n, int num_sms) {
     return static_cast<int>(max64(1, min64(want, ceil_div(n, kTile))));
 }
 
+int gather_splits(int heads, int32_t k, int num_sms) {
+    // about two waves of two CTAs per SM, every split at least one tile
+    const int64_t want = ceil_div(4LL * num_sms, heads);
+    return static_cast<int>(max64(1, min64(want, ceil_div(k, kTile))));
+}
+
+template <bool kGather>
+static cudaError_t launch_mma(const MmaAttendArgs& a, dim3 grid, cudaStream_t st) {
+    static std::atomic<uint64_t> done{0};
+    cudaError_t e = raise_smem_limit(attend_mma_kernel<kGather>, kSmem, done);
+    if (e != cudaSuccess) return e;
+    attend_mma_kernel<kGather><<<grid, kDW * 32, kSmem, st>>>(a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_dense_partial(const pariskv_config* cfg, const void* q, const void* K,
                                  const void* V, int64_t ld_tok, int64_t n, float scale,
-                                 float* work, int nsplit, cudaStream_t st) {
+                                 float* work, int nsplit, int split_base, int split_total,
+                                 cudaStream_t st) {
     if (cfg->group > kHeadsN) return cudaErrorInvalidValue;
-    static std::atomic<uint64_t> done{0};
-    cudaError_t e = raise_smem_limit(dense_attend_kernel, kSmem, done);
-    if (e != cudaSuccess) return e;
-    const int units = cfg->batch * cfg->num_kv_heads;
-    dense_attend_kernel<<<dim3(nsplit, units), kDW * 32, kSmem, st>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(K),
-        static_cast<const uint8_t*>(V), ld_tok, n, scale, cfg->group, nsplit, work);
-    return cudaGetLastError();
+    MmaAttendArgs a{static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(K),
+                    static_cast<const uint8_t*>(V), ld_tok, n, nullptr, 0, 0, scale,
+                    cfg->group, nsplit, split_base, split_total, work};
+    return launch_mma<false>(a, dim3(nsplit, cfg->batch * cfg->num_kv_heads), st);
+}
+
+cudaError_t launch_gather_partial(const pariskv_config* cfg, const void* q, const void* K,
+                                  const void* V, int64_t ld_tok, int64_t n, const int32_t* idx,
+                                  int32_t k, int32_t k_stride, float scale, float* work,
+                                  int nsplit, int split_base, int split_total, cudaStream_t st) {
+    MmaAttendArgs a{static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(K),
+                    static_cast<const uint8_t*>(V), ld_tok, n, idx, k, k_stride, scale,
+                    cfg->group, nsplit, split_base, split_total, work};
+    const int heads = cfg->batch * cfg->num_kv_heads * cfg->group;
+    return launch_mma<true>(a, dim3(nsplit, heads), st);
 }
 
 }  // namespace pkv

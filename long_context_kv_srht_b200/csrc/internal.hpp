@@ -131,10 +131,16 @@ cudaError_t launch_topk(const pariskv_index* ix, int64_t C, int32_t k, int32_t* 
 // attend.cu
 cudaError_t launch_read_stream(const void* src, int64_t bytes, uint32_t* sink,
                                cudaStream_t st);
+// Sparse attention has two kernels: with bf16 K/V in device memory, the tensor-core gather
+// kernel of dense.cu (`mma` = true); otherwise (K/V in pinned host memory, or fp32) the
+// latency-tolerant row-gather kernel of attend.cu. attend_splits gives the split count for
+// the chosen kernel; the launchers take the same choice.
+bool attend_uses_mma(const pariskv_config* cfg, bool kv_device);
+int attend_splits(int heads, int32_t k, int num_sms, bool mma);
 cudaError_t launch_attend(const pariskv_config* cfg, const void* q, const void* K,
                           const void* V, int64_t ld_tok, int64_t n, const int32_t* topk_idx,
                           int32_t k, float scale, void* out, int32_t out_dtype, float* work,
-                          int nsplit, cudaStream_t st);
+                          int nsplit, bool mma, cudaStream_t st);
 // the two halves of launch_attend: split-K partials of `k` indices per head (row `head` of
 // idx starts at head * k_stride) written to splits [split_base, split_base + nsplit) of
 // split_total per head, and the log-sum-exp merge of split_total splits per head
@@ -142,20 +148,26 @@ cudaError_t launch_attend_partial(const pariskv_config* cfg, const void* q, cons
                                   const void* V, int64_t ld_tok, int64_t n,
                                   const int32_t* idx, int32_t k, int32_t k_stride, float scale,
                                   float* work, int nsplit, int split_base, int split_total,
-                                  cudaStream_t st);
+                                  bool mma, cudaStream_t st);
 cudaError_t launch_attend_combine(int heads, const float* work, int split_total, void* out,
                                   int32_t out_dtype, cudaStream_t st);
-int attend_splits(int heads, int32_t k, int num_sms);
 // floats per split partial in the attention workspace: 128 accumulators, the running max
 // (natural-log units) and the denominator, padded so every partial starts 16-byte aligned
 constexpr int kAttendPart = 128 + 4;
 
-// dense.cu: split-K partials of dense attention over tokens [0, n) of every unit (bf16 K/V,
-// group <= 8), written like launch_attend_partial's with split_total = nsplit
+// dense.cu (tensor-core attention, bf16 K/V in device memory): split-K partials of dense
+// attention over rows [0, n) of every unit (group <= 8), and of the rows named by each head's
+// indices (gather mode), written like launch_attend_partial's
 int dense_splits(int units, int64_t n, int num_sms);
+int gather_splits(int heads, int32_t k, int num_sms);
 cudaError_t launch_dense_partial(const pariskv_config* cfg, const void* q, const void* K,
                                  const void* V, int64_t ld_tok, int64_t n, float scale,
-                                 float* work, int nsplit, cudaStream_t st);
+                                 float* work, int nsplit, int split_base, int split_total,
+                                 cudaStream_t st);
+cudaError_t launch_gather_partial(const pariskv_config* cfg, const void* q, const void* K,
+                                  const void* V, int64_t ld_tok, int64_t n, const int32_t* idx,
+                                  int32_t k, int32_t k_stride, float scale, float* work,
+                                  int nsplit, int split_base, int split_total, cudaStream_t st);
 // Allocation-free attention: floats in the fixed per-device workspace and its address on the
 // current device (looked up on first use per device).
 constexpr size_t kAttendScratchFloats = size_t(1) << 20;
