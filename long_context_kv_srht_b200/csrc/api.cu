@@ -504,7 +504,10 @@ pariskv_status pariskv_sparse_attend_noalloc(const pariskv_config* cfg, const vo
     if (fit < 1)
         return fail(PARISKV_EINVAL, "%d query heads exceed the fixed attention workspace "
                     "(at most %zu heads)", heads, kAttendScratchFloats / attend_workspace_floats(1, 1));
-    const bool mma = attend_uses_mma(cfg, device_memory(K) && device_memory(V));
+    // the tensor-core gather kernel needs a minimum split count; with too small a fixed
+    // workspace the row-gather kernel runs instead
+    const bool mma = attend_uses_mma(cfg, device_memory(K) && device_memory(V)) &&
+                     gather_min_splits(k) <= fit;
     const int nsplit = min(attend_splits(heads, k, sms, mma), fit);
     float* work = nullptr;
     cudaError_t e = attend_static_scratch(&work);

@@ -154,21 +154,34 @@ attend_partial_kernel(const T* __restrict__ q, const T* __restrict__ K, const T*
     }
 }
 
+// Log-sum-exp merge of one head's splits, one warp per head. Lane s (mod 32) reads split s's
+// max and denominator, so the global maximum and every split's weight take one round of
+// loads; the accumulators are then summed split by split, the weight broadcast by a
+// shuffle, with the float4 loads of eight splits in flight at a time.
 template <typename T>
 __global__ void __launch_bounds__(32)
 attend_combine_kernel(const float* __restrict__ work, int nsplit, T* __restrict__ out) {
     const int head = blockIdx.x, lane = threadIdx.x;
     const float* w = work + static_cast<int64_t>(head) * nsplit * kPart;
     float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, w[s * kPart + kMax]);
+    for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, w[s * kPart + kMax]);
+#pragma unroll
+    for (int x = 16; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x));
     float den = 0.0f, a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    for (int s = 0; s < nsplit; ++s) {
-        const float ms = w[s * kPart + kMax];
+    for (int s0 = 0; s0 < nsplit; s0 += 32) {
+        const int s = s0 + lane;
+        const float ms = s < nsplit ? w[s * kPart + kMax] : -INFINITY;
         const float f = ms == -INFINITY ? 0.0f : expf(ms - M);
-        den += w[s * kPart + kDen] * f;
-        const float4 v = *reinterpret_cast<const float4*>(w + s * kPart + 4 * lane);
-        a[0] += v.x * f; a[1] += v.y * f; a[2] += v.z * f; a[3] += v.w * f;
+        if (s < nsplit) den += w[s * kPart + kDen] * f;
+        const int cnt = min(32, nsplit - s0);
+#pragma unroll 8
+        for (int j = 0; j < cnt; ++j) {
+            const float fj = __shfl_sync(0xffffffffu, f, j);
+            const float4 v = *reinterpret_cast<const float4*>(w + (s0 + j) * kPart + 4 * lane);
+            a[0] += v.x * fj; a[1] += v.y * fj; a[2] += v.z * fj; a[3] += v.w * fj;
+        }
     }
+    den = warp_sum(den);
     const float inv = den > 0.0f ? 1.0f / den : 0.0f;
     float o[4];
 #pragma unroll

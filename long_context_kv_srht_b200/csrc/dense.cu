@@ -47,6 +47,7 @@ constexpr int kTileB = kTile * kRowB;         // 16 KiB per tensor and stage
 constexpr int kSmem = 2 * kStages * kTileB;
 constexpr int kHeadsN = 8;                    // N of the MMAs: query heads per KV head
 constexpr int kLoadsPerThread = 2 * kTile * (kRowB / 16) / (kDW * 32);
+constexpr int kMaxGatherTiles = 16;           // gather mode: tiles per CTA (indices in smem)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 static_assert(kDW * kHeadsN * kAttendPart * sizeof(float) <= static_cast<size_t>(kSmem),
@@ -104,6 +105,7 @@ __global__ void __launch_bounds__(kDW * 32, 2)
 attend_mma_kernel(const MmaAttendArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint8_t s_ok[kStages][kTile];   // gather mode: row holds a valid token
+    __shared__ int32_t s_idx[kGather ? kMaxGatherTiles * kTile : 1];  // gather: this CTA's rows
     uint8_t* sK = smem;
     uint8_t* sV = smem + kStages * kTileB;
     const int split = blockIdx.x;
@@ -121,6 +123,14 @@ attend_mma_kernel(const MmaAttendArgs a) {
     const int64_t ntile = tiles * (split + 1) / a.nsplit - tb0;
     const uint8_t* Kb = a.K + u * a.ld_tok * kRowB;
     const uint8_t* Vb = a.V + u * a.ld_tok * kRowB;
+    if (kGather) {
+        // the CTA's indices, once, coalesced (the host keeps ntile <= kMaxGatherTiles); -1
+        // past the end
+        const int64_t p0 = tb0 * kTile;
+        for (int i = tid; i < ntile * kTile; i += kDW * 32)
+            s_idx[i] = p0 + i < len ? hidx[p0 + i] : -1;
+        __syncthreads();
+    }
 
     // stage a tile: 2 tensors x 64 rows x 16 chunks of 16 bytes; missing rows are
     // zero-filled (and masked below)
@@ -134,7 +144,7 @@ attend_mma_kernel(const MmaAttendArgs a) {
             int64_t tok = pos;
             bool ok = pos < len;
             if (kGather) {
-                tok = ok ? hidx[pos] : -1;
+                tok = s_idx[(tile * kTile) + row];
                 ok = tok >= 0 && tok < n;
                 if (tensor == 0 && c == 0) s_ok[stage][row] = ok;
             }
@@ -306,10 +316,14 @@ int dense_splits(int units, int64_t n, int num_sms) {
 }
 
 int gather_splits(int heads, int32_t k, int num_sms) {
-    // about two waves of two CTAs per SM, every split at least one tile
-    const int64_t want = ceil_div(4LL * num_sms, heads);
-    return static_cast<int>(max64(1, min64(want, ceil_div(k, kTile))));
+    // about two waves of two CTAs per SM, every split at least one tile and at most
+    // kMaxGatherTiles
+    const int64_t tiles = ceil_div(k, kTile);
+    const int64_t want = max64(ceil_div(4LL * num_sms, heads), ceil_div(tiles, kMaxGatherTiles));
+    return static_cast<int>(max64(1, min64(want, tiles)));
 }
+
+int gather_min_splits(int32_t k) { return static_cast<int>(ceil_div(ceil_div(k, kTile), kMaxGatherTiles)); }
 
 template <bool kGather>
 static cudaError_t launch_mma(const MmaAttendArgs& a, dim3 grid, cudaStream_t st) {
@@ -335,6 +349,7 @@ cudaError_t launch_gather_partial(const pariskv_config* cfg, const void* q, cons
                                   const void* V, int64_t ld_tok, int64_t n, const int32_t* idx,
                                   int32_t k, int32_t k_stride, float scale, float* work,
                                   int nsplit, int split_base, int split_total, cudaStream_t st) {
+    if (nsplit < gather_min_splits(k)) return cudaErrorInvalidValue;   // s_idx holds 16 tiles
     MmaAttendArgs a{static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(K),
                     static_cast<const uint8_t*>(V), ld_tok, n, idx, k, k_stride, scale,
                     cfg->group, nsplit, split_base, split_total, work};

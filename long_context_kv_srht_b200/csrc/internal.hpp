@@ -160,6 +160,7 @@ constexpr int kAttendPart = 128 + 4;
 // indices (gather mode), written like launch_attend_partial's
 int dense_splits(int units, int64_t n, int num_sms);
 int gather_splits(int heads, int32_t k, int num_sms);
+int gather_min_splits(int32_t k);   // the gather kernel needs at least this many splits
 cudaError_t launch_dense_partial(const pariskv_config* cfg, const void* q, const void* K,
                                  const void* V, int64_t ld_tok, int64_t n, float scale,
                                  float* work, int nsplit, int split_base, int split_total,
