@@ -26,10 +26,12 @@ oracle is pinned only to its stated definitions and to the invariants they imply
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 import subprocess
 import threading
 from dataclasses import dataclass
+from typing import Optional
 
 import numpy as np
 
@@ -74,6 +76,8 @@ def _load():
             lib.orc_candidate_count.restype = i64
             lib.orc_select_candidates.argtypes = [P, i64, i64, P]
             lib.orc_rerank.argtypes = [i32, i32, P, P, P, P, i64, P, P]
+            lib.orc_encode_rotated_table.argtypes = [i32, i32, P, P, P, i64, P, P, P, P]
+            lib.orc_rerank_table.argtypes = [i32, i32, P, P, P, P, P, i64, P, P]
             lib.orc_topk.argtypes = [P, P, i64, i64, P, P]
             lib.orc_attend.argtypes = [i32, P, P, P, P, i64, ctypes.c_double, P]
             _lib = lib
@@ -123,6 +127,7 @@ class Encoded:
     mag: np.ndarray      # i32 [n, d]
     neg: np.ndarray      # u8  [n, d]
     factor: np.ndarray   # f32 [n, B]
+    table: Optional[np.ndarray] = None   # f32 [8] magnitude levels; None: uniform integers
 
     @property
     def codes(self) -> np.ndarray:
@@ -132,11 +137,18 @@ class Encoded:
 
     @property
     def vt(self) -> np.ndarray:
-        """Dequantised integer vectors (sign applied) as f64 [n, d]."""
+        """Dequantised vectors (sign applied) as f64 [n, d]: the integer levels, or the table's
+        levels for table-coded keys."""
+        if self.table is not None:
+            v = self.table.astype(np.float64)[self.mag]
+            return np.where(self.neg != 0, -v, v)
         return np.where(self.neg != 0, -self.mag, self.mag).astype(np.float64)
 
 
-def encode_rotated(y: np.ndarray, norm: np.ndarray, m: int, levels: int = 7) -> Encoded:
+def encode_rotated(y: np.ndarray, norm: np.ndarray, m: int, levels: int = 7,
+                   table: Optional[np.ndarray] = None) -> Encoded:
+    """Uniform integer levels 0..levels (R5), or, with `table` (8 ascending fp32 magnitudes),
+    the table-level codes of R24."""
     y = np.ascontiguousarray(y, dtype=np.float32)
     nr = np.ascontiguousarray(norm, dtype=np.float32)
     n, d = y.shape
@@ -145,6 +157,12 @@ def encode_rotated(y: np.ndarray, norm: np.ndarray, m: int, levels: int = 7) -> 
     mag = np.empty((n, d), np.int32)
     neg = np.empty((n, d), np.uint8)
     fac = np.empty((n, B), np.float32)
+    if table is not None:
+        table = np.ascontiguousarray(table, dtype=np.float32)
+        assert table.shape == (8,) and np.all(np.diff(table) > 0)
+        _load().orc_encode_rotated_table(d, m, _p(table), _p(y), _p(nr), n, _p(ids), _p(mag),
+                                         _p(neg), _p(fac))
+        return Encoded(ids, mag, neg, fac, table)
     _load().orc_encode_rotated(d, m, levels, _p(y), _p(nr), n, _p(ids), _p(mag), _p(neg),
                                _p(fac))
     return Encoded(ids, mag, neg, fac)
@@ -184,6 +202,10 @@ def rerank(enc: Encoded, cand: np.ndarray, qt: np.ndarray, m: int) -> np.ndarray
     qt = np.ascontiguousarray(qt, dtype=np.float32)
     d = qt.shape[0]
     S = np.empty((cand.shape[0],), np.float32)
+    if enc.table is not None:
+        _load().orc_rerank_table(d, m, _p(enc.table), _p(enc.mag), _p(enc.neg), _p(enc.factor),
+                                 _p(cand), cand.shape[0], _p(qt), _p(S))
+        return S
     _load().orc_rerank(d, m, _p(enc.mag), _p(enc.neg), _p(enc.factor), _p(cand),
                        cand.shape[0], _p(qt), _p(S))
     return S
@@ -223,10 +245,11 @@ class SearchParams:
     cand_bp: int = 500
 
 
-def build_unit(keys: np.ndarray, signs: np.ndarray, m: int) -> Encoded:
-    """Index of one (sequence, KV head): keys [n, d] -> Encoded."""
+def build_unit(keys: np.ndarray, signs: np.ndarray, m: int,
+               table: Optional[np.ndarray] = None) -> Encoded:
+    """Index of one (sequence, KV head): keys [n, d] -> Encoded (table: R24 levels)."""
     y, nr = normalize_rotate(keys, signs)
-    return encode_rotated(y, nr, m)
+    return encode_rotated(y, nr, m, table=table)
 
 
 def search_rotated(enc: Encoded, qt: np.ndarray, qnorm: float, k: int, p: SearchParams):
@@ -304,3 +327,54 @@ def cache_step_attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, regions: Cach
         rows, *_ = search(enc, q, signs, min(k, len(regions.retrieval)), p)
     toks = np.asarray(regions.dense() + [regions.retrieval[r] for r in rows], np.int32)
     return attend(q, K, V, toks, scale), rows
+
+
+# ---------------------------------------------------------------------------------------
+# Magnitude levels from the rotation prior ("Technical Summary: ParisKV", Core Algorithmic
+# Innovations 2, "Quantization": the 3-bit magnitude is derived from rotation-induced Beta
+# priors).
+# After the random rotation the direction of a subspace y_b is uniform on the sphere of
+# R^m, so each coordinate has u_j^2 ~ Beta(1/2, (m-1)/2); equivalently u = g / |g| with g
+# i.i.d. standard normal. The codes quantise r_j = |y_j| / max_i |y_i|, which does not depend
+# on |g|: r has the law of |g_j| / max_i |g_i| for i.i.d. half-normals. With psi the
+# half-normal density and Psi its CDF (erf(t / sqrt 2)), r has mass 1/m at 1 (the maximal
+# coordinate) and on [0, 1) the density
+#     f(x) = (m - 1) * integral_0^inf psi(t) psi(x t) t Psi(t)^(m-2) dt.
+# The levels are the 8-level Lloyd-Max quantiser of that law (nearest-level cells,
+# conditional-mean levels), reading R24.
+# ---------------------------------------------------------------------------------------
+def ratio_density(x: np.ndarray, m: int = 8, t_max: float = 9.0, nt: int = 4096) -> np.ndarray:
+    """f(x) above on [0, 1) by the midpoint rule in t (the integrand is below 1e-17 past
+    t = 9)."""
+    from scipy.special import erf
+    t = (np.arange(nt) + 0.5) * (t_max / nt)
+    psi = np.sqrt(2.0 / np.pi) * np.exp(-0.5 * t * t)
+    Psi = erf(t / np.sqrt(2.0))
+    w = psi * t * Psi ** (m - 2) * (t_max / nt)
+    xt = np.outer(np.asarray(x, dtype=np.float64), t)
+    return (m - 1) * (np.sqrt(2.0 / np.pi) * np.exp(-0.5 * xt * xt)) @ w
+
+
+@functools.lru_cache(maxsize=4)
+def ratio_levels(m: int = 8, nx: int = 16384, iters: int = 2000) -> np.ndarray:
+    """The 8 Lloyd-Max levels (ascending, fp32) of r = |y_j| / max_i |y_i| (reading R24).
+    Cell masses and first moments come from the cumulative integrals of f (trapezoid rule on
+    nx + 1 points), interpolated at the thresholds, so that cells are not snapped to a grid."""
+    x = np.linspace(0.0, 1.0, nx + 1)
+    f = ratio_density(x, m)
+    h = 1.0 / nx
+    F0 = np.concatenate([[0.0], np.cumsum(0.5 * h * (f[1:] + f[:-1]))])
+    xf = x * f
+    F1 = np.concatenate([[0.0], np.cumsum(0.5 * h * (xf[1:] + xf[:-1]))])
+    pm = 1.0 / m                                # point mass at r = 1
+    lv = (np.arange(8) + 0.5) / 8
+    for _ in range(iters):
+        edges = np.concatenate([[0.0], 0.5 * (lv[:-1] + lv[1:]), [1.0]])
+        c0 = np.interp(edges, x, F0)
+        c1 = np.interp(edges, x, F1)
+        s0 = np.diff(c0)
+        s1 = np.diff(c1)
+        s0[7] += pm                             # r = 1 always falls in the top cell
+        s1[7] += pm
+        lv = s1 / s0
+    return lv.astype(np.float32)

@@ -177,6 +177,78 @@ void orc_encode_rotated(int32_t d, int32_t m, int32_t levels, const float* y, co
 }
 
 /* ------------------------------------------------------------------------------------
+ * RSQ codes with a level table ("Beta-prior" levels). [TS] Core Algorithmic Innovations 2,
+ * "Quantization": the 3-bit magnitudes are "derived from rotation-induced Beta priors".
+ * [R24] Levels c_0 < ... < c_7 (fp32, a table given as input) for the ratio
+ *       r_j = |y_j| / max_i |y_i| of the subspace; thresholds t_i = fp32 of the exact
+ *       midpoint (c_{i-1} + c_i) / 2; mag_j = number of i in 1..7 with r_j >= t_i (r_j in
+ *       IEEE fp32: |y_j| / max); the signed level vt_j = (y_j < 0 ? -c : c)[mag_j]. The
+ *       factor is the same fold as with uniform levels, f = ||k|| * sum y^2 / sum vt y (fp32
+ *       FMA chains, j ascending), 0 for an all-zero subspace.
+ * ------------------------------------------------------------------------------------ */
+void orc_encode_rotated_table(int32_t d, int32_t m, const float* lv, const float* y,
+                              const float* knorm, int64_t n, uint8_t* ids, int32_t* mag,
+                              uint8_t* neg, float* factor)
+{
+    const int32_t B = d / m;
+    float th[8];
+    for (int32_t i = 1; i < 8; ++i) th[i] = (float)(((double)lv[i - 1] + (double)lv[i]) * 0.5);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; ++r) {
+        for (int32_t b = 0; b < B; ++b) {
+            const float* yb = y + r * d + (int64_t)b * m;
+            uint32_t id = 0;
+            float mx = 0.0f;
+            for (int32_t j = 0; j < m; ++j) {
+                if (yb[j] < 0.0f) id |= 1u << j;
+                float a = fabsf(yb[j]);
+                if (a > mx) mx = a;
+            }
+            ids[r * B + b] = (uint8_t)id;
+            float n2 = 0.0f, dot = 0.0f;
+            for (int32_t j = 0; j < m; ++j) {
+                const int64_t o = r * d + (int64_t)b * m + j;
+                int32_t q = 0;
+                if (mx != 0.0f) {
+                    const float ratio = fabsf(yb[j]) / mx;
+                    for (int32_t i = 1; i < 8; ++i) q += ratio >= th[i];
+                }
+                mag[o] = q;
+                neg[o] = (uint8_t)(yb[j] < 0.0f);
+                const float vt = neg[o] ? -lv[q] : lv[q];
+                n2 = fmaf(yb[j], yb[j], n2);
+                dot = fmaf(vt, yb[j], dot);
+            }
+            const float num = knorm[r] * n2;
+            factor[r * B + b] = (dot == 0.0f) ? 0.0f : num / dot;
+        }
+    }
+}
+
+/* The rerank of orc_rerank with table levels: vt_j = (neg ? -lv : lv)[mag_j], same chains. */
+void orc_rerank_table(int32_t d, int32_t m, const float* lv, const int32_t* mag,
+                      const uint8_t* neg, const float* factor, const int32_t* cand, int64_t C,
+                      const float* qt, float* S)
+{
+    const int32_t B = d / m;
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < C; ++c) {
+        const int64_t i = cand[c];
+        float s = 0.0f;
+        for (int32_t b = 0; b < B; ++b) {
+            float p = 0.0f;
+            for (int32_t j = 0; j < m; ++j) {
+                const int64_t o = i * d + (int64_t)b * m + j;
+                const float vt = neg[o] ? -lv[mag[o]] : lv[mag[o]];
+                p = fmaf(vt, qt[(int64_t)b * m + j], p);
+            }
+            s = fmaf(factor[i * B + b], p, s);
+        }
+        S[c] = s;
+    }
+}
+
+/* ------------------------------------------------------------------------------------
  * Query lookup table. [TS] "Coarse Candidate Generation": for a query, each subspace
  * selects the top-rho centroids most similar to the rotated query subspace; keys in those
  * buckets get tiered votes.

@@ -402,3 +402,110 @@ def test_cache_step_attend_is_dense_softmax_when_k_covers_retrieval():
     z = K.astype(np.float64) @ q.astype(np.float64) * 0.09
     w = np.exp(z - z.max())
     np.testing.assert_allclose(out, (w / w.sum()) @ V.astype(np.float64), rtol=1e-10, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- prior-derived levels
+def _gaussian_ratios(n, seed):
+    """r = |g_j| / max_i |g_i| over n i.i.d. Gaussian 8-vectors (all 8 coordinates)."""
+    g = np.abs(np.random.default_rng(seed).standard_normal((n, M)))
+    return (g / g.max(axis=1, keepdims=True)).ravel()
+
+
+def test_ratio_law_matches_rotated_directions():
+    """The density of r = |y_j| / max|y| (plus its mass 1/m at 1) integrates to one and its
+    CDF matches r measured on rotated random keys (the oracle's own rotation of
+    non-Gaussian keys, so the test also checks that the rotation makes subspace directions
+    uniform)."""
+    x = (np.arange(8192) + 0.5) / 8192
+    f = oracle.ratio_density(x)
+    assert abs(f.sum() / 8192 + 1 / M - 1.0) < 1e-6
+    rng = np.random.default_rng(21)
+    keys = rng.uniform(-1, 1, (20000, D)).astype(np.float32) ** 3      # far from Gaussian
+    y, _ = oracle.normalize_rotate(keys, _signs(D, 4))
+    a = np.abs(y.reshape(-1, M)).astype(np.float64)
+    r = np.sort((a / a.max(axis=1, keepdims=True)).ravel())
+    cdf_model = np.cumsum(f) / 8192                                     # P(r <= x), x < 1
+    cdf_emp = np.searchsorted(r, x, side="right") / r.size
+    assert np.max(np.abs(cdf_model - cdf_emp)) < 4e-3
+
+
+def test_ratio_levels_are_lloyd_max():
+    """Each level is the conditional mean of r over its nearest-level cell (independent
+    quadrature by scipy on the same law), and the table equals a Lloyd-Max fit to sampled
+    Gaussian ratios."""
+    from scipy.integrate import quad
+    lv = oracle.ratio_levels().astype(np.float64)
+    assert np.all(np.diff(lv) > 0) and 0 < lv[0] and lv[-1] < 1
+    th = np.concatenate([[0.0], 0.5 * (lv[:-1] + lv[1:]), [1.0]])
+    for i in range(8):
+        f = lambda x: float(oracle.ratio_density(np.array([x]))[0])
+        m0 = quad(f, th[i], th[i + 1], limit=200)[0]
+        m1 = quad(lambda x: x * f(x), th[i], th[i + 1], limit=200)[0]
+        if i == 7:
+            m0, m1 = m0 + 1 / M, m1 + 1 / M
+        assert abs(m1 / m0 - lv[i]) < 2e-5, (i, m1 / m0, lv[i])
+    r = _gaussian_ratios(400000, 3)
+    emp = (np.arange(8) + 0.5) / 8
+    for _ in range(300):
+        c = np.searchsorted(0.5 * (emp[:-1] + emp[1:]), r, side="right")
+        emp = np.bincount(c, r, 8) / np.bincount(c, None, 8)
+    np.testing.assert_allclose(lv, emp, atol=3e-3)
+
+
+def test_table_codes_nearest_level():
+    """Table-coded magnitudes are the nearest table level to r = |y_j| / max|y| (fp32 ratio,
+    fp32 midpoint thresholds), the signs are the coordinate signs, and the maximal coordinate
+    takes the top level."""
+    lv = oracle.ratio_levels()
+    rng = np.random.default_rng(22)
+    y = rng.standard_normal((3000, D)).astype(np.float32)
+    enc = oracle.encode_rotated(y, np.ones(3000, np.float32), M, table=lv)
+    a = np.abs(y.reshape(3000, B, M))
+    r = a / a.max(axis=2, keepdims=True)                       # fp32 IEEE division
+    th = (0.5 * (lv[:-1].astype(np.float64) + lv[1:].astype(np.float64))).astype(np.float32)
+    want = (r[..., None] >= th).sum(axis=-1)
+    np.testing.assert_array_equal(enc.mag.reshape(3000, B, M), want)
+    dist = np.abs(r[..., None].astype(np.float64) - lv.astype(np.float64))
+    np.testing.assert_array_equal(want, np.argmin(dist, axis=-1))   # nearest level
+    assert np.all(enc.mag.reshape(3000, B, M).max(axis=2) == 7)
+    np.testing.assert_array_equal(enc.neg, (y < 0).astype(np.uint8))
+
+
+def test_table_estimator_equals_literal_page_form_and_self_estimate():
+    """With table levels the folded factor still equals the literal w_{i,b} <v_b, q~_b>
+    (1e-5), and the estimate of <k, k> is ||k||^2 (2e-6)."""
+    lv = oracle.ratio_levels()
+    rng = np.random.default_rng(23)
+    sg = _signs(D, 13)
+    k = (rng.standard_normal((400, D)) * 2 + 0.5).astype(np.float32)
+    q = rng.standard_normal((1, D)).astype(np.float32)
+    y, kn = oracle.normalize_rotate(k, sg)
+    qt, qn = oracle.normalize_rotate(q, sg)
+    enc = oracle.encode_rotated(y, kn, M, table=lv)
+    lit = _literal_terms(enc, y, kn, qt[0])
+    cand = np.arange(400, dtype=np.int32)
+    S = oracle.rerank(enc, cand, qt[0], M).astype(np.float64)
+    assert np.max(np.abs(float(qn[0]) * S - float(qn[0]) * lit.sum(axis=1)) /
+                  (kn * qn[0])) <= 1e-5
+    for i in range(0, 400, 40):
+        S_ii = oracle.rerank(enc, np.array([i], np.int32), y[i], M)[0]
+        k2 = float(kn[i]) ** 2
+        assert abs(float(kn[i]) * float(S_ii) - k2) <= 2e-6 * k2
+
+
+def test_ratio_levels_quantise_directions_better_than_uniform():
+    """Over rotated random keys the table levels lose less of each subspace direction
+    (mean 1 - cos(y_b, v_b)) than the uniform levels: the point of deriving them from the
+    prior."""
+    lv = oracle.ratio_levels()
+    rng = np.random.default_rng(24)
+    y, kn = oracle.normalize_rotate(rng.standard_normal((20000, D)).astype(np.float32),
+                                    _signs(D, 5))
+    yb = y.reshape(-1, B, M).astype(np.float64)
+
+    def loss(enc):
+        v = enc.vt.reshape(-1, B, M)
+        cos = np.sum(v * yb, axis=2) / (np.linalg.norm(v, axis=2) * np.linalg.norm(yb, axis=2))
+        return float(np.mean(1 - cos))
+    uni, tab = loss(oracle.encode_rotated(y, kn, M)), loss(oracle.encode_rotated(y, kn, M, table=lv))
+    assert tab < 0.85 * uni, (tab, uni)
