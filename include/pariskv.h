@@ -54,7 +54,23 @@ enum { PARISKV_F32 = 0, PARISKV_BF16 = 1 };
  *   d == 128, m == 8, B * m == d (the kernels are specialised for d = 128, m = 8);
  *   1 <= rho <= 2^m; 0 <= w_rest <= w_rank1 <= 3, w_rank1 >= 1 (so a score fits 6 bits);
  *   1 <= cand_bp <= 10000; batch, num_kv_heads, group >= 1; capacity >= 0;
- *   dtype is PARISKV_F32 or PARISKV_BF16. */
+ *   dtype is PARISKV_F32 or PARISKV_BF16; levels is one of the PARISKV_LEVELS_* below.
+ *
+ * Magnitude levels of the 4-bit RSQ codes ("Candidate Reranking", Quantization: 1 sign bit
+ * and 3 magnitude bits, "derived from rotation-induced Beta priors"). Each code quantises
+ * r_j = |y_j| / max_i |y_i| over its 8-dim subspace of the rotated key:
+ *   PARISKV_LEVELS_UNIFORM: mag = min(7, floor(7 r + 1/2)) in IEEE fp32, signed level
+ *     vt = +-mag (8 uniform levels over [0, max]);
+ *   PARISKV_LEVELS_PRIOR: the 8 Lloyd-Max levels of the law of r under the rotation (a
+ *     subspace direction uniform on the sphere, u_j^2 ~ Beta(1/2, 7/2); r has the law of
+ *     half-normal ratios), computed by the library once per process;
+ *   PARISKV_LEVELS_TABLE: the caller's level_table (8 finite fp32 values,
+ *     0 <= c_0 < c_1 < ... < c_7).
+ * With a table, mag = the number of i in 1..7 with r_j >= t_i, r_j in IEEE fp32 and t_i the
+ * fp32 rounding of the exact midpoint (c_{i-1} + c_i) / 2 (the nearest level), and
+ * vt = +-c_mag. Everything else (factor fold, rerank chains) is the same for all three.
+ * level_table is ignored unless levels == PARISKV_LEVELS_TABLE. */
+enum { PARISKV_LEVELS_UNIFORM = 0, PARISKV_LEVELS_PRIOR = 1, PARISKV_LEVELS_TABLE = 2 };
 typedef struct {
     int32_t d;            /* head dimension */
     int32_t B;            /* number of subspaces */
@@ -68,14 +84,18 @@ typedef struct {
     int32_t group;        /* query heads per KV head (GQA group size) */
     int64_t capacity;     /* maximum tokens per (sequence, KV head) in the index */
     int32_t dtype;        /* element type of keys, queries, values and outputs */
-    int32_t reserved;     /* must be 0 */
+    int32_t levels;       /* magnitude levels of the codes: PARISKV_LEVELS_* (default 0) */
+    float level_table[8]; /* the levels when levels == PARISKV_LEVELS_TABLE */
 } pariskv_config;
 
 typedef struct pariskv_index pariskv_index;  /* opaque; owns device memory */
 
 /* Fills *cfg with d=128, B=16, m=8, rho=4, w_rank1=2, w_rest=1, cand_bp=500, batch=1,
- * num_kv_heads=1, group=1, capacity=0, dtype=PARISKV_BF16. */
+ * num_kv_heads=1, group=1, capacity=0, dtype=PARISKV_BF16, levels=PARISKV_LEVELS_UNIFORM. */
 PARISKV_API pariskv_status pariskv_config_default(pariskv_config* cfg);
+
+/* The 8 magnitude levels PARISKV_LEVELS_PRIOR uses (ascending), into out[0..7]. */
+PARISKV_API pariskv_status pariskv_prior_levels(float* out);
 
 /* Builds an index over the first n keys of every (sequence, KV head).
  * Definition: "Normalization and Rotation" and "Coarse Candidate Generation" /

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI of libpariskv.so: argument validation, memory ownership and the
 // launch sequence of each call. Every step of the retrieval path runs in the kernels of this
 // library; the host only validates, allocates and launches.
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -77,7 +78,14 @@ pariskv_status check_config(const pariskv_config* c) {
                     static_cast<long long>(c->capacity));
     if (c->dtype != PARISKV_F32 && c->dtype != PARISKV_BF16)
         return fail(PARISKV_EINVAL, "dtype %d unknown", c->dtype);
-    if (c->reserved != 0) return fail(PARISKV_EINVAL, "reserved field must be 0");
+    if (c->levels != PARISKV_LEVELS_UNIFORM && c->levels != PARISKV_LEVELS_PRIOR &&
+        c->levels != PARISKV_LEVELS_TABLE)
+        return fail(PARISKV_EINVAL, "levels=%d unknown", c->levels);
+    if (c->levels == PARISKV_LEVELS_TABLE)
+        for (int i = 0; i < 8; ++i)
+            if (!std::isfinite(c->level_table[i]) ||
+                (i == 0 ? c->level_table[0] < 0.0f : !(c->level_table[i] > c->level_table[i - 1])))
+                return fail(PARISKV_EINVAL, "level_table must be finite with 0 <= c0 < ... < c7");
     return PARISKV_OK;
 }
 
@@ -137,7 +145,7 @@ void free_index(pariskv_index* ix) {
     if (!ix) return;
     dfree(ix->signs); dfree(ix->ids); dfree(ix->rec); dfree(ix->lut); dfree(ix->qt);
     dfree(ix->qnorm); dfree(ix->scores); dfree(ix->hist); dfree(ix->thr); dfree(ix->cbase);
-    dfree(ix->cand); dfree(ix->S); dfree(ix->shist); dfree(ix->status);
+    dfree(ix->cand); dfree(ix->S); dfree(ix->shist); dfree(ix->status); dfree(ix->lvt);
     for (auto& e : ix->ev)
         if (e) cudaEventDestroy(e);
     delete ix;
@@ -169,7 +177,7 @@ pariskv_status create_index(const pariskv_config* cfg, const int8_t* signs, cuda
               dalloc(&ix->qnorm, heads) && dalloc(&ix->scores, up * ix->cap_pad) &&
               dalloc(&ix->hist, up * nch * PACK * NBINS) && dalloc(&ix->thr, heads * 4) &&
               dalloc(&ix->cbase, heads * nch * 2) && dalloc(&ix->shist, heads * SCOPIES * SBINS) &&
-              dalloc(&ix->status, 1);
+              dalloc(&ix->status, 1) && dalloc(&ix->lvt, kLevelTableFloats);
     if (!ok) {
         free_index(ix);
         return fail(PARISKV_ENOMEM, "device allocation for the index failed");
@@ -181,12 +189,20 @@ pariskv_status create_index(const pariskv_config* cfg, const int8_t* signs, cuda
         free_index(ix);
         return s;
     }
-    float hs[D];
+    float hs[D], tab[kLevelTableFloats];
     for (int j = 0; j < D; ++j) hs[j] = static_cast<float>(signs[j]);
+    if ((s = level_tables(cfg, tab)) != PARISKV_OK) {
+        free_index(ix);
+        return s;
+    }
+    if (cfg->levels == PARISKV_LEVELS_PRIOR)   // record the levels the index is coded with
+        for (int i = 0; i < 8; ++i) ix->cfg.level_table[i] = tab[i];
     cudaError_t e = cudaMemcpyAsync(ix->signs, hs, sizeof(hs), cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(ix->lvt, tab, sizeof(tab), cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(ix->lut, 0, up * NB * NC * sizeof(uint32_t), st);
     if (e == cudaSuccess) e = cudaMemsetAsync(ix->status, 0, sizeof(int), st);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(st);  // hs lives on this stack frame
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);  // hs, tab live on this stack frame
     if (e != cudaSuccess) {
         free_index(ix);
         return cuda_fail(e, "index initialisation");
@@ -524,7 +540,7 @@ pariskv_status pariskv_sparse_attend_noalloc(const pariskv_config* cfg, const vo
 namespace {
 
 constexpr char kMagic[8] = {'P', 'A', 'R', 'I', 'S', 'K', 'V', '\0'};
-constexpr uint32_t kImageVersion = 1;
+constexpr uint32_t kImageVersion = 2;
 
 struct ImageHeader {
     char magic[8];
@@ -535,9 +551,9 @@ struct ImageHeader {
     int32_t units;
     int32_t reserved;
     int8_t signs[D];
-    uint8_t pad[256 - 88 - D];
+    uint8_t pad[256 - 120 - D];
 };
-static_assert(sizeof(pariskv_config) == 56, "image header layout");
+static_assert(sizeof(pariskv_config) == 88, "image header layout");
 static_assert(sizeof(ImageHeader) == 256, "image header layout");
 
 constexpr size_t kKeyBytes = 16 + REC;   // bucket ids + code record per key
@@ -609,6 +625,8 @@ pariskv_status pariskv_import(const void* buf, size_t bytes, int64_t capacity, v
                     static_cast<long long>(capacity), static_cast<long long>(h.n));
     pariskv_config cfg = h.cfg;
     cfg.capacity = capacity;
+    // an index coded with the prior-derived levels keeps exactly the levels it was coded with
+    if (cfg.levels == PARISKV_LEVELS_PRIOR) cfg.levels = PARISKV_LEVELS_TABLE;
     pariskv_status s = check_config(&cfg);
     if (s != PARISKV_OK) return s;
     const size_t nid = static_cast<size_t>(h.n) * 16, nrec = static_cast<size_t>(h.n) * REC;
@@ -810,12 +828,14 @@ pariskv_status pariskv_debug_export_index(pariskv_index* ix, uint8_t* ids, uint8
                 const int64_t at = i * REC + 32 * (b >> 2) + 4 * (b & 3);
                 uint32_t w;
                 memcpy(&w, &hrec[at], 4);
-                // stored offset binary u = vt + 8; canonical code = sign << 3 | magnitude,
-                // the sign being bit j of the bucket id
+                // stored nibble u: uniform levels store vt + 8, table levels 8 + mag (y >= 0)
+                // or 7 - mag (y < 0); canonical code = sign << 3 | magnitude, the sign being
+                // bit j of the bucket id
+                const bool table = ix->cfg.levels != PARISKV_LEVELS_UNIFORM;
                 if (codes)
                     for (int j = 0; j < M; ++j) {
                         const int u = static_cast<int>((w >> (4 * j)) & 15u);
-                        const int mag = u >= 8 ? u - 8 : 8 - u;
+                        const int mag = u >= 8 ? u - 8 : (table ? 7 - u : 8 - u);
                         codes[o * D + b * M + j] =
                             static_cast<uint8_t>((((id >> j) & 1u) << 3) | static_cast<uint32_t>(mag));
                     }

@@ -8,7 +8,9 @@
 //    pattern, stored as one byte per subspace (bit j = dim j is negative).
 //  - 2 "Quantization": one 4-bit code per dim, a sign bit and a 3-bit magnitude; the
 //    magnitude is the nearest of 8 uniform levels over [0, max_j |y_j|] of its subspace:
-//    mag = min(7, floor(7|y| / max + 1/2)) in IEEE fp32, in that order.
+//    mag = min(7, floor(7|y| / max + 1/2)) in IEEE fp32, in that order; or, with a level
+//    table (levels derived from the rotation prior, or the caller's), the nearest table level
+//    to |y| / max (see encode_subspace_table).
 //  - 2 "Calibration": the per-(key, subspace) factor precomputed at prefill,
 //    f = ||k|| * sum_j y_j^2 / sum_j vt_j y_j  (vt the signed integer levels), which folds
 //    w_{i,b} = ||k|| ||y_b|| / <u_b, v_b> and the normalisation of v_b into one number so
@@ -71,11 +73,52 @@ __device__ __forceinline__ void encode_subspace(const float w[8], float knorm, u
     factor = (dot == 0.0f) ? 0.0f : __fdiv_rn(num, dot);
 }
 
-template <typename T, bool ROTATED>
+// The same with table levels (lv[0..7] ascending, th[i] = fp32 midpoint of lv[i-1], lv[i]):
+// r = |y| / max in IEEE fp32, mag = #{i in 1..7 : r >= th[i]}, vt = +-lv[mag]; the code
+// nibble is 8 + mag for y >= 0 and 7 - mag for y < 0, so that every (sign, magnitude) pair has
+// its own nibble (with a table the level of magnitude 0 is not zero).
+__device__ __forceinline__ void encode_subspace_table(const float w[8], float knorm,
+                                                      const float lv[8], const float th[8],
+                                                      uint32_t& id, uint32_t& code,
+                                                      float& factor) {
+    id = 0;
+    float mx = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        id |= (w[j] < 0.0f ? 1u : 0u) << j;
+        mx = fmaxf(mx, fabsf(w[j]));
+    }
+    code = 0;
+    float n2 = 0.0f, dot = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        int q = 0;
+        float c = lv[0];
+        if (mx != 0.0f) {
+            const float r = __fdiv_rn(fabsf(w[j]), mx);
+#pragma unroll
+            for (int i = 1; i < 8; ++i)
+                if (r >= th[i]) {
+                    q = i;
+                    c = lv[i];
+                }
+        }
+        const bool sgn = w[j] < 0.0f;
+        code |= static_cast<uint32_t>(sgn ? 7 - q : 8 + q) << (4 * j);
+        const float vt = sgn ? -c : c;
+        n2 = __fmaf_rn(w[j], w[j], n2);
+        dot = __fmaf_rn(vt, w[j], dot);
+    }
+    const float num = __fmul_rn(knorm, n2);
+    factor = (dot == 0.0f) ? 0.0f : __fdiv_rn(num, dot);
+}
+
+template <typename T, bool ROTATED, bool TABLE>
 __global__ void __launch_bounds__(kEncWarps * 32)
 encode_kernel(const T* __restrict__ src, const float* __restrict__ knorm_in, int64_t ld_tok,
               int64_t t, const float* __restrict__ signs, uint8_t* __restrict__ ids,
-              uint8_t* __restrict__ rec, int64_t cap_pad, int64_t pos0) {
+              uint8_t* __restrict__ rec, int64_t cap_pad, int64_t pos0,
+              const float* __restrict__ lvt) {
     const int lane = threadIdx.x & 31;
     const int64_t r = static_cast<int64_t>(blockIdx.x) * kEncWarps + (threadIdx.x >> 5);
     const int64_t unit = blockIdx.y;
@@ -106,7 +149,17 @@ encode_kernel(const T* __restrict__ src, const float* __restrict__ knorm_in, int
     }
     uint32_t id, code;
     float f;
-    encode_subspace(w, knorm, id, code, f);
+    if constexpr (TABLE) {
+        float lv[8], th[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            lv[i] = __ldg(lvt + i);
+            th[i] = __ldg(lvt + 8 + i);
+        }
+        encode_subspace_table(w, knorm, lv, th, id, code, f);
+    } else {
+        encode_subspace(w, knorm, id, code, f);
+    }
 
     if (!odd) {
         const int b = lane >> 1;
@@ -136,25 +189,35 @@ rotate_kernel(const T* __restrict__ x, int64_t n, const float* __restrict__ sign
 
 }  // namespace
 
+template <bool TABLE>
+static void launch_encode_t(const pariskv_index* ix, const void* keys, const float* knorm,
+                            int64_t ld_tok, int64_t t, int64_t pos0, bool rotated,
+                            cudaStream_t st) {
+    dim3 grid(static_cast<unsigned>(ceil_div(t, kEncWarps)), static_cast<unsigned>(ix->units));
+    dim3 block(kEncWarps * 32);
+    if (rotated) {
+        encode_kernel<float, true, TABLE><<<grid, block, 0, st>>>(
+            static_cast<const float*>(keys), knorm, ld_tok, t, ix->signs, ix->ids, ix->rec,
+            ix->cap_pad, pos0, ix->lvt);
+    } else if (ix->cfg.dtype == PARISKV_BF16) {
+        encode_kernel<__nv_bfloat16, false, TABLE><<<grid, block, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(keys), nullptr, ld_tok, t, ix->signs, ix->ids,
+            ix->rec, ix->cap_pad, pos0, ix->lvt);
+    } else {
+        encode_kernel<float, false, TABLE><<<grid, block, 0, st>>>(
+            static_cast<const float*>(keys), nullptr, ld_tok, t, ix->signs, ix->ids, ix->rec,
+            ix->cap_pad, pos0, ix->lvt);
+    }
+}
+
 cudaError_t launch_encode(const pariskv_index* ix, const void* keys, const float* knorm,
                           int64_t ld_tok, int64_t t, int64_t pos0, bool rotated,
                           cudaStream_t st) {
     if (t <= 0) return cudaSuccess;
-    dim3 grid(static_cast<unsigned>(ceil_div(t, kEncWarps)), static_cast<unsigned>(ix->units));
-    dim3 block(kEncWarps * 32);
-    if (rotated) {
-        encode_kernel<float, true><<<grid, block, 0, st>>>(
-            static_cast<const float*>(keys), knorm, ld_tok, t, ix->signs, ix->ids, ix->rec,
-            ix->cap_pad, pos0);
-    } else if (ix->cfg.dtype == PARISKV_BF16) {
-        encode_kernel<__nv_bfloat16, false><<<grid, block, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(keys), nullptr, ld_tok, t, ix->signs, ix->ids,
-            ix->rec, ix->cap_pad, pos0);
-    } else {
-        encode_kernel<float, false><<<grid, block, 0, st>>>(
-            static_cast<const float*>(keys), nullptr, ld_tok, t, ix->signs, ix->ids, ix->rec,
-            ix->cap_pad, pos0);
-    }
+    if (ix->cfg.levels == PARISKV_LEVELS_UNIFORM)
+        launch_encode_t<false>(ix, keys, knorm, ld_tok, t, pos0, rotated, st);
+    else
+        launch_encode_t<true>(ix, keys, knorm, ld_tok, t, pos0, rotated, st);
     return cudaGetLastError();
 }
 

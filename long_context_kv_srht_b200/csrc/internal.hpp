@@ -19,6 +19,8 @@ struct pariskv_index {
     int packs = 0;        // ceil(group / 4): vote-table packs per KV head
 
     int8_t hsigns[128] = {};    // the SRHT signs as given (host copy, for index images)
+    float* lvt = nullptr;       // [32] code levels: [0..7] magnitudes, [9..15] thresholds,
+                                //      [16..31] signed level of each code nibble
     float* signs = nullptr;     // [128] +-1.0f
     uint8_t* ids = nullptr;     // [units][cap_pad][16] bucket ids, byte-rotated per key
     uint8_t* rec = nullptr;     // [units][cap_pad][128] codes (64 B) + factors (16 x f32)
@@ -94,6 +96,12 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
                        cudaStream_t st, Args&&... args) {
     return launch_pdl_cluster(kernel, grid, block, smem, st, 1u, std::forward<Args>(args)...);
 }
+
+// levels.cu: the code level table of a config ([0..7] magnitude levels, [8 + i] the fp32
+// threshold between levels i-1 and i, [16 + u] the signed level of code nibble u)
+constexpr int kLevelTableFloats = 32;
+pariskv_status level_tables(const pariskv_config* cfg, float tab[kLevelTableFloats]);
+void prior_levels(float out[8]);
 
 // status helpers (defined in api.cu)
 pariskv_status fail(pariskv_status s, const char* fmt, ...);

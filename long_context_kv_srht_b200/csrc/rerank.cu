@@ -63,20 +63,39 @@ __device__ __forceinline__ uint64_t level_pair(uint32_t xa, uint32_t xb) {
                 kOff);
 }
 
+// table levels: nibble u (byte K of each word) -> dec[u], a 16-entry table in shared memory
+template <int K>
+__device__ __forceinline__ uint64_t table_pair(uint32_t xa, uint32_t xb, const float* dec) {
+    return pack2(dec[(xa >> (8 * K)) & 15u], dec[(xb >> (8 * K)) & 15u]);
+}
+
 // p chains of the subspace pair (a, b) from their code words, with the query pairs
 // q[j] = (q~_{a,j}, q~_{b,j}) for j = 0..7.
-__device__ __forceinline__ float2 pair_dots(uint32_t wa, uint32_t wb, const uint64_t q[8]) {
+template <bool TABLE>
+__device__ __forceinline__ float2 pair_dots(uint32_t wa, uint32_t wb, const uint64_t q[8],
+                                            const float* dec) {
     const uint32_t ea = wa & 0x0F0F0F0Fu, oa = (wa >> 4) & 0x0F0F0F0Fu;  // dims 0,2,4,6 | 1,3,5,7
     const uint32_t eb = wb & 0x0F0F0F0Fu, ob = (wb >> 4) & 0x0F0F0F0Fu;
     uint64_t p = pack2(0.0f, 0.0f);
-    p = fma2(level_pair<0>(ea, eb), q[0], p);
-    p = fma2(level_pair<0>(oa, ob), q[1], p);
-    p = fma2(level_pair<1>(ea, eb), q[2], p);
-    p = fma2(level_pair<1>(oa, ob), q[3], p);
-    p = fma2(level_pair<2>(ea, eb), q[4], p);
-    p = fma2(level_pair<2>(oa, ob), q[5], p);
-    p = fma2(level_pair<3>(ea, eb), q[6], p);
-    p = fma2(level_pair<3>(oa, ob), q[7], p);
+    if constexpr (TABLE) {
+        p = fma2(table_pair<0>(ea, eb, dec), q[0], p);
+        p = fma2(table_pair<0>(oa, ob, dec), q[1], p);
+        p = fma2(table_pair<1>(ea, eb, dec), q[2], p);
+        p = fma2(table_pair<1>(oa, ob, dec), q[3], p);
+        p = fma2(table_pair<2>(ea, eb, dec), q[4], p);
+        p = fma2(table_pair<2>(oa, ob, dec), q[5], p);
+        p = fma2(table_pair<3>(ea, eb, dec), q[6], p);
+        p = fma2(table_pair<3>(oa, ob, dec), q[7], p);
+    } else {
+        p = fma2(level_pair<0>(ea, eb), q[0], p);
+        p = fma2(level_pair<0>(oa, ob), q[1], p);
+        p = fma2(level_pair<1>(ea, eb), q[2], p);
+        p = fma2(level_pair<1>(oa, ob), q[3], p);
+        p = fma2(level_pair<2>(ea, eb), q[4], p);
+        p = fma2(level_pair<2>(oa, ob), q[5], p);
+        p = fma2(level_pair<3>(ea, eb), q[6], p);
+        p = fma2(level_pair<3>(oa, ob), q[7], p);
+    }
     return unpack2(p);
 }
 
@@ -92,8 +111,9 @@ __device__ __forceinline__ void load_qpairs(const uint64_t* qp, uint64_t q[8]) {
 // S of the kPerLane records in stage rows row0 + 32 u; qp = the head's 64 query pairs (pair
 // t at qp + 8 t). Each query pair is read once for all the lane's records; every record
 // keeps its own p and S chains in the defined order.
+template <bool TABLE>
 __device__ __forceinline__ void score_records(const uint8_t* st, int row0, const uint64_t* qp,
-                                              float S[kPerLane]) {
+                                              const float* dec, float S[kPerLane]) {
 #pragma unroll
     for (int u = 0; u < kPerLane; ++u) S[u] = 0.0f;
 #pragma unroll
@@ -108,14 +128,14 @@ __device__ __forceinline__ void score_records(const uint8_t* st, int row0, const
         load_qpairs(qp + 16 * c, q);
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
-            const float2 pa = pair_dots(cw[u].x, cw[u].y, q);
+            const float2 pa = pair_dots<TABLE>(cw[u].x, cw[u].y, q, dec);
             S[u] = __fmaf_rn(__uint_as_float(fw[u].x), pa.x, S[u]);
             S[u] = __fmaf_rn(__uint_as_float(fw[u].y), pa.y, S[u]);
         }
         load_qpairs(qp + 16 * c + 8, q);
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
-            const float2 pb = pair_dots(cw[u].z, cw[u].w, q);
+            const float2 pb = pair_dots<TABLE>(cw[u].z, cw[u].w, q, dec);
             S[u] = __fmaf_rn(__uint_as_float(fw[u].z), pb.x, S[u]);
             S[u] = __fmaf_rn(__uint_as_float(fw[u].w), pb.y, S[u]);
         }
@@ -148,12 +168,19 @@ struct StreamPos {
     const uint8_t* ubase;  // records of the head's unit
 };
 
+template <bool TABLE>
 __global__ void __launch_bounds__(kThr, kCtasPerSm)
 rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
               const float* __restrict__ qt, float* __restrict__ S, int32_t C, int64_t cmax,
               int64_t cap_pad, int64_t n, int group, int iph, int64_t items,
-              uint32_t* __restrict__ shist, int* status) {
+              uint32_t* __restrict__ shist, int* status, const float* __restrict__ lvt) {
     extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ float dec[16];   // table levels: code nibble -> signed level
+    if constexpr (TABLE) {
+        // the index's level table is written when the index is created, never by a search
+        if (threadIdx.x < 16) dec[threadIdx.x] = lvt[16 + threadIdx.x];
+        __syncthreads();
+    }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* ring = smem + warp * kWarpBytes;
     float2* qs = reinterpret_cast<float2*>(ring + kSlots * kStageBytes);
@@ -244,7 +271,7 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
         }
         const uint8_t* st = ring + slot * kStageBytes;
         float sv[kPerLane];
-        score_records(st, lane, qp, sv);
+        score_records<TABLE>(st, lane, qp, dec, sv);
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
             const int c = sc.c0 + kStageRecs * sc.s + 32 * u + lane;
@@ -272,8 +299,11 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
 
 cudaError_t launch_rerank(const pariskv_index* ix, int64_t C, cudaStream_t st) {
     if (C <= 0) return cudaSuccess;
-    static std::atomic<uint64_t> smem_raised{0};
-    if (cudaError_t e = raise_smem_limit(rerank_kernel, kSmem, smem_raised); e != cudaSuccess)
+    static std::atomic<uint64_t> smem_raised{0}, smem_raised_t{0};
+    const bool table = ix->cfg.levels != PARISKV_LEVELS_UNIFORM;
+    if (cudaError_t e = table ? raise_smem_limit(rerank_kernel<true>, kSmem, smem_raised_t)
+                              : raise_smem_limit(rerank_kernel<false>, kSmem, smem_raised);
+        e != cudaSuccess)
         return e;
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
@@ -283,9 +313,10 @@ cudaError_t launch_rerank(const pariskv_index* ix, int64_t C, cudaStream_t st) {
     const int64_t items = static_cast<int64_t>(heads) * iph;
     const int grid =
         static_cast<int>(max64(1, min64(int64_t{kCtasPerSm} * sms, ceil_div(items, kWarps))));
-    return launch_pdl(rerank_kernel, grid, kThr, kSmem, st, ix->rec, ix->cand, ix->qt, ix->S,
-                      static_cast<int32_t>(C), ix->cmax, ix->cap_pad, ix->n, ix->cfg.group, iph,
-                      items, ix->shist, ix->status);
+    return launch_pdl(table ? rerank_kernel<true> : rerank_kernel<false>, grid, kThr, kSmem, st,
+                      ix->rec, ix->cand, ix->qt, ix->S, static_cast<int32_t>(C), ix->cmax,
+                      ix->cap_pad, ix->n, ix->cfg.group, iph, items, ix->shist, ix->status,
+                      static_cast<const float*>(ix->lvt));
 }
 
 }  // namespace pkv

@@ -21,6 +21,7 @@ HEADERS = [os.path.join(os.path.dirname(_PKG), "include", h)
 
 OK, EINVAL, ENOMEM, ECUDA, ECAPACITY, ETIMEOUT = range(6)
 F32, BF16 = 0, 1
+LEVELS_UNIFORM, LEVELS_PRIOR, LEVELS_TABLE = range(3)
 
 
 class PariskvError(RuntimeError):
@@ -39,7 +40,7 @@ class Config(ctypes.Structure):
                 ("cand_bp", ctypes.c_int32), ("batch", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("group", ctypes.c_int32),
                 ("capacity", ctypes.c_int64), ("dtype", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("levels", ctypes.c_int32), ("level_table", ctypes.c_float * 8)]
 
     @property
     def num_q_heads(self) -> int:
@@ -74,6 +75,7 @@ _SIGS = {
     "pariskv_import": (_S, [_P, ctypes.c_size_t, _I64, _P, ctypes.POINTER(_P)]),
     "pariskv_dense_attend": (_S, [ctypes.POINTER(Config), _P, _P, _P, _I64, _I64, ctypes.c_float,
                                   _P, _I32, _P]),
+    "pariskv_prior_levels": (_S, [ctypes.POINTER(ctypes.c_float)]),
     "pariskv_sync": (_S, [_P, _P]),
     "pariskv_destroy": (_S, [_P]),
     "pariskv_size": (_I64, [_P]),
@@ -130,8 +132,19 @@ def config(**kw) -> Config:
     for k, v in kw.items():
         if k == "dtype" and isinstance(v, str):
             v = BF16 if v == "bf16" else F32
+        if k == "levels" and isinstance(v, str):
+            v = {"uniform": LEVELS_UNIFORM, "prior": LEVELS_PRIOR, "table": LEVELS_TABLE}[v]
+        if k == "level_table":
+            v = (ctypes.c_float * 8)(*[float(x) for x in v])
         setattr(c, k, v)
     return c
+
+
+def prior_levels() -> np.ndarray:
+    """pariskv_prior_levels: the 8 magnitude levels of PARISKV_LEVELS_PRIOR."""
+    out = (ctypes.c_float * 8)()
+    _check(lib.pariskv_prior_levels(out), "pariskv_prior_levels")
+    return np.array(out, dtype=np.float32)
 
 
 def _stream(stream) -> int:
@@ -286,9 +299,12 @@ def import_index(image, capacity: int = 0, stream=None) -> Index:
         st = _stream(stream)
     _check(lib.pariskv_import(buf.ctypes.data, buf.nbytes, capacity, st, ctypes.byref(h)),
            "pariskv_import")
-    cfg = Config.from_buffer_copy(bytes(buf[16:16 + ctypes.sizeof(Config)]))
-    cfg.capacity = capacity if capacity else max(1, int(np.frombuffer(
-        bytes(buf[72:80]), np.int64)[0]))
+    o = 16 + ctypes.sizeof(Config)              # header: magic, version, size, config, n
+    cfg = Config.from_buffer_copy(bytes(buf[16:o]))
+    cfg.capacity = capacity if capacity else max(1, int(np.frombuffer(bytes(buf[o:o + 8]),
+                                                                      np.int64)[0]))
+    if cfg.levels == LEVELS_PRIOR:              # imported with the levels it was coded with
+        cfg.levels = LEVELS_TABLE
     return Index(h.value, cfg)
 
 

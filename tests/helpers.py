@@ -7,9 +7,10 @@ import numpy as np
 import oracle
 
 
-def oracle_unit_from_rotated(y, kn, qts, qns, k, p: oracle.SearchParams):
-    """Oracle stages for one unit from rotated inputs: y [n, d], kn [n]; qts [G, d]."""
-    enc = oracle.encode_rotated(y, kn, p.m)
+def oracle_unit_from_rotated(y, kn, qts, qns, k, p: oracle.SearchParams, table=None):
+    """Oracle stages for one unit from rotated inputs: y [n, d], kn [n]; qts [G, d]; table:
+    the magnitude levels of table-coded keys (None: uniform levels)."""
+    enc = oracle.encode_rotated(y, kn, p.m, table=table)
     out = []
     for qt, qn in zip(qts, qns):
         lut = oracle.query_lut(qt, p.m, p.rho, p.w_rank1, p.w_rest)

@@ -26,13 +26,13 @@ def test_library_exports_every_declared_symbol():
 def test_config_default():
     c = pk.config()
     assert (c.d, c.B, c.m, c.rho, c.w_rank1, c.w_rest, c.cand_bp) == (128, 16, 8, 4, 2, 1, 500)
-    assert ctypes.sizeof(pk.Config) == 56
+    assert ctypes.sizeof(pk.Config) == 88
 
 
 @pytest.mark.parametrize("field,value", [("d", 64), ("m", 4), ("B", 8), ("rho", 0), ("rho", 257),
                                          ("w_rank1", 4), ("w_rest", 3), ("cand_bp", 0),
                                          ("cand_bp", 10001), ("batch", 0), ("group", 0),
-                                         ("capacity", -1), ("dtype", 7), ("reserved", 1)])
+                                         ("capacity", -1), ("dtype", 7), ("levels", 3)])
 def test_invalid_config_rejected(field, value):
     c = pk.config(capacity=10)
     setattr(c, field, value)
@@ -59,7 +59,7 @@ def test_status_strings_and_null_handles():
 
 
 # ------------------------------------------------------------------ index images (host checks)
-def _header(n=5, units=2, version=1, magic=b"PARISKV\0", **cfg_kw):
+def _header(n=5, units=2, version=2, magic=b"PARISKV\0", **cfg_kw):
     """A 256-byte image header laid out as include/pariskv.h describes it."""
     import numpy as np
     cfg = pk.config(batch=1, num_kv_heads=units, capacity=max(n, 1), **cfg_kw)
@@ -67,10 +67,10 @@ def _header(n=5, units=2, version=1, magic=b"PARISKV\0", **cfg_kw):
     h[0:8] = magic
     h[8:12] = int(version).to_bytes(4, "little")
     h[12:16] = (256).to_bytes(4, "little")
-    h[16:72] = bytes(cfg)
-    h[72:80] = int(n).to_bytes(8, "little", signed=True)
-    h[80:84] = int(units).to_bytes(4, "little", signed=True)
-    h[88:216] = np.ones(128, np.int8).tobytes()
+    h[16:104] = bytes(cfg)
+    h[104:112] = int(n).to_bytes(8, "little", signed=True)
+    h[112:116] = int(units).to_bytes(4, "little", signed=True)
+    h[120:248] = np.ones(128, np.int8).tobytes()
     return bytes(h)
 
 
@@ -86,10 +86,10 @@ def test_import_rejects_bad_images_on_the_host(case):
     elif case == "magic":
         img = _header(n, units, magic=b"PARISKW\0") + body
     elif case == "version":
-        img = _header(n, units, version=2) + body
+        img = _header(n, units, version=3) + body
     elif case == "units":
         img = _header(n, 3) + body          # header says 3 units, config says 3 KV heads
-        img = img[:16] + bytes(pk.config(batch=1, num_kv_heads=2, capacity=5)) + img[72:]
+        img = img[:16] + bytes(pk.config(batch=1, num_kv_heads=2, capacity=5)) + img[104:]
     elif case == "truncated":
         img = img[:-1]
     elif case == "capacity":
@@ -111,3 +111,24 @@ def test_import_accepts_a_well_formed_image_up_to_the_device():
     h = ctypes.c_void_p()
     st = pk.lib.pariskv_import(img, len(img), 0, None, ctypes.byref(h))
     assert st in (pk.ECUDA, pk.ENOMEM) and not h.value, (st, pk.last_error())
+
+
+def test_prior_levels_match_the_oracle():
+    """The library's prior-derived levels (its own quadrature and Lloyd-Max iteration, host
+    code) agree with the oracle's derivation of the same law."""
+    import numpy as np
+    import oracle
+    np.testing.assert_allclose(pk.prior_levels(), oracle.ratio_levels(), atol=1e-6)
+
+
+@pytest.mark.parametrize("table", [[0.1, 0.2, 0.3, 0.3, 0.5, 0.6, 0.7, 0.8],
+                                   [-0.1, 0.2, 0.3, 0.4, 0.5, 0.6, 0.7, 0.8],
+                                   [0.1, 0.2, 0.3, float("nan"), 0.5, 0.6, 0.7, 0.8]])
+def test_invalid_level_table_rejected(table):
+    import numpy as np
+    c = pk.config(capacity=10, levels="table", level_table=table)
+    signs = np.ones(128, np.int8)
+    h = ctypes.c_void_p()
+    st = pk.lib.pariskv_build_index(ctypes.byref(c), signs.ctypes.data, None, 0, 0, None,
+                                    ctypes.byref(h))
+    assert st == pk.EINVAL and not h.value and "level_table" in pk.last_error()

@@ -19,13 +19,16 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def _run(name, sample_units, sample_heads=None):
+def _run(name, sample_units, sample_heads=None, table=None):
+    """table: code with the oracle's prior-derived levels (given to the library as a table for
+    the bit-exact part; the end-to-end part uses the library's own prior levels)."""
     sp = workload.spec(name)
     d = workload.generate_torch(sp, DEV)
     signs = d["signs"].numpy()
     units, G, n = sp.batch * sp.num_kv_heads, sp.group, sp.n
+    lv = {} if table is None else {"levels": "table", "level_table": table}
     cfg = pk.config(batch=sp.batch, num_kv_heads=sp.num_kv_heads, group=G, capacity=n,
-                    dtype=sp.dtype, rho=sp.rho, cand_bp=sp.cand_bp)
+                    dtype=sp.dtype, rho=sp.rho, cand_bp=sp.cand_bp, **lv)
     keys = d["keys"].reshape(units, n, 128)
     y, kn = pk.rotate(cfg, signs, keys)
     y = y.reshape(units, n, 128)
@@ -49,7 +52,8 @@ def _run(name, sample_units, sample_heads=None):
         yo, no = host[u]
         heads = range(G) if sample_heads is None else sample_heads
         enc, outs = oracle_unit_from_rotated(yo, no, qt[u * G:(u + 1) * G][list(heads)],
-                                             qn[u * G:(u + 1) * G][list(heads)], k, p)
+                                             qn[u * G:(u + 1) * G][list(heads)], k, p,
+                                             table=table)
         for g, o in zip(heads, outs):
             h = u * G + g
             np.testing.assert_array_equal(gsc[h], o["scores"])
@@ -59,12 +63,14 @@ def _run(name, sample_units, sample_heads=None):
             np.testing.assert_array_equal(gest[h].view(np.uint32), o["est"].view(np.uint32))
     del ix, y, kn
     # end to end from raw inputs on one sampled unit (the library rotates keys and queries)
+    if table is not None:
+        cfg.levels = pk.LEVELS_PRIOR
     ixr = pk.build_index(cfg, signs, d["keys"])
     ridx, _ = ixr.search(d["queries"], k)
     ixr.sync()
     ridx = ridx.cpu().numpy()
     u = sample_units[0]
-    enc = oracle.encode_rotated(host[u][0], host[u][1], 8)   # the oracle's index of unit u
+    enc = oracle.encode_rotated(host[u][0], host[u][1], 8, table=table)   # oracle index of u
     hits = 0
     for g in range(G):
         o_idx, *_ = oracle.search(enc, q_host[u * G + g], signs, k, p)
@@ -82,3 +88,50 @@ def test_batched_64k_full_size():
 
 def test_million_offload_full_size():
     _run("million_offload", sample_units=[3], sample_heads=[0, 2])
+
+
+def test_llama3_8b_128k_full_size_prior_levels():
+    _run("llama3_8b_128k", sample_units=[0, 5], table=oracle.ratio_levels())
+
+
+def test_levels_against_exact_inner_products():
+    """Uniform levels against the rotation prior's levels at the llama3_8b_128k size, measured
+    against exact inner products (fp32, torch on the device):
+      - recall of the top-k against the exact top-k over all keys (bounded by the vote's
+        pruning, which the levels do not touch);
+      - recall against the exact top-k among each head's candidates (the rerank's own
+        accuracy, which the levels decide);
+      - the estimator's relative RMS error ||q|| S - <k, q> over the candidates.
+    The figures are printed for the record; the prior's levels must estimate more accurately
+    and rank candidates at least as well (within sampling noise)."""
+    sp = workload.spec("llama3_8b_128k")
+    d = workload.generate_torch(sp, DEV)
+    signs = d["signs"].numpy()
+    units, G, n, k = sp.batch * sp.num_kv_heads, sp.group, sp.n, sp.k
+    keys = d["keys"].reshape(units, n, 128).float()
+    q = d["queries"].reshape(units, G, 128).float()
+    dots = torch.einsum("ugd,und->ugn", q, keys).reshape(units * G, n)
+    exact = torch.topk(dots, k, dim=-1).indices.cpu().numpy()
+    qnorm = q.reshape(units * G, 128).norm(dim=-1)
+    out = {}
+    for levels in ("uniform", "prior"):
+        cfg = pk.config(batch=sp.batch, num_kv_heads=sp.num_kv_heads, group=G, capacity=n,
+                        dtype=sp.dtype, rho=sp.rho, cand_bp=sp.cand_bp, levels=levels)
+        ix = pk.build_index(cfg, signs, d["keys"])
+        idx, _ = ix.search(d["queries"], k)
+        got = idx.cpu().numpy()
+        _, _, cand, S = ix.export_search()
+        ct = torch.from_numpy(cand.astype(np.int64)).to(DEV)
+        cd = torch.gather(dots, 1, ct)                              # exact <k, q> of candidates
+        est = qnorm[:, None] * torch.from_numpy(S).to(DEV)
+        err = float(torch.sqrt(((est - cd) ** 2).mean() / (cd ** 2).mean()))
+        inner = torch.gather(ct, 1, torch.topk(cd, k, dim=-1).indices).cpu().numpy()
+        H = units * G
+        rec = np.mean([len(set(got[h].tolist()) & set(exact[h].tolist())) / k for h in range(H)])
+        rrec = np.mean([len(set(got[h].tolist()) & set(inner[h].tolist())) / k for h in range(H)])
+        out[levels] = {"recall": float(rec), "rerank_recall": float(rrec), "est_rel_rms": err}
+        ix.destroy()
+    print("levels vs exact inner products:", out)
+    assert out["prior"]["est_rel_rms"] < out["uniform"]["est_rel_rms"], out
+    assert out["prior"]["rerank_recall"] > out["uniform"]["rerank_recall"] - 0.002, out
+    assert abs(out["prior"]["recall"] - out["uniform"]["recall"]) < 0.01, out

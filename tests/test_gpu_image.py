@@ -51,7 +51,7 @@ def test_export_import_round_trip(name, n, extra):
     # exactly the appended keys
     img2 = b.export_image()
     assert img2.nbytes == img.nbytes + sp.batch * sp.num_kv_heads * extra * 144
-    assert bytes(img2[:72]) == bytes(img[:72])
+    assert bytes(img2[:104]) == bytes(img[:104])
 
 
 def test_import_capacity_rules():

@@ -18,21 +18,26 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def _cfg(batch, hkv, G, cap, dtype="f32", rho=4, w1=2, wr=1, bp=500):
+def _cfg(batch, hkv, G, cap, dtype="f32", rho=4, w1=2, wr=1, bp=500, table=None):
+    if table is None:
+        return pk.config(batch=batch, num_kv_heads=hkv, group=G, capacity=cap, dtype=dtype,
+                         rho=rho, w_rank1=w1, w_rest=wr, cand_bp=bp)
     return pk.config(batch=batch, num_kv_heads=hkv, group=G, capacity=cap, dtype=dtype, rho=rho,
-                     w_rank1=w1, w_rest=wr, cand_bp=bp)
+                     w_rank1=w1, w_rest=wr, cand_bp=bp, levels="table", level_table=table)
 
 
 def _t(a):
     return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
 
 
-def _compare_rotated(batch, hkv, G, n, k, keys, qs, signs, rho=4, w1=2, wr=1, bp=500, cap=None):
-    """Build + search from the oracle's rotated inputs; compare every stage bit for bit."""
+def _compare_rotated(batch, hkv, G, n, k, keys, qs, signs, rho=4, w1=2, wr=1, bp=500, cap=None,
+                     table=None):
+    """Build + search from the oracle's rotated inputs; compare every stage bit for bit
+    (table: code both sides with these magnitude levels)."""
     units = batch * hkv
     y, kn = rotate_all(keys.reshape(units, n, 128), signs)
     qt, qn = rotate_all(qs.reshape(units * G, 128), signs)
-    cfg = _cfg(batch, hkv, G, cap or n, rho=rho, w1=w1, wr=wr, bp=bp)
+    cfg = _cfg(batch, hkv, G, cap or n, rho=rho, w1=w1, wr=wr, bp=bp, table=table)
     ix = pk.build_index_rotated(cfg, signs, _t(y), _t(kn))
     idx, est = ix.search_rotated(_t(qt), _t(qn), k)
     torch.cuda.synchronize()
@@ -42,7 +47,7 @@ def _compare_rotated(batch, hkv, G, n, k, keys, qs, signs, rho=4, w1=2, wr=1, bp
     p = oracle.SearchParams(m=8, rho=rho, w_rank1=w1, w_rest=wr, cand_bp=bp)
     for u in range(units):
         enc, heads = oracle_unit_from_rotated(y[u], kn[u], qt[u * G:(u + 1) * G],
-                                              qn[u * G:(u + 1) * G], k, p)
+                                              qn[u * G:(u + 1) * G], k, p, table=table)
         np.testing.assert_array_equal(gids[u], enc.ids)
         np.testing.assert_array_equal(gcodes[u], enc.codes)
         np.testing.assert_array_equal(gfac[u].view(np.uint32), enc.factor.view(np.uint32))
@@ -91,6 +96,39 @@ def test_stages_bit_exact(batch, hkv, G, n, k, bp):
                        planted=min(32, max(1, n // (4 * G))), seed=n)
     w = workload.generate(sp)
     _compare_rotated(batch, hkv, G, n, k, w.keys, w.queries, w.signs, bp=bp)
+
+
+@pytest.mark.parametrize("batch,hkv,G,n,k,bp", [
+    (1, 1, 1, 4096, 64, 1000),
+    (1, 2, 4, 20000, 128, 500),
+    (2, 1, 5, 9000, 100, 500),
+    (1, 1, 2, 70000, 3000, 10000),
+])
+def test_table_levels_stages_bit_exact(batch, hkv, G, n, k, bp):
+    """Codes from the rotation prior's levels (the oracle's table, given to both sides):
+    every stage bit for bit, as with uniform levels."""
+    sp = workload.spec("tiny", batch=batch, num_kv_heads=hkv, group=G, n=n, dtype="f32",
+                       planted=min(32, max(1, n // (4 * G))), seed=n + 1)
+    w = workload.generate(sp)
+    _compare_rotated(batch, hkv, G, n, k, w.keys, w.queries, w.signs, bp=bp,
+                     table=oracle.ratio_levels())
+
+
+def test_table_levels_adversarial_and_zero_level():
+    """Table coding of zero keys and subspaces, -0, duplicates, and a table whose lowest level
+    is 0 (the two zero-magnitude nibbles then decode to +0 and -0)."""
+    rng = np.random.default_rng(15)
+    n, G = 3000, 4
+    keys = rng.standard_normal((n, 128)).astype(np.float32)
+    qs = rng.standard_normal((G, 128)).astype(np.float32)
+    keys[0:10] = 0.0
+    keys[10:40, 0:8] = 0.0
+    keys[40:60, 1::4] = -0.0
+    keys[100:300] = keys[99]
+    keys[500:520] = qs[0] * 2.0
+    for table in (oracle.ratio_levels(), np.array([0.0, 0.1, 0.2, 0.35, 0.5, 0.65, 0.8, 1.0],
+                                                   np.float32)):
+        _compare_rotated(1, 1, G, n, 300, keys, qs, random_signs(19), bp=1000, table=table)
 
 
 @pytest.mark.parametrize("rho,w1,wr", [(1, 2, 1), (16, 2, 1), (256, 2, 1), (4, 3, 0), (4, 1, 1)])
