@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cache", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--levels", choices=["uniform", "prior"], default="uniform",
+                    help="magnitude levels of the RSQ codes (uniform, or the rotation prior's)")
     return ap.parse_args()
 
 
@@ -441,7 +443,7 @@ def run_drift(args, ws, rank, local):
     bf = lambda a: torch.from_numpy(workload.bf16_bits(a)).view(torch.bfloat16).to(dev)
     pre, app, qs = bf(w.prefill[None]), bf(w.appended), bf(w.queries)
     cfg = pk.config(batch=1, num_kv_heads=H, group=1, capacity=n0 + T, dtype=sp.dtype,
-                    rho=sp.rho, cand_bp=sp.cand_bp)
+                    rho=sp.rho, cand_bp=sp.cand_bp, levels=args.levels)
     ix = pk.build_index(cfg, w.signs, pre)
     idx = torch.empty((H, k), dtype=torch.int32, device=dev)
     est = torch.empty((H, k), dtype=torch.float32, device=dev)
@@ -501,6 +503,7 @@ def run_drift(args, ws, rank, local):
             "config": {"workload": sp.name, "kv_heads": H, "q_heads_per_kv": 1, "d": sp.d,
                        "n_prefill": n0, "decode_steps": T, "k": k, "B": sp.B, "m": sp.m,
                        "rho": sp.rho, "cand_bp": sp.cand_bp, "key_dtype": sp.dtype,
+                       "levels": args.levels,
                        "step": "append one key per KV head + one search",
                        "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"},
             "decode_step": {"append_ms": app_ms, "search_ms": srch_ms},
@@ -542,7 +545,7 @@ def main():
     keys, vals, qs = data["keys"], data["values"], data["queries"]
     cfg = pk.config(batch=sp.batch, num_kv_heads=sp.num_kv_heads, group=sp.group,
                     capacity=sp.n + APPEND_SLACK, dtype=sp.dtype, rho=sp.rho,
-                    cand_bp=sp.cand_bp)
+                    cand_bp=sp.cand_bp, levels=args.levels)
     ix = pk.build_index(cfg, data["signs"], keys, n=sp.n)
     H = sp.batch * sp.num_q_heads
     k = sp.k
@@ -710,6 +713,7 @@ def main():
                        "kv_heads": sp.num_kv_heads, "d": sp.d, "n": sp.n, "k": k,
                        "candidates": C, "B": sp.B, "m": sp.m, "rho": sp.rho,
                        "key_dtype": sp.dtype, "kv_in": "pinned host" if kv_host else "HBM",
+                       "levels": args.levels,
                        "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"},
             "stage_ms": stage_avg,
             "host_enqueue_us_per_search": host_us,
