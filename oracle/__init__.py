@@ -16,12 +16,13 @@ Sources: "Technical Summary: ParisKV" (gist.science/paper/2602.07721), Methodolo
 System-Level Innovations; "ParisKV: Fast and Drift-Robust KV-Cache Retrieval for
 Long-Context LLMs" (ICML 2026 poster abstract).
 
-Parity status: every function here is pinned by tests in ``tests/test_oracle_pins.py``
-except the two readings the pages leave open and that no independent source fixes: the
-exact definition of the calibration weight w_{i,b} and the magnitude levels (the pages
-say "Beta priors"; the uniform levels used here are the stated reading). For those two the
-oracle is pinned only to its stated definitions and to the invariants they imply
-(parity unpinned against the pages).
+Parity status: every function here is pinned by tests in ``tests/test_oracle_pins.py``.
+Two readings the pages leave open are pinned only to their stated definitions and to the
+invariants and laws they imply, not to values the pages print (parity unpinned against the
+pages for these two): the exact definition of the calibration weight w_{i,b}, and the rule
+that turns the pages' "Beta priors" into magnitude levels (uniform levels, the default, and
+the prior-derived table levels of ``ratio_levels``; the law behind the latter is pinned
+against rotated keys and its Lloyd-Max conditions by independent quadrature).
 """
 from __future__ import annotations
 
