@@ -39,8 +39,11 @@ def _data(seed, hkv, G, total, dtype):
 
 
 def _run(dtype, hkv, G, n_sink, n_local, n_buffer, k, n0, steps, host_prefill, out_f32,
-         check_every, seed):
+         check_every, seed, batch=1):
     total = n0 + steps
+    if batch > 1:                      # sequences of a batch are further KV heads here
+        return _run_batched(dtype, batch, hkv, G, n_sink, n_local, n_buffer, k, n0, steps,
+                            seed)
     K, V, q = _data(seed, hkv, G, total, dtype)
     signs = random_signs(seed)
     cfg = pk.config(batch=1, num_kv_heads=hkv, group=G, capacity=1, dtype=dtype, rho=4,
@@ -111,6 +114,45 @@ def _run(dtype, hkv, G, n_sink, n_local, n_buffer, k, n0, steps, host_prefill, o
     return promotions
 
 
+def _run_batched(dtype, batch, hkv, G, n_sink, n_local, n_buffer, k, n0, steps, seed):
+    """batch > 1: the attention output against the oracle at every promotion and at the last
+    step, every sequence and head (region sizes are shared by all sequences)."""
+    total = n0 + steps
+    units = batch * hkv
+    K, V, q = _data(seed, units, G, total, dtype)            # [1, units, total, 128]
+    signs = random_signs(seed)
+    cfg = pk.config(batch=batch, num_kv_heads=hkv, group=G, capacity=1, dtype=dtype, rho=4,
+                    cand_bp=1000)
+    cache = pk.Cache(cfg, signs, n_sink, n_local, n_buffer, k, retrieval_capacity=total)
+    Kd, Vd = _conv(K, dtype).to(DEV), _conv(V, dtype).to(DEV)
+    qd = _conv(q, dtype).to(DEV)                              # [total, units * G, 128]
+    cache.prefill(Kd.view(batch, hkv, total, 128), Vd.view(batch, hkv, total, 128), n=n0)
+    model = oracle.CacheRegions(n_sink, n_local, n_buffer)
+    model.prefill(n0)
+    checked = 0
+    for t in range(steps):
+        tok = n0 + t
+        before = len(model.retrieval)
+        out, topk = cache.step(qd[tok].view(batch, hkv * G, 128),
+                               Kd[0, :, tok].contiguous().view(batch, hkv, 128),
+                               Vd[0, :, tok].contiguous().view(batch, hkv, 128), SCALE,
+                               out_dtype=torch.float32, want_topk=True)
+        model.append()
+        if len(model.retrieval) == before and t != steps - 1:
+            continue
+        checked += 1
+        got = out.cpu().numpy().reshape(units * G, 128)
+        gtop = topk.cpu().numpy()
+        k_eff = min(k, len(model.retrieval))
+        for h in range(units * G):
+            rows = gtop[h, :k_eff]
+            toks = np.asarray(model.dense() + [model.retrieval[r] for r in rows], np.int32)
+            ref = oracle.attend(q[tok, h], K[0, h // G], V[0, h // G], toks, SCALE)
+            assert np.all(np.abs(got[h] - ref) <= 2e-3), (t, h)
+    cache.destroy()
+    return checked
+
+
 @pytest.mark.parametrize("dtype,hkv,G,n_sink,n_local,n_buffer,k,n0,steps,host,out_f32", [
     ("bf16", 2, 4, 4, 128, 32, 64, 2000, 200, False, True),
     ("f32", 1, 2, 0, 64, 64, 256, 100, 150, True, False),
@@ -121,6 +163,12 @@ def test_cache_decode_matches_oracle(dtype, hkv, G, n_sink, n_local, n_buffer, k
     promotions = _run(dtype, hkv, G, n_sink, n_local, n_buffer, k, n0, steps, host, out_f32,
                       check_every=17, seed=n0 + steps)
     assert promotions >= 2
+
+
+def test_cache_batched_group_8():
+    """Two sequences of two KV heads with 8 query heads each (the widest group of the
+    tensor-core dense pass)."""
+    assert _run("bf16", 2, 8, 4, 64, 16, 32, 500, 70, False, True, 0, seed=9, batch=2) >= 3
 
 
 def test_cache_capacity_and_errors():
