@@ -79,6 +79,8 @@ def _load():
             lib.orc_rerank.argtypes = [i32, i32, P, P, P, P, i64, P, P]
             lib.orc_encode_rotated_table.argtypes = [i32, i32, P, P, P, i64, P, P, P, P]
             lib.orc_rerank_table.argtypes = [i32, i32, P, P, P, P, P, i64, P, P]
+            lib.orc_learned_ids.argtypes = [i32, i32, P, P, i64, P]
+            lib.orc_learned_lut.argtypes = [i32, i32, i32, i32, i32, P, P, P]
             lib.orc_topk.argtypes = [P, P, i64, i64, P, P]
             lib.orc_attend.argtypes = [i32, P, P, P, P, i64, ctypes.c_double, P]
             _lib = lib
@@ -244,6 +246,7 @@ class SearchParams:
     w_rank1: int = 2
     w_rest: int = 1
     cand_bp: int = 500
+    centroids: Optional[np.ndarray] = None   # learned centroids [B, 256, m] (R25), or analytic
 
 
 def build_unit(keys: np.ndarray, signs: np.ndarray, m: int,
@@ -254,9 +257,12 @@ def build_unit(keys: np.ndarray, signs: np.ndarray, m: int,
 
 
 def search_rotated(enc: Encoded, qt: np.ndarray, qnorm: float, k: int, p: SearchParams):
-    """One query head from its rotated query: returns (topk idx, S, est, candidates, scores)."""
+    """One query head from its rotated query: returns (topk idx, S, est, candidates, scores).
+    With p.centroids the coarse stage uses the learned centroids (enc.ids must be learned
+    ids, from learned_ids)."""
     n = enc.ids.shape[0]
-    lut = query_lut(qt, p.m, p.rho, p.w_rank1, p.w_rest)
+    lut = (query_lut(qt, p.m, p.rho, p.w_rank1, p.w_rest) if p.centroids is None else
+           learned_lut(qt, p.centroids, p.m, p.rho, p.w_rank1, p.w_rest))
     sc = vote(enc.ids, lut, p.m)
     C = candidate_count(n, k, p.cand_bp)
     cand = select_candidates(sc, C)
@@ -379,3 +385,59 @@ def ratio_levels(m: int = 8, nx: int = 16384, iters: int = 2000) -> np.ndarray:
         s1[7] += pm
         lv = s1 / s0
     return lv.astype(np.float32)
+
+
+# ---------------------------------------------------------------------------------------
+# Learned centroids: the comparator of the drift claim (reading R25; see pariskv_oracle.c)
+# ---------------------------------------------------------------------------------------
+def learned_ids(y: np.ndarray, cent: np.ndarray, m: int = 8) -> np.ndarray:
+    """ids [n, B]: argmax_c <y_b, mu_c> per subspace (fp32 chains, ties to the lower c)."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    cent = np.ascontiguousarray(cent, dtype=np.float32)
+    n, d = y.shape
+    ids = np.empty((n, d // m), np.uint8)
+    _load().orc_learned_ids(d, m, _p(cent), _p(y), n, _p(ids))
+    return ids
+
+
+def learned_lut(qt: np.ndarray, cent: np.ndarray, m: int = 8, rho: int = 4, w_rank1: int = 2,
+                w_rest: int = 1) -> np.ndarray:
+    """Vote table [B, 256] from the rho centroids with the largest <q~_b, mu_c>."""
+    qt = np.ascontiguousarray(qt, dtype=np.float32)
+    cent = np.ascontiguousarray(cent, dtype=np.float32)
+    lut = np.empty((qt.shape[0] // m, 1 << m), np.uint8)
+    _load().orc_learned_lut(qt.shape[0], m, rho, w_rank1, w_rest, _p(cent), _p(qt), _p(lut))
+    return lut
+
+
+def train_centroids(y: np.ndarray, iters: int, m: int = 8) -> np.ndarray:
+    """Spherical k-means (Lloyd) per subspace on the prefill keys' rotated directions
+    (reading R25): 256 unit-norm centroids; start from the directions of keys
+    floor(c n / 256); each iteration assigns every key by learned_ids and replaces each
+    centroid by the normalised sum (fp64) of its keys' unit directions (a centroid with no
+    key keeps its value). Returns fp32 [B, 256, m]."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    n, d = y.shape
+    B = d // m
+    yb = y.reshape(n, B, m).astype(np.float64)
+    nrm = np.linalg.norm(yb, axis=2, keepdims=True)
+    u = np.divide(yb, nrm, out=np.zeros_like(yb), where=nrm > 0)
+    cent = u[(np.arange(256) * n) // 256].transpose(1, 0, 2).astype(np.float32)   # [B, 256, m]
+    for _ in range(iters):
+        ids = learned_ids(y, cent, m)
+        new = cent.astype(np.float64).copy()
+        for b in range(B):
+            sums = np.zeros((256, m))
+            np.add.at(sums, ids[:, b], u[:, b])
+            norm = np.linalg.norm(sums, axis=1)
+            ok = norm > 0
+            new[b, ok] = sums[ok] / norm[ok, None]
+        cent = new.astype(np.float32)
+    return np.ascontiguousarray(cent)
+
+
+def sign_centroids(m: int = 8) -> np.ndarray:
+    """The analytic centroids as a table [B, 256, m]: c's sign pattern / sqrt(m)."""
+    c = np.arange(1 << m)
+    pat = np.where((c[:, None] >> np.arange(m)) & 1, -1.0, 1.0) / np.sqrt(m)
+    return np.ascontiguousarray(np.broadcast_to(pat, (128 // m, 1 << m, m)).astype(np.float32))

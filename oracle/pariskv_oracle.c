@@ -300,6 +300,78 @@ void orc_query_lut(int32_t d, int32_t m, int32_t rho, int32_t w_rank1, int32_t w
     free(e);
 }
 
+/* ------------------------------------------------------------------------------------
+ * Learned centroids (the comparator of the drift claim). [TS] Problem Statement 2
+ * ("Decoding Drift": centroids learned by clustering prefill keys go stale as decoding keys
+ * accumulate) and Key Contributions 1 (analytic centroids remove the need for them).
+ * [R25] The comparator replaces only the coarse stage's centroids: per (unit, subspace) 256
+ *       centroids mu_c in R^8 learned from the prefill keys' rotated subspace vectors.
+ *       A key's id is argmax_c <y_b, mu_c> (fp32 FMA chain over j ascending from 0.0f;
+ *       ties to the lower c); a query's top-rho are the rho largest <q~_b, mu_c> (same
+ *       chain; ties to the lower c), with the tiered weights of [R8]. Everything else (codes,
+ *       factors, vote, candidates, rerank, top-k) is unchanged.
+ * cent: [B][256][m] for one unit.
+ * ------------------------------------------------------------------------------------ */
+static float dot_chain(const float* a, const float* b, int32_t m)
+{
+    float s = 0.0f;
+    for (int32_t j = 0; j < m; ++j) s = fmaf(a[j], b[j], s);
+    return s;
+}
+
+void orc_learned_ids(int32_t d, int32_t m, const float* cent, const float* y, int64_t n,
+                     uint8_t* ids)
+{
+    const int32_t B = d / m, nc = 1 << m;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; ++r) {
+        for (int32_t b = 0; b < B; ++b) {
+            const float* yb = y + r * d + (int64_t)b * m;
+            const float* cb = cent + (int64_t)b * nc * m;
+            float best = dot_chain(cb, yb, m);
+            int32_t arg = 0;
+            for (int32_t c = 1; c < nc; ++c) {
+                const float v = dot_chain(cb + (int64_t)c * m, yb, m);
+                if (v > best) { best = v; arg = c; }
+            }
+            ids[r * B + b] = (uint8_t)arg;
+        }
+    }
+}
+
+typedef struct {
+    float s;
+    int32_t id;
+} sim_entry;
+
+static int cmp_sim(const void* a, const void* b)
+{
+    const sim_entry* x = (const sim_entry*)a;
+    const sim_entry* y = (const sim_entry*)b;
+    if (x->s != y->s) return (x->s < y->s) ? 1 : -1;
+    return (x->id > y->id) - (x->id < y->id);
+}
+
+void orc_learned_lut(int32_t d, int32_t m, int32_t rho, int32_t w_rank1, int32_t w_rest,
+                     const float* cent, const float* qt, uint8_t* lut)
+{
+    const int32_t B = d / m, nc = 1 << m;
+    sim_entry* e = (sim_entry*)malloc(sizeof(sim_entry) * (size_t)nc);
+    for (int32_t b = 0; b < B; ++b) {
+        const float* cb = cent + (int64_t)b * nc * m;
+        for (int32_t c = 0; c < nc; ++c) {
+            e[c].s = dot_chain(cb + (int64_t)c * m, qt + (int64_t)b * m, m);
+            e[c].id = c;
+        }
+        qsort(e, (size_t)nc, sizeof(sim_entry), cmp_sim);
+        uint8_t* lb = lut + (int64_t)b * nc;
+        for (int32_t c = 0; c < nc; ++c) lb[c] = 0;
+        for (int32_t r = 0; r < rho && r < nc; ++r)
+            lb[e[r].id] = (uint8_t)(r == 0 ? w_rank1 : w_rest);
+    }
+    free(e);
+}
+
 /* Collision vote. [TS] "Coarse Candidate Generation": votes are summed over subspaces into
  * an integer coarse score: score_i = sum_b lut[b][id_{i,b}]. */
 void orc_vote(int32_t B, int32_t m, const uint8_t* ids, int64_t n, const uint8_t* lut,

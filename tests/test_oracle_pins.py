@@ -509,3 +509,76 @@ def test_ratio_levels_quantise_directions_better_than_uniform():
         return float(np.mean(1 - cos))
     uni, tab = loss(oracle.encode_rotated(y, kn, M)), loss(oracle.encode_rotated(y, kn, M, table=lv))
     assert tab < 0.85 * uni, (tab, uni)
+
+
+# ----------------------------------------------------------------------------- learned centroids
+def test_learned_path_with_sign_centroids_is_the_analytic_path():
+    """With the 256 sign patterns / sqrt(m) as 'learned' centroids the comparator's ids, vote
+    tables and whole search equal the analytic ones (zero coordinates included: both break
+    ties toward the lower id)."""
+    rng = np.random.default_rng(31)
+    y = rng.standard_normal((3000, D)).astype(np.float32)
+    y[:50, ::5] = 0.0
+    sc = oracle.sign_centroids(M)
+    enc = oracle.encode_rotated(y, np.ones(3000, np.float32), M)
+    np.testing.assert_array_equal(oracle.learned_ids(y, sc, M), enc.ids)
+    for s in range(5):
+        qt = rng.standard_normal(D).astype(np.float32)
+        for rho in (1, 4, 16):
+            np.testing.assert_array_equal(oracle.learned_lut(qt, sc, M, rho),
+                                          oracle.query_lut(qt, M, rho))
+    qt = rng.standard_normal(D).astype(np.float32)
+    a = oracle.search_rotated(enc, qt, 1.0, 64, oracle.SearchParams(m=M))
+    b = oracle.search_rotated(enc, qt, 1.0, 64, oracle.SearchParams(m=M, centroids=sc))
+    for x, z in zip(a, b):
+        np.testing.assert_array_equal(x, z)
+
+
+def test_learned_ids_and_lut_brute_force():
+    """argmax / top-rho of fp64 inner products with arbitrary centroids (entries within 1e-6
+    of a tie excluded)."""
+    rng = np.random.default_rng(32)
+    cent = rng.standard_normal((B, 256, M)).astype(np.float32)
+    y = rng.standard_normal((500, D)).astype(np.float32)
+    ids = oracle.learned_ids(y, cent, M)
+    dots = np.einsum("nbj,bcj->nbc", y.reshape(500, B, M).astype(np.float64),
+                     cent.astype(np.float64))
+    srt = np.sort(dots, axis=2)
+    clear = srt[..., -1] - srt[..., -2] > 1e-6
+    assert clear.mean() > 0.99
+    np.testing.assert_array_equal(ids[clear], dots.argmax(axis=2)[clear])
+    qt = rng.standard_normal(D).astype(np.float32)
+    lut = oracle.learned_lut(qt, cent, M, rho=4, w_rank1=2, w_rest=1)
+    qd = np.einsum("bj,bcj->bc", qt.reshape(B, M).astype(np.float64), cent.astype(np.float64))
+    for b in range(B):
+        top = np.argsort(-qd[b], kind="stable")[:4]
+        want = np.zeros(256, np.uint8)
+        want[top[0]] = 2
+        want[top[1:]] = 1
+        np.testing.assert_array_equal(lut[b], want)
+
+
+def test_train_centroids_recovers_directions_and_improves_fit():
+    """Keys drawn as 4 copies each of 256 distinct directions per subspace (key i on
+    direction i // 4) are recovered exactly: the start picks one key of each direction and
+    every key then joins its own; on Gaussian keys the mean cosine to the assigned centroid
+    never decreases over iterations, and centroids stay unit vectors."""
+    rng = np.random.default_rng(33)
+    dirs = rng.standard_normal((B, 256, M))
+    dirs /= np.linalg.norm(dirs, axis=2, keepdims=True)
+    scale = rng.uniform(0.5, 2.0, (1024, B, 1))
+    y = (dirs[:, np.arange(1024) // 4].transpose(1, 0, 2) * scale).reshape(1024, D)
+    cent = oracle.train_centroids(y.astype(np.float32), 3, M)
+    np.testing.assert_allclose(cent, dirs.astype(np.float32), atol=1e-6)
+    g = rng.standard_normal((4000, D)).astype(np.float32)
+    u = g.reshape(4000, B, M) / np.linalg.norm(g.reshape(4000, B, M), axis=2, keepdims=True)
+    prev = -1.0
+    for it in range(0, 6):
+        c = oracle.train_centroids(g, it, M)
+        ids = oracle.learned_ids(g, c, M)
+        fit = float(np.mean(np.take_along_axis(
+            np.einsum("nbj,bcj->nbc", u, c.astype(np.float64)), ids[..., None].astype(np.int64),
+            axis=2)))
+        assert fit >= prev - 1e-12, (it, fit, prev)
+        prev = fit
+        np.testing.assert_allclose(np.linalg.norm(c, axis=2), 1.0, atol=1e-6)
