@@ -31,6 +31,7 @@ sys.path.insert(0, ROOT)
 
 L2_FLUSH_BYTES = 256 << 20
 APPEND_SLACK = 64
+LEARNED_ITERS = 10          # spherical k-means iterations of the learned-centroid comparator
 
 
 def parse():
@@ -45,6 +46,9 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cache", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--centroids", choices=["analytic", "learned"], default="analytic",
+                    help="drift_32k: coarse centroids (analytic, or learned from the prefill "
+                         "by spherical k-means: the comparator of the drift claim)")
     ap.add_argument("--levels", choices=["uniform", "prior"], default="uniform",
                     help="magnitude levels of the RSQ codes (uniform, or the rotation prior's)")
     return ap.parse_args()
@@ -444,7 +448,17 @@ def run_drift(args, ws, rank, local):
     pre, app, qs = bf(w.prefill[None]), bf(w.appended), bf(w.queries)
     cfg = pk.config(batch=1, num_kv_heads=H, group=1, capacity=n0 + T, dtype=sp.dtype,
                     rho=sp.rho, cand_bp=sp.cand_bp, levels=args.levels)
-    ix = pk.build_index(cfg, w.signs, pre)
+    train_ms = None
+    if args.centroids == "learned":
+        # the comparator: centroids learned from the prefill keys, then frozen
+        t0 = time.perf_counter()
+        cent = pk.train_centroids(cfg, w.signs, pre, LEARNED_ITERS)
+        train_ms = (time.perf_counter() - t0) * 1e3
+        ix = pk.build_index(cfg, w.signs, pre, n=0)
+        ix.set_centroids(cent)
+        ix.append(pre)
+    else:
+        ix = pk.build_index(cfg, w.signs, pre)
     idx = torch.empty((H, k), dtype=torch.int32, device=dev)
     est = torch.empty((H, k), dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -455,7 +469,7 @@ def run_drift(args, ws, rank, local):
     torch.cuda.synchronize()
 
     steps = T - W
-    sample = set(range(W, T, 4096)) | {T - 1}
+    sample = set(range(W, T, 2048)) | {T - 1}
     kept = {}
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     clocks = ClockSampler(local)
@@ -503,11 +517,13 @@ def run_drift(args, ws, rank, local):
             "config": {"workload": sp.name, "kv_heads": H, "q_heads_per_kv": 1, "d": sp.d,
                        "n_prefill": n0, "decode_steps": T, "k": k, "B": sp.B, "m": sp.m,
                        "rho": sp.rho, "cand_bp": sp.cand_bp, "key_dtype": sp.dtype,
-                       "levels": args.levels,
+                       "levels": args.levels, "centroids": args.centroids,
                        "step": "append one key per KV head + one search",
                        "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"},
             "decode_step": {"append_ms": app_ms, "search_ms": srch_ms},
             "recall_vs_exact_topk": rec,
+            "recall_mean": float(np.mean(list(rec.values()))),
+            "centroid_training_ms": train_ms,
             "roofline": None,
             "gpu_launches": launches,
             "clocks": clk,

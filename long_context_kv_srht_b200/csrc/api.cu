@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "internal.hpp"
 #include "pariskv_dense.h"
+#include "pariskv_learned.h"
 #include "pariskv_debug.h"
 
 using namespace pkv;
@@ -125,6 +126,7 @@ bool alloc_fault_injected() { return fault_alloc(); }
 pariskv_status check_device_pointer(const void* p, size_t align, const char* name) {
     return check_dev_ptr(p, align, name);
 }
+pariskv_status validate_config(const pariskv_config* cfg) { return check_config(cfg); }
 void set_last_launches(int32_t n) { g_launches = n; }
 int32_t last_launches() { return g_launches; }
 }  // namespace pkv
@@ -146,6 +148,7 @@ void free_index(pariskv_index* ix) {
     dfree(ix->signs); dfree(ix->ids); dfree(ix->rec); dfree(ix->lut); dfree(ix->qt);
     dfree(ix->qnorm); dfree(ix->scores); dfree(ix->hist); dfree(ix->thr); dfree(ix->cbase);
     dfree(ix->cand); dfree(ix->S); dfree(ix->shist); dfree(ix->status); dfree(ix->lvt);
+    dfree(ix->cent);
     for (auto& e : ix->ev)
         if (e) cudaEventDestroy(e);
     delete ix;
@@ -569,6 +572,7 @@ pariskv_status pariskv_export_bytes(const pariskv_index* ix, size_t* bytes) {
 pariskv_status pariskv_export(pariskv_index* ix, void* buf, size_t bytes, void* stream) {
     pariskv_status s = check_index(ix);
     if (s != PARISKV_OK) return s;
+    if (ix->cent) return fail(PARISKV_EINVAL, "an index with learned centroids has no image");
     size_t need = 0;
     pariskv_export_bytes(ix, &need);
     if (!buf) return fail(PARISKV_EINVAL, "buf is NULL");
@@ -653,6 +657,20 @@ pariskv_status pariskv_import(const void* buf, size_t bytes, int64_t capacity, v
     }
     ix->n = h.n;
     *out = ix;
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_set_centroids(pariskv_index* ix, const float* centroids, void* stream) {
+    pariskv_status s = check_index(ix);
+    if (s != PARISKV_OK) return s;
+    if (ix->n != 0) return fail(PARISKV_EINVAL, "centroids can only be set on an empty index");
+    if ((s = check_dev_ptr(centroids, 16, "centroids")) != PARISKV_OK) return s;
+    const size_t count = static_cast<size_t>(ix->units) * NB * NC * 8;
+    if (!ix->cent && !dalloc(&ix->cent, count))
+        return fail(PARISKV_ENOMEM, "centroid table");
+    cudaError_t e = cudaMemcpyAsync(ix->cent, centroids, count * sizeof(float),
+                                    cudaMemcpyDefault, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "centroid copy");
     return PARISKV_OK;
 }
 
@@ -836,8 +854,13 @@ pariskv_status pariskv_debug_export_index(pariskv_index* ix, uint8_t* ids, uint8
                     for (int j = 0; j < M; ++j) {
                         const int u = static_cast<int>((w >> (4 * j)) & 15u);
                         const int mag = u >= 8 ? u - 8 : (table ? 7 - u : 8 - u);
+                        // the nibble carries the sign except for a zero uniform level, whose
+                        // sign is the id bit (not recorded when ids come from learned
+                        // centroids: reported as +)
+                        const uint32_t neg = (table || u != 8) ? (u < 8 ? 1u : 0u)
+                                             : (ix->cent ? 0u : (id >> j) & 1u);
                         codes[o * D + b * M + j] =
-                            static_cast<uint8_t>((((id >> j) & 1u) << 3) | static_cast<uint32_t>(mag));
+                            static_cast<uint8_t>((neg << 3) | static_cast<uint32_t>(mag));
                     }
                 if (factors) memcpy(&factors[o * NB + b], &hrec[at + 16], 4);
             }

@@ -113,12 +113,38 @@ __device__ __forceinline__ void encode_subspace_table(const float w[8], float kn
     factor = (dot == 0.0f) ? 0.0f : __fdiv_rn(num, dot);
 }
 
+// Learned centroids (the comparator of the drift claim): the id of subspace b is the
+// centroid c of largest <y_b, mu_c> (fp32 FMA chain over the 8 dims, ties to the lower c).
+// Lanes 2b and 2b+1 both hold y_b; they scan centroids 0..127 and 128..255 and combine.
+__device__ __forceinline__ uint32_t learned_id(const float w[8], const float* __restrict__ cb,
+                                               bool odd) {
+    const float* c0 = cb + (odd ? 128 * 8 : 0);
+    float best = -INFINITY;
+    int arg = 0;
+#pragma unroll 4
+    for (int c = 0; c < 128; ++c) {
+        const float4 lo = __ldg(reinterpret_cast<const float4*>(c0 + 8 * c));
+        const float4 hi = __ldg(reinterpret_cast<const float4*>(c0 + 8 * c + 4));
+        float d = 0.0f;
+        d = __fmaf_rn(lo.x, w[0], d); d = __fmaf_rn(lo.y, w[1], d);
+        d = __fmaf_rn(lo.z, w[2], d); d = __fmaf_rn(lo.w, w[3], d);
+        d = __fmaf_rn(hi.x, w[4], d); d = __fmaf_rn(hi.y, w[5], d);
+        d = __fmaf_rn(hi.z, w[6], d); d = __fmaf_rn(hi.w, w[7], d);
+        if (d > best) { best = d; arg = c; }
+    }
+    arg += odd ? 128 : 0;
+    const float ob = __shfl_xor_sync(0xffffffffu, best, 1);
+    const int oa = __shfl_xor_sync(0xffffffffu, arg, 1);
+    if (ob > best || (ob == best && oa < arg)) arg = oa;
+    return static_cast<uint32_t>(arg);
+}
+
 template <typename T, bool ROTATED, bool TABLE>
 __global__ void __launch_bounds__(kEncWarps * 32)
 encode_kernel(const T* __restrict__ src, const float* __restrict__ knorm_in, int64_t ld_tok,
               int64_t t, const float* __restrict__ signs, uint8_t* __restrict__ ids,
               uint8_t* __restrict__ rec, int64_t cap_pad, int64_t pos0,
-              const float* __restrict__ lvt) {
+              const float* __restrict__ lvt, const float* __restrict__ cent) {
     const int lane = threadIdx.x & 31;
     const int64_t r = static_cast<int64_t>(blockIdx.x) * kEncWarps + (threadIdx.x >> 5);
     const int64_t unit = blockIdx.y;
@@ -160,6 +186,8 @@ encode_kernel(const T* __restrict__ src, const float* __restrict__ knorm_in, int
     } else {
         encode_subspace(w, knorm, id, code, f);
     }
+    if (cent)   // learned centroids replace the sign-pattern id (codes unchanged)
+        id = learned_id(w, cent + (unit * NB + (lane >> 1)) * NC * 8, odd);
 
     if (!odd) {
         const int b = lane >> 1;
@@ -198,15 +226,15 @@ static void launch_encode_t(const pariskv_index* ix, const void* keys, const flo
     if (rotated) {
         encode_kernel<float, true, TABLE><<<grid, block, 0, st>>>(
             static_cast<const float*>(keys), knorm, ld_tok, t, ix->signs, ix->ids, ix->rec,
-            ix->cap_pad, pos0, ix->lvt);
+            ix->cap_pad, pos0, ix->lvt, ix->cent);
     } else if (ix->cfg.dtype == PARISKV_BF16) {
         encode_kernel<__nv_bfloat16, false, TABLE><<<grid, block, 0, st>>>(
             static_cast<const __nv_bfloat16*>(keys), nullptr, ld_tok, t, ix->signs, ix->ids,
-            ix->rec, ix->cap_pad, pos0, ix->lvt);
+            ix->rec, ix->cap_pad, pos0, ix->lvt, ix->cent);
     } else {
         encode_kernel<float, false, TABLE><<<grid, block, 0, st>>>(
             static_cast<const float*>(keys), nullptr, ld_tok, t, ix->signs, ix->ids, ix->rec,
-            ix->cap_pad, pos0, ix->lvt);
+            ix->cap_pad, pos0, ix->lvt, ix->cent);
     }
 }
 

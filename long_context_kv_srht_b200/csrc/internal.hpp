@@ -21,6 +21,7 @@ struct pariskv_index {
     int8_t hsigns[128] = {};    // the SRHT signs as given (host copy, for index images)
     float* lvt = nullptr;       // [32] code levels: [0..7] magnitudes, [9..15] thresholds,
                                 //      [16..31] signed level of each code nibble
+    float* cent = nullptr;      // learned centroids [units][16][256][8], or NULL (analytic)
     float* signs = nullptr;     // [128] +-1.0f
     uint8_t* ids = nullptr;     // [units][cap_pad][16] bucket ids, byte-rotated per key
     uint8_t* rec = nullptr;     // [units][cap_pad][128] codes (64 B) + factors (16 x f32)
@@ -108,6 +109,7 @@ pariskv_status fail(pariskv_status s, const char* fmt, ...);
 pariskv_status cuda_fail(cudaError_t e, const char* what);
 bool alloc_fault_injected();   // PARISKV_FAULT=alloc: every device allocation fails
 pariskv_status check_device_pointer(const void* p, size_t align, const char* name);
+pariskv_status validate_config(const pariskv_config* cfg);   // the checks every call makes
 void set_last_launches(int32_t n);   // what pariskv_last_launch_count reports
 int32_t last_launches();
 

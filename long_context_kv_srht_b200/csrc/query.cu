@@ -32,7 +32,8 @@ __global__ void __launch_bounds__(32 * kQWarps)
 query_prep_kernel(const T* __restrict__ q, const float* __restrict__ qt_in,
                   const float* __restrict__ qn_in, const float* __restrict__ signs, int group,
                   int packs, int rho, int w1, int wr, float* __restrict__ qt_out,
-                  float* __restrict__ qn_out, uint8_t* __restrict__ lut8) {
+                  float* __restrict__ qn_out, uint8_t* __restrict__ lut8,
+                  const float* __restrict__ cent) {
     __shared__ float sq[D];
     const int head = blockIdx.x;  // unit * group + g
     const int unit = head / group, g = head % group;
@@ -71,15 +72,29 @@ query_prep_kernel(const T* __restrict__ q, const float* __restrict__ qt_in,
             c1 |= (x < 0.0f ? 1u : 0u) << j;
         }
         unsigned long long key[8];
+        if (cent) {
+            // learned centroids (the drift claim's comparator): rank by <mu_c, q~_b>
+            // (fp32 FMA chain over j ascending) descending, ties to the lower id
+            const float* cb = cent + (static_cast<int64_t>(unit) * NB + b) * NC * 8;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t c = static_cast<uint32_t>(lane + 32 * i);
-            const uint32_t diff = c ^ c1;
-            float pen = 0.0f;
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t c = static_cast<uint32_t>(lane + 32 * i);
+                float sim = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                if ((diff >> j) & 1u) pen = __fadd_rn(pen, a[j]);
-            key[i] = (static_cast<unsigned long long>(__float_as_uint(pen)) << 32) | c;
+                for (int j = 0; j < 8; ++j) sim = __fmaf_rn(cb[c * 8 + j], sq[8 * b + j], sim);
+                key[i] = (static_cast<unsigned long long>(~order_key(sim)) << 32) | c;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t c = static_cast<uint32_t>(lane + 32 * i);
+                const uint32_t diff = c ^ c1;
+                float pen = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    if ((diff >> j) & 1u) pen = __fadd_rn(pen, a[j]);
+                key[i] = (static_cast<unsigned long long>(__float_as_uint(pen)) << 32) | c;
+            }
         }
         uint32_t wgt[8];
 #pragma unroll
@@ -135,16 +150,17 @@ cudaError_t launch_query_prep(const pariskv_index* ix, const void* q, const floa
     if (rotated)
         return launch_pdl(query_prep_kernel<float, true>, heads, 32 * kQWarps, 0, st, nullptr, qt_in,
                           qn_in, ix->signs, c.group, ix->packs, c.rho, c.w_rank1, c.w_rest,
-                          ix->qt, ix->qnorm, lut8);
+                          ix->qt, ix->qnorm, lut8, static_cast<const float*>(ix->cent));
     else if (c.dtype == PARISKV_BF16)
         return launch_pdl(query_prep_kernel<__nv_bfloat16, false>, heads, 32 * kQWarps, 0, st,
                           static_cast<const __nv_bfloat16*>(q), nullptr, nullptr, ix->signs,
                           c.group, ix->packs, c.rho, c.w_rank1, c.w_rest, ix->qt, ix->qnorm,
-                          lut8);
+                          lut8, static_cast<const float*>(ix->cent));
     else
         return launch_pdl(query_prep_kernel<float, false>, heads, 32 * kQWarps, 0, st,
                           static_cast<const float*>(q), nullptr, nullptr, ix->signs, c.group,
-                          ix->packs, c.rho, c.w_rank1, c.w_rest, ix->qt, ix->qnorm, lut8);
+                          ix->packs, c.rho, c.w_rank1, c.w_rest, ix->qt, ix->qnorm, lut8,
+                          static_cast<const float*>(ix->cent));
 }
 
 }  // namespace pkv

@@ -1,5 +1,6 @@
 """Thin ctypes binding over libpariskv.so (the C ABI declared in include/pariskv.h,
-include/pariskv_cache.h, include/pariskv_dense.h and include/pariskv_debug.h).
+include/pariskv_cache.h, include/pariskv_dense.h, include/pariskv_learned.h and
+include/pariskv_debug.h).
 
 Only argument marshalling happens here: tensors become data pointers and strides become the
 library's slab strides; every step of the retrieval path runs in the library's CUDA kernels.
@@ -17,7 +18,8 @@ import numpy as np
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "_lib", "libpariskv.so")
 HEADERS = [os.path.join(os.path.dirname(_PKG), "include", h)
-           for h in ("pariskv.h", "pariskv_cache.h", "pariskv_dense.h", "pariskv_debug.h")]
+           for h in ("pariskv.h", "pariskv_cache.h", "pariskv_dense.h", "pariskv_learned.h",
+                     "pariskv_debug.h")]
 
 OK, EINVAL, ENOMEM, ECUDA, ECAPACITY, ETIMEOUT = range(6)
 F32, BF16 = 0, 1
@@ -76,6 +78,8 @@ _SIGS = {
     "pariskv_dense_attend": (_S, [ctypes.POINTER(Config), _P, _P, _P, _I64, _I64, ctypes.c_float,
                                   _P, _I32, _P]),
     "pariskv_prior_levels": (_S, [ctypes.POINTER(ctypes.c_float)]),
+    "pariskv_train_centroids": (_S, [ctypes.POINTER(Config), _P, _P, _I64, _I64, _I32, _P, _P]),
+    "pariskv_set_centroids": (_S, [_P, _P, _P]),
     "pariskv_sync": (_S, [_P, _P]),
     "pariskv_destroy": (_S, [_P]),
     "pariskv_size": (_I64, [_P]),
@@ -198,6 +202,11 @@ class Index:
     def sync(self, stream=None) -> None:
         _check(lib.pariskv_sync(self.handle, _stream(stream)), "pariskv_sync")
 
+    def set_centroids(self, centroids, stream=None) -> None:
+        """pariskv_set_centroids: learned centroids [units, 16, 256, 8] fp32 (empty index)."""
+        _check(lib.pariskv_set_centroids(self.handle, centroids.data_ptr(), _stream(stream)),
+               "pariskv_set_centroids")
+
     def export_image(self, stream=None) -> np.ndarray:
         """pariskv_export: the index image as a uint8 array (host memory)."""
         nb = ctypes.c_size_t(0)
@@ -306,6 +315,20 @@ def import_index(image, capacity: int = 0, stream=None) -> Index:
     if cfg.levels == LEVELS_PRIOR:              # imported with the levels it was coded with
         cfg.levels = LEVELS_TABLE
     return Index(h.value, cfg)
+
+
+def train_centroids(cfg: Config, signs, keys, iters: int, n: Optional[int] = None, stream=None):
+    """pariskv_train_centroids: spherical k-means centroids [units, 16, 256, 8] (fp32, on the
+    keys' device) from the first n keys of every (sequence, KV head)."""
+    import torch
+    n = keys.shape[-2] if n is None else n
+    units = cfg.batch * cfg.num_kv_heads
+    out = torch.empty((units, 16, 256, 8), dtype=torch.float32, device=keys.device)
+    sa, sp = _signs_ptr(signs)
+    _check(lib.pariskv_train_centroids(ctypes.byref(cfg), sp, keys.data_ptr(), _slab(keys), n,
+                                       int(iters), out.data_ptr(), _stream(stream)),
+           "pariskv_train_centroids")
+    return out
 
 
 def build_index_rotated(cfg: Config, signs, y, knorm, n: Optional[int] = None,
