@@ -55,7 +55,9 @@ def parse():
 
 
 # ------------------------------------------------------------------------------------ dist
-def dist_setup(args):
+def dist_setup(args=None):
+    """One process per GPU from the torchrun environment: NCCL over the local GPU, or gloo on
+    the host cores where no GPU is visible (the reference arm and the multi-rank tests)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -63,10 +65,21 @@ def dist_setup(args):
         import datetime
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout,
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timeout)
     return ws, rank, local
+
+
+def rank_spec(name: str, rank: int):
+    """The workload of one rank: weak scaling gives every rank its own sequences (the seed is
+    offset by 1000 per rank), the same shapes."""
+    from long_context_kv_srht_b200 import workload
+    return workload.spec(name, seed=workload.spec(name).seed + 1000 * rank)
 
 
 def dist_max(x: float, ws: int) -> float:
@@ -74,7 +87,8 @@ def dist_max(x: float, ws: int) -> float:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -440,8 +454,7 @@ def run_drift(args, ws, rank, local):
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    base = workload.spec("drift_32k")
-    sp = workload.spec("drift_32k", seed=base.seed + 1000 * rank)
+    sp = rank_spec("drift_32k", rank)
     T, H, n0, k = sp.decode_steps, sp.num_kv_heads, sp.n, sp.k
     w = workload.generate_drift(sp)
     bf = lambda a: torch.from_numpy(workload.bf16_bits(a)).view(torch.bfloat16).to(dev)
@@ -541,6 +554,9 @@ def main():
     ws, rank, local = dist_setup(args)
     if args.impl == "reference":
         run_reference(args, ws, rank)
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
         return
     if args.workload == "drift_32k":
         run_drift(args, ws, rank, local)
@@ -552,8 +568,7 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    base = workload.spec(args.workload)
-    sp = workload.spec(args.workload, seed=base.seed + 1000 * rank)
+    sp = rank_spec(args.workload, rank)
     kv_host = sp.name == "million_offload"
     # K/V hold APPEND_SLACK extra tokens after the n indexed ones: the decode-step measurement
     # appends them to the index, so every index the search can return has a K/V row
