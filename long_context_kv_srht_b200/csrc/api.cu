@@ -25,11 +25,24 @@ thread_local int32_t g_launches = 0;
 
 void set_err(const char* fmt, va_list ap) { vsnprintf(g_err, sizeof(g_err), fmt, ap); }
 
-// Test hook: PARISKV_FAULT=alloc makes every device allocation of the library fail, so the
-// ENOMEM paths (and their cleanup) can be exercised without exhausting a real device.
+// Test hooks (failures made on the host; no device fault is involved):
+//  PARISKV_FAULT=alloc makes every device allocation of the library fail, so the ENOMEM
+//  paths (and their cleanup) run without exhausting a real device;
+//  PARISKV_FAULT=launch makes every call that launches kernels (search, append, the
+//  attentions) fail with ECUDA before its first launch, as a launch error would, so that the
+//  callers' error paths and the index's unchanged state can be checked.
 bool fault_alloc() {
     const char* f = getenv("PARISKV_FAULT");
     return f && strcmp(f, "alloc") == 0;
+}
+
+bool fault_launch() {
+    const char* f = getenv("PARISKV_FAULT");
+    return f && strcmp(f, "launch") == 0;
+}
+
+pariskv_status injected_launch_failure() {
+    return fail(PARISKV_ECUDA, "injected launch failure (PARISKV_FAULT=launch)");
 }
 
 template <typename T>
@@ -241,6 +254,7 @@ pariskv_status run_search(pariskv_index* ix, const void* q, const float* qt, con
     const int64_t C = candidate_count(ix->n, k, ix->cfg.cand_bp);
     pariskv_status s = ensure_candidates(ix, C);
     if (s != PARISKV_OK) return s;
+    if (fault_launch()) return injected_launch_failure();
     g_launches = 0;
     int ne = 0;
     auto mark = [&]() {
@@ -348,6 +362,7 @@ static pariskv_status append_common(pariskv_index* ix, const void* keys, const f
     s = check_dev_ptr(keys, rotated ? 16 : (ix->cfg.dtype == PARISKV_BF16 ? 8 : 16), "keys");
     if (s != PARISKV_OK) return s;
     if (rotated && (s = check_dev_ptr(knorm, 4, "knorm")) != PARISKV_OK) return s;
+    if (fault_launch()) return injected_launch_failure();
     cudaError_t e = launch_encode(ix, keys, knorm, ld_tok, t, ix->n, rotated,
                                   static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "encode launch");
@@ -436,6 +451,7 @@ pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, c
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float* work = nullptr;
     if (fault_alloc()) return fail(PARISKV_ENOMEM, "attention workspace");
+    if (fault_launch()) return injected_launch_failure();
     cudaMemPool_t pool = nullptr;
     cudaError_t e = workspace_pool(&pool);
     if (e == cudaSuccess)
@@ -477,6 +493,7 @@ pariskv_status pariskv_dense_attend(const pariskv_config* cfg, const void* q, co
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float* work = nullptr;
     if (fault_alloc()) return fail(PARISKV_ENOMEM, "attention workspace");
+    if (fault_launch()) return injected_launch_failure();
     cudaMemPool_t pool = nullptr;
     cudaError_t e = workspace_pool(&pool);
     if (e == cudaSuccess)
@@ -529,6 +546,7 @@ pariskv_status pariskv_sparse_attend_noalloc(const pariskv_config* cfg, const vo
                      gather_min_splits(k) <= fit;
     const int nsplit = min(attend_splits(heads, k, sms, mma), fit);
     float* work = nullptr;
+    if (fault_launch()) return injected_launch_failure();
     cudaError_t e = attend_static_scratch(&work);
     if (e != cudaSuccess) return cuda_fail(e, "fixed attention workspace lookup");
     g_launches = 0;

@@ -290,3 +290,31 @@ def test_allocation_failure_is_reported(monkeypatch):
     ix = pk.build_index(_cfg(1, 1, 1, 100), w.signs, keys)
     idx, _ = ix.search(_t(w.queries), 10)
     assert idx.shape == (1, 10)
+
+
+def test_injected_launch_failure(monkeypatch):
+    """PARISKV_FAULT=launch: search, append and both attention calls fail with ECUDA before
+    launching, the index keeps its size and state, and once the hook is off the index
+    searches exactly as before."""
+    sp = workload.spec("tiny", n=2000, seed=41)
+    w = workload.generate(sp)
+    cfg = _cfg(1, 1, 1, 2100)
+    keys = _t(w.keys)
+    ix = pk.build_index(cfg, w.signs, keys)
+    q = _t(w.queries)
+    ref_idx, ref_est = ix.search(q, 50)
+    torch.cuda.synchronize()
+    monkeypatch.setenv("PARISKV_FAULT", "launch")
+    for call in (lambda: ix.search(q, 50), lambda: ix.append(keys[:, :, :10]),
+                 lambda: pk.sparse_attend(cfg, q, keys, keys, ref_idx, 50, 0.1),
+                 lambda: pk.sparse_attend_noalloc(cfg, q, keys, keys, ref_idx, 50, 0.1)):
+        with pytest.raises(pk.PariskvError) as e:
+            call()
+        assert e.value.status == pk.ECUDA and "injected" in pk.last_error()
+    assert ix.size == 2000
+    monkeypatch.delenv("PARISKV_FAULT")
+    idx, est = ix.search(q, 50)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx.cpu().numpy())
+    np.testing.assert_array_equal(est.cpu().numpy().view(np.uint32),
+                                  ref_est.cpu().numpy().view(np.uint32))
+    ix.sync()
