@@ -325,8 +325,8 @@ def decode_step(args, ix, cfg, sp, keys, vals, qs, idx, est, k, H, dev, kv_host)
 def dense_comparator(cfg, sp, data, ix, k, dev, peak_gbs):
     """Full attention over all n tokens (pariskv_dense_attend, K/V in HBM) against ParisKV's
     retrieval + sparse attention over the top-k with the same K/V in HBM (the one-key append,
-    about 0.02 ms, is in the decode-step figures): the synthetic analogue of the pages'
-    comparison with full attention. Both are
+    about 0.02 ms, is in the decode-step figures): the synthetic analogue of the comparison
+    with full attention in "Technical Summary: ParisKV" (Experimental Results). Both are
     timed with CUDA events around 20 steps enqueued back to back after 3 warm-up steps; K/V
     (4 GiB at the million-token workload) exceed L2, so no flush is needed between steps."""
     import numpy as np
@@ -378,8 +378,9 @@ def dense_comparator(cfg, sp, data, ix, k, dev, peak_gbs):
             "kv": "HBM (both)", "n": n, "k": k}
 
 
-# Region sizes of the four-region cache measurement (the pages give none; 64 sink tokens as in
-# the sink-token convention of the P4 page, a 2048-token local window, a 256-token buffer).
+# Region sizes of the four-region cache measurement ("Technical Summary: ParisKV" gives none;
+# 64 sink tokens as in the sink-token convention of "Self-Indexing KVCache", a 2048-token local
+# window, a 256-token buffer).
 CACHE_REGIONS = dict(n_sink=64, n_local=2048, n_buffer=256)
 
 
@@ -711,7 +712,7 @@ def main():
     if not args.no_decode:
         decode = decode_step(args, ix, cfg, sp, keys, vals, qs, idx, est, k, H, dev, kv_host)
 
-    # full attention over every token, the baseline the pages compare against
+    # full attention over every token, the baseline "Technical Summary: ParisKV" compares with
     dense = None
     if not args.no_dense:
         dense = dense_comparator(cfg, sp, data, ix, k, dev, measured_peaks()[0])
