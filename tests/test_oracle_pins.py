@@ -582,3 +582,29 @@ def test_train_centroids_recovers_directions_and_improves_fit():
         assert fit >= prev - 1e-12, (it, fit, prev)
         prev = fit
         np.testing.assert_allclose(np.linalg.norm(c, axis=2), 1.0, atol=1e-6)
+
+
+def test_table_levels_i_over_7_reproduce_uniform_codes():
+    """The table path with levels c_i = i / 7 is the uniform rule written another way: the
+    midpoints (2i - 1) / 14 give mag = floor(7 r + 1/2), so the codes agree (barring ratios
+    that land exactly on a midpoint), and since vt_table = vt_uniform / 7 the factor fold
+    absorbs the scale: S agrees to fp32 rounding. Two independent code paths in the oracle
+    checked against each other."""
+    rng = np.random.default_rng(34)
+    sg = _signs(D, 17)
+    k = (rng.standard_normal((2000, D)) * 2 + 0.3).astype(np.float32)
+    y, kn = oracle.normalize_rotate(k, sg)
+    uni = oracle.encode_rotated(y, kn, M)
+    tab = oracle.encode_rotated(y, kn, M, table=(np.arange(8) / 7).astype(np.float32))
+    a = np.abs(y.reshape(-1, B, M))
+    r = (a / a.max(axis=2, keepdims=True)).ravel()
+    on_mid = np.any(np.abs(r[:, None] * 14 - (2 * np.arange(1, 8) - 1)) < 1e-5, axis=1)
+    assert on_mid.mean() < 1e-3
+    same = ~on_mid.reshape(-1, B * M)
+    np.testing.assert_array_equal(uni.mag[same], tab.mag[same])
+    np.testing.assert_array_equal(uni.ids, tab.ids)
+    qt, _ = oracle.normalize_rotate(rng.standard_normal((1, D)).astype(np.float32), sg)
+    rows = np.where(same.all(axis=1))[0].astype(np.int32)
+    Su = oracle.rerank(uni, rows, qt[0], M).astype(np.float64)
+    St = oracle.rerank(tab, rows, qt[0], M).astype(np.float64)
+    np.testing.assert_allclose(St, Su, rtol=2e-5, atol=2e-6 * np.abs(Su).max())
