@@ -132,3 +132,37 @@ def test_invalid_level_table_rejected(table):
     st = pk.lib.pariskv_build_index(ctypes.byref(c), signs.ctypes.data, None, 0, 0, None,
                                     ctypes.byref(h))
     assert st == pk.EINVAL and not h.value and "level_table" in pk.last_error()
+
+
+@pytest.mark.parametrize("cc", [(-1, 8, 4, 4, 16), (2, 4, 8, 4, 16), (2, 8, 0, 4, 16),
+                                (2, 8, 4, 0, 16), (2, 8, 4, 4, 0)])
+def test_cache_config_rejected_on_the_host(cc):
+    """pariskv_cache_create validates the region sizes before it touches the device."""
+    import numpy as np
+    cfg = pk.config(capacity=1)
+    ccfg = pk.CacheConfig(*cc)
+    signs = np.ones(128, np.int8)
+    h = ctypes.c_void_p()
+    st = pk.lib.pariskv_cache_create(ctypes.byref(cfg), ctypes.byref(ccfg), signs.ctypes.data,
+                                     None, ctypes.byref(h))
+    assert st == pk.EINVAL and not h.value
+
+
+@pytest.mark.parametrize("field,value", [("dtype", 0), ("group", 9)])
+def test_dense_attend_config_rejected_on_the_host(field, value):
+    c = pk.config(capacity=64, **{field: value})
+    st = pk.lib.pariskv_dense_attend(ctypes.byref(c), None, None, None, 64, 64, 0.1, None, 0,
+                                     None)
+    assert st == pk.EINVAL
+
+
+def test_train_centroids_arguments_rejected_on_the_host():
+    import numpy as np
+    c = pk.config(capacity=64)
+    signs = np.ones(128, np.int8)
+    bad = signs.copy()
+    bad[5] = 0
+    for sg, n, iters in ((bad, 10, 1), (signs, 0, 1), (signs, 10, -1), (signs, 10, 1001)):
+        st = pk.lib.pariskv_train_centroids(ctypes.byref(c), sg.ctypes.data, None, 10, n, iters,
+                                            None, None)
+        assert st == pk.EINVAL
