@@ -608,3 +608,34 @@ def test_table_levels_i_over_7_reproduce_uniform_codes():
     Su = oracle.rerank(uni, rows, qt[0], M).astype(np.float64)
     St = oracle.rerank(tab, rows, qt[0], M).astype(np.float64)
     np.testing.assert_allclose(St, Su, rtol=2e-5, atol=2e-6 * np.abs(Su).max())
+
+
+def test_golden_basis_key():
+    """A hand-derived worked example (tests/golden/basis_key_e5.json, derivation and citation
+    inside): key 3 e_5 and query e_5 with all SRHT signs +1 -- ids, codes, factor, the
+    rho = 4 vote table and the estimate."""
+    import json
+    import os
+    fx = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "basis_key_e5.json")))
+    k = np.zeros((1, D), np.float32)
+    k[0, fx["basis_index"]] = fx["key_scale"]
+    q = np.zeros((1, D), np.float32)
+    q[0, fx["basis_index"]] = 1.0
+    s = np.ones(D, np.int8)
+    y, kn = oracle.normalize_rotate(k, s)
+    enc = oracle.encode_rotated(y, kn, M)
+    np.testing.assert_array_equal(enc.ids[0], fx["ids"])
+    np.testing.assert_array_equal(enc.mag[0], fx["magnitude"])
+    neg = np.zeros(M, np.uint8)
+    neg[fx["negative_dims_in_subspace"]] = 1
+    np.testing.assert_array_equal(enc.neg[0], np.tile(neg, B))
+    np.testing.assert_allclose(enc.factor[0], fx["factor"], rtol=1e-6)
+    qt, qn = oracle.normalize_rotate(q, s)
+    lut = oracle.query_lut(qt[0], M, 4)
+    want = np.zeros(256, np.uint8)
+    for c, wgt in fx["lut_rho4"].items():
+        want[int(c)] = wgt
+    for b in range(B):
+        np.testing.assert_array_equal(lut[b], want)
+    S = oracle.rerank(enc, np.array([0], np.int32), qt[0], M)[0]
+    assert abs(float(qn[0]) * float(S) - fx["estimate"]) <= 1e-5
