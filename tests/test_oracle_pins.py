@@ -639,3 +639,15 @@ def test_golden_basis_key():
         np.testing.assert_array_equal(lut[b], want)
     S = oracle.rerank(enc, np.array([0], np.int32), qt[0], M)[0]
     assert abs(float(qn[0]) * float(S) - fx["estimate"]) <= 1e-5
+
+
+def test_attend_saturated_logits_pick_the_best_row():
+    """Logits hundreds apart (scale 50 on unit-scale rows): the softmax is one-hot to fp64
+    precision, so the output is the value row of the largest logit, with no overflow."""
+    rng = np.random.default_rng(35)
+    K = rng.standard_normal((300, D)).astype(np.float32)
+    V = rng.standard_normal((300, D)).astype(np.float32)
+    q = K[123] * 4.0
+    idx = np.arange(0, 300, 3, dtype=np.int32)          # row 123 is among them
+    out = oracle.attend(q, K, V, idx, 50.0)
+    np.testing.assert_allclose(out, V[123].astype(np.float64), atol=1e-12)
