@@ -14,18 +14,15 @@ constexpr int M = 8;            // dims per subspace
 constexpr int NB = D / M;       // subspaces (16)
 constexpr int NC = 1 << M;      // sign centroids per subspace (256)
 constexpr int REC = 128;        // bytes per key record: 64 B of 4-bit codes + 16 fp32 factors
-constexpr int NBINS = 64;       // coarse scores are < 64 (B * w_rank1 <= 48)
+constexpr int NBINS = 64;       // histogram bins per head and chunk (scores <= B * w_rank1 <= 48)
 constexpr int SBINS_BITS = 11;  // first radix level of the top-k, counted by the rerank
 constexpr int SBINS = 1 << SBINS_BITS;
-constexpr int SCOPIES = 1;      // copies of that histogram (one copy per warp group spreads the reductions)
-constexpr int CHUNK = 8192;     // keys per coarse-score histogram chunk (a vote work item)
+constexpr int CHUNK = 16384;    // keys per coarse-score histogram chunk (a vote / compaction item)
 constexpr int PACK = 4;         // query heads whose vote weights share one 32-bit table entry
 
+// Device status word: ST_TIMEOUT when a bounded wait of the search kernel ran out,
+// ST_BADINDEX when a kernel found an index out of range (and skipped the access).
 enum : int { ST_OK = 0, ST_TIMEOUT = 5, ST_BADINDEX = 6 };
-
-// Upper bound for every device-side spin wait, in SM clock cycles (about 1 s at 2 GHz). A
-// wait that runs out records ST_TIMEOUT in the status word and returns.
-constexpr long long kSpinLimitCycles = 2000000000LL;
 
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ constexpr int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
@@ -153,19 +150,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         " selp.u32 %0, 1, 0, p;\n}\n"
         : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
-}
-// Bounded wait for the phase with the given parity. Returns false (and records a timeout in
-// *status) when the limit runs out.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* status) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kSpinLimitCycles) {
-            atomicExch(status, ST_TIMEOUT);
-            return false;
-        }
-    }
-    return true;
 }
 // Global -> shared bulk copy completing on an mbarrier (bytes and both addresses multiples
 // of 16). The destination is this CTA's own shared memory.
