@@ -67,6 +67,20 @@ PARISKV_API pariskv_status pariskv_debug_profile(pariskv_index* index, int32_t e
 PARISKV_API pariskv_status pariskv_debug_stage_ms(pariskv_index* index, float* ms,
                                                   int32_t* nstages);
 
+/* Bounds every device-side wait of later searches on this index to `cycles` SM clock cycles
+ * (0 restores the default of about one second). A wait that runs out makes pariskv_sync
+ * return PARISKV_ETIMEOUT, naming the control word it waited on. Used by tests of the
+ * timeout path. No counterpart on the pages. Errors: EINVAL. */
+PARISKV_API pariskv_status pariskv_debug_set_wait_limit(pariskv_index* index, int64_t cycles);
+
+/* Makes later searches on this index report, per CTA of the search kernel, the item it is
+ * working on into `board` (8 int32 per CTA: item number, kind, head or pack-unit, state 1 =
+ * claimed, -1 = its wait expired, 2 = done, 3 = exited; then the last checkpoint passed by
+ * threads 1, 32, 224 and 0 as 100 x loop iteration + checkpoint), a pinned host buffer the
+ * host may read while the kernel runs; NULL turns it off. The board must hold 8 ints for
+ * each of 2 x (number of SMs) CTAs. A debugging aid with no counterpart on the pages. Errors: EINVAL. */
+PARISKV_API pariskv_status pariskv_debug_set_progress(pariskv_index* index, int32_t* board);
+
 /* Phases of the last profiled search (pariskv_debug_profile on): the search runs as one
  * persistent kernel whose workers take items of several kinds; for each kind -- 0 query
  * prep, 1 vote, 2 compaction, 3 top-k, 4 threshold finalisation, 5 rerank, 6 vote-group

@@ -193,7 +193,7 @@ pariskv_status create_index(const pariskv_config* cfg, const int8_t* signs, cuda
               dalloc(&ix->qnorm, heads) && dalloc(&ix->scores, up * ix->cap_pad) &&
               dalloc(&ix->hist, up * nch * PACK * NBINS) && dalloc(&ix->thr, heads * 4) &&
               dalloc(&ix->cbase, heads * nch * 2) && dalloc(&ix->shist, heads * SBINS) &&
-              dalloc(&ix->status, 1) && dalloc(&ix->lvt, kLevelTableFloats) &&
+              dalloc(&ix->status, 4) && dalloc(&ix->lvt, kLevelTableFloats) &&
               dalloc(&ix->ctrl, search_ctrl_words(static_cast<int>(up)));
     if (!ok) {
         free_index(ix);
@@ -218,7 +218,7 @@ pariskv_status create_index(const pariskv_config* cfg, const int8_t* signs, cuda
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(ix->lvt, tab, sizeof(tab), cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(ix->lut, 0, up * NB * NC * sizeof(uint32_t), st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(ix->status, 0, sizeof(int), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ix->status, 0, 4 * sizeof(int), st);
     if (e == cudaSuccess)
         e = cudaMemsetAsync(ix->ctrl, 0, search_ctrl_words(static_cast<int>(up)) * sizeof(int), st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);  // hs, tab live on this stack frame
@@ -699,8 +699,13 @@ pariskv_status pariskv_sync(pariskv_index* index, void* stream) {
     e = cudaMemcpy(&st, index->status, sizeof(int), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "status read");
     if (st != ST_OK) {
-        cudaMemset(index->status, 0, sizeof(int));
-        if (st == ST_TIMEOUT) return fail(PARISKV_ETIMEOUT, "a bounded device-side wait expired");
+        int diag[4] = {};
+        cudaMemcpy(diag, index->status, sizeof(diag), cudaMemcpyDeviceToHost);
+        cudaMemset(index->status, 0, 4 * sizeof(int));
+        if (st == ST_TIMEOUT)
+            return fail(PARISKV_ETIMEOUT,
+                        "a bounded device-side wait expired (control word %d: waited for %d, saw %d)",
+                        diag[1], diag[2], diag[3]);
         return fail(PARISKV_ECUDA, "internal consistency check failed on the device (%d)", st);
     }
     return PARISKV_OK;
@@ -801,6 +806,22 @@ pariskv_status pariskv_debug_profile(pariskv_index* ix, int32_t enable) {
         return fail(PARISKV_ENOMEM, "search trace buffer");
     ix->profile = enable != 0;
     ix->nev = 0;
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_debug_set_progress(pariskv_index* ix, int32_t* board) {
+    pariskv_status s = check_index(ix);
+    if (s != PARISKV_OK) return s;
+    if (board && (s = check_dev_ptr(board, 16, "board")) != PARISKV_OK) return s;
+    ix->progress = board;
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_debug_set_wait_limit(pariskv_index* ix, int64_t cycles) {
+    pariskv_status s = check_index(ix);
+    if (s != PARISKV_OK) return s;
+    if (cycles < 0) return fail(PARISKV_EINVAL, "cycles < 0");
+    ix->spin_limit = cycles == 0 ? kDefaultSpinLimit : cycles;
     return PARISKV_OK;
 }
 

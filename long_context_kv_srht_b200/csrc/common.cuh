@@ -15,7 +15,7 @@ constexpr int NB = D / M;       // subspaces (16)
 constexpr int NC = 1 << M;      // sign centroids per subspace (256)
 constexpr int REC = 128;        // bytes per key record: 64 B of 4-bit codes + 16 fp32 factors
 constexpr int NBINS = 64;       // histogram bins per head and chunk (scores <= B * w_rank1 <= 48)
-constexpr int SBINS_BITS = 11;  // first radix level of the top-k, counted by the rerank
+constexpr int SBINS_BITS = 13;  // first radix level of the top-k, counted by the rerank
 constexpr int SBINS = 1 << SBINS_BITS;
 constexpr int CHUNK = 16384;    // keys per coarse-score histogram chunk (a vote / compaction item)
 constexpr int PACK = 4;         // query heads whose vote weights share one 32-bit table entry

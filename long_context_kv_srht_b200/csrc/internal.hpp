@@ -54,6 +54,7 @@ struct pariskv_index {
     // work queues of the persistent search kernel (search.cu)
     int* ctrl = nullptr;        // control block: queue counters, per-pack flags and counters
     unsigned long long* trace = nullptr;   // phase trace of profiled searches [kTraceWords]
+    int* progress = nullptr;    // debug: per-CTA item board in mapped host memory (not owned)
     long long spin_limit = kDefaultSpinLimit;   // bound of every device-side wait (cycles)
 
     // optional per-stage timing of searches (test and benchmark use)

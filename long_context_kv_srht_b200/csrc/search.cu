@@ -55,101 +55,56 @@ namespace {
 // ---------------------------------------------------------------------------------------
 // Shape of the kernel
 // ---------------------------------------------------------------------------------------
-constexpr int kVW = 8;                        // vote-group warps
-constexpr int kRW = 8;                        // rerank warps
-constexpr int kVT = 32 * kVW;                 // vote-group threads
-constexpr int kThreads = 32 * (kVW + kRW);
-constexpr int kBarV = 1;                      // named barrier of the vote group
+constexpr int kW = 8;                         // warps per CTA (two CTAs per SM)
+constexpr int kThreads = 32 * kW;
+constexpr int kVW = kW;                       // every item is worked on by the whole CTA
+constexpr int kVT = kThreads;
+constexpr int kBarV = 1;                      // named barrier of the CTA
 
 constexpr int kTileKeys = 64;                 // vote warp-tile: two keys per lane
-constexpr int kTiles = CHUNK / kTileKeys;     // tiles per chunk
 constexpr int kKeysPerThr = CHUNK / kVT;      // compaction: consecutive keys per thread
 constexpr int kCWords = kKeysPerThr / 32;     // 32-bit key masks per head and kind
-static_assert(kTiles % kVW == 0 && kKeysPerThr % 32 == 0, "chunk shape");
+static_assert(kKeysPerThr % 32 == 0, "chunk shape");
 
 constexpr int kStage = 32;                    // records per rerank stage (one per lane)
 constexpr int kSlots = 2;                     // stages per rerank warp ring
-constexpr int kRItem = 256;                   // candidates per rerank item
-constexpr int kBins = SBINS;                  // top-k radix bins (2048)
+constexpr int kRItem = 2048;                  // candidates per rerank item
+constexpr int kBins = 2048;                   // top-k radix bins of the later levels
+constexpr int kBins1 = SBINS;                 // first top-k level: counted by the rerank
+constexpr int kBits1 = SBINS_BITS;
 constexpr int kNR = 49;                       // byte-histogram rows per vote warp (scores 0..48)
-constexpr int kSub = 1024;                    // keys per streamed block of bucket ids (16 KB)
-constexpr int kVSlots = 3;                    // id blocks in the vote group's ring
+constexpr int kSub = 512;                     // keys per streamed block of bucket ids (8 KB)
+constexpr int kVSlots = 3;                    // id blocks in the vote ring
 
-// Dynamic shared memory (offsets from the dynamic base; `tab` depends on where the base
-// lies in the shared window, see Lay)
-//  vring   kVSlots blocks of ids streamed by bulk copies; also scratch of query prep,
-//          finalisation and compaction items (no copy is in flight during those)
-//  table   256 rows x 256 B at a 64 KB-aligned shared address (so one PRMT of an id byte and
-//          a column byte forms the full address of a vote lookup): row c, bytes 4 (2b + k):
-//          vote weights of centroid c, subspace b (copies k = 0, 1); bytes 128..255 of rows
-//          49 w .. 49 w + 48: byte counters of vote warp w < 4 (row s: one 32-bit word per
-//          lane, byte g = head g, score s)
-//  h2      the same counters of vote warps 4..7 (128-byte rows)
-//  everything from the dynamic base to the end of h2 is the scratch of a top-k item
-//  rring   per rerank warp kSlots stages of 32 records (128-byte rows, 16-byte piece c of
-//          row r at c ^ (r mod 8)); then per rerank warp 64 query pairs, the vote group's
-//          ring barriers, the rerank warps' stage records
-constexpr uint32_t kVRingBytes = kVSlots * kSub * 16;
+// Dynamic shared memory of a CTA (two CTAs per SM). Vote items, rerank items and top-k
+// items use the same bytes in turn (a vote item rebuilds its table and clears its counters
+// when another kind of item has used them since):
+//  table   256 rows x 256 B: row c, bytes 4 (2b + k): vote weights of centroid c, subspace b
+//          (copies k = 0, 1); bytes 128..255 of rows 49 w .. 49 w + 48: byte counters of
+//          warp w < 4 (row s: one 32-bit word per lane, byte g = head g, score s)
+//  h2      the same counters of warps 4..7 (128-byte rows)
+//  vring   kVSlots blocks of bucket ids streamed by bulk copies; between vote items also the
+//          scratch of query-prep, finalisation and compaction items
+//  a rerank item's per-warp rings (kSlots stages of 32 records, 128-byte rows, 16-byte
+//  piece c of row r at c ^ (r mod 8)) and query pairs start at 0; a top-k item uses it all
+constexpr uint32_t kOffTab = 0;
 constexpr uint32_t kTabBytes = 256 * 256;
+constexpr uint32_t kOffH2 = kOffTab + kTabBytes;
 constexpr uint32_t kH2Bytes = 4 * kNR * 128;
+constexpr uint32_t kOffVRing = kOffH2 + kH2Bytes;
+constexpr uint32_t kVRingBytes = kVSlots * kSub * 16;
+constexpr uint32_t kOffScr = kOffVRing;
+constexpr int kSmem = static_cast<int>(kOffVRing + kVRingBytes);
 constexpr int kRingWarp = kSlots * kStage * REC;
-constexpr uint32_t kAfterTab = kTabBytes + kH2Bytes + kRW * kRingWarp + kRW * 512 + 32 +
-                               kRW * kSlots * 16 + 256;
-constexpr uint32_t kMaxBase = 65536 - kVRingBytes;   // largest dynamic base the layout allows
-constexpr int kSmem = 65536 + kAfterTab;
-struct Lay {
-    uint32_t tab, h2, ring, qry, vbar, desc;   // offsets from the dynamic base
-    uint32_t hi;                               // byte 2 of the table's shared address
-};
-__device__ __forceinline__ Lay make_lay(uint32_t base) {
-    Lay l;
-    const uint32_t ta = (base + kVRingBytes + 65535u) & ~65535u;   // table shared address
-    l.tab = ta - base;
-    l.h2 = l.tab + kTabBytes;
-    l.ring = l.h2 + kH2Bytes;
-    l.qry = l.ring + kRW * kRingWarp;
-    l.vbar = l.qry + kRW * 512;
-    l.desc = l.vbar + 32;
-    l.hi = ta >> 16;
-    return l;
-}
-constexpr uint32_t kOffVRing = 0;
-constexpr uint32_t kOffScr = 0;
+constexpr uint32_t kOffRing = 0;
+constexpr uint32_t kOffQry = kW * kRingWarp;
+static_assert(kOffQry + 512 <= static_cast<uint32_t>(kSmem), "rerank rings");
 static_assert(2 * kBins * 4 + 1024 <= kVRingBytes, "item scratch");
-
-// items of the vote-group queue
-enum : int { IT_NONE = -1, IT_Q = 0, IT_V = 1, IT_C = 2, IT_K = 3 };
-struct VItem {
-    int type, x, y;   // Q, K: query head x; V, C: pack-unit x, chunk y
-};
-
-// The vote-group queue, computed from the item number: Q(h) for every query head h; then
-// the vote items pack by pack, with the compaction items of pack p placed after the vote
-// items of pack p + kLag (so that the vote group claiming them rarely finds pack p
-// unfinished); then the compaction items of the last kLag packs; then one top-k item per
-// query head.
-constexpr int kLag = 2;
-__device__ inline VItem vqueue_item(int i, int P, int nc, int heads) {
-    if (i < heads) return {IT_Q, i, 0};
-    int j = i - heads;
-    const int lead = min(P, kLag), mid = P - lead;
-    if (j < lead * nc) return {IT_V, j / nc, j % nc};
-    j -= lead * nc;
-    if (j < mid * 2 * nc) {
-        const int p = kLag + j / (2 * nc), o = j % (2 * nc);
-        return o < nc ? VItem{IT_V, p, o} : VItem{IT_C, p - kLag, o - nc};
-    }
-    j -= mid * 2 * nc;
-    if (j < lead * nc) return {IT_C, mid + j / nc, j % nc};
-    j -= lead * nc;
-    if (j < heads) return {IT_K, j, 0};
-    return {IT_NONE, 0, 0};
-}
 
 // Optional phase trace (a measurement aid, off when SearchArgs::trace is NULL): per kind of
 // work, the earliest start (stored as ~t so that atomicMax keeps the minimum), the latest
 // end and the summed busy time, in %globaltimer nanoseconds.
-enum : int { TR_Q = IT_Q, TR_V = IT_V, TR_C = IT_C, TR_K = IT_K, TR_F = 4, TR_R = 5,
+enum : int { TR_Q = 0, TR_V = 1, TR_C = 2, TR_K = 3, TR_F = 4, TR_R = 5,
              TR_VWAIT = 6, TR_RWAIT = 7, TR_KERNEL = 8, TR_POLLS = 9, TR_KSEL = 10,
              TR_KWRITE = 11, TR_SLOTS = 12 };
 __device__ __forceinline__ uint64_t gtime() {
@@ -190,6 +145,7 @@ struct SearchArgs {
     int* ctrl;
     int* status;
     unsigned long long* trace;   // phase trace [TR_SLOTS][3], or NULL
+    int* progress;               // per-CTA item board in mapped host memory, or NULL
     int64_t n, cap_pad, cmax;
     long long spin_limit;
     int units, G, packs, P, nc, nch, heads;
@@ -201,7 +157,7 @@ struct SearchArgs {
 // control block: one 128-byte line per word (queue counters and flags polled by many warps
 // must not share lines): queue counters, exit count, then per pack-unit p the query-prep
 // count, the threshold-ready flag and the vote, compaction and rerank done-counts
-enum : int { CT_VQ = 0, CT_RQ = 1, CT_EXIT = 2, CT_HDR = 4 };
+enum : int { CT_Q = 0, CT_EXIT = 2, CT_HDR = 4 };
 constexpr int kCtlStride = 32;
 enum : int { PK_Q = 0, PK_F = 1, PK_V = 2, PK_C = 3, PK_R = 4, PK_N = 5 };
 __device__ __forceinline__ int* ctl(const SearchArgs& a, int word) { return a.ctrl + word * kCtlStride; }
@@ -209,16 +165,79 @@ __device__ __forceinline__ int* pk(const SearchArgs& a, int kind, int p) {
     return a.ctrl + (CT_HDR + kind * a.P + p) * kCtlStride;
 }
 
+// ---------------------------------------------------------------------------------------
+// The work queue
+// ---------------------------------------------------------------------------------------
+// Every CTA takes items from one queue, in this order: the query-prep item Q(h) of every
+// query head; then segments s = 0, 1, ...: the compaction items C(s - 2, .) of pack-unit
+// s - 2, the vote items V(s, .) of pack-unit s and the rerank items R(., .) of the heads of
+// pack-unit s - 3 (evenly interleaved, so that the two CTAs of an SM usually stream ids and
+// gather records at the same time), and the top-k items K(h) of the heads of pack-unit
+// s - 4. Each item waits only for items handed out before it: V(p) for the Q items of p, C(p)
+// for the finalisation of p (done by the CTA that completed its last vote item), R for all
+// C of its pack-unit, K for all R of its pack-unit.
+enum : int { IT_NONE = -1, IT_Q = 0, IT_V = 1, IT_C = 2, IT_K = 3, IT_R = 4 };
+struct Item {
+    int type, x, y;   // Q, K: query head x; V, C: pack-unit x, chunk y; R: head x, range y
+};
+constexpr int kLagC = 2, kLagR = 3, kLagK = 4;
+__device__ __forceinline__ int heads_of(const SearchArgs& a, int p) {
+    return min(PACK, a.G - (p % a.packs) * PACK);
+}
+// query heads of pack-units [0, q)
+__device__ __forceinline__ int heads_before(const SearchArgs& a, int q) {
+    return (q / a.packs) * a.G + min(PACK * (q % a.packs), a.G);
+}
+__device__ __forceinline__ int64_t seg_start(const SearchArgs& a, int s) {
+    auto cl = [&](int v) { return max(0, min(v, a.P)); };
+    return static_cast<int64_t>(a.heads) + static_cast<int64_t>(a.nc) * (cl(s) + cl(s - kLagC)) +
+           static_cast<int64_t>(a.nrh) * heads_before(a, cl(s - kLagR)) +
+           heads_before(a, cl(s - kLagK));
+}
+__device__ Item queue_item(const SearchArgs& a, int64_t i) {
+    if (i < a.heads) return {IT_Q, static_cast<int>(i), 0};
+    const int S = a.P + kLagK;   // segments 0 .. S - 1
+    if (i >= seg_start(a, S)) return {IT_NONE, 0, 0};
+    int lo = 0, hi = S - 1;      // the last segment starting at or before i
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) / 2;
+        if (seg_start(a, mid) <= i) lo = mid;
+        else hi = mid - 1;
+    }
+    const int s = lo;
+    int64_t o = i - seg_start(a, s);
+    const int pc = s - kLagC, pr = s - kLagR, pkk = s - kLagK;
+    const int nC = (pc >= 0 && pc < a.P) ? a.nc : 0;
+    if (o < nC) return {IT_C, pc, static_cast<int>(o)};
+    o -= nC;
+    const int64_t nV = s < a.P ? a.nc : 0;
+    const int64_t nR = (pr >= 0 && pr < a.P) ? static_cast<int64_t>(heads_of(a, pr)) * a.nrh : 0;
+    if (o < nV + nR) {
+        const int64_t N = nV + nR;
+        const int64_t v0 = o * nV / N, v1 = (o + 1) * nV / N;
+        if (v1 > v0) return {IT_V, s, static_cast<int>(v0)};
+        const int r = static_cast<int>(o - v0);   // rerank item within the pack-unit
+        const int unit = pr / a.packs, pack = pr % a.packs;
+        return {IT_R, unit * a.G + pack * PACK + r / a.nrh, r % a.nrh};
+    }
+    o -= nV + nR;
+    const int unit = pkk / a.packs, pack = pkk % a.packs;
+    return {IT_K, unit * a.G + pack * PACK + static_cast<int>(o), 0};
+}
+
 
 // The kernel's dynamic shared memory, referenced directly by the hot loops so that its
 // (constant) shared-window address folds into the load instructions.
-extern __shared__ __align__(1024) uint8_t g_smem[];
+extern __shared__ __align__(128) uint8_t g_smem[];
 
 // ---------------------------------------------------------------------------------------
 // Small helpers
 // ---------------------------------------------------------------------------------------
+// The non-aligned form: thread 0 often reaches a barrier later than the other lanes of its
+// warp (it claims items and waits on flags alone), and an aligned barrier reached by a
+// diverged warp may count the warp before all of its threads have arrived.
 __device__ __forceinline__ void bar_v() {
-    asm volatile("bar.sync %0, %1;" :: "n"(kBarV), "n"(kVT) : "memory");
+    asm volatile("barrier.sync %0, %1;" :: "n"(kBarV), "n"(kVT) : "memory");
 }
 // Loads that bypass L1: data written by other CTAs during this kernel.
 __device__ __forceinline__ uint32_t ldcg_u32(const void* p) {
@@ -253,7 +272,7 @@ __device__ __forceinline__ int ld_relaxed(const int* p) {
     return v;
 }
 __device__ bool wait_flag(const int* flag, int target, bool geq, long long limit, int* status,
-                          unsigned long long* trace) {
+                          unsigned long long* trace, const int* ctrl) {
     int v = ld_acquire(flag);
     if (geq ? v >= target : v == target) return true;
     // relaxed polling with exponential backoff (many warps may wait on one flag: keep its
@@ -270,7 +289,11 @@ __device__ bool wait_flag(const int* flag, int target, bool geq, long long limit
             return true;
         }
         if (clock64() - t0 > limit) {
-            atomicExch(status, ST_TIMEOUT);
+            if (atomicExch(status, ST_TIMEOUT) != ST_TIMEOUT) {   // the first expiry: where and what
+                status[1] = static_cast<int>(flag - ctrl) / kCtlStride;
+                status[2] = target;
+                status[3] = v;
+            }
             return false;
         }
     }
@@ -283,17 +306,15 @@ __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, l
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
         if (clock64() - t0 > limit) {
-            atomicExch(status, ST_TIMEOUT);
+            if (atomicExch(status, ST_TIMEOUT) != ST_TIMEOUT) status[1] = -1;   // an mbarrier
             return false;
         }
     }
     return true;
 }
 
-__device__ __forceinline__ uint32_t tab_ld(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
+__device__ __forceinline__ uint32_t tab_ld(uint32_t off) {
+    return *reinterpret_cast<const uint32_t*>(g_smem + kOffTab + off);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -428,12 +449,11 @@ __device__ __forceinline__ u32x8 ldg_ids(const uint8_t* p) {
     return v;
 }
 
-// Shared address of the table entry of step t: byte0 <- column (byte t % 3 of colp[t / 3]),
-// byte1 <- id byte t % 4 (row id, 256-byte rows), byte2 <- the top byte of colp[t / 3] (the
-// table's 64 KB page), byte3 <- that byte's sign replicated (zero).
+// Table entry of step t: byte0 <- column (byte t % 3 of colp[t / 3]), byte1 <- id byte t % 4,
+// bytes 2, 3 <- the zero top byte of colp[t / 3]: row id, 256-byte rows.
 template <int T>
 __device__ __forceinline__ uint32_t look(const uint32_t* wd, const uint32_t* colp) {
-    constexpr uint32_t sel = 0xF700u | ((T & 3u) << 4) | (4u + (T % 3));
+    constexpr uint32_t sel = 0x7700u | ((T & 3u) << 4) | (4u + (T % 3));
     return tab_ld(prmt_i<sel>(wd[T >> 2], colp[T / 3]));
 }
 
@@ -470,9 +490,9 @@ __device__ void load_table(const SearchArgs& a, int p, uint8_t* tab) {
 // word whose byte g counts head g's keys with that score (one bank per lane, so the
 // increments of a warp never conflict). Warps 0..3 keep theirs in the upper halves of the
 // table rows 49 w + s, warps 4..7 in h2 rows 49 (w - 4) + s.
-__device__ __forceinline__ uint32_t counter_base(uint8_t* smem, const Lay& L, int warp, int lane) {
-    return warp < 4 ? smem_addr(smem + L.tab + 49 * warp * 256 + 128 + 4 * lane)
-                    : smem_addr(smem + L.h2 + 49 * (warp - 4) * 128 + 4 * lane);
+__device__ __forceinline__ uint32_t counter_base(uint8_t* smem, int warp, int lane) {
+    return warp < 4 ? smem_addr(smem + kOffTab + 49 * warp * 256 + 128 + 4 * lane)
+                    : smem_addr(smem + kOffH2 + 49 * (warp - 4) * 128 + 4 * lane);
 }
 
 // Counts one key's HP packed scores (byte g of acc = head g's score) in this lane's byte
@@ -510,12 +530,12 @@ struct VRing {
 };
 
 __device__ __forceinline__ void v_item(const SearchArgs& a, int p, int c, uint8_t* smem,
-                                      const Lay& L, const uint32_t colp[6], VRing& vr) {
+                                      const uint32_t colp[6], VRing& vr) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int unit = p / a.packs, pack = p % a.packs;
     const int hp = min(PACK, a.G - pack * PACK);
     const uint32_t pitch = warp < 4 ? 256u : 128u;
-    const uint32_t cb = counter_base(smem, L, warp, lane);
+    const uint32_t cb = counter_base(smem, warp, lane);
 
     const int64_t k0 = static_cast<int64_t>(c) * CHUNK;
     const int nkeys = static_cast<int>(min64(a.n - k0, CHUNK));
@@ -540,24 +560,24 @@ __device__ __forceinline__ void v_item(const SearchArgs& a, int p, int c, uint8_
         const uint32_t par = static_cast<uint32_t>((vr.seq + b) / kVSlots) & 1u;
         mbar_wait_limit(vr.bar0 + 8 * slot, par, a.spin_limit, a.status);
         const uint8_t* blk = smem + kOffVRing + slot * kSub * 16;
-        // warp w scores tiles 2w and 2w + 1 of the block: four keys per lane at once
-        const int kb = b * kSub + 2 * warp * kTileKeys;      // first key of the warp's tiles
+        // warp w scores tile w of the block: keys lane and lane + 32
+        const int kb = b * kSub + warp * kTileKeys;      // first key of the warp's tile
         if (kb < nkeys) {
-            uint32_t acc[4];
+            uint32_t acc[2];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint4 x = *reinterpret_cast<const uint4*>(blk + (2 * warp * kTileKeys + 32 * i + lane) * 16);
+            for (int i = 0; i < 2; ++i) {
+                const uint4 x = *reinterpret_cast<const uint4*>(blk + (warp * kTileKeys + 32 * i + lane) * 16);
                 const uint32_t wd[4] = {x.x, x.y, x.z, x.w};
                 acc[i] = score_key(wd, colp);
             }
-            if (kb + 2 * kTileKeys <= nkeys && hp == PACK) {
+            if (kb + kTileKeys <= nkeys && hp == PACK) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) sc_out[kb + 32 * i + lane] = acc[i];
+                for (int i = 0; i < 2; ++i) sc_out[kb + 32 * i + lane] = acc[i];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) count_scores<PACK>(acc[i], cb, pitch);
+                for (int i = 0; i < 2; ++i) count_scores<PACK>(acc[i], cb, pitch);
             } else {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < 2; ++i) {
                     if (kb + 32 * i + lane < nkeys) {
                         sc_out[kb + 32 * i + lane] = acc[i];
                         if (hp == 4) count_scores<4>(acc[i], cb, pitch);
@@ -583,8 +603,8 @@ __device__ __forceinline__ void v_item(const SearchArgs& a, int p, int c, uint8_
 #pragma unroll
         for (int w = 0; w < kVW; ++w) {
             uint32_t* q = reinterpret_cast<uint32_t*>(
-                w < 4 ? smem + L.tab + (49 * w + sv) * 256 + 128 + 4 * lane
-                      : smem + L.h2 + (49 * (w - 4) + sv) * 128 + 4 * lane);
+                w < 4 ? smem + kOffTab + (49 * w + sv) * 256 + 128 + 4 * lane
+                      : smem + kOffH2 + (49 * (w - 4) + sv) * 128 + 4 * lane);
             const uint32_t x = *q;
             *q = 0u;
             lo += x & 0x00ff00ffu;
@@ -754,7 +774,7 @@ __device__ void f_item(const SearchArgs& a, int p, uint8_t* scr) {
         bar_v();
     }
     // the top-k's first radix level is counted by the rerank: start it at zero
-    for (int i = t; i < hp * kBins; i += kVT) a.shist[static_cast<int64_t>(head0) * kBins + i] = 0u;
+    for (int i = t; i < hp * kBins1; i += kVT) a.shist[static_cast<int64_t>(head0) * kBins1 + i] = 0u;
     __threadfence();
     bar_v();
     if (t == 0) st_release(pk(a, PK_F, p), 1);
@@ -966,10 +986,11 @@ __device__ void k_item(const SearchArgs& a, int head, uint8_t* kscr, uint32_t ks
     uint32_t lo = 0u, hi = 0xffffffffu;
     // finds, from each thread's BPT bins, the bin holding the krem-th largest value and
     // narrows [lo, hi] to it (every thread makes the same choice)
-    auto choose = [&](const uint32_t h[BPT], int sh) {
+    auto choose = [&](const auto& h, int sh) {
+        constexpr int NB = sizeof(h) / sizeof(h[0]);   // bins per thread
         uint32_t mine = 0;
 #pragma unroll
-        for (int j = 0; j < BPT; ++j) mine += h[j];
+        for (int j = 0; j < NB; ++j) mine += h[j];
         uint32_t x = mine;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -988,17 +1009,24 @@ __device__ void k_item(const SearchArgs& a, int head, uint8_t* kscr, uint32_t ks
             }
             if (lane < kVW) wb[lane] = y - tv;
         }
+        if (t == 0) pick[0] = 0xffffffffu;
         bar_v();
         uint32_t above = wb[warp] + x - mine;
 #pragma unroll
-        for (int j = BPT - 1; j >= 0; --j) {
+        for (int j = NB - 1; j >= 0; --j) {
             if (above < krem && krem <= above + h[j]) {
-                pick[0] = BPT * t + j;
+                pick[0] = NB * t + j;
                 pick[1] = above;
             }
             above += h[j];
         }
         bar_v();
+        if (pick[0] == 0xffffffffu) {   // the counts do not hold the k-th value: give up
+            if (t == 0) atomicExch(a.status, ST_BADINDEX);
+            lo = hi;
+            bar_v();
+            return;
+        }
         const uint32_t b = pick[0];
         krem -= pick[1];
         const uint32_t nlo = lo + (b << sh);
@@ -1007,18 +1035,21 @@ __device__ void k_item(const SearchArgs& a, int head, uint8_t* kscr, uint32_t ks
         hi = static_cast<uint32_t>(min(static_cast<uint64_t>(hi), bin_hi));
         bar_v();
     };
-    // 1. first level, counted by the rerank
+    // 1. first level, counted by the rerank (kBins1 bins of the top kBits1 bits)
     {
-        uint32_t h[BPT];
-        const uint32_t* hs = a.shist + static_cast<int64_t>(head) * kBins + BPT * t;
-        const uint4 v = ldcg_u128(hs), w = ldcg_u128(hs + 4);
-        h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
-        h[4] = w.x; h[5] = w.y; h[6] = w.z; h[7] = w.w;
-        choose(h, 32 - SBINS_BITS);
+        constexpr int NB1 = kBins1 / kVT;
+        uint32_t h[NB1];
+        const uint32_t* hs = a.shist + static_cast<int64_t>(head) * kBins1 + NB1 * t;
+#pragma unroll
+        for (int i = 0; i < NB1 / 4; ++i) {
+            const uint4 v = ldcg_u128(hs + 4 * i);
+            h[4 * i] = v.x; h[4 * i + 1] = v.y; h[4 * i + 2] = v.z; h[4 * i + 3] = v.w;
+        }
+        choose(h, 32 - kBits1);
     }
     // 2. radix levels until the k-th largest value is isolated
     bool listed = false;   // the list holds every value inside [lo, hi]
-    while (lo != hi) {
+    for (int level = 0; lo != hi && level < 4; ++level) {
         const uint32_t span = hi - lo;
         const int bitlen = 32 - __clz(span);
         const int sh = bitlen > 11 ? bitlen - 11 : 0;
@@ -1247,105 +1278,45 @@ __device__ __forceinline__ float score_record(const uint8_t* row, int sw, const 
     return S;
 }
 
-struct StageDesc {
-    int32_t head;   // query head, or -1
-    int32_t pos;    // first candidate
-    int32_t cnt;    // candidates in the stage
-    int32_t last;   // 1 when the stage ends its item
-};
-
-constexpr int kRdyWords = 32;   // per-CTA bitmap of pack-units whose compaction is complete
-
-// One rerank warp: claims items of 256 candidates of one query head, cuts them into stages
-// of 32, gathers each stage's records with 16-byte cp.async copies (eight lanes per record,
-// so one warp instruction moves four records) into a ring of kSlots stages, and scores one
-// record per lane. Exactly one copy group is committed per ring step, empty when nothing
-// could be issued (the next item's pack is not compacted yet), so the wait counts stay
-// fixed; the warp blocks on a pack only when no stage of its own is in flight.
+// ---------------------------------------------------------------------------------------
+// R: rerank of one range of up to kRItem candidates of one query head (whole CTA)
+// ---------------------------------------------------------------------------------------
+// Warp w takes the stages w, w + 8, ... of 32 candidates; each warp gathers its stages' records
+// with 16-byte cp.async copies (eight lanes per record, so one warp instruction moves four
+// records) into a ring of kSlots stages and scores one record per lane. Every value is also
+// counted, by the top 13 bits of its order-preserving image, into the head's first top-k
+// level (lanes with the same bin are grouped by a warp match; one global add per group).
 template <bool TABLE>
-__device__ void r_warp(const SearchArgs& a, uint8_t* smem, const Lay& L, const float* dec,
-                       unsigned* rdy, bool& aborted) {
-    const int warp = (threadIdx.x >> 5) - kVW, lane = threadIdx.x & 31;
-    uint8_t* ring = smem + L.ring + warp * kRingWarp;
-    float2* qs = reinterpret_cast<float2*>(smem + L.qry + warp * 512);
+__device__ void r_item(const SearchArgs& a, int head, int r, uint8_t* smem, const float* dec) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c0 = r * kRItem, c1 = min(a.C, c0 + kRItem);
+    const int nst = (c1 - c0 + kStage - 1) / kStage;
+    uint8_t* ring = smem + kOffRing + warp * kRingWarp;
+    float2* qs = reinterpret_cast<float2*>(smem + kOffQry);
     const uint64_t* qp = reinterpret_cast<const uint64_t*>(qs);
-    StageDesc* desc = reinterpret_cast<StageDesc*>(smem + L.desc + warp * kSlots * 16);
-    const int64_t nitems = static_cast<int64_t>(a.heads) * a.nrh;
-
-    int staged = -1;              // head whose query is in qs
-    int it_head = -1, it_pos = 0, it_end = 0;
-    bool exhausted = false, ready = false;
-    int inflight = 0;             // stages issued and not yet scored
-    int g = 0;                    // ring steps committed
-
-    auto claim = [&]() -> bool {  // next item into (it_head, it_pos, it_end); false when none
-        int it = 0;
-        if (lane == 0) it = atomicAdd(ctl(a, CT_RQ), 1);
-        it = __shfl_sync(0xffffffffu, it, 0);
-        if (it >= nitems) return false;
-        it_head = it / a.nrh;
-        const int r = it - it_head * a.nrh;
-        it_pos = r * kRItem;
-        it_end = min(a.C, it_pos + kRItem);
-        ready = false;
-        return true;
-    };
-    // Has the compaction of the item's pack-unit finished? (non-blocking unless `block`).
-    // Packs seen ready are remembered in the CTA's bitmap, so the warps of a CTA poll the
-    // global flag only until one of them has seen it.
-    auto pack_ready = [&](bool block) -> int {   // 1 ready, 0 not yet, -1 timed out
-        const int unit = it_head / a.G, gg = it_head - unit * a.G;
-        const int p = unit * a.packs + gg / PACK;
-        int ok = 0;
-        if (lane == 0) {
-            const bool cached = p < 32 * kRdyWords && ((rdy[p >> 5] >> (p & 31)) & 1u);
-            const int* f = pk(a, PK_C, p);
-            if (cached) {
-                ok = 1;
-            } else if (block) {
-                const uint64_t tw = a.trace ? gtime() : 0;
-                ok = wait_flag(f, a.nc, true, a.spin_limit, a.status, a.trace) ? 1 : -1;
-                if (a.trace) trace_add(a.trace, TR_RWAIT, tw, gtime());
-            } else {
-                ok = ld_relaxed(f) >= a.nc ? 1 : 0;
-                if (ok) __threadfence();
-            }
-            if (ok == 1 && !cached && p < 32 * kRdyWords) atomicOr(&rdy[p >> 5], 1u << (p & 31));
-        }
-        return __shfl_sync(0xffffffffu, ok, 0);
-    };
-    // commits one ring step: the next stage's copies, or an empty group
-    auto issue_next = [&]() {
-        const int slot = g % kSlots;
-        int head = -1, pos = 0, cnt = 0, last = 0;
-        while (!exhausted) {
-            if (it_head < 0 || it_pos >= it_end) {
-                if (!claim()) { exhausted = true; break; }
-            }
-            if (!ready) {
-                const int r = pack_ready(inflight == 0);
-                if (r < 0) { aborted = true; exhausted = true; break; }
-                if (r == 0) break;
-                ready = true;
-            }
-            head = it_head;
-            pos = it_pos;
-            cnt = min(kStage, it_end - it_pos);
-            last = pos + cnt >= it_end ? 1 : 0;
-            it_pos += cnt;
-            break;
-        }
-        if (head >= 0) {
-            const uint8_t* ubase = a.rec + static_cast<int64_t>(head / a.G) * a.cap_pad * REC;
+    if (threadIdx.x < 64) {   // the head's rotated query as (subspace 2t, 2t + 1) pairs
+        const float* qh = a.qt + static_cast<int64_t>(head) * D;
+        const int tt = threadIdx.x >> 3, j = threadIdx.x & 7;
+        qs[threadIdx.x] = make_float2(ldcg_f32(qh + 16 * tt + j), ldcg_f32(qh + 16 * tt + 8 + j));
+    }
+    bar_v();
+    const uint8_t* ubase = a.rec + static_cast<int64_t>(head / a.G) * a.cap_pad * REC;
+    const int32_t* cbase = a.cand + static_cast<int64_t>(head) * a.cmax;
+    const int nmine = nst > warp ? (nst - warp + kW - 1) / kW : 0;   // this warp's stages
+    // commits one ring step: the copies of this warp's k-th stage, or an empty group
+    auto issue = [&](int k) {
+        if (k < nmine) {
+            const int pos = c0 + (warp + kW * k) * kStage;
+            const int cnt = min(kStage, c1 - pos);
             uint32_t idx = 0xffffffffu;
             if (lane < cnt) {
-                idx = static_cast<uint32_t>(ldcg_i32(a.cand + static_cast<int64_t>(head) * a.cmax + pos + lane));
+                idx = static_cast<uint32_t>(ldcg_i32(cbase + pos + lane));
                 if (idx >= static_cast<uint64_t>(a.n)) {
                     atomicExch(a.status, ST_BADINDEX);   // never taken when selection is consistent
                     idx = 0xffffffffu;
                 }
             }
-            uint8_t* dst0 = ring + slot * (kStage * REC);
+            uint8_t* dst0 = ring + (k % kSlots) * (kStage * REC);
             const int piece = lane & 7, sub = lane >> 3;
 #pragma unroll
             for (int j = 0; j < kStage / 4; ++j) {
@@ -1357,183 +1328,191 @@ __device__ void r_warp(const SearchArgs& a, uint8_t* smem, const Lay& L, const f
                     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(srcp) : "memory");
                 }
             }
-            ++inflight;
         }
-        if (lane == 0) desc[slot] = StageDesc{head, pos, cnt, last};
         asm volatile("cp.async.commit_group;" ::: "memory");
-        ++g;
     };
-
-    const uint64_t tr0 = a.trace ? gtime() : 0;
-    for (int i = 0; i < kSlots; ++i) issue_next();
-    for (int sg = 0;; ++sg) {
-        if (inflight == 0 && exhausted) break;
+    for (int k = 0; k < kSlots; ++k) issue(k);
+    for (int k = 0; k < nmine; ++k) {
         asm volatile("cp.async.wait_group %0;" :: "n"(kSlots - 1) : "memory");
         __syncwarp();
-        const int slot = sg % kSlots;
-        const StageDesc d = desc[slot];
-        if (d.head >= 0) {
-            if (d.head != staged) {
-                const float* qh = a.qt + static_cast<int64_t>(d.head) * D;
-#pragma unroll
-                for (int e = lane; e < 64; e += 32) {
-                    const int tt = e >> 3, j = e & 7;
-                    qs[e] = make_float2(ldcg_f32(qh + 16 * tt + j), ldcg_f32(qh + 16 * tt + 8 + j));
-                }
-                __syncwarp();
-                staged = d.head;
-            }
-            if (lane < d.cnt) {
-                const DecodeConsts dc = decode_consts();
-                const float sv = score_record<TABLE>(ring + slot * (kStage * REC) + lane * REC, lane & 7, qp, dec, dc);
-                a.S[static_cast<int64_t>(d.head) * a.cmax + d.pos + lane] = sv;
-                const uint32_t bin = order_key(sv) >> (32 - SBINS_BITS);
-                const uint32_t peers = __match_any_sync(__activemask(), bin);
-                if (lane == __ffs(peers) - 1)
-                    atomicAdd(&a.shist[static_cast<int64_t>(d.head) * kBins + bin], static_cast<uint32_t>(__popc(peers)));
-            }
-            --inflight;
-            if (d.last) {
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) {
-                    const int unit = d.head / a.G, gg = d.head - unit * a.G;
-                    atomicAdd(pk(a, PK_R, unit * a.packs + gg / PACK), 1);
-                }
-            }
+        const int pos = c0 + (warp + kW * k) * kStage;
+        const int cnt = min(kStage, c1 - pos);
+        if (lane < cnt) {
+            const DecodeConsts dc = decode_consts();
+            const float sv = score_record<TABLE>(ring + (k % kSlots) * (kStage * REC) + lane * REC,
+                                                 lane & 7, qp, dec, dc);
+            a.S[static_cast<int64_t>(head) * a.cmax + pos + lane] = sv;
+            const uint32_t bin = order_key(sv) >> (32 - kBits1);
+            const uint32_t peers = __match_any_sync(__activemask(), bin);
+            if (lane == __ffs(peers) - 1)
+                atomicAdd(&a.shist[static_cast<int64_t>(head) * kBins1 + bin],
+                          static_cast<uint32_t>(__popc(peers)));
         }
-        __syncwarp();   // every lane has read the slot and the query
-        issue_next();
+        __syncwarp();   // every lane has read the slot
+        issue(k + kSlots);
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");   // no copy in flight at exit
-    if (a.trace && lane == 0) trace_add(a.trace, TR_R, tr0, gtime());
+    asm volatile("cp.async.wait_all;" ::: "memory");   // no copy in flight past the item
+    __threadfence();
+    bar_v();
+    if (threadIdx.x == 0) {
+        const int unit = head / a.G, g = head - unit * a.G;
+        atomicAdd(pk(a, PK_R, unit * a.packs + g / PACK), 1);
+    }
 }
+
+}  // namespace
 
 // ---------------------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------------------
+namespace {
+
+// Progress board checkpoints (debugging aid): threads 1, 32, 224 and 0 report 100 * (loop
+// iteration) + checkpoint into words 4..7 of their CTA's board entry.
+__device__ __forceinline__ void mark(const SearchArgs& a, int iter, int v) {
+    if (!a.progress) return;
+    const int t = threadIdx.x;
+    const int slot = t == 0 ? 7 : t == 1 ? 4 : t == 32 ? 5 : t == 224 ? 6 : -1;
+    if (slot >= 0) reinterpret_cast<volatile int*>(a.progress)[8 * blockIdx.x + slot] = 100 * iter + v;
+}
+
 template <bool TABLE>
-__global__ void __launch_bounds__(kThreads, 1) search_kernel(const SearchArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) search_kernel(const SearchArgs a) {
     uint8_t* smem = g_smem;
-    const Lay L = make_lay(smem_addr(g_smem));
     __shared__ float dec[16];
-    __shared__ int vbuf[4];      // vote group: claimed item, abort flag
-    __shared__ unsigned rdy[kRdyWords];
+    __shared__ int vbuf[4];      // claimed item (type, x, y), abort flag
+    __shared__ __align__(8) uint64_t vbar[kVSlots];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x < 16) dec[threadIdx.x] = TABLE ? a.lvt[16 + threadIdx.x] : 0.0f;
-    // byte-histogram counters start at zero; rerank rings get their barriers
-    if (smem_addr(g_smem) > kMaxBase) {   // the layout needs the table's 64 KB page
-        if (threadIdx.x == 0) atomicExch(a.status, ST_BADINDEX);
-        return;
-    }
-    for (int i = threadIdx.x; i < 256 * 8; i += kThreads)   // upper halves of the table rows
-        *reinterpret_cast<uint4*>(smem + L.tab + (i >> 3) * 256 + 128 + 16 * (i & 7)) =
-            make_uint4(0, 0, 0, 0);
-    for (int i = threadIdx.x; i < static_cast<int>(kH2Bytes / 16); i += kThreads)
-        reinterpret_cast<uint4*>(smem + L.h2)[i] = make_uint4(0, 0, 0, 0);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kVSlots; ++s) mbar_init(smem_addr(smem + L.vbar + 8 * s), 1);
+        vbuf[3] = 0;
+        for (int s = 0; s < kVSlots; ++s) mbar_init(smem_addr(&vbar[s]), 1);
         mbar_fence_init();
     }
-    if (threadIdx.x == 0) vbuf[1] = 0;
-    if (threadIdx.x < kRdyWords) rdy[threadIdx.x] = 0u;
     const uint64_t tk0 = a.trace ? gtime() : 0;
     __syncthreads();
 
-    if (warp < kVW) {
-        // ---------------- vote group ----------------
-        uint32_t colp[6];
+    // per-lane address parts of the vote lookups: at step t lane L reads subspace
+    // (t + L / 2) mod 16 of both its keys (the encoder rotates key i's bytes by (i / 2) mod
+    // 16), in copy L mod 2, which owns bank column 2 * subspace + copy; three columns per
+    // register with a zero top byte, so one PRMT builds an address
+    uint32_t colp[6];
 #pragma unroll
-        for (int r = 0; r < 6; ++r) {
-            uint32_t w = 0;
+    for (int r = 0; r < 6; ++r) {
+        uint32_t w = 0;
 #pragma unroll
-            for (int j = 0; j < 3; ++j) {
-                const int tt = 3 * r + j;
-                if (tt < 16) w |= (4u * (2u * ((tt + (lane >> 1)) & 15) + (lane & 1))) << (8 * j);
-            }
-            colp[r] = w | (L.hi << 24);   // top byte: the table's 64 KB page
+        for (int j = 0; j < 3; ++j) {
+            const int tt = 3 * r + j;
+            if (tt < 16) w |= (4u * (2u * ((tt + (lane >> 1)) & 15) + (lane & 1))) << (8 * j);
         }
-        int cur_table = -1;     // pack-unit whose vote table is in the table area
-        VRing vr{smem_addr(smem + L.vbar), 0};
-        uint8_t* scr = smem + kOffScr;
-        for (;;) {
-            uint64_t tw = 0;
-            if (threadIdx.x == 0) {
-                const int it = atomicAdd(ctl(a, CT_VQ), 1);
-                const VItem vi = vqueue_item(it, a.P, a.nc, a.heads);
-                vbuf[0] = vi.type;
-                vbuf[2] = vi.x;
-                vbuf[3] = vi.y;
-                if (a.trace) tw = gtime();
-                bool ok = true;
-                if (vi.type == IT_V && vi.x != cur_table)
-                    ok = wait_flag(pk(a, PK_Q, vi.x), min(PACK, a.G - (vi.x % a.packs) * PACK),
-                                   true, a.spin_limit, a.status, a.trace);
-                else if (vi.type == IT_C)
-                    ok = wait_flag(pk(a, PK_F, vi.x), 1, false, a.spin_limit, a.status, a.trace);
-                else if (vi.type == IT_K) {
-                    const int unit = vi.x / a.G, g = vi.x - unit * a.G;
-                    const int p = unit * a.packs + g / PACK;
-                    const int hp = min(PACK, a.G - (g / PACK) * PACK);
-                    ok = wait_flag(pk(a, PK_R, p), hp * a.nrh, true,
-                                   a.spin_limit, a.status, a.trace);
-                }
-                if (!ok) vbuf[1] = 1;
-                if (a.trace && vi.type != IT_NONE) trace_add(a.trace, TR_VWAIT, tw, gtime());
-            }
-            bar_v();
-            const int type = vbuf[0], x = vbuf[2], y = vbuf[3];
-            if (type == IT_NONE || vbuf[1]) break;
-            const uint64_t t0 = a.trace ? gtime() : 0;
-            if (type == IT_Q) {
-                q_item(a, x, scr);
-            } else if (type == IT_V) {
-                if (x != cur_table) {
-                    load_table(a, x, smem + L.tab);
-                    cur_table = x;
-                    bar_v();
-                }
-                v_item(a, x, y, smem, L, colp, vr);
-                __threadfence();
-                bar_v();
-                if (threadIdx.x == 0) {
-                    vbuf[2] = atomicAdd(pk(a, PK_V, x), 1);
-                    __threadfence();   // the other vote items' histograms are visible after this
-                }
-                bar_v();
-                if (vbuf[2] == a.nc - 1) {
-                    if (a.trace && threadIdx.x == 0) trace_add(a.trace, TR_V, t0, gtime());
-                    const uint64_t t1 = a.trace ? gtime() : 0;
-                    f_item(a, x, scr);
-                    if (a.trace && threadIdx.x == 0) trace_add(a.trace, TR_F, t1, gtime());
-                    bar_v();
-                    continue;
-                }
-            } else if (type == IT_C) {
-                c_item(a, x, y, scr);
-            } else {
-                k_item(a, x, smem, L.ring);
-                cur_table = -1;   // the table area was scratch
-            }
-            if (a.trace && threadIdx.x == 0) trace_add(a.trace, type, t0, gtime());
-            bar_v();
-        }
-    } else {
-        // ---------------- rerank warps ----------------
-        bool aborted = false;
-        r_warp<TABLE>(a, smem, L, dec, rdy, aborted);
+        colp[r] = w;
     }
-
+    int cur_table = -1;          // pack-unit whose vote table is in shared memory
+    bool counters_clean = false; // the vote counters are zero (cleared lazily)
+    VRing vr{smem_addr(&vbar[0]), 0};
+    uint8_t* scr = smem + kOffScr;
+    for (int iter = 0;; ++iter) {
+        mark(a, iter, 1);
+        if (threadIdx.x == 0) {
+            const int64_t it = atomicAdd(ctl(a, CT_Q), 1);
+            const Item vi = queue_item(a, it);
+            vbuf[0] = vi.type;
+            vbuf[1] = vi.x;
+            vbuf[2] = vi.y;
+            const uint64_t tw = a.trace ? gtime() : 0;
+            bool ok = true;
+            if (vi.type == IT_V && vi.x != cur_table) {
+                ok = wait_flag(pk(a, PK_Q, vi.x), heads_of(a, vi.x), true, a.spin_limit, a.status, a.trace, a.ctrl);
+            } else if (vi.type == IT_C) {
+                ok = wait_flag(pk(a, PK_F, vi.x), 1, false, a.spin_limit, a.status, a.trace, a.ctrl);
+            } else if (vi.type == IT_R || vi.type == IT_K) {
+                const int unit = vi.x / a.G, g = vi.x - unit * a.G;
+                const int p = unit * a.packs + g / PACK;
+                ok = vi.type == IT_R
+                         ? wait_flag(pk(a, PK_C, p), a.nc, true, a.spin_limit, a.status, a.trace, a.ctrl)
+                         : wait_flag(pk(a, PK_R, p), heads_of(a, p) * a.nrh, true, a.spin_limit,
+                                     a.status, a.trace, a.ctrl);
+            }
+            if (!ok) vbuf[3] = 1;
+            if (a.progress) {
+                volatile int* pb = a.progress + 8 * blockIdx.x;
+                pb[0] = static_cast<int>(it); pb[1] = vi.type; pb[2] = vi.x; pb[3] = ok ? 1 : -1;
+            }
+            if (a.trace && vi.type != IT_NONE)
+                trace_add(a.trace, vi.type == IT_R ? TR_RWAIT : TR_VWAIT, tw, gtime());
+        }
+        __syncwarp();
+        bar_v();
+        mark(a, iter, 2);
+        const int type = vbuf[0], x = vbuf[1], y = vbuf[2];
+        if (type == IT_NONE || vbuf[3]) break;
+        const uint64_t t0 = a.trace ? gtime() : 0;
+        if (type == IT_Q) {
+            q_item(a, x, scr);
+        } else if (type == IT_V) {
+            if (!counters_clean) {
+                for (int i = threadIdx.x; i < 256 * 8; i += kThreads)   // upper halves of the table rows
+                    *reinterpret_cast<uint4*>(smem + kOffTab + (i >> 3) * 256 + 128 + 16 * (i & 7)) =
+                        make_uint4(0, 0, 0, 0);
+                for (int i = threadIdx.x; i < static_cast<int>(kH2Bytes / 16); i += kThreads)
+                    reinterpret_cast<uint4*>(smem + kOffH2)[i] = make_uint4(0, 0, 0, 0);
+                counters_clean = true;
+            }
+            if (x != cur_table) {
+                bar_v();
+                load_table(a, x, smem + kOffTab);
+                cur_table = x;
+            }
+            bar_v();
+            mark(a, iter, 5);
+            v_item(a, x, y, smem, colp, vr);
+            mark(a, iter, 6);
+            __threadfence();
+            bar_v();
+            if (threadIdx.x == 0) {
+                vbuf[2] = atomicAdd(pk(a, PK_V, x), 1);
+                __threadfence();   // the other vote items' histograms are visible after this
+            }
+            bar_v();
+            mark(a, iter, 7);
+            if (vbuf[2] == a.nc - 1) {
+                if (a.trace && threadIdx.x == 0) trace_add(a.trace, TR_V, t0, gtime());
+                const uint64_t t1 = a.trace ? gtime() : 0;
+                f_item(a, x, scr);
+                mark(a, iter, 8);
+                if (a.trace && threadIdx.x == 0) trace_add(a.trace, TR_F, t1, gtime());
+                bar_v();
+                continue;
+            }
+        } else if (type == IT_C) {
+            c_item(a, x, y, scr);
+        } else if (type == IT_R) {
+            r_item<TABLE>(a, x, y, smem, dec);
+            counters_clean = false;
+            cur_table = -1;
+        } else {
+            k_item(a, x, smem, kSmem);
+            counters_clean = false;
+            cur_table = -1;
+        }
+        if (a.trace && threadIdx.x == 0)
+            trace_add(a.trace, type == IT_R ? TR_R : type, t0, gtime());
+        if (a.progress && threadIdx.x == 0) reinterpret_cast<volatile int*>(a.progress)[8 * blockIdx.x + 3] = 2;
+        mark(a, iter, 9);
+        bar_v();
+    }
+    mark(a, 99, 3);
     __syncthreads();
+    mark(a, 99, 4);
     if (threadIdx.x == 0) {
+        if (a.progress) reinterpret_cast<volatile int*>(a.progress)[8 * blockIdx.x + 3] = 3;
         if (a.trace) trace_add(a.trace, TR_KERNEL, tk0, gtime());
         __threadfence();
         const int done = atomicAdd(ctl(a, CT_EXIT), 1);
         if (done == static_cast<int>(gridDim.x) - 1) {
-            // the last CTA out resets the queues and counters for the next search
-            *ctl(a, CT_VQ) = 0;
-            *ctl(a, CT_RQ) = 0;
+            // the last CTA out resets the queue and the per-pack counters for the next search
+            *ctl(a, CT_Q) = 0;
             for (int i = 0; i < PK_N * a.P; ++i) *ctl(a, CT_HDR + i) = 0;
             __threadfence();
             *ctl(a, CT_EXIT) = 0;
@@ -1572,6 +1551,7 @@ cudaError_t launch_search(pariskv_index* ix, const void* q, const float* qt_in,
     a.hist = ix->hist; a.thr = ix->thr; a.cbase = ix->cbase; a.cand = ix->cand; a.S = ix->S;
     a.shist = ix->shist; a.topk_idx = topk_idx; a.topk_est = topk_est;
     a.ctrl = ix->ctrl; a.status = ix->status; a.trace = ix->profile ? ix->trace : nullptr;
+    a.progress = ix->progress;
     a.n = ix->n; a.cap_pad = ix->cap_pad; a.cmax = ix->cmax;
     a.spin_limit = ix->spin_limit;
     a.units = ix->units; a.G = c.group; a.packs = ix->packs; a.P = P; a.nc = nc;
@@ -1584,7 +1564,7 @@ cudaError_t launch_search(pariskv_index* ix, const void* q, const float* qt_in,
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(sms));
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * sms));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmem;
     cfg.stream = st;

@@ -96,6 +96,8 @@ _SIGS = {
     "pariskv_debug_profile": (_S, [_P, _I32]),
     "pariskv_debug_stage_ms": (_S, [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_I32)]),
     "pariskv_debug_search_phases": (_S, [_P, ctypes.POINTER(ctypes.c_double)]),
+    "pariskv_debug_set_wait_limit": (_S, [_P, ctypes.c_int64]),
+    "pariskv_debug_set_progress": (_S, [_P, _P]),
     "pariskv_debug_read_stream": (_S, [_P, _I64, _P, _P]),
     "pariskv_cache_create": (_S, [ctypes.POINTER(Config), ctypes.POINTER(CacheConfig), _P, _P,
                                   ctypes.POINTER(_P)]),
@@ -260,6 +262,15 @@ class Index:
         _check(lib.pariskv_debug_stage_ms(self.handle, ms, ctypes.byref(n)),
                "pariskv_debug_stage_ms")
         return {STAGES[i]: float(ms[i]) for i in range(n.value)}
+
+    def set_progress(self, board) -> None:
+        """Per-CTA item board (a pinned host int32 tensor of 4 x 2 x SMs), or None."""
+        _check(lib.pariskv_debug_set_progress(self.handle, None if board is None else board.data_ptr()),
+               "pariskv_debug_set_progress")
+
+    def set_wait_limit(self, cycles: int) -> None:
+        """Bounds the device-side waits of later searches (0 restores the default)."""
+        _check(lib.pariskv_debug_set_wait_limit(self.handle, int(cycles)), "pariskv_debug_set_wait_limit")
 
     def search_phases(self) -> dict:
         """Per kind of work of the last profiled search: first start, last end (us after the
