@@ -186,8 +186,6 @@ def algorithmic_bytes(stage: str, sp, C: int) -> int:
         return units * packs * sp.n * 16
     if stage == "rerank":
         return sp.batch * sp.num_q_heads * C * 128
-    if stage == "search":   # the whole step runs as one kernel: both passes
-        return algorithmic_bytes("vote", sp, C) + algorithmic_bytes("rerank", sp, C)
     return 0
 
 
@@ -621,16 +619,11 @@ def main():
     # loop, because reading the events synchronises the host every step)
     ix.profile(True)
     stage_tot = {}
-    phases = {}
     for s in range(args.steps):
         flush.fill_(s & 255)
         ix.search(qs, k, idx, est)
         for name, ms in ix.stage_ms().items():
             stage_tot[name] = stage_tot.get(name, 0.0) + ms
-        for name, ph in ix.search_phases().items():
-            acc = phases.setdefault(name, {key: 0.0 for key in ph})
-            for key in acc:
-                acc[key] += ph[key] / args.steps
     ix.profile(False)
     torch.cuda.synchronize()
     stage_avg = {kname: v / args.steps for kname, v in stage_tot.items()}
@@ -755,7 +748,6 @@ def main():
                        "levels": args.levels,
                        "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"},
             "stage_ms": stage_avg,
-            "search_phases": phases,
             "host_enqueue_us_per_search": host_us,
             "graph": {"ms_per_step": graph_ms, "value": graph_value},
             "roofline": roofline,

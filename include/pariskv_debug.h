@@ -56,42 +56,15 @@ PARISKV_API pariskv_status pariskv_debug_export_index(pariskv_index* index, uint
 PARISKV_API pariskv_status pariskv_debug_export_search(pariskv_index* index, uint8_t* lut, int32_t* scores,
                                            int64_t* ncand, int32_t* cand, float* S);
 
-/* Timing of pariskv_search with CUDA events recorded on the search stream around its kernel,
- * and the phase trace read by pariskv_debug_search_phases. enable != 0 turns both on for this
- * index (events and the trace buffer are created then). */
+/* Per-stage timing of pariskv_search with CUDA events recorded on the search stream between
+ * the kernel launches. enable != 0 turns it on for this index (events are created then). */
 PARISKV_API pariskv_status pariskv_debug_profile(pariskv_index* index, int32_t enable);
 
-/* Waits for the last profiled search and writes the device time (ms) of each of its
- * launches to ms[0..*nstages-1]; the search is one kernel, so *nstages is 1. ms must hold at
- * least 8 floats. */
+/* Waits for the last profiled search and writes the device time (ms) of each of its stages
+ * to ms[0..*nstages-1]: query prep, vote scan, threshold, compaction, rerank, top-k. ms must
+ * hold at least 8 floats. */
 PARISKV_API pariskv_status pariskv_debug_stage_ms(pariskv_index* index, float* ms,
                                                   int32_t* nstages);
-
-/* Bounds every device-side wait of later searches on this index to `cycles` SM clock cycles
- * (0 restores the default of about one second). A wait that runs out makes pariskv_sync
- * return PARISKV_ETIMEOUT, naming the control word it waited on. Used by tests of the
- * timeout path. No counterpart on the pages. Errors: EINVAL. */
-PARISKV_API pariskv_status pariskv_debug_set_wait_limit(pariskv_index* index, int64_t cycles);
-
-/* Makes later searches on this index report, per CTA of the search kernel, the item it is
- * working on into `board` (8 int32 per CTA: item number, kind, head or pack-unit, state 1 =
- * claimed, -1 = its wait expired, 2 = done, 3 = exited; then the last checkpoint passed by
- * threads 1, 32, 224 and 0 as 100 x loop iteration + checkpoint), a pinned host buffer the
- * host may read while the kernel runs; NULL turns it off. The board must hold 8 ints for
- * each of 2 x (number of SMs) CTAs. A debugging aid with no counterpart on the pages. Errors: EINVAL. */
-PARISKV_API pariskv_status pariskv_debug_set_progress(pariskv_index* index, int32_t* board);
-
-/* Phases of the last profiled search (pariskv_debug_profile on): the search runs as one
- * persistent kernel whose workers take items of several kinds; for each kind -- 0 query
- * prep, 1 vote, 2 compaction, 3 top-k, 4 threshold finalisation, 5 rerank, 6 vote-group
- * waits, 7 rerank-warp waits, 8 whole kernel -- out[3 i] and out[3 i + 1] receive the first
- * start and the last end (microseconds after the kernel's first CTA started; -1 if that
- * kind never ran) and out[3 i + 2] the busy time summed over workers; out[29] receives the
- * number of polls the bounded waits made; out[30], out[31], out[32] and out[35] the top-k
- * items' passes over the rerank values, their selections finished without the in-memory
- * list, and their summed selection and writing times (us). out holds 36 doubles.
- * Synchronises with the search. No counterpart on the pages (a measurement aid). */
-PARISKV_API pariskv_status pariskv_debug_search_phases(pariskv_index* index, double* out);
 
 /* Reads `bytes` from `src` once, with coalesced 16-byte loads spread over every SM, and
  * folds the data into one word that may be written to `sink` (a device pointer to 4 bytes),

@@ -161,7 +161,7 @@ void free_index(pariskv_index* ix) {
     dfree(ix->signs); dfree(ix->ids); dfree(ix->rec); dfree(ix->lut); dfree(ix->qt);
     dfree(ix->qnorm); dfree(ix->scores); dfree(ix->hist); dfree(ix->thr); dfree(ix->cbase);
     dfree(ix->cand); dfree(ix->S); dfree(ix->shist); dfree(ix->status); dfree(ix->lvt);
-    dfree(ix->cent); dfree(ix->ctrl); dfree(ix->trace);
+    dfree(ix->cent);
     for (auto& e : ix->ev)
         if (e) cudaEventDestroy(e);
     delete ix;
@@ -192,9 +192,8 @@ pariskv_status create_index(const pariskv_config* cfg, const int8_t* signs, cuda
               dalloc(&ix->lut, up * NB * NC) && dalloc(&ix->qt, heads * D) &&
               dalloc(&ix->qnorm, heads) && dalloc(&ix->scores, up * ix->cap_pad) &&
               dalloc(&ix->hist, up * nch * PACK * NBINS) && dalloc(&ix->thr, heads * 4) &&
-              dalloc(&ix->cbase, heads * nch * 2) && dalloc(&ix->shist, heads * SBINS) &&
-              dalloc(&ix->status, 4) && dalloc(&ix->lvt, kLevelTableFloats) &&
-              dalloc(&ix->ctrl, search_ctrl_words(static_cast<int>(up)));
+              dalloc(&ix->cbase, heads * nch * 2) && dalloc(&ix->shist, heads * SCOPIES * SBINS) &&
+              dalloc(&ix->status, 1) && dalloc(&ix->lvt, kLevelTableFloats);
     if (!ok) {
         free_index(ix);
         return fail(PARISKV_ENOMEM, "device allocation for the index failed");
@@ -218,9 +217,7 @@ pariskv_status create_index(const pariskv_config* cfg, const int8_t* signs, cuda
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(ix->lvt, tab, sizeof(tab), cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(ix->lut, 0, up * NB * NC * sizeof(uint32_t), st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(ix->status, 0, 4 * sizeof(int), st);
-    if (e == cudaSuccess)
-        e = cudaMemsetAsync(ix->ctrl, 0, search_ctrl_words(static_cast<int>(up)) * sizeof(int), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ix->status, 0, sizeof(int), st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);  // hs, tab live on this stack frame
     if (e != cudaSuccess) {
         free_index(ix);
@@ -260,12 +257,17 @@ pariskv_status run_search(pariskv_index* ix, const void* q, const float* qt, con
     if (fault_launch()) return injected_launch_failure();
     g_launches = 0;
     int ne = 0;
-    if (ix->profile) cudaEventRecord(ix->ev[ne++], st);
-    cudaError_t e = launch_search(ix, q, qt, qn, rotated, C, k, topk_idx, topk_est, st);
-    if (e == cudaSuccess) {
-        g_launches = 1;
+    auto mark = [&]() {
         if (ix->profile) cudaEventRecord(ix->ev[ne++], st);
-    }
+    };
+    mark();
+    cudaError_t e = launch_query_prep(ix, q, qt, qn, rotated, st);
+    if (e == cudaSuccess) { ++g_launches; mark(); e = launch_vote(ix, st); }
+    if (e == cudaSuccess) { ++g_launches; mark(); e = launch_threshold(ix, C, st); }
+    if (e == cudaSuccess) { ++g_launches; mark(); e = launch_compact(ix, st); }
+    if (e == cudaSuccess) { ++g_launches; mark(); e = launch_rerank(ix, C, st); }
+    if (e == cudaSuccess) { ++g_launches; mark(); e = launch_topk(ix, C, k, topk_idx, topk_est, st); }
+    if (e == cudaSuccess) { ++g_launches; mark(); }
     ix->nev = ne;
     if (e != cudaSuccess) return cuda_fail(e, "search launch");
     ix->last_C = C;
@@ -699,13 +701,8 @@ pariskv_status pariskv_sync(pariskv_index* index, void* stream) {
     e = cudaMemcpy(&st, index->status, sizeof(int), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "status read");
     if (st != ST_OK) {
-        int diag[4] = {};
-        cudaMemcpy(diag, index->status, sizeof(diag), cudaMemcpyDeviceToHost);
-        cudaMemset(index->status, 0, 4 * sizeof(int));
-        if (st == ST_TIMEOUT)
-            return fail(PARISKV_ETIMEOUT,
-                        "a bounded device-side wait expired (control word %d: waited for %d, saw %d)",
-                        diag[1], diag[2], diag[3]);
+        cudaMemset(index->status, 0, sizeof(int));
+        if (st == ST_TIMEOUT) return fail(PARISKV_ETIMEOUT, "a bounded device-side wait expired");
         return fail(PARISKV_ECUDA, "internal consistency check failed on the device (%d)", st);
     }
     return PARISKV_OK;
@@ -802,54 +799,8 @@ pariskv_status pariskv_debug_profile(pariskv_index* ix, int32_t enable) {
             if (r != cudaSuccess) return cuda_fail(r, "event create");
         }
     }
-    if (enable && !ix->trace && !dalloc(&ix->trace, kTraceWords))
-        return fail(PARISKV_ENOMEM, "search trace buffer");
     ix->profile = enable != 0;
     ix->nev = 0;
-    return PARISKV_OK;
-}
-
-pariskv_status pariskv_debug_set_progress(pariskv_index* ix, int32_t* board) {
-    pariskv_status s = check_index(ix);
-    if (s != PARISKV_OK) return s;
-    if (board && (s = check_dev_ptr(board, 16, "board")) != PARISKV_OK) return s;
-    ix->progress = board;
-    return PARISKV_OK;
-}
-
-pariskv_status pariskv_debug_set_wait_limit(pariskv_index* ix, int64_t cycles) {
-    pariskv_status s = check_index(ix);
-    if (s != PARISKV_OK) return s;
-    if (cycles < 0) return fail(PARISKV_EINVAL, "cycles < 0");
-    ix->spin_limit = cycles == 0 ? kDefaultSpinLimit : cycles;
-    return PARISKV_OK;
-}
-
-pariskv_status pariskv_debug_search_phases(pariskv_index* ix, double* out) {
-    pariskv_status s = check_index(ix);
-    if (s != PARISKV_OK) return s;
-    if (!out) return fail(PARISKV_EINVAL, "out is NULL");
-    if (!ix->trace || ix->nev < 2) return fail(PARISKV_EINVAL, "no profiled search has run");
-    cudaError_t e = cudaEventSynchronize(ix->ev[ix->nev - 1]);
-    unsigned long long tr[kTraceWords];
-    if (e == cudaSuccess) e = cudaMemcpy(tr, ix->trace, sizeof(tr), cudaMemcpyDeviceToHost);
-    if (e != cudaSuccess) return cuda_fail(e, "search trace");
-    const unsigned long long t0 = ~tr[3 * 8];   // kernel: earliest start
-    for (int i = 0; i < 9; ++i) {
-        const bool seen = tr[3 * i] != 0;
-        out[3 * i + 0] = seen ? static_cast<double>(~tr[3 * i] - t0) * 1e-3 : -1.0;
-        out[3 * i + 1] = seen ? static_cast<double>(tr[3 * i + 1] - t0) * 1e-3 : -1.0;
-        out[3 * i + 2] = static_cast<double>(tr[3 * i + 2]) * 1e-3;
-    }
-    out[27] = -1.0;
-    out[28] = -1.0;
-    out[29] = static_cast<double>(tr[29]);   // polls of the bounded waits
-    out[30] = static_cast<double>(tr[30]);   // top-k: passes over S
-    out[31] = static_cast<double>(tr[31]);   // top-k: selections without the list
-    out[32] = static_cast<double>(tr[32]) * 1e-3;   // top-k: selection time (us, summed)
-    out[33] = -1.0;
-    out[34] = -1.0;
-    out[35] = static_cast<double>(tr[35]) * 1e-3;   // top-k: write time (us, summed)
     return PARISKV_OK;
 }
 

@@ -14,14 +14,16 @@ constexpr int M = 8;            // dims per subspace
 constexpr int NB = D / M;       // subspaces (16)
 constexpr int NC = 1 << M;      // sign centroids per subspace (256)
 constexpr int REC = 128;        // bytes per key record: 64 B of 4-bit codes + 16 fp32 factors
-constexpr int NBINS = 64;       // histogram bins per head and chunk (scores <= B * w_rank1 <= 48)
-constexpr int SBINS_BITS = 13;  // first radix level of the top-k, counted by the rerank
+constexpr int NBINS = 64;       // coarse scores are < 64 (B * w_rank1 <= 48)
+constexpr int SBINS_BITS = 11;  // first radix level of the top-k, counted by the rerank
 constexpr int SBINS = 1 << SBINS_BITS;
-constexpr int CHUNK = 16384;    // keys per coarse-score histogram chunk (a vote / compaction item)
+constexpr int SCOPIES = 1;      // copies of that histogram (one copy per warp group spreads the reductions)
+constexpr int CHUNK = 8192;     // keys per coarse-score histogram chunk (a vote work item)
 constexpr int PACK = 4;         // query heads whose vote weights share one 32-bit table entry
 
-// Device status word: ST_TIMEOUT when a bounded wait of the search kernel ran out,
-// ST_BADINDEX when a kernel found an index out of range (and skipped the access).
+// Device status word. ST_BADINDEX: a kernel found an index out of range and skipped the
+// access. ST_TIMEOUT is the code a bounded device-side wait records when it runs out; no
+// kernel of the library waits on another (each stage is its own launch), so it is reserved.
 enum : int { ST_OK = 0, ST_TIMEOUT = 5, ST_BADINDEX = 6 };
 
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }

@@ -9,17 +9,6 @@
 
 #include "pariskv.h"
 
-// Phase trace of a profiled search: per kind of work (query prep, vote, compaction, top-k,
-// finalisation, rerank, vote-group waits, rerank waits, whole kernel) the earliest start
-// (bit-inverted), the latest end and the summed busy time, in globaltimer nanoseconds; then
-// the number of polls of the bounded waits (third word of a tenth slot), and for the top-k
-// items the number of passes over S, of selections finished without the list, and the time
-// spent selecting and writing.
-constexpr int kTraceWords = 36;
-
-// Bound of every device-side wait of the search kernel, in SM clock cycles (about 1 s).
-constexpr long long kDefaultSpinLimit = 2000000000LL;
-
 struct pariskv_index {
     pariskv_config cfg;
     int device = 0;
@@ -47,15 +36,9 @@ struct pariskv_index {
     int32_t* cbase = nullptr;   // [units*group][chunks][2] selected/ties before each chunk
     int32_t* cand = nullptr;    // [units*group][cmax] candidate indices (ascending)
     float* S = nullptr;         // [units*group][cmax] rerank values
-    uint32_t* shist = nullptr;  // [units*group][SBINS] counts of S by its top order-key bits
+    uint32_t* shist = nullptr;  // [units*group][SCOPIES][SBINS] counts of S by its top order-key bits
     int64_t cmax = 0;
-    int* status = nullptr;      // device status word (ST_OK / ST_TIMEOUT / ST_BADINDEX)
-
-    // work queues of the persistent search kernel (search.cu)
-    int* ctrl = nullptr;        // control block: queue counters, per-pack flags and counters
-    unsigned long long* trace = nullptr;   // phase trace of profiled searches [kTraceWords]
-    int* progress = nullptr;    // debug: per-CTA item board in mapped host memory (not owned)
-    long long spin_limit = kDefaultSpinLimit;   // bound of every device-side wait (cycles)
+    int* status = nullptr;      // device status word (ST_OK / ST_TIMEOUT)
 
     // optional per-stage timing of searches (test and benchmark use)
     bool profile = false;
@@ -137,12 +120,23 @@ cudaError_t launch_encode(const pariskv_index* ix, const void* keys, const float
 cudaError_t launch_rotate(const pariskv_config* cfg, const float* signs, const void* x,
                           int64_t n, float* y, float* norm, cudaStream_t st);
 
-// search.cu: the whole retrieval step as one persistent kernel (query prep, vote, select,
-// rerank, top-k); search_ctrl_words gives the control block's size for P pack-units.
-int search_ctrl_words(int P);
-cudaError_t launch_search(pariskv_index* ix, const void* q, const float* qt_in,
-                          const float* qn_in, bool rotated, int64_t C, int32_t k,
-                          int32_t* topk_idx, float* topk_est, cudaStream_t st);
+// query.cu
+cudaError_t launch_query_prep(const pariskv_index* ix, const void* q, const float* qt_in,
+                              const float* qn_in, bool rotated, cudaStream_t st);
+
+// vote.cu
+cudaError_t launch_vote(const pariskv_index* ix, cudaStream_t st);
+
+// select.cu
+cudaError_t launch_threshold(const pariskv_index* ix, int64_t C, cudaStream_t st);
+cudaError_t launch_compact(const pariskv_index* ix, cudaStream_t st);
+
+// rerank.cu
+cudaError_t launch_rerank(const pariskv_index* ix, int64_t C, cudaStream_t st);
+
+// topk.cu
+cudaError_t launch_topk(const pariskv_index* ix, int64_t C, int32_t k, int32_t* topk_idx,
+                        float* topk_est, cudaStream_t st);
 
 // attend.cu
 cudaError_t launch_read_stream(const void* src, int64_t bytes, uint32_t* sink,

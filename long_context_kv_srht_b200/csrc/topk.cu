@@ -1,0 +1,298 @@
+// topk.cu -- final top-k of the reranked candidates.
+//
+// "Technical Summary: ParisKV", Problem Statement (attention over a Top-k subset of past
+// tokens) and Key Contributions 2 (Top-k selection directly on compressed codes); "ParisKV:
+// Fast and Drift-Robust KV-Cache Retrieval for Long-Context LLMs" (on-demand top-k fetch).
+// The k candidates with the largest rerank value S are kept, ties going to the lower key
+// index, and returned in ascending key order with est = ||q|| * S.
+//
+// Exact selection on the order-preserving 32-bit image u of S (flip all bits of negative
+// values, set the sign bit of the others). A head's candidates are split over CL CTAs: one
+// CTA when they fit its shared memory (up to 8192) -- 1024 threads when there are no more
+// heads than SMs, else 256 threads (with a 4096-value slice when it suffices, so four CTAs
+// share an SM and even many heads run in about one wave) -- and otherwise a cluster of four
+// 1024-thread CTAs:
+//  - CTA r copies the r-th part of the head's S values and candidate indices into shared
+//    memory with asynchronous copies, all in flight at once, and turns S into u in place
+//    (parts longer than the slice stay in global memory and are re-read on every pass);
+//  - the first radix level, the top 11 bits of u, was counted by the rerank as it wrote S
+//    (per head, SCOPIES copies of a 2048-bin histogram in global memory), so it costs one
+//    round of reads here;
+//  - then range-adaptive radix levels: the current interval [lo, hi] is cut into at most 2048
+//    power-of-two-wide bins, every CTA histograms its part, and every CTA sums the CL
+//    histograms bin by bin (over DSMEM in a cluster) and runs the same suffix scan, so all
+//    pick the same bin (the one holding the k-th largest) without further exchange.
+//    Histograms alternate between two buffers, so one barrier per level suffices; the 21
+//    bits left after the first level take at most two more levels;
+//  - with T the k-th largest value and E the number of T-valued candidates to keep, each
+//    thread counts a contiguous run of values, the counts are scanned over the CTA and the
+//    cluster, and each thread then writes its run's values above T and its ties at T while
+//    fewer than E ties precede them, in ascending key order (the candidates are stored in
+//    key order); est comes from u itself.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+#include "internal.hpp"
+
+namespace pkv {
+
+namespace cg = cooperative_groups;
+
+namespace {
+
+constexpr int kBins = 2048;
+
+template <int CL, int T, int SLICE, bool RES>
+__global__ void __launch_bounds__(T, 1)
+topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
+            const float* __restrict__ qnorm, const uint32_t* __restrict__ shist, int32_t C,
+            int64_t cmax, int32_t k, int32_t* __restrict__ out_idx, float* __restrict__ out_est,
+            int* status) {
+    constexpr int kWarps = T / 32;
+    constexpr int BPT = kBins / T;     // bins per thread: thread t owns bins BPT t .. BPT t + BPT - 1
+    static_assert(kWarps <= 32 && kBins % T == 0 && (BPT == 2 || BPT == 8), "layout");
+    extern __shared__ __align__(16) uint32_t dyn[];
+    __shared__ __align__(16) uint32_t hist[2][kBins];
+    __shared__ uint32_t wa[kWarps], wb[kWarps];
+    __shared__ uint32_t ctot[2];       // this CTA's candidates above T / ties at T
+    __shared__ uint32_t pick[2];
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = CL > 1 ? static_cast<int>(cluster.block_rank()) : 0;
+    const int head = blockIdx.x / CL;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int s0 = static_cast<int>(static_cast<int64_t>(C) * rank / CL);
+    const int s1 = static_cast<int>(static_cast<int64_t>(C) * (rank + 1) / CL);
+    const int L = s1 - s0;
+    const float* Sh = S + head * cmax + s0;
+    const int32_t* ch = cand + head * cmax + s0;
+    uint32_t* keys = dyn;                                   // [SLICE] u
+    int32_t* idx = reinterpret_cast<int32_t*>(dyn + SLICE);  // [SLICE] candidate index
+    auto key_at = [&](int i) -> uint32_t { return RES ? keys[i] : order_key(Sh[i]); };
+    auto idx_at = [&](int i) -> int32_t { return RES ? idx[i] : ch[i]; };
+    auto sync_all = [&]() {
+        if constexpr (CL > 1) cluster.sync();
+        else __syncthreads();
+    };
+    // this thread's BPT bins of a histogram buffer (uint2 / uint4 loads)
+    auto load_bins = [&](const uint32_t* hb, uint32_t h[BPT]) {
+        if constexpr (BPT == 2) {
+            const uint2 v = reinterpret_cast<const uint2*>(hb)[threadIdx.x];
+            h[0] = v.x; h[1] = v.y;
+        } else {
+            const uint4 v = reinterpret_cast<const uint4*>(hb)[2 * threadIdx.x];
+            const uint4 w = reinterpret_cast<const uint4*>(hb)[2 * threadIdx.x + 1];
+            h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
+            h[4] = w.x; h[5] = w.y; h[6] = w.z; h[7] = w.w;
+        }
+    };
+    pdl_wait();
+    pdl_launch_dependents();
+
+    // 1. this CTA's part into shared memory (asynchronous 4-byte copies, all in flight at
+    //    once); then u in place
+    if (RES) {
+        for (int i = threadIdx.x; i < L; i += T) {
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(keys + i)),
+                         "l"(Sh + i) : "memory");
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(idx + i)),
+                         "l"(ch + i) : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        for (int i = threadIdx.x; i < L; i += T)   // each thread converts what it copied
+            keys[i] = order_key(__uint_as_float(keys[i]));
+    }
+
+    // 2. radix levels. The first (the top SBINS_BITS bits of u) was counted by the rerank;
+    //    the following ones are range-adaptive histograms over the head's CTAs. choose()
+    //    finds, from each thread's bins, the bin holding the krem-th largest value and
+    //    narrows [lo, hi] to it; every CTA sees the same counts and makes the same choice.
+    uint32_t krem = static_cast<uint32_t>(k);
+    uint32_t lo = 0u, hi = 0xffffffffu;
+    auto choose = [&](const uint32_t h[BPT], int sh) {
+        uint32_t mine = 0;
+#pragma unroll
+        for (int j = 0; j < BPT; ++j) mine += h[j];
+        uint32_t x = mine;             // suffix counts over the threads' bin ranges
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
+            if (lane + o < 32) x += y;
+        }
+        if (lane == 0) wa[warp] = x;   // warp totals
+        __syncthreads();
+        if (warp == 0) {               // exclusive suffix sums of the warp totals
+            const uint32_t t = lane < kWarps ? wa[lane] : 0u;
+            uint32_t y = t;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t z = __shfl_down_sync(0xffffffffu, y, o);
+                if (lane + o < 32) y += z;
+            }
+            if (lane < kWarps) wb[lane] = y - t;
+        }
+        __syncthreads();
+        uint32_t above = wb[warp] + x - mine;   // strictly above this thread's bins
+#pragma unroll
+        for (int j = BPT - 1; j >= 0; --j) {
+            if (above < krem && krem <= above + h[j]) {
+                pick[0] = BPT * threadIdx.x + j;
+                pick[1] = above;
+            }
+            above += h[j];
+        }
+        __syncthreads();
+        const uint32_t b = pick[0];
+        krem -= pick[1];
+        const uint32_t nlo = lo + (b << sh);
+        const uint64_t bin_hi = static_cast<uint64_t>(nlo) + ((uint64_t{1} << sh) - 1u);
+        lo = nlo;
+        hi = static_cast<uint32_t>(min(static_cast<uint64_t>(hi), bin_hi));
+        __syncthreads();   // pick[], wa[] and wb[] are rewritten by the next level
+    };
+    static_assert(SBINS == kBins, "the first level uses the same bins");
+    {
+        uint32_t h[BPT] = {}, v[BPT];
+        const uint32_t* hs = shist + static_cast<int64_t>(head) * SCOPIES * SBINS;
+#pragma unroll
+        for (int r = 0; r < SCOPIES; ++r) {
+            load_bins(hs + r * SBINS, v);
+#pragma unroll
+            for (int j = 0; j < BPT; ++j) h[j] += v[j];
+        }
+        choose(h, 32 - SBINS_BITS);
+    }
+    int level = 0;
+    while (lo != hi) {
+        uint32_t* hb = hist[level & 1];
+        const uint32_t span = hi - lo;
+        const int bitlen = 32 - __clz(span);
+        const int sh = bitlen > 11 ? bitlen - 11 : 0;   // (span >> sh) < 2048
+#pragma unroll
+        for (int j = 0; j < BPT; ++j) hb[threadIdx.x + T * j] = 0u;
+        __syncthreads();
+        if (RES && (L & 3) == 0) {
+            const uint4* k4 = reinterpret_cast<const uint4*>(keys);
+            for (int i = threadIdx.x; i < (L >> 2); i += T) {
+                const uint4 v = k4[i];
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (u[j] >= lo && u[j] <= hi) atomicAdd(&hb[(u[j] - lo) >> sh], 1u);
+            }
+        } else {
+            for (int i = threadIdx.x; i < L; i += T) {
+                const uint32_t u = key_at(i);
+                if (u >= lo && u <= hi) atomicAdd(&hb[(u - lo) >> sh], 1u);
+            }
+        }
+        sync_all();   // every part's histogram is complete
+        uint32_t h[BPT] = {}, v[BPT];
+#pragma unroll
+        for (int q = 0; q < CL; ++q) {
+            load_bins(CL > 1 ? cluster.map_shared_rank(hb, q) : hb, v);
+#pragma unroll
+            for (int j = 0; j < BPT; ++j) h[j] += v[j];
+        }
+        choose(h, sh);
+        ++level;
+    }
+    const uint32_t Tv = lo;
+    const uint32_t E = krem;   // ties at Tv to keep, in key order
+
+    // 3. counts per thread-contiguous run, then offsets over the CTA (block scan) and over
+    //    the head's CTAs
+    const int a = static_cast<int>(static_cast<int64_t>(L) * threadIdx.x / T);
+    const int b = static_cast<int>(static_cast<int64_t>(L) * (threadIdx.x + 1) / T);
+    uint32_t ngt = 0, neq = 0;
+    for (int i = a; i < b; ++i) {
+        const uint32_t u = key_at(i);
+        ngt += u > Tv;
+        neq += u == Tv;
+    }
+    // inclusive warp scans of (gt, eq), then warp totals
+    uint32_t xg = ngt, xe = neq;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t yg = __shfl_up_sync(0xffffffffu, xg, o);
+        const uint32_t ye = __shfl_up_sync(0xffffffffu, xe, o);
+        if (lane >= o) { xg += yg; xe += ye; }
+    }
+    if (lane == 31) { wa[warp] = xg; wb[warp] = xe; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t g = 0, e = 0;
+        for (int w = 0; w < kWarps; ++w) { g += wa[w]; e += wb[w]; }
+        ctot[0] = g;
+        ctot[1] = e;
+    }
+    sync_all();
+    uint32_t gt_run = xg - ngt, eq_run = xe - neq;   // above Tv / ties before this thread
+    if constexpr (CL > 1) {
+        for (int q = 0; q < rank; ++q) {
+            const uint32_t* r = cluster.map_shared_rank(ctot, q);
+            gt_run += r[0];
+            eq_run += r[1];
+        }
+    }
+    for (int w = 0; w < warp; ++w) { gt_run += wa[w]; eq_run += wb[w]; }
+    if constexpr (CL > 1) cluster.barrier_arrive();   // no remote read of this CTA follows
+
+    // 4. this thread's winners in key order: every value above Tv, and the ties at Tv while
+    //    fewer than E ties precede them
+    const float qn = qnorm[head];
+    uint32_t pos = gt_run + min(eq_run, E);
+    if (pos + ngt + (E > eq_run ? min(E - eq_run, neq) : 0u) > static_cast<uint32_t>(k)) {
+        atomicExch(status, ST_BADINDEX);   // never taken when the counts are consistent
+    } else {
+        int32_t* oi = out_idx + static_cast<int64_t>(head) * k;
+        float* oe = out_est ? out_est + static_cast<int64_t>(head) * k : nullptr;
+        for (int i = a; i < b; ++i) {
+            const uint32_t u = key_at(i);
+            bool take = u > Tv;
+            if (u == Tv) take = eq_run++ < E;
+            if (take) {
+                oi[pos] = idx_at(i);
+                if (oe) oe[pos] = __fmul_rn(qn, value_of(u));
+                ++pos;
+            }
+        }
+    }
+    if constexpr (CL > 1) cluster.barrier_wait();
+}
+
+template <int CL, int T, int SLICE, bool RES>
+cudaError_t launch_cfg(const pariskv_index* ix, int64_t C, int32_t k, int32_t* topk_idx,
+                       float* topk_est, cudaStream_t st) {
+    constexpr int kDyn = RES ? 2 * SLICE * 4 : 0;
+    static std::atomic<uint64_t> smem_raised{0};
+    if (kDyn > 0) {   // static + dynamic shared memory can pass the 48 KB default
+        cudaError_t e = raise_smem_limit(topk_kernel<CL, T, SLICE, RES>, kDyn, smem_raised);
+        if (e != cudaSuccess) return e;
+    }
+    const int heads = ix->units * ix->cfg.group;
+    return launch_pdl_cluster(topk_kernel<CL, T, SLICE, RES>, dim3(heads * CL), dim3(T), kDyn,
+                              st, static_cast<unsigned>(CL), ix->S, ix->cand, ix->qnorm,
+                              ix->shist, static_cast<int32_t>(C), ix->cmax, k, topk_idx,
+                              topk_est, ix->status);
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const pariskv_index* ix, int64_t C, int32_t k, int32_t* topk_idx,
+                        float* topk_est, cudaStream_t st) {
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int heads = ix->units * ix->cfg.group;
+    if (C <= 8192 && heads <= sms)   // at most one head per SM: use all of its threads
+        return launch_cfg<1, 1024, 8192, true>(ix, C, k, topk_idx, topk_est, st);
+    if (C <= 4096) return launch_cfg<1, 256, 4096, true>(ix, C, k, topk_idx, topk_est, st);
+    if (C <= 8192) return launch_cfg<1, 256, 8192, true>(ix, C, k, topk_idx, topk_est, st);
+    if (C <= 4 * 16384)
+        return launch_cfg<4, 1024, 16384, true>(ix, C, k, topk_idx, topk_est, st);
+    return launch_cfg<4, 1024, 16384, false>(ix, C, k, topk_idx, topk_est, st);
+}
+
+}  // namespace pkv

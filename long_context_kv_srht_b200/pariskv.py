@@ -95,9 +95,6 @@ _SIGS = {
     "pariskv_debug_export_search": (_S, [_P, _P, _P, ctypes.POINTER(_I64), _P, _P]),
     "pariskv_debug_profile": (_S, [_P, _I32]),
     "pariskv_debug_stage_ms": (_S, [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_I32)]),
-    "pariskv_debug_search_phases": (_S, [_P, ctypes.POINTER(ctypes.c_double)]),
-    "pariskv_debug_set_wait_limit": (_S, [_P, ctypes.c_int64]),
-    "pariskv_debug_set_progress": (_S, [_P, _P]),
     "pariskv_debug_read_stream": (_S, [_P, _I64, _P, _P]),
     "pariskv_cache_create": (_S, [ctypes.POINTER(Config), ctypes.POINTER(CacheConfig), _P, _P,
                                   ctypes.POINTER(_P)]),
@@ -108,10 +105,7 @@ _SIGS = {
     "pariskv_cache_destroy": (_S, [_P]),
 }
 
-STAGES = ("search",)
-# kinds of work in the trace of a profiled search (pariskv_debug_search_phases)
-PHASES = ("query_prep", "vote", "compact", "topk", "finalise", "rerank", "vote_wait",
-          "rerank_wait", "kernel", "polls")
+STAGES = ("query_prep", "vote", "threshold", "compact", "rerank", "topk")
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
     _f.restype = _res
@@ -262,27 +256,6 @@ class Index:
         _check(lib.pariskv_debug_stage_ms(self.handle, ms, ctypes.byref(n)),
                "pariskv_debug_stage_ms")
         return {STAGES[i]: float(ms[i]) for i in range(n.value)}
-
-    def set_progress(self, board) -> None:
-        """Per-CTA item board (a pinned host int32 tensor of 4 x 2 x SMs), or None."""
-        _check(lib.pariskv_debug_set_progress(self.handle, None if board is None else board.data_ptr()),
-               "pariskv_debug_set_progress")
-
-    def set_wait_limit(self, cycles: int) -> None:
-        """Bounds the device-side waits of later searches (0 restores the default)."""
-        _check(lib.pariskv_debug_set_wait_limit(self.handle, int(cycles)), "pariskv_debug_set_wait_limit")
-
-    def search_phases(self) -> dict:
-        """Per kind of work of the last profiled search: first start, last end (us after the
-        kernel started) and busy time summed over workers (us)."""
-        out = (ctypes.c_double * 36)()
-        _check(lib.pariskv_debug_search_phases(self.handle, out), "pariskv_debug_search_phases")
-        ph = {name: {"start_us": out[3 * i], "end_us": out[3 * i + 1], "busy_us": out[3 * i + 2]}
-              for i, name in enumerate(PHASES[:-1])}
-        ph["polls"] = {"start_us": -1.0, "end_us": -1.0, "busy_us": out[29]}
-        ph["topk_detail"] = {"passes": out[30], "unlisted": out[31], "select_us": out[32],
-                             "write_us": out[35]}
-        return ph
 
     def export_index(self):
         units = self.cfg.batch * self.cfg.num_kv_heads
