@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cache", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the search and dense-comparator lines of the other workloads")
     ap.add_argument("--centroids", choices=["analytic", "learned"], default="analytic",
                     help="drift_32k: coarse centroids (analytic, or learned from the prefill "
                          "by spherical k-means: the comparator of the drift claim)")
@@ -276,6 +278,7 @@ def decode_step(args, ix, cfg, sp, keys, vals, qs, idx, est, k, H, dev, kv_host)
     nwarm, nrep = 3, 10        # warm-up steps touch the host pages (GPU TLB) before timing
     out = torch.empty(qs.shape, dtype=torch.float32, device=dev)
     assert nwarm + nrep <= APPEND_SLACK
+    pk.union_rows()   # reset the union-row counter of the group-union attention
     for s in range(nwarm + nrep):
         new_k = keys[:, :, ix.size:ix.size + 1].to(dev)
         e0.record()
@@ -295,10 +298,16 @@ def decode_step(args, ix, cfg, sp, keys, vals, qs, idx, est, k, H, dev, kv_host)
         app_ms += e0.elapsed_time(ea) / nrep
         srch_ms += ea.elapsed_time(es) / nrep
         att_ms += es.elapsed_time(e1) / nrep
-    kv_bytes = H * k * 2 * sp.d * 2
+    # K/V rows the attention fetched per step: the GQA-group union when it is used (each row
+    # once per KV head), else every head's own k rows
+    urows = pk.union_rows() / (nwarm + nrep)
+    rows = urows if urows else H * k
+    kv_bytes = int(rows * 2 * sp.d * 2)
     decode = {"append_ms": app_ms, "search_ms": srch_ms, "sparse_attend_ms": att_ms,
               "total_ms": app_ms + srch_ms + att_ms,
               "kv_source": "pinned host (UVA)" if kv_host else "HBM",
+              "attend_rows_per_step": rows, "attend_rows_per_head_selection": H * k,
+              "attend_kv_bytes_per_step": kv_bytes,
               "attend_gbs": kv_bytes / (att_ms / 1e3) / 1e9}
     if kv_host:
         # the PCIe roofline of the attention: one coalesced pass over 256 MiB of the pinned K
@@ -376,6 +385,57 @@ def dense_comparator(cfg, sp, data, ix, k, dev, peak_gbs):
             "paris_hbm_ms": paris_ms, "speedup_vs_dense_hbm": dense_ms / paris_ms,
             "speedup_vs_dense_roofline": kv_bytes / (peak_gbs * 1e9) * 1e3 / paris_ms,
             "kv": "HBM (both)", "n": n, "k": k}
+
+
+def side_workload(name, args, dev, flush):
+    """The search of another workload (K/V in HBM), timed like the headline (L2 flushed
+    between steps, CUDA events per step), with its roofline fraction and the ParisKV step
+    (search + sparse attention) against full attention on the same K/V."""
+    import numpy as np
+    import torch
+    from long_context_kv_srht_b200 import pariskv as pk
+    from long_context_kv_srht_b200 import workload
+    sp = workload.spec(name)
+    data = workload.generate_torch(sp, dev, n=sp.n)
+    cfg = pk.config(batch=sp.batch, num_kv_heads=sp.num_kv_heads, group=sp.group,
+                    capacity=sp.n, dtype=sp.dtype, rho=sp.rho, cand_bp=sp.cand_bp,
+                    levels=args.levels)
+    ix = pk.build_index(cfg, data["signs"], data["keys"], n=sp.n)
+    H, k = sp.batch * sp.num_q_heads, sp.k
+    C = candidate_count(sp.n, k, sp.cand_bp)
+    idx = torch.empty((H, k), dtype=torch.int32, device=dev)
+    est = torch.empty((H, k), dtype=torch.float32, device=dev)
+    qs = data["queries"]
+    for _ in range(max(3, args.warmup)):
+        ix.search(qs, k, idx, est)
+    torch.cuda.synchronize()
+    steps = max(10, min(args.steps, 50))
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for s in range(steps):
+        flush.fill_(s & 255)
+        ev0[s].record()
+        ix.search(qs, k, idx, est)
+        ev1[s].record()
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev0, ev1)]))
+    peak = measured_peaks()[0]
+    step_bytes = algorithmic_bytes("vote", sp, C) + algorithmic_bytes("rerank", sp, C)
+    out = {"ms_per_step": ms, "keys_per_s": H * sp.n / (ms / 1e3), "steps": steps,
+           "step_algorithmic_bytes": step_bytes,
+           "step_frac": step_bytes / (ms / 1e3) / 1e9 / peak,
+           "config": {"batch": sp.batch, "q_heads": sp.num_q_heads, "kv_heads": sp.num_kv_heads,
+                      "n": sp.n, "k": k, "candidates": C, "key_dtype": sp.dtype, "kv_in": "HBM"}}
+    dense = dense_comparator(cfg, sp, data, ix, k, dev, peak)
+    if dense:
+        out["dense_ms"] = dense["dense_ms"]
+        out["paris_step_ms"] = dense["paris_hbm_ms"]
+        out["paris_vs_dense"] = dense["speedup_vs_dense_hbm"]
+    ix.sync()
+    ix.destroy()
+    del data
+    torch.cuda.empty_cache()
+    return out
 
 
 # Region sizes of the four-region cache measurement ("Technical Summary: ParisKV" gives none;
@@ -725,7 +785,12 @@ def main():
     if not args.no_cache:
         cache_step = cache_decode(cfg, sp, data, k, dev)
 
-    cpu = None
+    # the search on the other workloads of the pages' tables (one GPU, rank 0 only)
+    others = None
+    if rank == 0 and ws == 1 and not args.no_workloads and sp.name == "million_offload":
+        others = {name: side_workload(name, args, dev, flush)
+                  for name in ("llama3_8b_128k", "batched_64k")}
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         v, dt, cores = oracle_sample(sp, data, reps=1)
@@ -756,6 +821,7 @@ def main():
             "decode_step": decode,
             "cache_step": cache_step,
             "dense_comparator": dense,
+            "workloads": others,
             "gpu_launches": launches,
             "clocks": clk,
         }

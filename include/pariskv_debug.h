@@ -66,6 +66,48 @@ PARISKV_API pariskv_status pariskv_debug_profile(pariskv_index* index, int32_t e
 PARISKV_API pariskv_status pariskv_debug_stage_ms(pariskv_index* index, float* ms,
                                                   int32_t* nstages);
 
+/* Test hook: the next pariskv_search on this index writes `value` (which must not be a valid
+ * key index: negative or >= the index size) into candidate slot `pos` of query head `head`
+ * (row s * Hq + h) after the compaction, as a selection bug would. The rerank and the top-k
+ * skip the out-of-range record instead of reading it; pariskv_sync then reports ECUDA with
+ * the device status ST_BADINDEX, and the results of every other query head are unaffected.
+ * One search consumes the hook. pos must be below that search's candidate count C (else
+ * the search fails with EINVAL), with one exception that tests the guard bytes (see
+ * pariskv_debug_check_guards): with guards on, a slot of the last head that falls in the
+ * guard after the candidate buffer is written there. No counterpart on the pages.
+ * Errors: EINVAL. */
+PARISKV_API pariskv_status pariskv_debug_inject_bad_candidate(pariskv_index* index, int32_t head,
+                                                               int64_t pos, int32_t value);
+
+/* Forces the launch shapes of later searches on this index, for tests that require the same
+ * bits from every shape: vote_ctas / rerank_ctas = the number of CTAs of the vote scan and of
+ * the rerank (0: automatic; any positive count is valid, work is split over the CTAs), and
+ * topk_mode = 1 one 1024-thread CTA per head (C <= 8192), 2 one 256-thread CTA per head
+ * (C <= 8192), 3 a cluster of four 1024-thread CTAs holding the values in shared memory
+ * (C <= 65536), 4 the same cluster reading them from global memory (any C), 0 automatic. A
+ * search whose C does not fit the forced top-k shape fails with EINVAL. No counterpart on the
+ * pages. Errors: EINVAL. */
+PARISKV_API pariskv_status pariskv_debug_set_launch(pariskv_index* index, int32_t vote_ctas,
+                                                    int32_t rerank_ctas, int32_t topk_mode);
+
+/* K/V rows fetched by pariskv_sparse_attend's GQA-group union since the last call, on the
+ * current device (synchronises the device, then resets the count). The row-gather attention
+ * (K/V in pinned host memory, or fp32) with 1 < group <= 8 merges the group's top-k lists
+ * into one union of rows per (sequence, KV head) and fetches each union row once for every
+ * query head that selected it; this count is the number of rows it read, so the bytes that
+ * crossed PCIe are rows x 2 x 128 x the element size. PARISKV_ATTEND_UNION=0 in the
+ * environment turns the union off (each query head then fetches its own rows). A measurement
+ * aid with no counterpart on the pages. Errors: EINVAL, ECUDA. */
+PARISKV_API pariskv_status pariskv_debug_union_rows(int64_t* rows);
+
+/* Guard bytes: when PARISKV_GUARD=1 is in the environment before the library's first index
+ * allocation, every device buffer an index owns is allocated with 256 bytes of a fixed
+ * pattern before and after it. This call synchronises the device and checks the guards of
+ * every live buffer (buffers freed since the last call were checked when freed); ECUDA names
+ * the first overrun seen, with the buffer's size and side. A stand-in for a memory checker,
+ * with no counterpart on the pages. Errors: EINVAL (guards off), ECUDA. */
+PARISKV_API pariskv_status pariskv_debug_check_guards(void);
+
 /* Reads `bytes` from `src` once, with coalesced 16-byte loads spread over every SM, and
  * folds the data into one word that may be written to `sink` (a device pointer to 4 bytes),
  * on `stream`. Timed with CUDA events around the call it measures how fast the device reads

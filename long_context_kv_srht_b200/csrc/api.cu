@@ -45,22 +45,103 @@ pariskv_status injected_launch_failure() {
     return fail(PARISKV_ECUDA, "injected launch failure (PARISKV_FAULT=launch)");
 }
 
+// Guard bytes (a test aid standing in for a memory checker): with PARISKV_GUARD=1 in the
+// environment when the library makes its first index allocation, every device buffer an
+// index owns gets kGuard bytes of a fixed pattern before and after it. They are checked when
+// the buffer is freed and by pariskv_debug_check_guards; a kernel that wrote past either end
+// of a buffer is reported there by the buffer's size and the side it overran.
+constexpr size_t kGuard = 256;            // keeps the buffer 256-byte aligned
+constexpr unsigned char kGuardByte = 0xA5;
+struct Guarded {
+    char* base;
+    size_t bytes;
+};
+std::mutex g_guard_mu;
+std::vector<Guarded> g_guarded;           // live guarded buffers
+char g_guard_bad[256] = "";               // first overrun seen (empty: none)
+
+bool guards_on() {
+    static const bool on = [] {
+        const char* v = getenv("PARISKV_GUARD");
+        return v && v[0] == '1';
+    }();
+    return on;
+}
+
+// Checks one buffer's guards (synchronous); records the first overrun in g_guard_bad.
+bool guard_ok(const Guarded& g) {
+    unsigned char h[2][kGuard];
+    if (cudaMemcpy(h[0], g.base, kGuard, cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemcpy(h[1], g.base + kGuard + g.bytes, kGuard, cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return true;   // unreadable (device error): reported by the call that failed
+    }
+    for (int side = 0; side < 2; ++side)
+        for (size_t i = 0; i < kGuard; ++i)
+            if (h[side][i] != kGuardByte) {
+                if (!g_guard_bad[0])
+                    snprintf(g_guard_bad, sizeof(g_guard_bad),
+                             "guard bytes %s a %zu-byte index buffer were overwritten (byte %zu)",
+                             side ? "after" : "before", g.bytes, i);
+                return false;
+            }
+    return true;
+}
+
+void* raw_alloc(size_t bytes) {
+    void* p = nullptr;
+    if (!guards_on()) {
+        if (cudaMalloc(&p, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        return p;
+    }
+    char* base = nullptr;
+    if (cudaMalloc(reinterpret_cast<void**>(&base), bytes + 2 * kGuard) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (cudaMemset(base, kGuardByte, kGuard) != cudaSuccess ||
+        cudaMemset(base + kGuard + bytes, kGuardByte, kGuard) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(base);
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lk(g_guard_mu);
+    g_guarded.push_back({base, bytes});
+    return base + kGuard;
+}
+
+void raw_free(void* p) {
+    if (!p) return;
+    if (guards_on()) {
+        std::lock_guard<std::mutex> lk(g_guard_mu);
+        for (size_t i = 0; i < g_guarded.size(); ++i)
+            if (g_guarded[i].base + kGuard == p) {
+                cudaDeviceSynchronize();
+                guard_ok(g_guarded[i]);
+                cudaFree(g_guarded[i].base);
+                g_guarded[i] = g_guarded.back();
+                g_guarded.pop_back();
+                return;
+            }
+    }
+    cudaFree(p);
+}
+
 template <typename T>
 bool dalloc(T** p, size_t count) {
     *p = nullptr;
     if (count == 0) count = 1;
     if (fault_alloc()) return false;
-    if (cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T)) != cudaSuccess) {
-        cudaGetLastError();
-        *p = nullptr;
-        return false;
-    }
-    return true;
+    *p = static_cast<T*>(raw_alloc(count * sizeof(T)));
+    return *p != nullptr;
 }
 
 template <typename T>
 void dfree(T*& p) {
-    if (p) cudaFree(p);
+    raw_free(p);
     p = nullptr;
 }
 
@@ -254,6 +335,20 @@ pariskv_status run_search(pariskv_index* ix, const void* q, const float* qt, con
     const int64_t C = candidate_count(ix->n, k, ix->cfg.cand_bp);
     pariskv_status s = ensure_candidates(ix, C);
     if (s != PARISKV_OK) return s;
+    // a slot past C is refused, except (with guard bytes on) one inside the guard that
+    // follows the candidate buffer, which tests that an overrun is detected
+    const int64_t slot = static_cast<int64_t>(ix->inject_head) * ix->cmax + ix->inject_pos;
+    const int64_t cand_end = static_cast<int64_t>(ix->units) * ix->cfg.group * ix->cmax;
+    const bool into_guard = guards_on() && slot >= cand_end &&
+                            slot < cand_end + static_cast<int64_t>(kGuard / sizeof(int32_t));
+    if (ix->inject_head >= 0 && ix->inject_pos >= C && !into_guard) {
+        ix->inject_head = -1;
+        return fail(PARISKV_EINVAL, "injected candidate position %lld >= C = %lld",
+                    static_cast<long long>(ix->inject_pos), static_cast<long long>(C));
+    }
+    if (ix->topk_mode != 0 && !topk_mode_fits(ix->topk_mode, C))
+        return fail(PARISKV_EINVAL, "top-k launch shape %d cannot hold C = %lld candidates",
+                    ix->topk_mode, static_cast<long long>(C));
     if (fault_launch()) return injected_launch_failure();
     g_launches = 0;
     int ne = 0;
@@ -265,6 +360,10 @@ pariskv_status run_search(pariskv_index* ix, const void* q, const float* qt, con
     if (e == cudaSuccess) { ++g_launches; mark(); e = launch_vote(ix, st); }
     if (e == cudaSuccess) { ++g_launches; mark(); e = launch_threshold(ix, C, st); }
     if (e == cudaSuccess) { ++g_launches; mark(); e = launch_compact(ix, st); }
+    if (e == cudaSuccess && ix->inject_head >= 0) {   // test hook: one bad candidate index
+        e = launch_poke(ix->cand + ix->inject_head * ix->cmax + ix->inject_pos, ix->inject_value, st);
+        ix->inject_head = -1;
+    }
     if (e == cudaSuccess) { ++g_launches; mark(); e = launch_rerank(ix, C, st); }
     if (e == cudaSuccess) { ++g_launches; mark(); e = launch_topk(ix, C, k, topk_idx, topk_est, st); }
     if (e == cudaSuccess) { ++g_launches; mark(); }
@@ -447,7 +546,11 @@ pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, c
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int heads = cfg->batch * cfg->num_kv_heads * cfg->group;
     const bool mma = attend_uses_mma(cfg, device_memory(K) && device_memory(V));
-    const int nsplit = attend_splits(heads, k, sms, mma);
+    // the row-gather kernel fetches each row of a GQA group's union once when it can
+    const size_t ubytes = mma ? 0 : union_workspace_bytes(cfg, n, k);
+    const int nsplit = ubytes ? union_splits(cfg->batch * cfg->num_kv_heads, cfg->group, k, sms)
+                              : attend_splits(heads, k, sms, mma);
+    const size_t pbytes = round_up(attend_workspace_floats(heads, nsplit) * sizeof(float), 256);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     float* work = nullptr;
     if (fault_alloc()) return fail(PARISKV_ENOMEM, "attention workspace");
@@ -455,14 +558,18 @@ pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, c
     cudaMemPool_t pool = nullptr;
     cudaError_t e = workspace_pool(&pool);
     if (e == cudaSuccess)
-        e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&work),
-                                    attend_workspace_floats(heads, nsplit) * sizeof(float), pool,
-                                    st);
+        e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&work), pbytes + ubytes, pool, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention workspace");
     g_launches = 0;
-    e = launch_attend(cfg, q, K, V, ld_tok, n, topk_idx, k, scale, out, out_dtype, work, nsplit,
-                      mma, st);
-    if (e == cudaSuccess) g_launches = 2;
+    if (ubytes) {
+        e = launch_attend_union(cfg, q, K, V, ld_tok, n, topk_idx, k, scale, out, out_dtype, work,
+                                nsplit, reinterpret_cast<char*>(work) + pbytes, st);
+        if (e == cudaSuccess) g_launches = 4;
+    } else {
+        e = launch_attend(cfg, q, K, V, ld_tok, n, topk_idx, k, scale, out, out_dtype, work,
+                          nsplit, mma, st);
+        if (e == cudaSuccess) g_launches = 2;
+    }
     cudaFreeAsync(work, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
     return PARISKV_OK;
@@ -703,6 +810,10 @@ pariskv_status pariskv_sync(pariskv_index* index, void* stream) {
     if (st != ST_OK) {
         cudaMemset(index->status, 0, sizeof(int));
         if (st == ST_TIMEOUT) return fail(PARISKV_ETIMEOUT, "a bounded device-side wait expired");
+        if (st == ST_BADINDEX)
+            return fail(PARISKV_ECUDA,
+                        "a kernel found an index out of range and skipped the access (device "
+                        "status %d); the results of the affected heads are invalid", st);
         return fail(PARISKV_ECUDA, "internal consistency check failed on the device (%d)", st);
     }
     return PARISKV_OK;
@@ -801,6 +912,59 @@ pariskv_status pariskv_debug_profile(pariskv_index* ix, int32_t enable) {
     }
     ix->profile = enable != 0;
     ix->nev = 0;
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_debug_inject_bad_candidate(pariskv_index* ix, int32_t head, int64_t pos,
+                                                 int32_t value) {
+    pariskv_status s = check_index(ix);
+    if (s != PARISKV_OK) return s;
+    const int heads = ix->units * ix->cfg.group;
+    if (head < 0 || head >= heads) return fail(PARISKV_EINVAL, "head %d not in [0, %d)", head, heads);
+    if (pos < 0) return fail(PARISKV_EINVAL, "pos < 0");
+    if (value >= 0 && value < ix->n)
+        return fail(PARISKV_EINVAL, "value %d is a valid key index (size %lld)", value,
+                    static_cast<long long>(ix->n));
+    ix->inject_head = head;
+    ix->inject_pos = pos;
+    ix->inject_value = value;
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_debug_set_launch(pariskv_index* ix, int32_t vote_ctas, int32_t rerank_ctas,
+                                        int32_t topk_mode) {
+    pariskv_status s = check_index(ix);
+    if (s != PARISKV_OK) return s;
+    if (vote_ctas < 0 || rerank_ctas < 0 || topk_mode < 0 || topk_mode > kTopkModes)
+        return fail(PARISKV_EINVAL, "launch shape (%d, %d, %d) out of range", vote_ctas,
+                    rerank_ctas, topk_mode);
+    ix->vote_ctas = vote_ctas;
+    ix->rerank_ctas = rerank_ctas;
+    ix->topk_mode = topk_mode;
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_debug_union_rows(int64_t* rows) {
+    if (!rows) return fail(PARISKV_EINVAL, "rows is NULL");
+    cudaError_t e = cudaDeviceSynchronize();
+    unsigned long long r = 0;
+    if (e == cudaSuccess) e = read_union_rows(&r);
+    if (e != cudaSuccess) return cuda_fail(e, "union row counter");
+    *rows = static_cast<int64_t>(r);
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_debug_check_guards(void) {
+    if (!guards_on()) return fail(PARISKV_EINVAL, "guard bytes are off (PARISKV_GUARD=1 not set)");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "device synchronise");
+    std::lock_guard<std::mutex> lk(g_guard_mu);
+    for (const Guarded& g : g_guarded) guard_ok(g);
+    if (g_guard_bad[0]) {
+        const pariskv_status r = fail(PARISKV_ECUDA, "%s", g_guard_bad);
+        g_guard_bad[0] = 0;
+        return r;
+    }
     return PARISKV_OK;
 }
 

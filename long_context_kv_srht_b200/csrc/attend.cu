@@ -17,6 +17,7 @@
 // memory and the CTA writes (128 accumulators, max, denominator) to the workspace; a second
 // kernel merges the splits with the log-sum-exp rule and writes the output in the input
 // dtype.
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -189,6 +190,192 @@ attend_combine_kernel(const float* __restrict__ work, int nsplit, T* __restrict_
     store4<T>(out + static_cast<int64_t>(head) * D + 4 * lane, o);
 }
 
+// ---------------------------------------------------------------------------------------
+// GQA-group union: the G query heads of a KV head often select the same rows; each union row
+// is fetched once (over PCIe when K/V live in pinned host memory) and scored for every head
+// that selected it.
+// ---------------------------------------------------------------------------------------
+constexpr int kUnionT = 1024;     // threads of the union-building CTA (one per unit)
+
+__device__ unsigned long long g_union_rows;   // union rows fetched, summed until read
+
+// bit (row mod 32) of word row / 32 of head's bitmap, for every valid index of the head
+__global__ void __launch_bounds__(256)
+union_mark_kernel(const int32_t* __restrict__ topk, int32_t k, int64_t n, int64_t nw,
+                  uint32_t* __restrict__ bits) {
+    const int64_t head = blockIdx.y;
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= k) return;
+    const int32_t r = topk[head * k + i];
+    if (r < 0 || r >= n) return;   // skipped like the per-head kernel skips them
+    atomicOr(bits + head * nw + (r >> 5), 1u << (r & 31));
+}
+
+// One CTA per unit: the OR of the group's bitmaps, scanned into the ascending union row list
+// with each row's membership mask (bit g = query head g of the group selected it).
+__global__ void __launch_bounds__(kUnionT)
+union_build_kernel(const uint32_t* __restrict__ bits, int G, int64_t nw, int64_t cap,
+                   int32_t* __restrict__ rows, uint8_t* __restrict__ masks,
+                   int32_t* __restrict__ count) {
+    __shared__ uint32_t wsum[kUnionT / 32];
+    const int64_t unit = blockIdx.x;
+    const uint32_t* b = bits + unit * G * nw;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t per = (nw + kUnionT - 1) / kUnionT;
+    const int64_t w0 = min64(nw, per * threadIdx.x), w1 = min64(nw, w0 + per);
+    uint32_t c = 0;
+    for (int64_t w = w0; w < w1; ++w) {
+        uint32_t u = 0;
+        for (int g = 0; g < G; ++g) u |= b[g * nw + w];
+        c += __popc(u);
+    }
+    uint32_t x = c;   // inclusive scan over the warp, then over the warps
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    uint32_t before = 0, total = 0;
+    for (int i = 0; i < kUnionT / 32; ++i) {
+        before += i < warp ? wsum[i] : 0u;
+        total += wsum[i];
+    }
+    int64_t pos = unit * cap + before + x - c;
+    for (int64_t w = w0; w < w1; ++w) {
+        uint32_t bg[8], u = 0;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            bg[g] = g < G ? b[g * nw + w] : 0u;
+            u |= bg[g];
+        }
+        while (u) {
+            const int bit = __ffs(u) - 1;
+            u &= u - 1u;
+            uint32_t m = 0;
+#pragma unroll
+            for (int g = 0; g < 8; ++g) m |= ((bg[g] >> bit) & 1u) << g;
+            rows[pos] = static_cast<int32_t>(32 * w + bit);
+            masks[pos] = static_cast<uint8_t>(m);
+            ++pos;
+        }
+    }
+    if (threadIdx.x == 0) {
+        count[unit] = static_cast<int32_t>(total);
+        atomicAdd(&g_union_rows, static_cast<unsigned long long>(total));
+    }
+}
+
+// Split-K partials over a unit's union rows: CTA (split, unit) takes a contiguous slice of
+// the union; each warp walks every 8th row of it, a lane holding 4 of the 128 dims, with the
+// row fetches pipelined as in attend_partial_kernel, and keeps one online-softmax state per
+// query head of the group (GM >= G, a compile-time bound so the states stay in registers).
+// Each head's partial goes where the per-head kernel would put it, so the same merge follows.
+template <typename T, int GM>
+__global__ void __launch_bounds__(kAW * 32)
+attend_union_kernel(const T* __restrict__ q, const T* __restrict__ K, const T* __restrict__ V,
+                    int64_t ld_tok, const int32_t* __restrict__ rows,
+                    const uint8_t* __restrict__ masks, const int32_t* __restrict__ count,
+                    int64_t cap, float scale, int G, int nsplit, float* __restrict__ work) {
+    __shared__ __align__(16) float sm[kAW][kPart];
+    const int64_t unit = blockIdx.y;
+    const int split = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t u = count[unit];
+    const int64_t t0 = u * split / nsplit, t1 = u * (split + 1) / nsplit;
+    float qv[GM][4], mx[GM], den[GM], acc[GM][4];
+#pragma unroll
+    for (int g = 0; g < GM; ++g) {
+        if (g < G) Elem<T>::load4(q + (unit * G + g) * D + 4 * lane, qv[g]);
+        mx[g] = -INFINITY;
+        den[g] = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[g][i] = 0.0f;
+    }
+    const T* Kb = K + unit * ld_tok * D + 4 * lane;
+    const T* Vb = V + unit * ld_tok * D + 4 * lane;
+    const int32_t* ur = rows + unit * cap;
+    const uint8_t* um = masks + unit * cap;
+    const int64_t mine = t1 - t0 > warp ? (t1 - t0 - warp + kAW - 1) / kAW : 0;
+    for (int64_t b0 = 0; b0 < mine; b0 += 64) {
+        const int cnt = static_cast<int>(min64(64, mine - b0));
+        int32_t ir[2];
+        uint32_t im[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int j = 32 * h + lane;
+            const int64_t t = t0 + warp + (b0 + j) * kAW;
+            ir[h] = j < cnt ? ur[t] : -1;
+            im[h] = j < cnt ? um[t] : 0u;
+        }
+        auto row_of = [&](int j) -> int32_t {
+            const int32_t a = __shfl_sync(0xffffffffu, ir[0], j & 31);
+            const int32_t b = __shfl_sync(0xffffffffu, ir[1], j & 31);
+            return j < cnt ? (j < 32 ? a : b) : -1;
+        };
+        auto mask_of = [&](int j) -> uint32_t {
+            const uint32_t a = __shfl_sync(0xffffffffu, im[0], j & 31);
+            const uint32_t b = __shfl_sync(0xffffffffu, im[1], j & 31);
+            return j < cnt ? (j < 32 ? a : b) : 0u;
+        };
+        float kv[2][kUnroll][4], vv[2][kUnroll][4];
+        uint32_t mw[2][kUnroll];
+        auto load_stage = [&](int buf, int j0) {
+#pragma unroll
+            for (int e = 0; e < kUnroll; ++e) {
+                const int32_t row = row_of(j0 + e);
+                mw[buf][e] = row >= 0 ? mask_of(j0 + e) : 0u;
+                if (row >= 0) {
+                    Elem<T>::load4(Kb + static_cast<int64_t>(row) * D, kv[buf][e]);
+                    Elem<T>::load4(Vb + static_cast<int64_t>(row) * D, vv[buf][e]);
+                }
+            }
+        };
+        auto consume = [&](int buf) {
+#pragma unroll
+            for (int e = 0; e < kUnroll; ++e)
+#pragma unroll
+                for (int g = 0; g < GM; ++g)
+                    if ((mw[buf][e] >> g) & 1u)
+                        softmax_step(qv[g], kv[buf][e], vv[buf][e], scale, mx[g], den[g], acc[g]);
+        };
+        load_stage(0, 0);
+        for (int j0 = 0; j0 < cnt; j0 += 2 * kUnroll) {
+            if (j0 + kUnroll < cnt) load_stage(1, j0 + kUnroll);
+            consume(0);
+            if (j0 + kUnroll >= cnt) break;
+            if (j0 + 2 * kUnroll < cnt) load_stage(0, j0 + 2 * kUnroll);
+            consume(1);
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < GM; ++g) {
+        if (g >= G) break;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sm[warp][4 * lane + i] = acc[g][i];
+        if (lane == 0) { sm[warp][kMax] = mx[g]; sm[warp][kDen] = den[g]; }
+        __syncthreads();
+        if (warp == 0) {
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kAW; ++w) M = fmaxf(M, sm[w][kMax]);
+            float dsum = 0.0f, a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int w = 0; w < kAW; ++w) {
+                const float f = sm[w][kMax] == -INFINITY ? 0.0f : expf(sm[w][kMax] - M);
+                dsum += sm[w][kDen] * f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) a[i] += sm[w][4 * lane + i] * f;
+            }
+            float* out = work + ((unit * G + g) * nsplit + split) * kPart;
+            *reinterpret_cast<float4*>(out + 4 * lane) = make_float4(a[0], a[1], a[2], a[3]);
+            if (lane == 0) { out[kMax] = M; out[kDen] = dsum; }
+        }
+        __syncthreads();
+    }
+}
+
 // Fixed workspace of the allocation-free attention entry point: split-K partials in a
 // file-scope device array, so a call needs no allocator. Every device that loads the library
 // holds these 4 MiB until the process exits; all calls on a device share them.
@@ -291,6 +478,82 @@ cudaError_t launch_attend_combine(int heads, const float* work, int split_total,
         attend_combine_kernel<float><<<heads, 32, 0, st>>>(work, split_total,
                                                            static_cast<float*>(out));
     return cudaGetLastError();
+}
+
+// The union scratch: group bitmaps [units][G][ceil(n / 32)] words, then the union rows
+// [units][G k] (int32), their masks [units][G k] (u8) and the counts [units]. Used for
+// 1 < group <= 8 while the bitmaps stay within kUnionBitmapBytes, unless the environment has
+// PARISKV_ATTEND_UNION=0.
+constexpr size_t kUnionBitmapBytes = size_t(256) << 20;
+
+static size_t union_bitmap_words(const pariskv_config* cfg, int64_t n) {
+    return static_cast<size_t>(cfg->batch) * cfg->num_kv_heads * cfg->group *
+           static_cast<size_t>((n + 31) / 32);
+}
+
+size_t union_workspace_bytes(const pariskv_config* cfg, int64_t n, int32_t k) {
+    const char* env = getenv("PARISKV_ATTEND_UNION");
+    if (env && env[0] == '0') return 0;
+    if (cfg->group < 2 || cfg->group > 8) return 0;
+    const size_t words = union_bitmap_words(cfg, n);
+    if (words * 4 > kUnionBitmapBytes) return 0;
+    const size_t units = static_cast<size_t>(cfg->batch) * cfg->num_kv_heads;
+    const size_t cap = static_cast<size_t>(cfg->group) * k;
+    const size_t b = words * 4 + units * cap * 4 + round_up(units * cap, 16) + units * 4;
+    return round_up(b, 256);
+}
+
+int union_splits(int units, int group, int32_t k, int num_sms) {
+    // one wave of one CTA per SM (the kernel keeps G softmax states and two register stages
+    // of rows per lane: one 8-warp CTA fills an SM's registers)
+    const int want = static_cast<int>(static_cast<int64_t>(num_sms) / units);
+    const int most = static_cast<int>(ceil_div(static_cast<int64_t>(group) * k, 64));
+    return max(1, min(want, most));
+}
+
+cudaError_t launch_attend_union(const pariskv_config* cfg, const void* q, const void* K,
+                                const void* V, int64_t ld_tok, int64_t n, const int32_t* topk,
+                                int32_t k, float scale, void* out, int32_t out_dtype,
+                                float* work, int nsplit, void* scratch, cudaStream_t st) {
+    const int G = cfg->group;
+    const int units = cfg->batch * cfg->num_kv_heads;
+    const int64_t nw = (n + 31) / 32, cap = static_cast<int64_t>(G) * k;
+    const size_t words = union_bitmap_words(cfg, n);
+    uint32_t* bits = static_cast<uint32_t*>(scratch);
+    int32_t* rows = reinterpret_cast<int32_t*>(bits + words);
+    uint8_t* masks = reinterpret_cast<uint8_t*>(rows + static_cast<size_t>(units) * cap);
+    int32_t* count = reinterpret_cast<int32_t*>(masks + round_up(static_cast<size_t>(units) * cap, 16));
+    cudaError_t e = cudaMemsetAsync(bits, 0, words * 4, st);
+    if (e != cudaSuccess) return e;
+    union_mark_kernel<<<dim3(static_cast<unsigned>(ceil_div(k, 256)), units * G), 256, 0, st>>>(
+        topk, k, n, nw, bits);
+    union_build_kernel<<<units, kUnionT, 0, st>>>(bits, G, nw, cap, rows, masks, count);
+    dim3 grid(nsplit, units);
+    const bool bf = cfg->dtype == PARISKV_BF16;
+#define PKV_UNION_LAUNCH(TT, GM)                                                              \
+    attend_union_kernel<TT, GM><<<grid, kAW * 32, 0, st>>>(                                   \
+        static_cast<const TT*>(q), static_cast<const TT*>(K), static_cast<const TT*>(V),      \
+        ld_tok, rows, masks, count, cap, scale, G, nsplit, work)
+    if (bf) {
+        if (G <= 2) PKV_UNION_LAUNCH(__nv_bfloat16, 2);
+        else if (G <= 4) PKV_UNION_LAUNCH(__nv_bfloat16, 4);
+        else PKV_UNION_LAUNCH(__nv_bfloat16, 8);
+    } else {
+        if (G <= 2) PKV_UNION_LAUNCH(float, 2);
+        else if (G <= 4) PKV_UNION_LAUNCH(float, 4);
+        else PKV_UNION_LAUNCH(float, 8);
+    }
+#undef PKV_UNION_LAUNCH
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_attend_combine(units * G, work, nsplit, out, out_dtype, st);
+}
+
+cudaError_t read_union_rows(unsigned long long* rows) {
+    cudaError_t e = cudaMemcpyFromSymbol(rows, g_union_rows, sizeof(*rows));
+    if (e != cudaSuccess) return e;
+    const unsigned long long zero = 0;
+    return cudaMemcpyToSymbol(g_union_rows, &zero, sizeof(zero));
 }
 
 cudaError_t launch_attend(const pariskv_config* cfg, const void* q, const void* K,

@@ -40,6 +40,13 @@ struct pariskv_index {
     int64_t cmax = 0;
     int* status = nullptr;      // device status word (ST_OK / ST_TIMEOUT)
 
+    // test hooks: one out-of-range candidate index written before the next rerank (head < 0:
+    // none), and launch shapes forced for the determinism tests (0: automatic)
+    int32_t inject_head = -1;
+    int64_t inject_pos = 0;
+    int32_t inject_value = 0;
+    int32_t vote_ctas = 0, rerank_ctas = 0, topk_mode = 0;
+
     // optional per-stage timing of searches (test and benchmark use)
     bool profile = false;
     cudaEvent_t ev[8] = {};
@@ -130,6 +137,13 @@ cudaError_t launch_vote(const pariskv_index* ix, cudaStream_t st);
 // select.cu
 cudaError_t launch_threshold(const pariskv_index* ix, int64_t C, cudaStream_t st);
 cudaError_t launch_compact(const pariskv_index* ix, cudaStream_t st);
+// writes `value` to *dst on the stream (the bad-candidate test hook)
+cudaError_t launch_poke(int32_t* dst, int32_t value, cudaStream_t st);
+// top-k launch shapes that pariskv_debug_set_launch may force: 1 one 1024-thread CTA per head
+// (C <= 8192), 2 one 256-thread CTA (C <= 8192), 3 a cluster of four 1024-thread CTAs with the
+// values in shared memory (C <= 65536), 4 the same cluster reading global memory (any C)
+constexpr int kTopkModes = 4;
+bool topk_mode_fits(int mode, int64_t C);
 
 // rerank.cu
 cudaError_t launch_rerank(const pariskv_index* ix, int64_t C, cudaStream_t st);
@@ -161,6 +175,18 @@ cudaError_t launch_attend_partial(const pariskv_config* cfg, const void* q, cons
                                   bool mma, cudaStream_t st);
 cudaError_t launch_attend_combine(int heads, const float* work, int split_total, void* out,
                                   int32_t out_dtype, cudaStream_t st);
+// GQA-group union (attend.cu): for the row-gather kernel with 1 < group <= 8, the group's
+// top-k lists are merged into one ascending union of rows per unit with a membership mask per
+// row; each union row is fetched once and scored for every query head that selected it.
+// union_workspace_bytes is the scratch launch_attend_union needs (0: the union is not used for
+// this shape); the partials then take union_splits splits per head.
+size_t union_workspace_bytes(const pariskv_config* cfg, int64_t n, int32_t k);
+int union_splits(int units, int group, int32_t k, int num_sms);
+cudaError_t launch_attend_union(const pariskv_config* cfg, const void* q, const void* K,
+                                const void* V, int64_t ld_tok, int64_t n, const int32_t* topk,
+                                int32_t k, float scale, void* out, int32_t out_dtype,
+                                float* work, int nsplit, void* scratch, cudaStream_t st);
+cudaError_t read_union_rows(unsigned long long* rows);   // rows fetched since the last read
 // floats per split partial in the attention workspace: 128 accumulators, the running max
 // (natural-log units) and the denominator, padded so every partial starts 16-byte aligned
 constexpr int kAttendPart = 128 + 4;

@@ -29,9 +29,12 @@
 // (subspace 2t, subspace 2t + 1) fp32 pairs, each read once by broadcast for both records; a
 // lane walks the 8 subspace pairs in order, two p chains advancing together in Blackwell's
 // packed fp32x2 FMA (each half an ordinary IEEE fp32 FMA), and extends each record's S chain
-// after every pair. Decoding is exact integer arithmetic: the stored offset-binary nibbles
-// u = vt + 8 are split into even and odd dims with two masks, a PRMT places u in the
-// mantissa of 2^23, and one packed subtraction of 2^23 + 8 gives vt exactly as fp32.
+// after every pair. Decoding is exact integer arithmetic on the code words of the two
+// subspaces, which one shared-memory load leaves in a register pair: one LOP3 per half puts
+// the offset-binary nibble u = vt + 8 of a dimension into the mantissa of 2^23 (scaled by a
+// power of 16 that the staged query undoes exactly), and one packed subtraction gives vt as
+// fp32. (Placing the nibbles with PRMT into two single registers needed about one register
+// move per value to form the pair, 20 % more instructions per record.)
 #include "common.cuh"
 #include "internal.hpp"
 
@@ -46,7 +49,7 @@ constexpr int kSlots = 2;               // stages in flight per warp
 constexpr int kPerLane = 2;             // records scored per lane and stage
 constexpr int kStageRecs = 32 * kPerLane;
 constexpr int kStageBytes = kStageRecs * REC;
-constexpr int kQBytes = D * 4;          // one head's rotated query
+constexpr int kQBytes = 2 * D * 4;      // one head's rotated query, plain and scaled pairs
 constexpr int kWarpBytes = kSlots * kStageBytes + kQBytes;
 constexpr int kSmem = kWarps * kWarpBytes;
 static_assert(kWarpBytes % 128 == 0, "warp areas stay 128-byte aligned");
@@ -99,6 +102,46 @@ __device__ __forceinline__ float2 pair_dots(uint32_t wa, uint32_t wb, const uint
     return unpack2(p);
 }
 
+// Scaled decode (uniform levels): the code words of subspaces a and b form one 64-bit value
+// w = {wa, wb} (a register pair as loaded), and dim j's nibble u sits at bits 4 j of each
+// half. For j <= 4, (w & (15 << 4 j)) | bits(2^23) holds 2^23 + u 16^j in both halves;
+// dims 5..7 take the same from w >> 16 with j - 4. Subtracting 2^23 + 8 16^e (e = j or
+// j - 4) leaves vt 16^e exactly, and the query pair of dim j is staged as q~ 16^-e, so each
+// FMA of the chain gets the exact product vt q~ and rounds exactly as fma(vt, q~, p) does.
+// The scaling is exact while no query component is a nonzero value below 2^-100 (checked
+// when the query is staged; such a query takes the unscaled path).
+// The mask and the exponent bits live in registers (opaque to the compiler's constant
+// folding), and each half is one LOP3 (w & m) | e writing straight into the pair that the
+// packed subtraction reads, so no register moves are needed to form the pair.
+__device__ __forceinline__ uint64_t opaque64(uint64_t v) {
+    uint64_t r;
+    asm volatile("mov.b64 %0, %1;" : "=l"(r) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ uint64_t lev_scaled(uint64_t w, int sh, uint64_t kc) {
+    const uint64_t m = opaque64(0x0000000F0000000Full << sh);
+    const uint64_t e = opaque64(0x4B0000004B000000ull);
+    uint64_t r;
+    asm("{\n .reg .b32 wl, wh, ml, mh, el, eh, rl, rh;\n mov.b64 {wl, wh}, %1;\n mov.b64 {ml, mh}, %2;\n"
+        " mov.b64 {el, eh}, %3;\n lop3.b32 rl, wl, ml, el, 0xEA;\n lop3.b32 rh, wh, mh, eh, 0xEA;\n"
+        " mov.b64 %0, {rl, rh};\n}" : "=l"(r) : "l"(w), "l"(m), "l"(e));
+    return add2(r, kc);
+}
+__device__ __forceinline__ float2 pair_dots_scaled(uint64_t w, const uint64_t q[8],
+                                                   const uint64_t kc[5]) {
+    uint64_t p = 0;   // (0.0f, 0.0f)
+    p = fma2(lev_scaled(w, 0, kc[0]), q[0], p);
+    p = fma2(lev_scaled(w, 4, kc[1]), q[1], p);
+    p = fma2(lev_scaled(w, 8, kc[2]), q[2], p);
+    p = fma2(lev_scaled(w, 12, kc[3]), q[3], p);
+    p = fma2(lev_scaled(w, 16, kc[4]), q[4], p);
+    const uint64_t v = w >> 16;
+    p = fma2(lev_scaled(v, 4, kc[1]), q[5], p);
+    p = fma2(lev_scaled(v, 8, kc[2]), q[6], p);
+    p = fma2(lev_scaled(v, 12, kc[3]), q[7], p);
+    return unpack2(p);
+}
+
 __device__ __forceinline__ void load_qpairs(const uint64_t* qp, uint64_t q[8]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -109,50 +152,70 @@ __device__ __forceinline__ void load_qpairs(const uint64_t* qp, uint64_t q[8]) {
 }
 
 // S of the kPerLane records in stage rows row0 + 32 u; qp = the head's 64 query pairs (pair
-// t at qp + 8 t). Each query pair is read once for all the lane's records; every record
-// keeps its own p and S chains in the defined order.
-template <bool TABLE>
+// t at qp + 8 t), qs_scaled the same pairs scaled for the scaled decode. Each query pair is
+// read once for all the lane's records; every record keeps its own p and S chains in the
+// defined order.
+template <bool TABLE, bool SCALED>
 __device__ __forceinline__ void score_records(const uint8_t* st, int row0, const uint64_t* qp,
                                               const float* dec, float S[kPerLane]) {
+    const uint64_t kc[5] = {pack2(-8388616.0f, -8388616.0f), pack2(-8388736.0f, -8388736.0f),
+                            pack2(-8390656.0f, -8390656.0f), pack2(-8421376.0f, -8421376.0f),
+                            pack2(-8912896.0f, -8912896.0f)};   // -(2^23 + 8 16^e)
 #pragma unroll
     for (int u = 0; u < kPerLane; ++u) S[u] = 0.0f;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {   // chunk c: subspaces 4c..4c+3
-        uint4 cw[kPerLane], fw[kPerLane];
+        ulonglong2 cw[kPerLane];
+        uint4 fw[kPerLane];
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
-            cw[u] = *reinterpret_cast<const uint4*>(st + piece_at(row0 + 32 * u, 2 * c));
+            cw[u] = *reinterpret_cast<const ulonglong2*>(st + piece_at(row0 + 32 * u, 2 * c));
             fw[u] = *reinterpret_cast<const uint4*>(st + piece_at(row0 + 32 * u, 2 * c + 1));
         }
         uint64_t q[8];
         load_qpairs(qp + 16 * c, q);
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
-            const float2 pa = pair_dots<TABLE>(cw[u].x, cw[u].y, q, dec);
+            const float2 pa =
+                SCALED ? pair_dots_scaled(cw[u].x, q, kc)
+                       : pair_dots<TABLE>(static_cast<uint32_t>(cw[u].x),
+                                          static_cast<uint32_t>(cw[u].x >> 32), q, dec);
             S[u] = __fmaf_rn(__uint_as_float(fw[u].x), pa.x, S[u]);
             S[u] = __fmaf_rn(__uint_as_float(fw[u].y), pa.y, S[u]);
         }
         load_qpairs(qp + 16 * c + 8, q);
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
-            const float2 pb = pair_dots<TABLE>(cw[u].z, cw[u].w, q, dec);
+            const float2 pb =
+                SCALED ? pair_dots_scaled(cw[u].y, q, kc)
+                       : pair_dots<TABLE>(static_cast<uint32_t>(cw[u].y),
+                                          static_cast<uint32_t>(cw[u].y >> 32), q, dec);
             S[u] = __fmaf_rn(__uint_as_float(fw[u].z), pb.x, S[u]);
             S[u] = __fmaf_rn(__uint_as_float(fw[u].w), pb.y, S[u]);
         }
     }
 }
 
-// Stages head h's rotated query into the warp's pair table: entry 8 t + j holds
-// (q~[16 t + j], q~[16 t + 8 + j]).
-__device__ __forceinline__ void stage_query(const float* __restrict__ qt, int64_t h,
-                                            float2* qs, int lane) {
+// Stages head h's rotated query into the warp's pair tables: entry 8 t + j of qs holds
+// (q~[16 t + j], q~[16 t + 8 + j]) and of qss the same pair times 16^-e (e = j for j <= 4,
+// else j - 4) for the scaled decode. Returns whether the scaling is exact for this query.
+__device__ __forceinline__ bool stage_query(const float* __restrict__ qt, int64_t h, float2* qs,
+                                            float2* qss, int lane) {
     const float* qh = qt + h * D;
+    bool tiny = false;
 #pragma unroll
     for (int e = lane; e < 64; e += 32) {
         const int t = e >> 3, j = e & 7;
-        qs[e] = make_float2(qh[16 * t + j], qh[16 * t + 8 + j]);
+        const float a = qh[16 * t + j], b = qh[16 * t + 8 + j];
+        qs[e] = make_float2(a, b);
+        const float sc = j == 0 ? 1.0f : j == 1 || j == 5 ? 0.0625f : j == 2 || j == 6 ? 0.00390625f
+                       : j == 3 || j == 7 ? 0.000244140625f : 1.52587890625e-05f;   // 16^-e
+        qss[e] = make_float2(__fmul_rn(a, sc), __fmul_rn(b, sc));
+        tiny |= (a != 0.0f && fabsf(a) < 7.8886091e-31f) || (b != 0.0f && fabsf(b) < 7.8886091e-31f);
     }
+    const bool ok = !__any_sync(0xffffffffu, tiny);   // 7.8886091e-31 = 2^-100
     __syncwarp();
+    return ok;
 }
 
 // Work is cut into items of kItem consecutive candidates of one query head; warp g of the
@@ -184,7 +247,9 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* ring = smem + warp * kWarpBytes;
     float2* qs = reinterpret_cast<float2*>(ring + kSlots * kStageBytes);
+    float2* qss = qs + 64;
     const uint64_t* qp = reinterpret_cast<const uint64_t*>(qs);
+    const uint64_t* qps = reinterpret_cast<const uint64_t*>(qss);
     const int64_t W = static_cast<int64_t>(gridDim.x) * kWarps;
     const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
 
@@ -257,7 +322,8 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
         pend = load_idx(iss);
     }
 
-    int staged = -1;   // head whose query is in qs
+    int staged = -1;       // head whose query is in qs
+    bool scaled = false;   // its scaled pairs are exact
 #pragma unroll 1
     for (int g = 0; sc.it < items; ++g) {
         const int slot = g % kSlots;
@@ -266,12 +332,13 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
         asm volatile("cp.async.wait_group %0;" :: "n"(kSlots - 1) : "memory");
         __syncwarp();
         if (sc.head != staged) {
-            stage_query(qt, sc.head, qs, lane);
+            scaled = stage_query(qt, sc.head, qs, qss, lane);
             staged = sc.head;
         }
         const uint8_t* st = ring + slot * kStageBytes;
         float sv[kPerLane];
-        score_records<TABLE>(st, lane, qp, dec, sv);
+        if (!TABLE && scaled) score_records<false, true>(st, lane, qps, dec, sv);
+        else score_records<TABLE, false>(st, lane, qp, dec, sv);
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
             const int c = sc.c0 + kStageRecs * sc.s + 32 * u + lane;

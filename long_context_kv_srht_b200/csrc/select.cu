@@ -351,6 +351,13 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
 
 }  // namespace
 
+static __global__ void poke_kernel(int32_t* dst, int32_t value) { *dst = value; }
+
+cudaError_t launch_poke(int32_t* dst, int32_t value, cudaStream_t st) {
+    poke_kernel<<<1, 1, 0, st>>>(dst, value);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_threshold(const pariskv_index* ix, int64_t C, cudaStream_t st) {
     const int64_t nchunks = ceil_div(ix->n, CHUNK);
     const int heads = ix->units * ix->cfg.group;

@@ -280,8 +280,19 @@ cudaError_t launch_cfg(const pariskv_index* ix, int64_t C, int32_t k, int32_t* t
 
 }  // namespace
 
+bool topk_mode_fits(int mode, int64_t C) {
+    return mode == 1 || mode == 2 ? C <= 8192 : mode == 3 ? C <= 4 * 16384 : mode == 4;
+}
+
 cudaError_t launch_topk(const pariskv_index* ix, int64_t C, int32_t k, int32_t* topk_idx,
                         float* topk_est, cudaStream_t st) {
+    switch (ix->topk_mode) {   // a launch shape forced by the determinism tests
+        case 1: return launch_cfg<1, 1024, 8192, true>(ix, C, k, topk_idx, topk_est, st);
+        case 2: return launch_cfg<1, 256, 8192, true>(ix, C, k, topk_idx, topk_est, st);
+        case 3: return launch_cfg<4, 1024, 16384, true>(ix, C, k, topk_idx, topk_est, st);
+        case 4: return launch_cfg<4, 1024, 16384, false>(ix, C, k, topk_idx, topk_est, st);
+        default: break;
+    }
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

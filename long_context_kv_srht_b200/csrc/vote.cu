@@ -220,7 +220,7 @@ cudaError_t launch_vote(const pariskv_index* ix, cudaStream_t st) {
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int grid = static_cast<int>(min64(items, 2LL * sms));
+    const int grid = static_cast<int>(min64(items, ix->vote_ctas > 0 ? ix->vote_ctas : 2LL * sms));
     return launch_pdl(vote_kernel, grid, kThreads, kSmemBytes, st, ix->ids, ix->lut, ix->scores,
                       ix->hist, ix->n, ix->cap_pad, ix->packs, ix->cfg.group, nchunks, items,
                       ix->status);

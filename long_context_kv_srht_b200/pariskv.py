@@ -96,6 +96,10 @@ _SIGS = {
     "pariskv_debug_profile": (_S, [_P, _I32]),
     "pariskv_debug_stage_ms": (_S, [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_I32)]),
     "pariskv_debug_read_stream": (_S, [_P, _I64, _P, _P]),
+    "pariskv_debug_inject_bad_candidate": (_S, [_P, _I32, _I64, _I32]),
+    "pariskv_debug_set_launch": (_S, [_P, _I32, _I32, _I32]),
+    "pariskv_debug_check_guards": (_S, []),
+    "pariskv_debug_union_rows": (_S, [ctypes.POINTER(_I64)]),
     "pariskv_cache_create": (_S, [ctypes.POINTER(Config), ctypes.POINTER(CacheConfig), _P, _P,
                                   ctypes.POINTER(_P)]),
     "pariskv_cache_prefill": (_S, [_P, _P, _P, _I64, _I64, _P]),
@@ -247,6 +251,16 @@ class Index:
                "pariskv_debug_search_rotated")
         return idx, est
 
+    def inject_bad_candidate(self, head: int, pos: int, value: int) -> None:
+        """pariskv_debug_inject_bad_candidate (test hook, consumed by the next search)."""
+        _check(lib.pariskv_debug_inject_bad_candidate(self.handle, head, pos, value),
+               "pariskv_debug_inject_bad_candidate")
+
+    def set_launch(self, vote_ctas: int = 0, rerank_ctas: int = 0, topk_mode: int = 0) -> None:
+        """pariskv_debug_set_launch: force the launch shapes of later searches (0: automatic)."""
+        _check(lib.pariskv_debug_set_launch(self.handle, vote_ctas, rerank_ctas, topk_mode),
+               "pariskv_debug_set_launch")
+
     def profile(self, enable: bool = True) -> None:
         _check(lib.pariskv_debug_profile(self.handle, int(enable)), "pariskv_debug_profile")
 
@@ -352,6 +366,20 @@ def rotate(cfg: Config, signs, x, stream=None):
     _check(lib.pariskv_debug_rotate(ctypes.byref(cfg), sp, x.data_ptr(), n, y.data_ptr(),
                                     nr.data_ptr(), _stream(stream)), "pariskv_debug_rotate")
     return y, nr
+
+
+def check_guards() -> None:
+    """pariskv_debug_check_guards: the guard bytes around every live index buffer are intact
+    (requires PARISKV_GUARD=1 in the environment before the first index is created)."""
+    _check(lib.pariskv_debug_check_guards(), "pariskv_debug_check_guards")
+
+
+def union_rows() -> int:
+    """pariskv_debug_union_rows: K/V rows the GQA-group union attention fetched since the
+    last call (current device)."""
+    r = _I64(0)
+    _check(lib.pariskv_debug_union_rows(ctypes.byref(r)), "pariskv_debug_union_rows")
+    return int(r.value)
 
 
 def sparse_attend(cfg: Config, q, K, V, topk_idx, k: int, scale: float, n: Optional[int] = None,

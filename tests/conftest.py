@@ -7,6 +7,10 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+# Guard bytes around every device buffer an index owns (a stand-in for a memory checker):
+# set before the library makes its first allocation; checked after every GPU test below.
+os.environ.setdefault("PARISKV_GUARD", "1")
+
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
@@ -37,3 +41,13 @@ def pytest_sessionstart(session):
     kbuild.build()
     import oracle
     oracle.build()
+
+
+@pytest.fixture(autouse=True)
+def _guard_bytes_intact(request):
+    """After each GPU test: no kernel wrote past either end of an index buffer."""
+    yield
+    if "gpu" not in request.keywords or not _has_gpu() or os.environ.get("PARISKV_GUARD") != "1":
+        return
+    from long_context_kv_srht_b200 import pariskv as pk
+    pk.check_guards()

@@ -107,9 +107,9 @@ def _run(dtype, hkv, G, n_sink, n_local, n_buffer, k, n0, steps, host_prefill, o
             ref = oracle.attend(q[tok, h], K[0, h // G], V[0, h // G], toks, SCALE)
             tol = 2e-3 if out_f32 else 2e-3 + np.abs(ref) * 2.0 ** -8
             assert np.all(np.abs(got[h] - ref) <= tol), (t, h, np.abs(got[h] - ref).max())
-    # raw inputs: the GPU rotates in fp32, the oracle in fp64, so near-tied keys may differ
+    # raw inputs: the GPU rotates in fp32, the oracle in fp64, so a near-tied key may differ
     if want:
-        assert hits / want >= 0.995, hits / want
+        assert hits / want >= 0.999, hits / want
     cache.destroy()
     return promotions
 

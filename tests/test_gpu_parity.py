@@ -31,12 +31,15 @@ def _t(a):
 
 
 def _compare_rotated(batch, hkv, G, n, k, keys, qs, signs, rho=4, w1=2, wr=1, bp=500, cap=None,
-                     table=None):
+                     table=None, edit_qt=None):
     """Build + search from the oracle's rotated inputs; compare every stage bit for bit
-    (table: code both sides with these magnitude levels)."""
+    (table: code both sides with these magnitude levels; edit_qt(qt) may change the rotated
+    queries in place before both sides see them)."""
     units = batch * hkv
     y, kn = rotate_all(keys.reshape(units, n, 128), signs)
     qt, qn = rotate_all(qs.reshape(units * G, 128), signs)
+    if edit_qt is not None:
+        edit_qt(qt)
     cfg = _cfg(batch, hkv, G, cap or n, rho=rho, w1=w1, wr=wr, bp=bp, table=table)
     ix = pk.build_index_rotated(cfg, signs, _t(y), _t(kn))
     idx, est = ix.search_rotated(_t(qt), _t(qn), k)
@@ -154,6 +157,27 @@ def test_adversarial_keys_bit_exact():
     _compare_rotated(1, 1, G, n, 400, keys, qs, random_signs(9), bp=1000)
 
 
+def test_tiny_query_components_bit_exact():
+    """Rotated queries with components near the bottom of the fp32 range (2^-110, normal
+    values below 2^-100, subnormals), exact zeros and -0: the rerank stages the query scaled
+    by powers of 16 only when that is exact, and every stage stays bit for bit."""
+    rng = np.random.default_rng(23)
+    n, G = 5000, 4
+    keys = rng.standard_normal((n, 128)).astype(np.float32)
+    qs = rng.standard_normal((G, 128)).astype(np.float32)
+
+    def edit(qt):
+        qt[0, 3] = np.float32(2.0 ** -110)
+        qt[0, 77] = np.float32(-3.0e-36)
+        qt[1, 5] = np.float32(1.0e-40)               # subnormal
+        qt[1, 100] = np.float32(-2.0 ** -101)
+        qt[2, 0:16] = 0.0
+        qt[2, 16:20] = -0.0
+        qt[3, 9] = np.float32(2.0 ** -99)             # just above the exactness bound
+
+    _compare_rotated(1, 1, G, n, 300, keys, qs, random_signs(29), bp=1000, edit_qt=edit)
+
+
 def test_append_equals_build():
     sp = workload.spec("tiny", num_kv_heads=2, group=4, n=12000, seed=21)
     w = workload.generate(sp)
@@ -252,6 +276,57 @@ def test_sparse_attend_matches_oracle(dtype, G, n, k, host_kv, out_f32):
                                 topk[b * hkv * G + h].astype(np.int32), 1 / np.sqrt(128))
             tol = 2e-3 if out_f32 else 2e-3 + np.abs(ref) * 2.0 ** -8
             assert np.all(np.abs(got[b, h] - ref) <= tol)
+
+
+@pytest.mark.parametrize("dtype,G,host_kv", [("bf16", 4, True), ("f32", 4, False),
+                                             ("bf16", 8, True), ("bf16", 3, True),
+                                             ("bf16", 2, True)])
+def test_group_union_attention_shares_rows(dtype, G, host_kv, monkeypatch):
+    """The query heads of a group select overlapping rows (a common core, a shared pool and
+    rows of their own); the row-gather attention fetches each row of the group's union once
+    and still matches the oracle per head at 2e-3. The fetched-row count equals the union
+    size, and turning the union off gives the same outputs within the same bound."""
+    rng = np.random.default_rng(31 + G)
+    batch, hkv, n, k = 2, 2, 20000, 1024
+    K = rng.standard_normal((batch, hkv, n, 128)).astype(np.float32) * 0.5
+    V = rng.standard_normal((batch, hkv, n, 128)).astype(np.float32)
+    q = rng.standard_normal((batch, hkv * G, 128)).astype(np.float32)
+    if dtype == "bf16":
+        K, V, q = workload.bf16_round(K), workload.bf16_round(V), workload.bf16_round(q)
+        conv = lambda a: torch.from_numpy(workload.bf16_bits(a)).view(torch.bfloat16)
+    else:
+        conv = lambda a: torch.from_numpy(np.ascontiguousarray(a))
+    topk, union = [], 0
+    for u in range(batch * hkv):
+        core = rng.choice(n, k // 2, replace=False)            # every head of the group
+        pool = np.setdiff1d(rng.choice(n, 2 * k, replace=False), core)
+        rows = set()
+        for g in range(G):
+            own = rng.choice(pool, k - k // 2, replace=False)   # partly shared, partly not
+            sel = np.sort(np.concatenate([core, own]))
+            assert len(np.unique(sel)) == k
+            topk.append(sel)
+            rows |= set(sel.tolist())
+        union += len(rows)
+    topk = np.stack(topk).astype(np.int32)
+    cfg = _cfg(batch, hkv, G, n, dtype=dtype)
+    Kt, Vt = conv(K), conv(V)
+    Kt, Vt = (Kt.pin_memory(), Vt.pin_memory()) if host_kv else (Kt.to(DEV), Vt.to(DEV))
+    pk.union_rows()                                            # reset the counter
+    out = pk.sparse_attend(cfg, conv(q).to(DEV), Kt, Vt, _t(topk), k, 1 / np.sqrt(128),
+                           out_dtype=torch.float32)
+    assert pk.union_rows() == union < batch * hkv * G * k
+    got = out.cpu().numpy()
+    for b in range(batch):
+        for h in range(hkv * G):
+            ref = oracle.attend(q[b, h], K[b, h // G], V[b, h // G],
+                                topk[b * hkv * G + h], 1 / np.sqrt(128))
+            assert np.all(np.abs(got[b, h] - ref) <= 2e-3)
+    monkeypatch.setenv("PARISKV_ATTEND_UNION", "0")
+    per_head = pk.sparse_attend(cfg, conv(q).to(DEV), Kt, Vt, _t(topk), k, 1 / np.sqrt(128),
+                                out_dtype=torch.float32)
+    assert pk.union_rows() == 0
+    assert (per_head - out).abs().max().item() <= 2e-3
 
 
 # ------------------------------------------------------------------------------- errors
