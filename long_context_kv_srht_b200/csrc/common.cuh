@@ -26,6 +26,20 @@ constexpr int PACK = 4;         // query heads whose vote weights share one 32-b
 // kernel of the library waits on another (each stage is its own launch), so it is reserved.
 enum : int { ST_OK = 0, ST_TIMEOUT = 5, ST_BADINDEX = 6 };
 
+// The checked build (-DPKV_CHECK=1, libpariskv_check.so) adds device-side checks of values
+// that are correct by construction in a consistent run (score bytes, output positions and
+// indices); a failed check records ST_BADINDEX and skips the access. Never a trap.
+#ifndef PKV_CHECK
+#define PKV_CHECK 0
+#endif
+__device__ __forceinline__ bool pkv_check(bool ok, int* status) {
+    if (PKV_CHECK && !ok) {
+        atomicExch(status, ST_BADINDEX);
+        return false;
+    }
+    return true;
+}
+
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 __host__ __device__ constexpr int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 __host__ __device__ constexpr int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }

@@ -342,7 +342,7 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
             const int c = sc.c0 + kStageRecs * sc.s + 32 * u + lane;
-            const bool ok = c < sc.cend;
+            const bool ok = c < sc.cend && pkv_check(c < cmax, status);   // (checked build)
             if (ok) S[sc.head * cmax + c] = sv[u];
             // the top-k's first radix level: count the values by their top order-key bits,
             // one global reduction per distinct bin in the warp (values cluster in few bins)

@@ -332,6 +332,7 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
 #pragma unroll
         for (int w = 0; w < kWords; ++w) nsel += __popc(sel[w]);
         const int32_t start = cbase[hb + 0] + gbefore + min(B, ebefore);
+        if (!pkv_check(start >= 0, status)) continue;   // (checked build)
         if (start + nsel > C) {               // never taken when the histograms are consistent
             atomicExch(status, ST_BADINDEX);
             continue;

@@ -177,7 +177,9 @@ vote_kernel(const uint8_t* __restrict__ ids, const uint32_t* __restrict__ lut,
                 if (kk + 32 * j < nkeys) sc_out[kk + 32 * j] = acc[j];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                if (kk + 32 * j < nkeys) {
+                // (checked build) every packed score byte is below 64: a larger one would
+                // count into the next head's histogram rows
+                if (kk + 32 * j < nkeys && pkv_check((acc[j] & 0xC0C0C0C0u) == 0u, status)) {
                     const uint32_t sc = acc[j] + 0xC0804000u;  // byte h -> 64 h + score_h
                     hist_inc<0>(tab, sc, hcol);
                     if (hp > 1) hist_inc<1>(tab, sc, hcol);

@@ -16,7 +16,10 @@ from typing import Optional
 import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "_lib", "libpariskv.so")
+# PARISKV_LIBRARY=check loads the checked build (extra device-side bounds checks; see
+# build.py); the default is the product library.
+LIB_PATH = os.path.join(_PKG, "_lib", "libpariskv_check.so" if os.environ.get(
+    "PARISKV_LIBRARY") == "check" else "libpariskv.so")
 HEADERS = [os.path.join(os.path.dirname(_PKG), "include", h)
            for h in ("pariskv.h", "pariskv_cache.h", "pariskv_dense.h", "pariskv_learned.h",
                      "pariskv_debug.h")]

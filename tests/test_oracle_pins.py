@@ -452,6 +452,40 @@ def test_ratio_levels_are_lloyd_max():
     np.testing.assert_allclose(lv, emp, atol=3e-3)
 
 
+def test_ratio_law_closed_forms_for_two_and_three_dims():
+    """For m = 2, r = |g_j| / max|g| is 1 with probability 1/2 and otherwise the ratio of
+    two half-normals, whose density on [0, 1) is 2 / (pi (1 + x^2)) (the half-Cauchy law
+    of |g_1 / g_2|). For m = 3 the t-integral has the closed form
+    integral_0^inf t exp(-a t^2) erf(b t) dt = b / (2 a sqrt(a + b^2)), which gives
+    f(x) = 4 / (pi (1 + x^2) sqrt(2 + x^2)), of mass 2/3 on [0, 1). Both pin the density
+    formula (the factor m - 1, the two half-normal densities and the Psi^(m - 2) term)
+    without the oracle's own quadrature."""
+    x = (np.arange(2000) + 0.5) / 2000
+    np.testing.assert_allclose(oracle.ratio_density(x, m=2), 2 / (np.pi * (1 + x * x)),
+                               atol=5e-7)
+    np.testing.assert_allclose(oracle.ratio_density(x, m=3),
+                               4 / (np.pi * (1 + x * x) * np.sqrt(2 + x * x)), atol=1e-9)
+    assert abs(4 / np.pi * np.arctan(1 / np.sqrt(3)) - 2 / 3) < 1e-15   # the m = 3 mass
+
+
+def test_ratio_levels_two_dims_by_closed_form_lloyd():
+    """The level recipe (cell masses and moments from cumulative integrals, interpolated at
+    the thresholds; the point mass at 1 in the top cell; Lloyd to convergence) against the
+    same fixed point computed from the m = 2 law's closed-form integrals
+    F0(x) = (2 / pi) atan x and F1(x) = ln(1 + x^2) / pi."""
+    lv = oracle.ratio_levels(m=2).astype(np.float64)
+    F0 = lambda t: 2 / np.pi * np.arctan(t)
+    F1 = lambda t: np.log1p(t * t) / np.pi
+    ref = (np.arange(8) + 0.5) / 8
+    for _ in range(5000):
+        e = np.concatenate([[0.0], 0.5 * (ref[:-1] + ref[1:]), [1.0]])
+        s0, s1 = np.diff(F0(e)), np.diff(F1(e))
+        s0[7] += 0.5
+        s1[7] += 0.5
+        ref = s1 / s0
+    np.testing.assert_allclose(lv, ref, atol=1e-6)
+
+
 def test_table_codes_nearest_level():
     """Table-coded magnitudes are the nearest table level to r = |y_j| / max|y| (fp32 ratio,
     fp32 midpoint thresholds), the signs are the coordinate signs, and the maximal coordinate
