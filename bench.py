@@ -48,6 +48,15 @@ def parse():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the search and dense-comparator lines of the other workloads")
+    ap.add_argument("--profile-run", action="store_true",
+                    help="for profilers: build the index, run --warmup + --steps searches (and "
+                         "with --attend the sparse attention over the top-k) and exit; no "
+                         "timing, no JSON line, no extra device buffers")
+    ap.add_argument("--attend", action="store_true",
+                    help="with --profile-run: also run the sparse attention after each search")
+    ap.add_argument("--n", type=int, default=None,
+                    help="with --profile-run: index this many keys instead of the workload's n "
+                         "(a reduced case for captures that replay each launch many times)")
     ap.add_argument("--centroids", choices=["analytic", "learned"], default="analytic",
                     help="drift_32k: coarse centroids (analytic, or learned from the prefill "
                          "by spherical k-means: the comparator of the drift claim)")
@@ -610,6 +619,41 @@ def run_drift(args, ws, rank, local):
         dist.destroy_process_group()
 
 
+def profile_run(args, local):
+    """The search (and optionally the sparse attention) of the workload, untimed, for an
+    ncu capture: K/V in pinned host memory at the million-token workload as in the bench,
+    on the device otherwise; --n reduces the number of keys."""
+    import numpy as np
+    import torch
+    from long_context_kv_srht_b200 import pariskv as pk
+    from long_context_kv_srht_b200 import workload
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(local)
+    sp = workload.spec(args.workload)
+    if args.n:
+        sp = workload.spec(args.workload, n=args.n)
+    kv_host = sp.name == "million_offload"
+    data = workload.generate_torch(sp, dev, n=sp.n, kv_on_host=kv_host)
+    cfg = pk.config(batch=sp.batch, num_kv_heads=sp.num_kv_heads, group=sp.group,
+                    capacity=sp.n, dtype=sp.dtype, rho=sp.rho, cand_bp=sp.cand_bp,
+                    levels=args.levels)
+    ix = pk.build_index(cfg, data["signs"], data["keys"], n=sp.n)
+    H, k = sp.batch * sp.num_q_heads, min(sp.k, sp.n)
+    idx = torch.empty((H, k), dtype=torch.int32, device=dev)
+    est = torch.empty((H, k), dtype=torch.float32, device=dev)
+    out = torch.empty(data["queries"].shape, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup + args.steps):
+        ix.search(data["queries"], k, idx, est)
+        if args.attend:
+            pk.sparse_attend(cfg, data["queries"], data["keys"], data["values"], idx, k,
+                             1.0 / float(np.sqrt(sp.d)), out=out)
+    torch.cuda.synchronize()
+    ix.sync()
+    ix.destroy()
+    print(f"profile run: {sp.name}, n = {sp.n}, {args.warmup + args.steps} searches"
+          + (" + attention" if args.attend else ""), flush=True)
+
+
 def main():
     args = parse()
     ws, rank, local = dist_setup(args)
@@ -621,6 +665,9 @@ def main():
         return
     if args.workload == "drift_32k":
         run_drift(args, ws, rank, local)
+        return
+    if args.profile_run:
+        profile_run(args, local)
         return
     import numpy as np
     import torch
