@@ -22,8 +22,8 @@ constexpr int CHUNK = 8192;     // keys per coarse-score histogram chunk (a vote
 constexpr int PACK = 4;         // query heads whose vote weights share one 32-bit table entry
 
 // Device status word. ST_BADINDEX: a kernel found an index out of range and skipped the
-// access. ST_TIMEOUT is the code a bounded device-side wait records when it runs out; no
-// kernel of the library waits on another (each stage is its own launch), so it is reserved.
+// access. ST_TIMEOUT: a bounded device-side wait ran out (the top-k's wait for its own bulk
+// copies; no kernel of the library waits on another, each stage is its own launch).
 enum : int { ST_OK = 0, ST_TIMEOUT = 5, ST_BADINDEX = 6 };
 
 // The checked build (-DPKV_CHECK=1, libpariskv_check.so) adds device-side checks of values

@@ -13,8 +13,10 @@
 // share an SM and even many heads run in about one wave) -- and otherwise a cluster of four
 // 1024-thread CTAs:
 //  - CTA r copies the r-th part of the head's S values and candidate indices into shared
-//    memory with asynchronous copies, all in flight at once, and turns S into u in place
-//    (parts longer than the slice stay in global memory and are re-read on every pass);
+//    memory with two bulk asynchronous copies (each a contiguous range, from the 16-byte
+//    boundary at or below the part's start) completing on one mbarrier, and turns S into u
+//    in place (parts longer than the slice stay in global memory and are re-read on every
+//    pass);
 //  - the first radix level, the top 11 bits of u, was counted by the rerank as it wrote S
 //    (per head, SCOPIES copies of a 2048-bin histogram in global memory), so it costs one
 //    round of reads here;
@@ -53,6 +55,7 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
     static_assert(kWarps <= 32 && kBins % T == 0 && (BPT == 2 || BPT == 8), "layout");
     extern __shared__ __align__(16) uint32_t dyn[];
     __shared__ __align__(16) uint32_t hist[2][kBins];
+    __shared__ __align__(8) uint64_t lbar;   // completion of the part's bulk copies
     __shared__ uint32_t wa[kWarps], wb[kWarps];
     __shared__ uint32_t ctot[2];       // this CTA's candidates above T / ties at T
     __shared__ uint32_t pick[2];
@@ -66,8 +69,12 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
     const int L = s1 - s0;
     const float* Sh = S + head * cmax + s0;
     const int32_t* ch = cand + head * cmax + s0;
-    uint32_t* keys = dyn;                                   // [SLICE] u
-    int32_t* idx = reinterpret_cast<int32_t*>(dyn + SLICE);  // [SLICE] candidate index
+    // the part is copied from a 16-byte boundary (rows start on one: cmax is a multiple of
+    // 32), so it sits `off` = s0 mod 4 words into each buffer
+    const int off = RES ? (s0 & 3) : 0;
+    uint32_t* keys = dyn + off;                                    // [SLICE] u
+    // (a copied range is at most L + 6 words long: buffers of SLICE + 8 words)
+    int32_t* idx = reinterpret_cast<int32_t*>(dyn + SLICE + 8) + off;   // [SLICE] candidate index
     auto key_at = [&](int i) -> uint32_t { return RES ? keys[i] : order_key(Sh[i]); };
     auto idx_at = [&](int i) -> int32_t { return RES ? idx[i] : ch[i]; };
     auto sync_all = [&]() {
@@ -89,18 +96,35 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
     pdl_wait();
     pdl_launch_dependents();
 
-    // 1. this CTA's part into shared memory (asynchronous 4-byte copies, all in flight at
-    //    once); then u in place
+    // 1. this CTA's part into shared memory: two bulk asynchronous copies (values and
+    //    indices, from the 16-byte boundary at or below s0 to the one at or above s1, which
+    //    stays inside the row) completing on one mbarrier; then u in place
     if (RES) {
-        for (int i = threadIdx.x; i < L; i += T) {
-            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(keys + i)),
-                         "l"(Sh + i) : "memory");
-            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(idx + i)),
-                         "l"(ch + i) : "memory");
+        const uint32_t bar = smem_addr(&lbar);
+        const int a0 = s0 & ~3, a1 = (s1 + 3) & ~3;
+        const uint32_t bytes = static_cast<uint32_t>(a1 - a0) * 4u;
+        if (threadIdx.x == 0) {
+            mbar_init(bar, 1);
+            mbar_fence_init();
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        for (int i = threadIdx.x; i < L; i += T)   // each thread converts what it copied
+        __syncthreads();
+        if (threadIdx.x == 0 && bytes) {
+            mbar_arrive_expect_tx(bar, 2 * bytes);
+            bulk_g2s(smem_addr(dyn), S + head * cmax + a0, bytes, bar);
+            bulk_g2s(smem_addr(dyn + SLICE + 8), cand + head * cmax + a0, bytes, bar);
+        }
+        if (bytes) {
+            // bounded: past about a second of polling the part is treated as lost and the
+            // status word records a timeout (never taken while the copies complete)
+            long long spins = 0;
+            while (!mbar_try_wait(bar, 0u)) {
+                if (++spins > (1LL << 26)) {
+                    atomicExch(status, ST_TIMEOUT);
+                    break;
+                }
+            }
+        }
+        for (int i = threadIdx.x; i < L; i += T)   // each thread converts a strided share
             keys[i] = order_key(__uint_as_float(keys[i]));
     }
 
@@ -172,7 +196,7 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
 #pragma unroll
         for (int j = 0; j < BPT; ++j) hb[threadIdx.x + T * j] = 0u;
         __syncthreads();
-        if (RES && (L & 3) == 0) {
+        if (RES && off == 0 && (L & 3) == 0) {
             const uint4* k4 = reinterpret_cast<const uint4*>(keys);
             for (int i = threadIdx.x; i < (L >> 2); i += T) {
                 const uint4 v = k4[i];
@@ -265,7 +289,7 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
 template <int CL, int T, int SLICE, bool RES>
 cudaError_t launch_cfg(const pariskv_index* ix, int64_t C, int32_t k, int32_t* topk_idx,
                        float* topk_est, cudaStream_t st) {
-    constexpr int kDyn = RES ? 2 * SLICE * 4 : 0;
+    constexpr int kDyn = RES ? 2 * (SLICE + 8) * 4 : 0;
     static std::atomic<uint64_t> smem_raised{0};
     if (kDyn > 0) {   // static + dynamic shared memory can pass the 48 KB default
         cudaError_t e = raise_smem_limit(topk_kernel<CL, T, SLICE, RES>, kDyn, smem_raised);
