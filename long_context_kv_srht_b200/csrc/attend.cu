@@ -277,7 +277,8 @@ __global__ void __launch_bounds__(kAW * 32)
 attend_union_kernel(const T* __restrict__ q, const T* __restrict__ K, const T* __restrict__ V,
                     int64_t ld_tok, const int32_t* __restrict__ rows,
                     const uint8_t* __restrict__ masks, const int32_t* __restrict__ count,
-                    int64_t cap, float scale, int G, int nsplit, float* __restrict__ work) {
+                    int64_t cap, float scale, int G, int nsplit, int split_base,
+                    int split_total, float* __restrict__ work) {
     __shared__ __align__(16) float sm[kAW][kPart];
     const int64_t unit = blockIdx.y;
     const int split = blockIdx.x;
@@ -368,7 +369,7 @@ attend_union_kernel(const T* __restrict__ q, const T* __restrict__ K, const T* _
 #pragma unroll
                 for (int i = 0; i < 4; ++i) a[i] += sm[w][4 * lane + i] * f;
             }
-            float* out = work + ((unit * G + g) * nsplit + split) * kPart;
+            float* out = work + ((unit * G + g) * split_total + split_base + split) * kPart;
             *reinterpret_cast<float4*>(out + 4 * lane) = make_float4(a[0], a[1], a[2], a[3]);
             if (lane == 0) { out[kMax] = M; out[kDen] = dsum; }
         }
@@ -511,10 +512,11 @@ int union_splits(int units, int group, int32_t k, int num_sms) {
     return max(1, min(want, most));
 }
 
-cudaError_t launch_attend_union(const pariskv_config* cfg, const void* q, const void* K,
-                                const void* V, int64_t ld_tok, int64_t n, const int32_t* topk,
-                                int32_t k, float scale, void* out, int32_t out_dtype,
-                                float* work, int nsplit, void* scratch, cudaStream_t st) {
+cudaError_t launch_union_partial(const pariskv_config* cfg, const void* q, const void* K,
+                                 const void* V, int64_t ld_tok, int64_t n, const int32_t* topk,
+                                 int32_t k, float scale, float* work, int nsplit,
+                                 int split_base, int split_total, void* scratch,
+                                 cudaStream_t st) {
     const int G = cfg->group;
     const int units = cfg->batch * cfg->num_kv_heads;
     const int64_t nw = (n + 31) / 32, cap = static_cast<int64_t>(G) * k;
@@ -533,7 +535,7 @@ cudaError_t launch_attend_union(const pariskv_config* cfg, const void* q, const 
 #define PKV_UNION_LAUNCH(TT, GM)                                                              \
     attend_union_kernel<TT, GM><<<grid, kAW * 32, 0, st>>>(                                   \
         static_cast<const TT*>(q), static_cast<const TT*>(K), static_cast<const TT*>(V),      \
-        ld_tok, rows, masks, count, cap, scale, G, nsplit, work)
+        ld_tok, rows, masks, count, cap, scale, G, nsplit, split_base, split_total, work)
     if (bf) {
         if (G <= 2) PKV_UNION_LAUNCH(__nv_bfloat16, 2);
         else if (G <= 4) PKV_UNION_LAUNCH(__nv_bfloat16, 4);
@@ -544,9 +546,18 @@ cudaError_t launch_attend_union(const pariskv_config* cfg, const void* q, const 
         else PKV_UNION_LAUNCH(float, 8);
     }
 #undef PKV_UNION_LAUNCH
-    e = cudaGetLastError();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attend_union(const pariskv_config* cfg, const void* q, const void* K,
+                                const void* V, int64_t ld_tok, int64_t n, const int32_t* topk,
+                                int32_t k, float scale, void* out, int32_t out_dtype,
+                                float* work, int nsplit, void* scratch, cudaStream_t st) {
+    cudaError_t e = launch_union_partial(cfg, q, K, V, ld_tok, n, topk, k, scale, work, nsplit, 0,
+                                         nsplit, scratch, st);
     if (e != cudaSuccess) return e;
-    return launch_attend_combine(units * G, work, nsplit, out, out_dtype, st);
+    return launch_attend_combine(cfg->batch * cfg->num_kv_heads * cfg->group, work, nsplit, out,
+                                 out_dtype, st);
 }
 
 cudaError_t read_union_rows(unsigned long long* rows) {

@@ -44,6 +44,7 @@ struct pariskv_cache {
     int32_t* dense_idx = nullptr; // device [P]: 0, 1, ..., P - 1 (every head reads it)
     int32_t* topk = nullptr;      // device [heads][k]
     float* work = nullptr;        // device [heads][max_splits][partial]
+    void* uscratch = nullptr;     // GQA-group union of the retrieved rows (NULL: per head)
     int max_splits = 0;           // per source (dense, retrieved)
     int sms = 0;
     pariskv_index* ix = nullptr;
@@ -115,6 +116,7 @@ void free_cache(pariskv_cache* c) {
     cudaFree(c->dense_idx);
     cudaFree(c->topk);
     cudaFree(c->work);
+    cudaFree(c->uscratch);
     if (c->hostK) cudaFreeHost(c->hostK);
     if (c->hostV) cudaFreeHost(c->hostV);
     delete c;
@@ -213,8 +215,13 @@ pariskv_status attend(pariskv_cache* c, const void* q, float scale, int32_t k_ef
                              : min(attend_splits(c->heads, static_cast<int32_t>(n_dense), c->sms,
                                                  false),
                                    c->max_splits);
-    const int nr = k_eff > 0 ? min(attend_splits(c->heads, k_eff, c->sms, false), c->max_splits)
-                             : 0;
+    // the retrieved rows: over the GQA group's union (each row read once over PCIe) when the
+    // cache has its scratch, else per head
+    const int nr = k_eff <= 0 ? 0
+                   : c->uscratch ? min(union_splits(c->units, c->cfg.group, k_eff, c->sms),
+                                       c->max_splits)
+                                 : min(attend_splits(c->heads, k_eff, c->sms, false),
+                                       c->max_splits);
     cudaError_t e =
         dense_mma ? launch_dense_partial(&c->cfg, q, c->poolK, c->poolV, c->P, n_dense, scale,
                                          c->work, nd, 0, nd + nr, st)
@@ -223,10 +230,17 @@ pariskv_status attend(pariskv_cache* c, const void* q, float scale, int32_t k_ef
                                           c->work, nd, 0, nd + nr, false, st);
     *launches += 1;
     if (e == cudaSuccess && nr > 0) {
-        e = launch_attend_partial(&c->cfg, q, c->hostK, c->hostV, c->cc.retrieval_capacity,
-                                  c->retr, c->topk, k_eff, k_eff, scale, c->work, nr, nd,
-                                  nd + nr, false, st);
-        *launches += 1;
+        if (c->uscratch) {
+            e = launch_union_partial(&c->cfg, q, c->hostK, c->hostV, c->cc.retrieval_capacity,
+                                     c->retr, c->topk, k_eff, scale, c->work, nr, nd, nd + nr,
+                                     c->uscratch, st);
+            *launches += 3;
+        } else {
+            e = launch_attend_partial(&c->cfg, q, c->hostK, c->hostV, c->cc.retrieval_capacity,
+                                      c->retr, c->topk, k_eff, k_eff, scale, c->work, nr, nd,
+                                      nd + nr, false, st);
+            *launches += 1;
+        }
     }
     if (e == cudaSuccess) {
         e = launch_attend_combine(c->heads, c->work, nd + nr, out, out_dtype, st);
@@ -285,6 +299,10 @@ pariskv_status pariskv_cache_create(const pariskv_config* cfg, const pariskv_cac
         dev_alloc(&c->topk, static_cast<size_t>(c->heads) * cc->k * 4) &&
         dev_alloc(&c->work, attend_workspace_floats(c->heads, 2 * c->max_splits) * 4) &&
         host_alloc(&c->hostK, host) && host_alloc(&c->hostV, host);
+    // the union scratch for the Retrieval zone (bitmaps over its capacity, union lists for k
+    // rows per head); skipped (per-head fetching) when the union does not apply
+    const size_t ub = union_workspace_bytes(&icfg, cc->retrieval_capacity, cc->k);
+    if (ok && ub && !dev_alloc(&c->uscratch, ub)) c->uscratch = nullptr;
     if (!ok) {
         free_cache(c);
         return fail(PARISKV_ENOMEM, "cache allocation failed");

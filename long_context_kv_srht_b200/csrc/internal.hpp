@@ -186,6 +186,13 @@ cudaError_t launch_attend_union(const pariskv_config* cfg, const void* q, const 
                                 const void* V, int64_t ld_tok, int64_t n, const int32_t* topk,
                                 int32_t k, float scale, void* out, int32_t out_dtype,
                                 float* work, int nsplit, void* scratch, cudaStream_t st);
+// the union's split-K partials only, into splits [split_base, split_base + nsplit) of
+// split_total per head (the four-region cache merges them with its dense rows' partials)
+cudaError_t launch_union_partial(const pariskv_config* cfg, const void* q, const void* K,
+                                 const void* V, int64_t ld_tok, int64_t n, const int32_t* topk,
+                                 int32_t k, float scale, float* work, int nsplit,
+                                 int split_base, int split_total, void* scratch,
+                                 cudaStream_t st);
 cudaError_t read_union_rows(unsigned long long* rows);   // rows fetched since the last read
 // floats per split partial in the attention workspace: 128 accumulators, the running max
 // (natural-log units) and the denominator, padded so every partial starts 16-byte aligned
