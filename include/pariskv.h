@@ -148,13 +148,18 @@ PARISKV_API pariskv_status pariskv_search(pariskv_index* index, const void* q, i
  *   out[s][h] = sum_{t in topk[s][h]} softmax_t(scale * <q[s][h], K[s][h/group][t]>) V[..][t]
  *   q:        device pointer [batch][Hq][d]; K, V: device or pinned-host pointers with the
  *             layout of pariskv_build_index's keys (slab stride ld_tok, n valid tokens);
- *   topk_idx: device pointer [batch][Hq][k]; entries outside [0, n) are skipped;
+ *   topk_idx: device pointer [batch][Hq][k]; entries outside [0, n) are skipped; the valid
+ *             entries of one head are distinct (as pariskv_search returns them: a repeated
+ *             index may be attended once or twice depending on the kernel chosen);
  *   out:      device pointer [batch][Hq][d] of element type out_dtype (PARISKV_F32 keeps the
  *             fp32 accumulator precision; PARISKV_BF16 rounds to nearest even).
- * q, K and V have element type cfg->dtype; accumulation is fp32. The split-K partials live in
- * a stream-ordered workspace allocated and freed on `stream` from a memory pool the library
- * keeps per device (it keeps its memory mapped between calls; it holds at most the largest
- * workspaces in flight at once).
+ * q, K and V have element type cfg->dtype; accumulation is fp32. With K/V in pinned host
+ * memory (or fp32) and 1 < group <= 8, the rows the group's query heads selected are merged
+ * into one union per (sequence, KV head) and each union row is fetched once for every head
+ * that selected it. The split-K partials (and that union's bitmaps) live in a stream-ordered
+ * workspace allocated and freed on `stream` from a memory pool the library keeps per device
+ * (it keeps its memory mapped between calls; it holds at most the largest workspaces in
+ * flight at once).
  * Errors: EINVAL, ENOMEM, ECUDA. */
 PARISKV_API pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q,
                                                  const void* K, const void* V, int64_t ld_tok,

@@ -74,13 +74,31 @@ def test_noalloc_matches_oracle_on_two_calls(dtype, host_kv):
 
 
 def test_noalloc_many_heads_near_the_workspace_limit():
-    # 4096 query heads (batch 512 x 8 KV heads): more than half of the heads the workspace
-    # holds; every head against the oracle
-    batch, hkv, G, n, k = 512, 8, 1, 256, 64
-    cfg, q, K, V, topk, host = _case(14, batch, hkv, G, n, k, "bf16")
+    # 4096 query heads (batch 512 x 8 KV heads) with k = 4096 on bf16 K/V in HBM: the fixed
+    # workspace then holds one split per head, fewer than the tensor-core gather needs, so
+    # the call falls back to the row-gather kernel with a single split. K/V (4.3 GB) are
+    # drawn on the device; 64 heads spread over the batch are checked against the oracle.
+    batch, hkv, G, n, k = 512, 8, 1, 4096, 4096
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(14)
+    K = (torch.randn((batch, hkv, n, 128), generator=gen, device=DEV) * 0.5).to(torch.bfloat16)
+    V = torch.randn((batch, hkv, n, 128), generator=gen, device=DEV).to(torch.bfloat16)
+    q = torch.randn((batch, hkv * G, 128), generator=gen, device=DEV).to(torch.bfloat16)
+    topk = torch.arange(n, dtype=torch.int32, device=DEV).repeat(batch * hkv * G, 1)
+    cfg = pk.config(batch=batch, num_kv_heads=hkv, group=G, capacity=n, dtype="bf16")
     got = pk.sparse_attend_noalloc(cfg, q, K, V, topk, k, SCALE, out_dtype=torch.float32)
     torch.cuda.synchronize()
-    _check_against_oracle(got, host, G)
+    assert pk.last_launch_count() == 2
+    rows = np.arange(n, dtype=np.int32)
+    worst = 0.0
+    for i in np.linspace(0, batch * hkv * G - 1, 64).astype(int):
+        b, h = divmod(int(i), hkv * G)
+        ref = oracle.attend(q[b, h].float().cpu().numpy(), K[b, h // G].float().cpu().numpy(),
+                            V[b, h // G].float().cpu().numpy(), rows, SCALE)
+        worst = max(worst, float(np.abs(got[b, h].cpu().numpy() - ref).max()))
+    assert worst <= 2e-3, worst
+    del K, V
+    torch.cuda.empty_cache()
 
 
 def test_noalloc_rejects_requests_beyond_its_workspace():
