@@ -564,7 +564,7 @@ pariskv_status pariskv_sparse_attend(const pariskv_config* cfg, const void* q, c
     if (ubytes) {
         e = launch_attend_union(cfg, q, K, V, ld_tok, n, topk_idx, k, scale, out, out_dtype, work,
                                 nsplit, reinterpret_cast<char*>(work) + pbytes, st);
-        if (e == cudaSuccess) g_launches = 4;
+        if (e == cudaSuccess) g_launches = 5;   // mark, count, write, attention, merge
     } else {
         e = launch_attend(cfg, q, K, V, ld_tok, n, topk_idx, k, scale, out, out_dtype, work,
                           nsplit, mma, st);

@@ -195,7 +195,8 @@ attend_combine_kernel(const float* __restrict__ work, int nsplit, T* __restrict_
 // is fetched once (over PCIe when K/V live in pinned host memory) and scored for every head
 // that selected it.
 // ---------------------------------------------------------------------------------------
-constexpr int kUnionT = 1024;     // threads of the union-building CTA (one per unit)
+constexpr int kUnionT = 256;      // threads of a union-building CTA
+constexpr int kUnionBlocks = 32;  // union-building CTAs per unit
 
 __device__ unsigned long long g_union_rows;   // union rows fetched, summed until read
 
@@ -211,25 +212,23 @@ union_mark_kernel(const int32_t* __restrict__ topk, int32_t k, int64_t n, int64_
     atomicOr(bits + head * nw + (r >> 5), 1u << (r & 31));
 }
 
-// One CTA per unit: the OR of the group's bitmaps, scanned into the ascending union row list
-// with each row's membership mask (bit g = query head g of the group selected it).
-__global__ void __launch_bounds__(kUnionT)
-union_build_kernel(const uint32_t* __restrict__ bits, int G, int64_t nw, int64_t cap,
-                   int32_t* __restrict__ rows, uint8_t* __restrict__ masks,
-                   int32_t* __restrict__ count) {
-    __shared__ uint32_t wsum[kUnionT / 32];
-    const int64_t unit = blockIdx.x;
-    const uint32_t* b = bits + unit * G * nw;
+// The union of the group's bitmaps, scanned into the ascending union row list with each row's
+// membership mask (bit g = query head g of the group selected it), over kUnionBlocks CTAs per
+// unit: union_count_kernel counts each block's rows, union_write_kernel offsets a block by the
+// counts of the unit's earlier blocks and writes its rows in order.
+__device__ __forceinline__ void union_block_range(int64_t nw, int b, int64_t* w0, int64_t* w1,
+                                                  int64_t* per) {
+    const int64_t wb = (nw + kUnionBlocks - 1) / kUnionBlocks;   // words per block
+    const int64_t b0 = min64(nw, wb * b), b1 = min64(nw, b0 + wb);
+    *per = (b1 - b0 + kUnionT - 1) / kUnionT;                      // words per thread
+    *w0 = min64(b1, b0 + *per * threadIdx.x);
+    *w1 = min64(b1, *w0 + *per);
+}
+
+__device__ __forceinline__ uint32_t union_block_scan(uint32_t c, uint32_t* total,
+                                                     uint32_t* wsum /* [kUnionT / 32] */) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t per = (nw + kUnionT - 1) / kUnionT;
-    const int64_t w0 = min64(nw, per * threadIdx.x), w1 = min64(nw, w0 + per);
-    uint32_t c = 0;
-    for (int64_t w = w0; w < w1; ++w) {
-        uint32_t u = 0;
-        for (int g = 0; g < G; ++g) u |= b[g * nw + w];
-        c += __popc(u);
-    }
-    uint32_t x = c;   // inclusive scan over the warp, then over the warps
+    uint32_t x = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
@@ -237,12 +236,61 @@ union_build_kernel(const uint32_t* __restrict__ bits, int G, int64_t nw, int64_t
     }
     if (lane == 31) wsum[warp] = x;
     __syncthreads();
-    uint32_t before = 0, total = 0;
+    uint32_t before = 0, tot = 0;
+#pragma unroll
     for (int i = 0; i < kUnionT / 32; ++i) {
         before += i < warp ? wsum[i] : 0u;
-        total += wsum[i];
+        tot += wsum[i];
     }
-    int64_t pos = unit * cap + before + x - c;
+    *total = tot;
+    return before + x - c;
+}
+
+__global__ void __launch_bounds__(kUnionT)
+union_count_kernel(const uint32_t* __restrict__ bits, int G, int64_t nw,
+                   uint32_t* __restrict__ bcount) {
+    __shared__ uint32_t wsum[kUnionT / 32];
+    const int64_t unit = blockIdx.y;
+    const uint32_t* b = bits + unit * G * nw;
+    int64_t w0, w1, per;
+    union_block_range(nw, blockIdx.x, &w0, &w1, &per);
+    uint32_t c = 0;
+    for (int64_t w = w0; w < w1; ++w) {
+        uint32_t u = 0;
+        for (int g = 0; g < G; ++g) u |= b[g * nw + w];
+        c += __popc(u);
+    }
+    uint32_t total;
+    union_block_scan(c, &total, wsum);
+    if (threadIdx.x == 0) bcount[unit * kUnionBlocks + blockIdx.x] = total;
+}
+
+__global__ void __launch_bounds__(kUnionT)
+union_write_kernel(const uint32_t* __restrict__ bits, int G, int64_t nw, int64_t cap,
+                   const uint32_t* __restrict__ bcount, int32_t* __restrict__ rows,
+                   uint8_t* __restrict__ masks, int32_t* __restrict__ count) {
+    __shared__ uint32_t wsum[kUnionT / 32];
+    __shared__ uint32_t sbase;
+    const int64_t unit = blockIdx.y;
+    const uint32_t* b = bits + unit * G * nw;
+    if (threadIdx.x < 32) {   // the unit's rows in the blocks before this one
+        uint32_t x = 0;
+        for (int i = threadIdx.x; i < blockIdx.x; i += 32) x += bcount[unit * kUnionBlocks + i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (threadIdx.x == 0) sbase = x;
+    }
+    int64_t w0, w1, per;
+    union_block_range(nw, blockIdx.x, &w0, &w1, &per);
+    uint32_t c = 0;
+    for (int64_t w = w0; w < w1; ++w) {
+        uint32_t u = 0;
+        for (int g = 0; g < G; ++g) u |= b[g * nw + w];
+        c += __popc(u);
+    }
+    uint32_t total;
+    const uint32_t before = union_block_scan(c, &total, wsum);   // (its barrier orders sbase)
+    int64_t pos = unit * cap + sbase + before;
     for (int64_t w = w0; w < w1; ++w) {
         uint32_t bg[8], u = 0;
 #pragma unroll
@@ -261,9 +309,10 @@ union_build_kernel(const uint32_t* __restrict__ bits, int G, int64_t nw, int64_t
             ++pos;
         }
     }
-    if (threadIdx.x == 0) {
-        count[unit] = static_cast<int32_t>(total);
-        atomicAdd(&g_union_rows, static_cast<unsigned long long>(total));
+    if (blockIdx.x == kUnionBlocks - 1 && threadIdx.x == 0) {
+        const uint32_t all = sbase + total;
+        count[unit] = static_cast<int32_t>(all);
+        atomicAdd(&g_union_rows, static_cast<unsigned long long>(all));
     }
 }
 
@@ -500,7 +549,8 @@ size_t union_workspace_bytes(const pariskv_config* cfg, int64_t n, int32_t k) {
     if (words * 4 > kUnionBitmapBytes) return 0;
     const size_t units = static_cast<size_t>(cfg->batch) * cfg->num_kv_heads;
     const size_t cap = static_cast<size_t>(cfg->group) * k;
-    const size_t b = words * 4 + units * cap * 4 + round_up(units * cap, 16) + units * 4;
+    const size_t b = words * 4 + units * cap * 4 + round_up(units * cap, 16) + units * 4 +
+                     units * kUnionBlocks * 4;
     return round_up(b, 256);
 }
 
@@ -512,6 +562,30 @@ int union_splits(int units, int group, int32_t k, int num_sms) {
     return max(1, min(want, most));
 }
 
+cudaError_t launch_union_build(const pariskv_config* cfg, int64_t n, const int32_t* topk,
+                               int32_t k, void* scratch, cudaStream_t st, UnionLists* out) {
+    const int G = cfg->group;
+    const int units = cfg->batch * cfg->num_kv_heads;
+    const int64_t nw = (n + 31) / 32, cap = static_cast<int64_t>(G) * k;
+    const size_t words = union_bitmap_words(cfg, n);
+    uint32_t* bits = static_cast<uint32_t*>(scratch);
+    out->cap = cap;
+    out->rows = reinterpret_cast<int32_t*>(bits + words);
+    out->masks = reinterpret_cast<uint8_t*>(out->rows + static_cast<size_t>(units) * cap);
+    out->count = reinterpret_cast<int32_t*>(out->masks +
+                                            round_up(static_cast<size_t>(units) * cap, 16));
+    cudaError_t e = cudaMemsetAsync(bits, 0, words * 4, st);
+    if (e != cudaSuccess) return e;
+    union_mark_kernel<<<dim3(static_cast<unsigned>(ceil_div(k, 256)), units * G), 256, 0, st>>>(
+        topk, k, n, nw, bits);
+    uint32_t* bcount = reinterpret_cast<uint32_t*>(out->count + units);
+    union_count_kernel<<<dim3(kUnionBlocks, units), kUnionT, 0, st>>>(bits, G, nw, bcount);
+    union_write_kernel<<<dim3(kUnionBlocks, units), kUnionT, 0, st>>>(bits, G, nw, cap, bcount,
+                                                                      out->rows, out->masks,
+                                                                      out->count);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_union_partial(const pariskv_config* cfg, const void* q, const void* K,
                                  const void* V, int64_t ld_tok, int64_t n, const int32_t* topk,
                                  int32_t k, float scale, float* work, int nsplit,
@@ -519,17 +593,13 @@ cudaError_t launch_union_partial(const pariskv_config* cfg, const void* q, const
                                  cudaStream_t st) {
     const int G = cfg->group;
     const int units = cfg->batch * cfg->num_kv_heads;
-    const int64_t nw = (n + 31) / 32, cap = static_cast<int64_t>(G) * k;
-    const size_t words = union_bitmap_words(cfg, n);
-    uint32_t* bits = static_cast<uint32_t*>(scratch);
-    int32_t* rows = reinterpret_cast<int32_t*>(bits + words);
-    uint8_t* masks = reinterpret_cast<uint8_t*>(rows + static_cast<size_t>(units) * cap);
-    int32_t* count = reinterpret_cast<int32_t*>(masks + round_up(static_cast<size_t>(units) * cap, 16));
-    cudaError_t e = cudaMemsetAsync(bits, 0, words * 4, st);
+    UnionLists ul;
+    cudaError_t e = launch_union_build(cfg, n, topk, k, scratch, st, &ul);
     if (e != cudaSuccess) return e;
-    union_mark_kernel<<<dim3(static_cast<unsigned>(ceil_div(k, 256)), units * G), 256, 0, st>>>(
-        topk, k, n, nw, bits);
-    union_build_kernel<<<units, kUnionT, 0, st>>>(bits, G, nw, cap, rows, masks, count);
+    const int32_t* rows = ul.rows;
+    const uint8_t* masks = ul.masks;
+    const int32_t* count = ul.count;
+    const int64_t cap = ul.cap;
     dim3 grid(nsplit, units);
     const bool bf = cfg->dtype == PARISKV_BF16;
 #define PKV_UNION_LAUNCH(TT, GM)                                                              \

@@ -234,7 +234,7 @@ pariskv_status attend(pariskv_cache* c, const void* q, float scale, int32_t k_ef
             e = launch_union_partial(&c->cfg, q, c->hostK, c->hostV, c->cc.retrieval_capacity,
                                      c->retr, c->topk, k_eff, scale, c->work, nr, nd, nd + nr,
                                      c->uscratch, st);
-            *launches += 3;
+            *launches += 4;   // the union's mark, count and write kernels, then the partials
         } else {
             e = launch_attend_partial(&c->cfg, q, c->hostK, c->hostV, c->cc.retrieval_capacity,
                                       c->retr, c->topk, k_eff, k_eff, scale, c->work, nr, nd,

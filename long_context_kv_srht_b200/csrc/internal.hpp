@@ -186,6 +186,16 @@ cudaError_t launch_attend_union(const pariskv_config* cfg, const void* q, const 
                                 const void* V, int64_t ld_tok, int64_t n, const int32_t* topk,
                                 int32_t k, float scale, void* out, int32_t out_dtype,
                                 float* work, int nsplit, void* scratch, cudaStream_t st);
+// the union lists of a call (inside its scratch): rows [units][cap], masks [units][cap],
+// count [units]; launch_union_build fills them from the heads' top-k lists
+struct UnionLists {
+    int32_t* rows;
+    uint8_t* masks;
+    int32_t* count;
+    int64_t cap;
+};
+cudaError_t launch_union_build(const pariskv_config* cfg, int64_t n, const int32_t* topk,
+                               int32_t k, void* scratch, cudaStream_t st, UnionLists* out);
 // the union's split-K partials only, into splits [split_base, split_base + nsplit) of
 // split_total per head (the four-region cache merges them with its dense rows' partials)
 cudaError_t launch_union_partial(const pariskv_config* cfg, const void* q, const void* K,

@@ -204,7 +204,7 @@ def test_cache_capacity_and_errors():
 
 def test_cache_step_launch_count():
     """A step is one token-copy kernel, the search's launches, two attention partials and one
-    merge, plus (group > 1) the two kernels that build the GQA group's union of retrieved rows;
+    merge, plus (group > 1) the three kernels that build the GQA group's union of retrieved rows;
     a step that evicts to the Retrieval zone adds the spill, encode and slide kernels."""
     K, V, q = _data(2, 2, 2, 600, "bf16")
     signs = random_signs(2)
@@ -221,5 +221,5 @@ def test_cache_step_launch_count():
         cache.step(qd[t].view(1, 4, 128), Kd[:, :, t].contiguous(), Vd[:, :, t].contiguous(),
                    SCALE)
         seen.append(pk.last_launch_count())
-    assert seen.count(search_launches + 6) == 14 and seen.count(search_launches + 9) == 2
+    assert seen.count(search_launches + 7) == 14 and seen.count(search_launches + 10) == 2
     cache.destroy()
