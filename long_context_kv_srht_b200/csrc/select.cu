@@ -15,8 +15,11 @@
 //    writes for every 8192-key chunk how many candidates and how many score-T keys precede
 //    it (one thread per chunk reads its 64 bins with vector loads; exclusive scans over
 //    chunks).
-//  compact_kernel (one CTA per chunk and vote pack): each thread owns 64 consecutive keys
-//    (read coalesced and transposed through shared memory). SWAR byte arithmetic tests the
+//  compact_kernel (one CTA per chunk and vote pack, seven per SM so that the million-token
+//    search's 1024 CTAs run in one wave): each thread owns 64 consecutive keys, read
+//    coalesced and transposed through shared memory in two halves of 32 (the first half
+//    before the wait for the threshold kernel, the second once the first is consumed; a
+//    single 64-key buffer would allow only six CTAs per SM). SWAR byte arithmetic tests the
 //    four packed scores of a key against the four heads' thresholds at once, and the test
 //    bits are sliced into 32-bit masks per head (above T, at T) over the thread's keys.
 //    POPC gives the counts; one block-wide scan of them gives every thread where its
@@ -177,7 +180,7 @@ constexpr int kKeys = 64;                       // consecutive keys per thread
 constexpr int kWords = kKeys / 32;              // 32-bit key masks per head and kind
 constexpr int kCW = CHUNK / (32 * kKeys);       // compaction: warps per block (one chunk)
 constexpr int kCThr = 32 * kCW;
-constexpr int kRow = kKeys + 1;                 // transposed row stride (conflict-free)
+constexpr int kRow = 33;                        // transposed row stride (conflict-free)
 static_assert(kCW * 32 * kKeys == CHUNK, "one chunk per block");
 
 // Block-wide exclusive scan of two 64-bit values at once (4 packed 16-bit counters each,
@@ -200,12 +203,12 @@ __device__ __forceinline__ void block_excl_scan2(uint64_t& a, uint64_t& b,
     b = by + y - b;
 }
 
-__global__ void __launch_bounds__(kCThr)
+__global__ void __launch_bounds__(kCThr, 7)
 compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ thr,
                const int32_t* __restrict__ cbase, int32_t* __restrict__ cand, int64_t n,
                int64_t cap_pad, int group, int packs, int64_t nchunks, int64_t cmax,
                uint32_t* __restrict__ shist, int* status) {
-    __shared__ uint32_t tr[kCW][32 * kRow];
+    __shared__ uint32_t tr[kCW][32 * kRow];   // one half (32 keys per lane) at a time
     __shared__ uint64_t scan_sh[kCW + 1][2];
     const int64_t c = blockIdx.x;
     const int64_t up = blockIdx.y;
@@ -217,28 +220,27 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
     const int64_t k0 = kw + static_cast<int64_t>(lane) * kKeys;                // thread's first key
     const int nv = static_cast<int>(max64(0, min64(kKeys, n - k0)));          // its valid keys
 
-    // coalesced load of the warp's 32 x kKeys packed scores, transposed so that lane l then
-    // reads keys kKeys l .. kKeys l + kKeys - 1 (row stride kKeys + 1 words: both directions
-    // are conflict-free). Asynchronous 4-byte copies, all in flight at once; keys at or past
-    // n read as 0 (zero fill, src-size 0); their address stays inside the padded capacity.
-    {
-        const uint32_t* src = scores + up * cap_pad + kw + lane;
-        const int nw = static_cast<int>(max64(0, min64(32 * kKeys, n - kw)));
+    // half w of the warp's keys (32 per lane: lane l's keys kKeys l + 32 w .. + 31) into the
+    // transposition buffer: copy t moves lane t's 32 keys, 128 contiguous bytes, so every
+    // warp instruction is one coalesced line; lane l then reads row l (stride 33 words:
+    // conflict-free both ways). Keys at or past n read as 0 (zero fill, src-size 0); their
+    // address stays inside the padded capacity.
+    auto load_half = [&](int w) {
+        const uint32_t* src = scores + up * cap_pad + kw + 32 * w + lane;
 #pragma unroll
-        for (int t = 0; t < kKeys; ++t) {
-            const int key = 32 * t + lane;                 // within the warp's range
-            const uint32_t dst = smem_addr(&tr[warp][(key / kKeys) * kRow + key % kKeys]);
-            const uint32_t bytes = key < nw ? 4u : 0u;
+        for (int t = 0; t < 32; ++t) {
+            const int64_t key = kw + static_cast<int64_t>(kKeys) * t + 32 * w + lane;
+            const uint32_t dst = smem_addr(&tr[warp][t * kRow + lane]);
+            const uint32_t bytes = key < n ? 4u : 0u;
             asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst),
-                         "l"(src + 32 * t), "r"(bytes) : "memory");
+                         "l"(src + kKeys * t), "r"(bytes) : "memory");
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        __syncwarp();
-    }
+    };
+    // the first half is loaded before the wait for the threshold kernel (the scores were
+    // written two kernels back); the second once the first has been consumed
+    load_half(0);
     const uint32_t* s = &tr[warp][lane * kRow];
-    // the scores above were written two kernels back; thresholds and offsets come from the
-    // threshold kernel just before this one
     pdl_wait();
     pdl_launch_dependents();
     // the rerank that follows counts its values per head into shist: start it at zero
@@ -262,13 +264,19 @@ compact_kernel(const uint32_t* __restrict__ scores, const int32_t* __restrict__ 
     uint32_t gm[PACK][kWords], em[PACK][kWords];
 #pragma unroll
     for (int w = 0; w < kWords; ++w) {
+        if (w > 0) {
+            __syncwarp();            // every lane has read the previous half
+            load_half(w);
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncwarp();
         uint32_t G[4], GE[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             uint32_t a = 0, b = 0;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const uint32_t sv = s[32 * w + 8 * q + i];
+                const uint32_t sv = s[8 * q + i];
                 a |= (((sv + gt_add) >> 7) & 0x01010101u) << i;
                 b |= (((sv + ge_add) >> 7) & 0x01010101u) << i;
             }
