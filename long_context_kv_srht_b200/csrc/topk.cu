@@ -56,9 +56,9 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
     extern __shared__ __align__(16) uint32_t dyn[];
     __shared__ __align__(16) uint32_t hist[2][kBins];
     __shared__ __align__(8) uint64_t lbar;   // completion of the part's bulk copies
-    __shared__ uint32_t wa[kWarps], wb[kWarps];
+    __shared__ uint32_t wa[2][kWarps], wb[kWarps];   // wa: per-level warp totals (two sets)
     __shared__ uint32_t ctot[2];       // this CTA's candidates above T / ties at T
-    __shared__ uint32_t pick[2];
+    __shared__ uint32_t pick[2][2];    // per level (two sets): chosen bin, count above it
 
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = CL > 1 ? static_cast<int>(cluster.block_rank()) : 0;
@@ -134,6 +134,10 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
     //    narrows [lo, hi] to it; every CTA sees the same counts and makes the same choice.
     uint32_t krem = static_cast<uint32_t>(k);
     uint32_t lo = 0u, hi = 0xffffffffu;
+    // The shared words a level writes (warp totals, the pick) come in two sets used by
+    // alternate levels, so no barrier is needed between one level's last read and the next
+    // level's first write (the next level's own barriers come first).
+    int par = 0;
     auto choose = [&](const uint32_t h[BPT], int sh) {
         uint32_t mine = 0;
 #pragma unroll
@@ -144,38 +148,35 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
             const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
             if (lane + o < 32) x += y;
         }
-        if (lane == 0) wa[warp] = x;   // warp totals
+        if (lane == 0) wa[par][warp] = x;   // warp totals
         __syncthreads();
-        if (warp == 0) {               // exclusive suffix sums of the warp totals
-            const uint32_t t = lane < kWarps ? wa[lane] : 0u;
-            uint32_t y = t;
+        // the warps after this one, summed by every warp for itself
+        uint32_t aw = lane < kWarps && lane > warp ? wa[par][lane] : 0u;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t z = __shfl_down_sync(0xffffffffu, y, o);
-                if (lane + o < 32) y += z;
-            }
-            if (lane < kWarps) wb[lane] = y - t;
-        }
-        __syncthreads();
-        uint32_t above = wb[warp] + x - mine;   // strictly above this thread's bins
+        for (int o = 16; o > 0; o >>= 1) aw += __shfl_xor_sync(0xffffffffu, aw, o);
+        uint32_t above = aw + x - mine;   // strictly above this thread's bins
 #pragma unroll
         for (int j = BPT - 1; j >= 0; --j) {
             if (above < krem && krem <= above + h[j]) {
-                pick[0] = BPT * threadIdx.x + j;
-                pick[1] = above;
+                pick[par][0] = BPT * threadIdx.x + j;
+                pick[par][1] = above;
             }
             above += h[j];
         }
         __syncthreads();
-        const uint32_t b = pick[0];
-        krem -= pick[1];
+        const uint32_t b = pick[par][0];
+        krem -= pick[par][1];
         const uint32_t nlo = lo + (b << sh);
         const uint64_t bin_hi = static_cast<uint64_t>(nlo) + ((uint64_t{1} << sh) - 1u);
         lo = nlo;
         hi = static_cast<uint32_t>(min(static_cast<uint64_t>(hi), bin_hi));
-        __syncthreads();   // pick[], wa[] and wb[] are rewritten by the next level
+        par ^= 1;
     };
     static_assert(SBINS == kBins, "the first level uses the same bins");
+    // the first histogram buffer starts at zero (the first choose's barriers order this
+    // before the first pass); each later level clears the buffer of the level after it
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) hist[0][threadIdx.x + T * j] = 0u;
     {
         uint32_t h[BPT] = {}, v[BPT];
         const uint32_t* hs = shist + static_cast<int64_t>(head) * SCOPIES * SBINS;
@@ -193,9 +194,6 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
         const uint32_t span = hi - lo;
         const int bitlen = 32 - __clz(span);
         const int sh = bitlen > 11 ? bitlen - 11 : 0;   // (span >> sh) < 2048
-#pragma unroll
-        for (int j = 0; j < BPT; ++j) hb[threadIdx.x + T * j] = 0u;
-        __syncthreads();
         if (RES && off == 0 && (L & 3) == 0) {
             const uint4* k4 = reinterpret_cast<const uint4*>(keys);
             for (int i = threadIdx.x; i < (L >> 2); i += T) {
@@ -212,6 +210,10 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
             }
         }
         sync_all();   // every part's histogram is complete
+        // the other buffer was last read (by every CTA of the head) before this barrier:
+        // clear it for the next level
+#pragma unroll
+        for (int j = 0; j < BPT; ++j) hist[(level + 1) & 1][threadIdx.x + T * j] = 0u;
         uint32_t h[BPT] = {}, v[BPT];
 #pragma unroll
         for (int q = 0; q < CL; ++q) {
@@ -243,11 +245,11 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
         const uint32_t ye = __shfl_up_sync(0xffffffffu, xe, o);
         if (lane >= o) { xg += yg; xe += ye; }
     }
-    if (lane == 31) { wa[warp] = xg; wb[warp] = xe; }
+    if (lane == 31) { wa[par][warp] = xg; wb[warp] = xe; }
     __syncthreads();
     if (threadIdx.x == 0) {
         uint32_t g = 0, e = 0;
-        for (int w = 0; w < kWarps; ++w) { g += wa[w]; e += wb[w]; }
+        for (int w = 0; w < kWarps; ++w) { g += wa[par][w]; e += wb[w]; }
         ctot[0] = g;
         ctot[1] = e;
     }
@@ -260,7 +262,7 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
             eq_run += r[1];
         }
     }
-    for (int w = 0; w < warp; ++w) { gt_run += wa[w]; eq_run += wb[w]; }
+    for (int w = 0; w < warp; ++w) { gt_run += wa[par][w]; eq_run += wb[w]; }
     if constexpr (CL > 1) cluster.barrier_arrive();   // no remote read of this CTA follows
 
     // 4. this thread's winners in key order: every value above Tv, and the ties at Tv while
