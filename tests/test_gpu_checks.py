@@ -60,8 +60,11 @@ def test_bad_candidate_is_reported_and_other_heads_are_unchanged():
     ix.destroy()
 
 
-@pytest.mark.parametrize("n,k,modes", [(60000, 256, (1, 2, 3, 4)), (200000, 512, (3, 4))])
+@pytest.mark.parametrize("n,k,modes", [(60000, 256, (1, 2, 3, 4)), (60030, 256, (1, 2, 3, 4)),
+                                       (200000, 512, (3, 4))])
 def test_every_launch_shape_gives_the_same_bits(n, k, modes):
+    # (n = 60030 gives C = 6003, so the four-CTA top-k parts start 0, 1 and 2 words past a
+    # 16-byte boundary: the bulk copies' offset path)
     ix, q, cfg = _index(n)
     ref_idx, ref_est = ix.search(q, k)
     ix.sync()

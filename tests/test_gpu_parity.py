@@ -278,16 +278,20 @@ def test_sparse_attend_matches_oracle(dtype, G, n, k, host_kv, out_f32):
             assert np.all(np.abs(got[b, h] - ref) <= tol)
 
 
-@pytest.mark.parametrize("dtype,G,host_kv", [("bf16", 4, True), ("f32", 4, False),
-                                             ("bf16", 8, True), ("bf16", 3, True),
-                                             ("bf16", 2, True)])
-def test_group_union_attention_shares_rows(dtype, G, host_kv, monkeypatch):
+@pytest.mark.parametrize("dtype,G,host_kv,n,k", [("bf16", 4, True, 20000, 1024),
+                                                 ("f32", 4, False, 20000, 1024),
+                                                 ("bf16", 8, True, 20000, 1024),
+                                                 ("bf16", 3, True, 20000, 1024),
+                                                 ("bf16", 2, True, 20000, 1024),
+                                                 ("bf16", 4, True, 20001, 999),
+                                                 ("f32", 2, False, 70, 33)])
+def test_group_union_attention_shares_rows(dtype, G, host_kv, n, k, monkeypatch):
     """The query heads of a group select overlapping rows (a common core, a shared pool and
     rows of their own); the row-gather attention fetches each row of the group's union once
     and still matches the oracle per head at 2e-3. The fetched-row count equals the union
     size, and turning the union off gives the same outputs within the same bound."""
-    rng = np.random.default_rng(31 + G)
-    batch, hkv, n, k = 2, 2, 20000, 1024
+    rng = np.random.default_rng(31 + G + n)
+    batch, hkv = 2, 2
     K = rng.standard_normal((batch, hkv, n, 128)).astype(np.float32) * 0.5
     V = rng.standard_normal((batch, hkv, n, 128)).astype(np.float32)
     q = rng.standard_normal((batch, hkv * G, 128)).astype(np.float32)
