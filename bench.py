@@ -749,6 +749,28 @@ def main():
                 "step_frac": step_bytes / (step_ms_max / 1e3) / 1e9 / peak,
                 "step_frac_of_nominal_8tbs": step_bytes / (step_ms_max / 1e3) / 8e12}
 
+    # the rerank's gathers alone: the last search's candidate records read once per query head
+    # with the rerank's access pattern and no arithmetic, timed like the stages (L2 flushed).
+    # A random 128-byte gather cannot reach the copy rate, so this rate is the rerank's
+    # practical ceiling; the rerank's fraction of it shows what its arithmetic costs.
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(3):
+        ix.gather_candidates(sink)
+    for s in range(args.steps):
+        flush.fill_(s & 255)
+        ev0[s].record()
+        ix.gather_candidates(sink)
+        ev1[s].record()
+    torch.cuda.synchronize()
+    gather_ms = dist_max(float(np.mean([a.elapsed_time(b) for a, b in zip(ev0, ev1)])), ws)
+    rbytes = algorithmic_bytes("rerank", sp, C)
+    gather_gbs = rbytes / (gather_ms / 1e3) / 1e9
+    rerank_gbs = rbytes / (stage_avg["rerank"] / 1e3) / 1e9
+    roofline["gather_ceiling"] = {"kernel": "record gather without arithmetic",
+                                  "ms": gather_ms, "achieved": gather_gbs, "unit": "GB/s",
+                                  "frac_of_peak": gather_gbs / peak,
+                                  "rerank_frac_of_ceiling": rerank_gbs / gather_gbs}
+
     # host cost of enqueueing one search (the device is kept busy meanwhile), and the same
     # search replayed as a CUDA graph (one launch per step, no host work between kernels)
     ix.profile(False)

@@ -108,6 +108,15 @@ PARISKV_API pariskv_status pariskv_debug_union_rows(int64_t* rows);
  * with no counterpart on the pages. Errors: EINVAL (guards off), ECUDA. */
 PARISKV_API pariskv_status pariskv_debug_check_guards(void);
 
+/* Reads the 128-byte records of the last search's candidates once, for every query head (the
+ * rerank's memory access: sorted random records of a 1 GiB-scale array, 16-byte loads, eight
+ * lanes per record), with no arithmetic on them, on `stream`; `sink` (a device pointer to 4
+ * bytes) may receive a fold of the data. Timed with CUDA events it measures the gather rate
+ * that bounds the rerank, next to the copy rate of MEASURED peaks. No counterpart on the
+ * pages (a measurement aid). Errors: EINVAL (no search yet), ECUDA. */
+PARISKV_API pariskv_status pariskv_debug_gather_candidates(pariskv_index* index, uint32_t* sink,
+                                                           void* stream);
+
 /* Reads `bytes` from `src` once, with coalesced 16-byte loads spread over every SM, and
  * folds the data into one word that may be written to `sink` (a device pointer to 4 bytes),
  * on `stream`. Timed with CUDA events around the call it measures how fast the device reads

@@ -968,6 +968,19 @@ pariskv_status pariskv_debug_check_guards(void) {
     return PARISKV_OK;
 }
 
+pariskv_status pariskv_debug_gather_candidates(pariskv_index* ix, uint32_t* sink, void* stream) {
+    pariskv_status s = check_index(ix);
+    if (s != PARISKV_OK) return s;
+    if (!ix->searched) return fail(PARISKV_EINVAL, "no search has run on this index");
+    if ((s = check_dev_ptr(sink, 4, "sink")) != PARISKV_OK) return s;
+    const int64_t heads = static_cast<int64_t>(ix->units) * ix->cfg.group;
+    cudaError_t e = launch_gather_candidates(ix->rec, ix->cap_pad, ix->cand, ix->cmax,
+                                             static_cast<int32_t>(ix->last_C), ix->cfg.group,
+                                             heads, ix->n, sink, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+    return PARISKV_OK;
+}
+
 pariskv_status pariskv_debug_read_stream(const void* src, int64_t bytes, uint32_t* sink,
                                         void* stream) {
     if (bytes <= 0 || bytes % 16 != 0)

@@ -448,7 +448,52 @@ read_stream_kernel(const uint4* __restrict__ p, int64_t n16, uint32_t* __restric
     if (acc == 0x9E3779B9u) *sink = acc;   // keeps the loads; almost never stores
 }
 
+// The rerank's memory access alone: every (query head, candidate) pair's 128-byte record is
+// read with 16-byte loads (eight lanes per record, four records per warp instruction, eight
+// instructions in flight per lane) and folded into one word; no arithmetic on the data.
+// Warps take groups of 32 candidates of one head in turn.
+__global__ void __launch_bounds__(256)
+gather_candidates_kernel(const uint8_t* __restrict__ rec, int64_t cap_pad,
+                         const int32_t* __restrict__ cand, int64_t cmax, int32_t C, int group,
+                         int64_t heads, int64_t n, uint32_t* __restrict__ sink) {
+    const int lane = threadIdx.x & 31;
+    const int64_t gpr = (C + 31) / 32;                        // groups per head
+    const int64_t groups = heads * gpr;
+    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    uint32_t acc = 0;
+    for (int64_t gi = w0; gi < groups; gi += nw) {
+        const int64_t h = gi / gpr, j0 = (gi - h * gpr) * 32;
+        const uint8_t* base = rec + (h / group) * cap_pad * 128;
+        const int64_t j = j0 + lane;
+        const int32_t idx = j < C ? cand[h * cmax + j] : -1;
+        uint4 v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int32_t r = __shfl_sync(0xffffffffu, idx, 4 * i + (lane >> 3));
+            v[i] = (r >= 0 && r < n)
+                       ? __ldcs(reinterpret_cast<const uint4*>(base + static_cast<int64_t>(r) * 128) +
+                                (lane & 7))
+                       : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc ^= v[i].x ^ v[i].y ^ v[i].z ^ v[i].w;
+    }
+    if (acc == 0x9E3779B9u) *sink = acc;   // keeps the loads; almost never stores
+}
+
 }  // namespace
+
+cudaError_t launch_gather_candidates(const uint8_t* rec, int64_t cap_pad, const int32_t* cand,
+                                     int64_t cmax, int32_t C, int group, int64_t heads,
+                                     int64_t n, uint32_t* sink, cudaStream_t st) {
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    gather_candidates_kernel<<<4 * sms, 256, 0, st>>>(rec, cap_pad, cand, cmax, C, group, heads, n,
+                                                      sink);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_read_stream(const void* src, int64_t bytes, uint32_t* sink,
                                cudaStream_t st) {

@@ -155,6 +155,10 @@ cudaError_t launch_topk(const pariskv_index* ix, int64_t C, int32_t k, int32_t* 
 // attend.cu
 cudaError_t launch_read_stream(const void* src, int64_t bytes, uint32_t* sink,
                                cudaStream_t st);
+// the rerank's record gathers alone (no arithmetic): the candidates' records of every head
+cudaError_t launch_gather_candidates(const uint8_t* rec, int64_t cap_pad, const int32_t* cand,
+                                     int64_t cmax, int32_t C, int group, int64_t heads,
+                                     int64_t n, uint32_t* sink, cudaStream_t st);
 // Sparse attention has two kernels: with bf16 K/V in device memory, the tensor-core gather
 // kernel of dense.cu (`mma` = true); otherwise (K/V in pinned host memory, or fp32) the
 // latency-tolerant row-gather kernel of attend.cu. attend_splits gives the split count for

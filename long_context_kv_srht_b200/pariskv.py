@@ -99,6 +99,7 @@ _SIGS = {
     "pariskv_debug_profile": (_S, [_P, _I32]),
     "pariskv_debug_stage_ms": (_S, [_P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_I32)]),
     "pariskv_debug_read_stream": (_S, [_P, _I64, _P, _P]),
+    "pariskv_debug_gather_candidates": (_S, [_P, _P, _P]),
     "pariskv_debug_inject_bad_candidate": (_S, [_P, _I32, _I64, _I32]),
     "pariskv_debug_set_launch": (_S, [_P, _I32, _I32, _I32]),
     "pariskv_debug_check_guards": (_S, []),
@@ -263,6 +264,12 @@ class Index:
         """pariskv_debug_set_launch: force the launch shapes of later searches (0: automatic)."""
         _check(lib.pariskv_debug_set_launch(self.handle, vote_ctas, rerank_ctas, topk_mode),
                "pariskv_debug_set_launch")
+
+    def gather_candidates(self, sink, stream=None) -> None:
+        """pariskv_debug_gather_candidates: the last search's candidate records read once,
+        without arithmetic (the rerank's gathers alone); ``sink`` a device tensor (4 bytes)."""
+        _check(lib.pariskv_debug_gather_candidates(self.handle, sink.data_ptr(), _stream(stream)),
+               "pariskv_debug_gather_candidates")
 
     def profile(self, enable: bool = True) -> None:
         _check(lib.pariskv_debug_profile(self.handle, int(enable)), "pariskv_debug_profile")

@@ -112,3 +112,20 @@ def test_guard_bytes_catch_a_write_past_a_buffer():
     with pytest.raises(pk.PariskvError):
         pk.check_guards()
     pk.check_guards()
+
+
+def test_candidate_gather_needs_a_search_and_leaves_results_alone():
+    n, k = 20000, 256
+    ix, q, cfg = _index(n)
+    sink = torch.zeros(1, dtype=torch.int32, device=DEV)
+    with pytest.raises(pk.PariskvError) as e:
+        ix.gather_candidates(sink)
+    assert e.value.status == pk.EINVAL
+    ref_idx, ref_est = ix.search(q, k)
+    ix.sync()
+    ref_idx, ref_est = ref_idx.clone(), ref_est.clone()
+    ix.gather_candidates(sink)
+    idx, est = ix.search(q, k)
+    ix.sync()
+    assert torch.equal(idx, ref_idx) and torch.equal(est, ref_est)
+    ix.destroy()
