@@ -79,6 +79,15 @@ PARISKV_API pariskv_status pariskv_debug_stage_ms(pariskv_index* index, float* m
 PARISKV_API pariskv_status pariskv_debug_inject_bad_candidate(pariskv_index* index, int32_t head,
                                                                int64_t pos, int32_t value);
 
+/* Test hook for the bounded device-side wait: the next pariskv_search's top-k arms the
+ * barrier of its part's bulk copies for 16 bytes more than the copies deliver, so the barrier
+ * never completes (the copies themselves do) and each CTA's wait runs out after about one
+ * second; the kernel then records a timeout and finishes, and pariskv_sync returns
+ * PARISKV_ETIMEOUT. The hook is consumed by that search. A search whose top-k stages no
+ * copies (C > 65,536 candidates, or launch shape 4) refuses it with EINVAL. No counterpart on
+ * the pages. Errors: EINVAL. */
+PARISKV_API pariskv_status pariskv_debug_inject_wait_timeout(pariskv_index* index);
+
 /* Forces the launch shapes of later searches on this index, for tests that require the same
  * bits from every shape: vote_ctas / rerank_ctas = the number of CTAs of the vote scan and of
  * the rerank (0: automatic; any positive count is valid, work is split over the CTAs), and

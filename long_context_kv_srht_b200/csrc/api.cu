@@ -346,6 +346,11 @@ pariskv_status run_search(pariskv_index* ix, const void* q, const float* qt, con
         return fail(PARISKV_EINVAL, "injected candidate position %lld >= C = %lld",
                     static_cast<long long>(ix->inject_pos), static_cast<long long>(C));
     }
+    if (ix->inject_wait && (ix->topk_mode == 4 || C > 4 * 16384)) {
+        ix->inject_wait = false;
+        return fail(PARISKV_EINVAL, "the top-k of C = %lld candidates stages no copies to wait for",
+                    static_cast<long long>(C));
+    }
     if (ix->topk_mode != 0 && !topk_mode_fits(ix->topk_mode, C))
         return fail(PARISKV_EINVAL, "top-k launch shape %d cannot hold C = %lld candidates",
                     ix->topk_mode, static_cast<long long>(C));
@@ -366,6 +371,7 @@ pariskv_status run_search(pariskv_index* ix, const void* q, const float* qt, con
     }
     if (e == cudaSuccess) { ++g_launches; mark(); e = launch_rerank(ix, C, st); }
     if (e == cudaSuccess) { ++g_launches; mark(); e = launch_topk(ix, C, k, topk_idx, topk_est, st); }
+    ix->inject_wait = false;
     if (e == cudaSuccess) { ++g_launches; mark(); }
     ix->nev = ne;
     if (e != cudaSuccess) return cuda_fail(e, "search launch");
@@ -928,6 +934,13 @@ pariskv_status pariskv_debug_inject_bad_candidate(pariskv_index* ix, int32_t hea
     ix->inject_head = head;
     ix->inject_pos = pos;
     ix->inject_value = value;
+    return PARISKV_OK;
+}
+
+pariskv_status pariskv_debug_inject_wait_timeout(pariskv_index* ix) {
+    pariskv_status s = check_index(ix);
+    if (s != PARISKV_OK) return s;
+    ix->inject_wait = true;
     return PARISKV_OK;
 }
 

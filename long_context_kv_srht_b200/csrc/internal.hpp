@@ -45,6 +45,7 @@ struct pariskv_index {
     int32_t inject_head = -1;
     int64_t inject_pos = 0;
     int32_t inject_value = 0;
+    bool inject_wait = false;   // test hook: the next top-k's copy wait runs out
     int32_t vote_ctas = 0, rerank_ctas = 0, topk_mode = 0;
 
     // optional per-stage timing of searches (test and benchmark use)

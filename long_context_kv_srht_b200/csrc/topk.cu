@@ -43,13 +43,22 @@ namespace cg = cooperative_groups;
 namespace {
 
 constexpr int kBins = 2048;
+// limit of the wait for the part's bulk copies: far above any copy's latency (microseconds),
+// short enough that a lost completion costs the caller about a second, not a hang
+constexpr uint64_t kCopyWaitNs = 1000000000ull;
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
 
 template <int CL, int T, int SLICE, bool RES>
 __global__ void __launch_bounds__(T, 1)
 topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
             const float* __restrict__ qnorm, const uint32_t* __restrict__ shist, int32_t C,
             int64_t cmax, int32_t k, int32_t* __restrict__ out_idx, float* __restrict__ out_est,
-            int* status) {
+            int* status, uint32_t extra_tx) {
     constexpr int kWarps = T / 32;
     constexpr int BPT = kBins / T;     // bins per thread: thread t owns bins BPT t .. BPT t + BPT - 1
     static_assert(kWarps <= 32 && kBins % T == 0 && (BPT == 2 || BPT == 8), "layout");
@@ -109,16 +118,18 @@ topk_kernel(const float* __restrict__ S, const int32_t* __restrict__ cand,
         }
         __syncthreads();
         if (threadIdx.x == 0 && bytes) {
-            mbar_arrive_expect_tx(bar, 2 * bytes);
+            // (extra_tx, normally 0, is a test hook: bytes no copy delivers, so the barrier
+            // never completes and the wait below runs out)
+            mbar_arrive_expect_tx(bar, 2 * bytes + extra_tx);
             bulk_g2s(smem_addr(dyn), S + head * cmax + a0, bytes, bar);
             bulk_g2s(smem_addr(dyn + SLICE + 8), cand + head * cmax + a0, bytes, bar);
         }
         if (bytes) {
-            // bounded: past about a second of polling the part is treated as lost and the
-            // status word records a timeout (never taken while the copies complete)
-            long long spins = 0;
+            // bounded: past kCopyWaitNs of polling the part is treated as lost and the status
+            // word records a timeout (never taken while the copies complete)
+            const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(bar, 0u)) {
-                if (++spins > (1LL << 26)) {
+                if (globaltimer_ns() - t0 > kCopyWaitNs) {
                     atomicExch(status, ST_TIMEOUT);
                     break;
                 }
@@ -301,7 +312,8 @@ cudaError_t launch_cfg(const pariskv_index* ix, int64_t C, int32_t k, int32_t* t
     return launch_pdl_cluster(topk_kernel<CL, T, SLICE, RES>, dim3(heads * CL), dim3(T), kDyn,
                               st, static_cast<unsigned>(CL), ix->S, ix->cand, ix->qnorm,
                               ix->shist, static_cast<int32_t>(C), ix->cmax, k, topk_idx,
-                              topk_est, ix->status);
+                              topk_est, ix->status,
+                              static_cast<uint32_t>(ix->inject_wait ? 16 : 0));
 }
 
 }  // namespace

@@ -102,6 +102,7 @@ _SIGS = {
     "pariskv_debug_gather_candidates": (_S, [_P, _P, _P]),
     "pariskv_debug_inject_bad_candidate": (_S, [_P, _I32, _I64, _I32]),
     "pariskv_debug_set_launch": (_S, [_P, _I32, _I32, _I32]),
+    "pariskv_debug_inject_wait_timeout": (_S, [_P]),
     "pariskv_debug_check_guards": (_S, []),
     "pariskv_debug_union_rows": (_S, [ctypes.POINTER(_I64)]),
     "pariskv_cache_create": (_S, [ctypes.POINTER(Config), ctypes.POINTER(CacheConfig), _P, _P,
@@ -264,6 +265,11 @@ class Index:
         """pariskv_debug_set_launch: force the launch shapes of later searches (0: automatic)."""
         _check(lib.pariskv_debug_set_launch(self.handle, vote_ctas, rerank_ctas, topk_mode),
                "pariskv_debug_set_launch")
+
+    def inject_wait_timeout(self) -> None:
+        """pariskv_debug_inject_wait_timeout: the next search's top-k copy wait runs out."""
+        _check(lib.pariskv_debug_inject_wait_timeout(self.handle),
+               "pariskv_debug_inject_wait_timeout")
 
     def gather_candidates(self, sink, stream=None) -> None:
         """pariskv_debug_gather_candidates: the last search's candidate records read once,

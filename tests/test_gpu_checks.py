@@ -6,7 +6,9 @@
   split over any number of CTAs, top-k on one CTA, on a cluster, from shared or global
   memory): no result depends on scheduling;
 * the guard bytes around the index's device buffers catch a write past a buffer's end (the
-  autouse fixture in conftest.py checks them after every GPU test).
+  autouse fixture in conftest.py checks them after every GPU test);
+* the top-k's bounded wait for its bulk copies runs out when a test hook arms its barrier for
+  bytes that never arrive, and the timeout reaches the caller as PARISKV_ETIMEOUT.
 """
 import numpy as np
 import pytest
@@ -128,4 +130,39 @@ def test_candidate_gather_needs_a_search_and_leaves_results_alone():
     idx, est = ix.search(q, k)
     ix.sync()
     assert torch.equal(idx, ref_idx) and torch.equal(est, ref_est)
+    ix.destroy()
+
+
+def test_bounded_copy_wait_runs_out_and_is_reported():
+    # the hook arms the top-k's copy barrier for 16 bytes that never arrive: every CTA's wait
+    # runs out after about a second, the kernel finishes, and the status word reports it
+    import time
+    n, k = 20000, 256
+    ix, q, cfg = _index(n)
+    ref_idx, ref_est = ix.search(q, k)
+    ix.sync()
+    ref_idx, ref_est = ref_idx.clone(), ref_est.clone()
+    for mode in (0, 3):          # one CTA per head; a four-CTA cluster per head
+        ix.set_launch(0, 0, mode)
+        ix.inject_wait_timeout()
+        t0 = time.perf_counter()
+        ix.search(q, k)
+        with pytest.raises(pk.PariskvError) as e:
+            ix.sync()
+        waited = time.perf_counter() - t0
+        assert e.value.status == pk.ETIMEOUT, e.value
+        assert 0.9 <= waited < 30.0, waited
+        # consumed: the next search is clean and gives the reference bits
+        idx, est = ix.search(q, k)
+        ix.sync()
+        assert torch.equal(idx, ref_idx) and torch.equal(est, ref_est)
+    # a top-k that reads its part from global memory has no copy to wait for
+    ix.set_launch(0, 0, 4)
+    ix.inject_wait_timeout()
+    with pytest.raises(pk.PariskvError) as e:
+        ix.search(q, k)
+    assert e.value.status == pk.EINVAL
+    ix.set_launch(0, 0, 0)
+    ix.search(q, k)
+    ix.sync()
     ix.destroy()
