@@ -218,16 +218,16 @@ __device__ __forceinline__ bool stage_query(const float* __restrict__ qt, int64_
     return ok;
 }
 
-// Work is cut into items of kItem consecutive candidates of one query head; warp g of the
-// grid takes items g, g + W, g + 2 W, ... (W warps in all), so within a stage the head, its
-// unit's record base and its rotated query are the same for every lane.
-constexpr int kItem = 256;
+// Work is cut into stages of kStageRecs consecutive candidates of one query head, numbered
+// head by head; warp g of the grid (W warps in all) takes the contiguous run of stages
+// [total g / W, total (g + 1) / W), so every warp has the same number of stages to within
+// one, and within a stage the head, its unit's record base and its rotated query are the
+// same for every lane.
 constexpr uint32_t kNoRec = 0xffffffffu;
 
 struct StreamPos {
-    int64_t it;            // item
-    int s, nst;            // stage within the item, stages in the item
-    int head, c0, cend;    // query head, first candidate, one past the item's last
+    int64_t t;             // stage (over all heads)
+    int head, c0, cend;    // query head, first candidate, one past the stage's last
     const uint8_t* ubase;  // records of the head's unit
 };
 
@@ -235,7 +235,7 @@ template <bool TABLE>
 __global__ void __launch_bounds__(kThr, kCtasPerSm)
 rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
               const float* __restrict__ qt, float* __restrict__ S, int32_t C, int64_t cmax,
-              int64_t cap_pad, int64_t n, int group, int iph, int64_t items,
+              int64_t cap_pad, int64_t n, int group, int64_t total,
               uint32_t* __restrict__ shist, int* status, const float* __restrict__ lvt) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ float dec[16];   // table levels: code nibble -> signed level
@@ -253,20 +253,24 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
     const int64_t W = static_cast<int64_t>(gridDim.x) * kWarps;
     const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
 
-    auto start_item = [&](StreamPos& p) {
-        if (p.it >= items) return;
-        p.head = static_cast<int>(p.it / iph);
-        p.c0 = static_cast<int>(p.it - static_cast<int64_t>(p.head) * iph) * kItem;
-        p.cend = min(C, p.c0 + kItem);
-        p.nst = (p.cend - p.c0 + kStageRecs - 1) / kStageRecs;
-        p.s = 0;
+    const int64_t nst = (C + kStageRecs - 1) / kStageRecs;   // stages per head
+    const int64_t t_end = total * (gw + 1) / W;
+    auto start_at = [&](StreamPos& p, int64_t t) {
+        p.t = t;
+        p.head = static_cast<int>(t / nst);
+        p.c0 = static_cast<int>(t - p.head * nst) * kStageRecs;
+        p.cend = min(C, p.c0 + kStageRecs);
         p.ubase = rec + static_cast<int64_t>(p.head / group) * cap_pad * REC;
     };
     auto advance = [&](StreamPos& p) {
-        if (++p.s == p.nst) {
-            p.it += W;
-            start_item(p);
+        ++p.t;
+        p.c0 += kStageRecs;
+        if (p.c0 >= C) {
+            ++p.head;
+            p.c0 = 0;
+            p.ubase = rec + static_cast<int64_t>(p.head / group) * cap_pad * REC;
         }
+        p.cend = min(C, p.c0 + kStageRecs);
     };
     // candidate indices of this lane's records (rows lane, lane + 32) in the stage at p,
     // loaded one stage ahead of their use so the loads overlap the scoring of a stage
@@ -275,16 +279,16 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
         Idx r;
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
-            const int c = p.c0 + kStageRecs * p.s + 32 * u + lane;
-            r.v[u] = (p.it < items && c < p.cend) ? static_cast<uint32_t>(cand[p.head * cmax + c])
-                                                  : kNoRec;
+            const int c = p.c0 + 32 * u + lane;
+            r.v[u] = (p.t < t_end && c < p.cend) ? static_cast<uint32_t>(cand[p.head * cmax + c])
+                                                 : kNoRec;
         }
         return r;
     };
     // stage refill: for copy instruction j, lanes 8g..8g+7 move the 8 16-byte pieces of
     // record 4j + g (whose index lane (4j + g) mod 32 holds)
     auto issue = [&](int slot, const StreamPos& p, Idx idx) {
-        if (p.it < items) {
+        if (p.t < t_end) {
 #pragma unroll
             for (int u = 0; u < kPerLane; ++u) {
                 if (idx.v[u] != kNoRec && idx.v[u] >= static_cast<uint64_t>(n)) {
@@ -311,21 +315,21 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
 
     pdl_wait();
     pdl_launch_dependents();
-    StreamPos iss{gw, 0, 0, 0, 0, 0, rec}, sc{gw, 0, 0, 0, 0, 0, rec};
-    start_item(iss);
-    start_item(sc);
+    StreamPos iss, sc;
+    start_at(iss, total * gw / W);
+    start_at(sc, total * gw / W);
     // prologue: fill the ring
     Idx pend = load_idx(iss);
     for (int g = 0; g < kSlots; ++g) {
         issue(g, iss, pend);
-        if (iss.it < items) advance(iss);
+        if (iss.t < t_end) advance(iss);
         pend = load_idx(iss);
     }
 
     int staged = -1;       // head whose query is in qs
     bool scaled = false;   // its scaled pairs are exact
 #pragma unroll 1
-    for (int g = 0; sc.it < items; ++g) {
+    for (int g = 0; sc.t < t_end; ++g) {
         const int slot = g % kSlots;
         // the oldest committed group is this stage's; each lane waits for its own pieces and
         // the warp barrier makes every lane's pieces visible
@@ -341,7 +345,7 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
         else score_records<TABLE, false>(st, lane, qp, dec, sv);
 #pragma unroll
         for (int u = 0; u < kPerLane; ++u) {
-            const int c = sc.c0 + kStageRecs * sc.s + 32 * u + lane;
+            const int c = sc.c0 + 32 * u + lane;
             const bool ok = c < sc.cend && pkv_check(c < cmax, status);   // (checked build)
             if (ok) S[sc.head * cmax + c] = sv[u];
             // the top-k's first radix level: count the values by their top order-key bits,
@@ -355,7 +359,7 @@ rerank_kernel(const uint8_t* __restrict__ rec, const int32_t* __restrict__ cand,
         }
         __syncwarp();                        // every lane has read the slot and the query
         issue(slot, iss, pend);
-        if (iss.it < items) advance(iss);
+        if (iss.t < t_end) advance(iss);
         pend = load_idx(iss);
         advance(sc);
     }
@@ -376,13 +380,14 @@ cudaError_t launch_rerank(const pariskv_index* ix, int64_t C, cudaStream_t st) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int heads = ix->units * ix->cfg.group;
-    const int iph = static_cast<int>(ceil_div(C, kItem));
-    const int64_t items = static_cast<int64_t>(heads) * iph;
-    const int grid =
-        static_cast<int>(max64(1, min64(int64_t{kCtasPerSm} * sms, ceil_div(items, kWarps))));
+    const int64_t total = static_cast<int64_t>(heads) * ceil_div(C, kStageRecs);
+    const int grid = ix->rerank_ctas > 0   // (a launch shape forced by the determinism tests)
+                         ? ix->rerank_ctas
+                         : static_cast<int>(max64(1, min64(int64_t{kCtasPerSm} * sms,
+                                                           ceil_div(total, kWarps))));
     return launch_pdl(table ? rerank_kernel<true> : rerank_kernel<false>, grid, kThr, kSmem, st,
                       ix->rec, ix->cand, ix->qt, ix->S, static_cast<int32_t>(C), ix->cmax,
-                      ix->cap_pad, ix->n, ix->cfg.group, iph, items, ix->shist, ix->status,
+                      ix->cap_pad, ix->n, ix->cfg.group, total, ix->shist, ix->status,
                       static_cast<const float*>(ix->lvt));
 }
 
