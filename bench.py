@@ -30,8 +30,26 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 L2_FLUSH_BYTES = 256 << 20
+L2_NOTE = (f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write, then "
+           f"{L2_FLUSH_BYTES >> 20} MiB read of another buffer)")
 APPEND_SLACK = 64
 LEARNED_ITERS = 10          # spherical k-means iterations of the learned-centroid comparator
+
+
+class L2Flush:
+    """Evicts the step's data from L2 between timed steps: writes a buffer larger than L2,
+    then reads another buffer as large, so that L2 is left holding clean lines (the write's
+    dirty lines are written back here, outside the timed region, rather than during the
+    next step's own DRAM traffic)."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+
+    def __call__(self, s: int) -> None:
+        self.w.fill_(s & 255)
+        self.r.sum()
 
 
 def parse():
@@ -422,7 +440,7 @@ def side_workload(name, args, dev, flush):
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     for s in range(steps):
-        flush.fill_(s & 255)
+        flush(s)
         ev0[s].record()
         ix.search(qs, k, idx, est)
         ev1[s].record()
@@ -544,7 +562,7 @@ def run_drift(args, ws, rank, local):
         ix = pk.build_index(cfg, w.signs, pre)
     idx = torch.empty((H, k), dtype=torch.int32, device=dev)
     est = torch.empty((H, k), dtype=torch.float32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     W = max(0, min(args.warmup, T - 1))
     for t in range(W):
         ix.append(app[t].view(1, H, 1, 128))
@@ -562,7 +580,7 @@ def run_drift(args, ws, rank, local):
     torch.cuda.synchronize()
     launches = 0
     for i, t in enumerate(range(W, T)):
-        flush.fill_(t & 255)
+        flush(t)
         ev[i][0].record()
         ix.append(app[t].view(1, H, 1, 128))
         ev[i][1].record()
@@ -602,7 +620,7 @@ def run_drift(args, ws, rank, local):
                        "rho": sp.rho, "cand_bp": sp.cand_bp, "key_dtype": sp.dtype,
                        "levels": args.levels, "centroids": args.centroids,
                        "step": "append one key per KV head + one search",
-                       "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"},
+                       "l2": L2_NOTE},
             "decode_step": {"append_ms": app_ms, "search_ms": srch_ms},
             "recall_vs_exact_topk": rec,
             "recall_mean": float(np.mean(list(rec.values()))),
@@ -691,7 +709,7 @@ def main():
     C = candidate_count(sp.n, k, sp.cand_bp)
     idx = torch.empty((H, k), dtype=torch.int32, device=dev)
     est = torch.empty((H, k), dtype=torch.float32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     for _ in range(args.warmup):
         ix.search(qs, k, idx, est)
     torch.cuda.synchronize()
@@ -707,7 +725,7 @@ def main():
     ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     launches = 0
     for s in range(args.steps):
-        flush.fill_(s & 255)                    # L2 flushed between timed steps
+        flush(s)                    # L2 flushed between timed steps
         ev0[s].record()
         ix.search(qs, k, idx, est)
         ev1[s].record()
@@ -727,7 +745,7 @@ def main():
     ix.profile(True)
     stage_tot = {}
     for s in range(args.steps):
-        flush.fill_(s & 255)
+        flush(s)
         ix.search(qs, k, idx, est)
         for name, ms in ix.stage_ms().items():
             stage_tot[name] = stage_tot.get(name, 0.0) + ms
@@ -757,7 +775,7 @@ def main():
     for _ in range(3):
         ix.gather_candidates(sink)
     for s in range(args.steps):
-        flush.fill_(s & 255)
+        flush(s)
         ev0[s].record()
         ix.gather_candidates(sink)
         ev1[s].record()
@@ -797,7 +815,7 @@ def main():
     torch.cuda.synchronize()
     gtimes = []
     for s in range(args.steps):
-        flush.fill_(s & 255)
+        flush(s)
         ev0[s].record()
         graph.replay()
         ev1[s].record()
@@ -820,7 +838,7 @@ def main():
         tot = 0.0
         nrep = max(3, min(args.steps, 50))
         for s in range(nrep + 2):
-            flush.fill_(s & 255)
+            flush(s)
             e0.record()
             q_dev.copy_(q_host, non_blocking=True)
             ix.search(q_dev, k, idx, est)
@@ -880,7 +898,7 @@ def main():
                        "candidates": C, "B": sp.B, "m": sp.m, "rho": sp.rho,
                        "key_dtype": sp.dtype, "kv_in": "pinned host" if kv_host else "HBM",
                        "levels": args.levels,
-                       "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)"},
+                       "l2": L2_NOTE},
             "stage_ms": stage_avg,
             "host_enqueue_us_per_search": host_us,
             "graph": {"ms_per_step": graph_ms, "value": graph_value},
