@@ -56,6 +56,11 @@ def test_status_strings_and_null_handles():
     assert pk.lib.pariskv_size(None) == -1
     assert pk.lib.pariskv_destroy(None) == pk.OK
     assert pk.lib.pariskv_search(None, None, 1, None, None, None) == pk.EINVAL
+    # the debug hooks refuse a NULL index before touching the device
+    assert pk.lib.pariskv_debug_inject_wait_timeout(None) == pk.EINVAL
+    assert pk.lib.pariskv_debug_inject_bad_candidate(None, 0, 0, -2) == pk.EINVAL
+    assert pk.lib.pariskv_debug_set_launch(None, 0, 0, 0) == pk.EINVAL
+    assert pk.lib.pariskv_debug_gather_candidates(None, None, None) == pk.EINVAL
 
 
 # ------------------------------------------------------------------ index images (host checks)
